@@ -1,0 +1,507 @@
+"""Plain CPU float64 oracle for RBS block selection, block-sparse prefill
+attention, Block-attention lists and RoPE position re-encoding.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this module.  It shares no code with the CUDA library: it reads the same bf16
+input bytes (widened exactly to float64) and computes every step from its
+plain definition with numpy, one step per function, in the order the sources
+give them.  It is slow on purpose.
+
+Sources (web pages; cited by title and section):
+
+* [RBS-en] "RBS-Attention: How a Geometric Rescue Branch Fixes Sparse Prefill
+  for Long-Context LLMs" -- sections "The Standard Approach and Its Blind
+  Spot" (centroid = average of the block's keys; radius = largest distance of
+  a key from the centroid) and "The Fix: A Radius-Adaptive Rescue Branch"
+  (centroid branch q^T c_b; rescue branch q^T c_b + |q|_2 r_b beta_b with
+  beta_b in [0, 1] taken from the radius distribution; branches thresholded
+  independently, masks combined; Cauchy-Schwarz bound; exact block-sparse
+  attention on the result).
+* [RBS-id] "RBS-Attention Bikin Prefill LLM Gede 20x Lebih Cepat, Tanpa
+  Training Lagi?" -- section "Dual-Branch Selection: Centroid Base + Rescue
+  Branch" (radius distribution per prompt, per layer, per head; the two
+  branches thresholded independently; masks merged).
+* [BA] "Block-Attention for Efficient Prefilling" -- 2.1 Main idea, 2.2 Block
+  segmentation, 2.3 Position re-encoding, 2.4 Block fine-tune (mask), 2.5
+  Inference.
+
+Readings of points the pages leave open (each is a parameter here):
+  query representative = mean of the query block's queries; raw dot-product
+  scores (no 1/sqrt(d)); beta = per (prompt, KV head) min-max normalisation of
+  the radii with quantiles (p_lo, p_hi) (type-7, linear interpolation), a
+  degenerate range giving beta = 1; per-branch threshold = keep the
+  k_i = ceil(rho * n_i) best of the n_i causally visible blocks, ties to the
+  lower block index; the diagonal block is always kept and does not count
+  toward k_i; RoPE = rotate-half pairs (m, m + d/2) with
+  inv_freq_m = theta^(-2m/d).
+
+Pins: every function here is checked in tests/test_oracle_pins.py against a
+closed form, a library routine, an invariant the pages state, or brute force.
+Parity unpinned: none of the functions below.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# bf16 storage -> float64
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def as_f64(x: np.ndarray) -> np.ndarray:
+    """Accept either bf16 bits (uint16) or floating arrays; return float64."""
+    if x.dtype == np.uint16:
+        return bf16_to_f64(x)
+    return np.asarray(x, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# Parameters of the selection (mirrors the C struct field by field)
+
+
+@dataclasses.dataclass
+class SelectParams:
+    block_q: int = 128
+    block_k: int = 128
+    rho_centroid: float = 0.05
+    rho_rescue: float = 0.05
+    beta_mode: int = 0  # 0 = RANGE (quantile min-max of the radii), 1 = CONST
+    beta_const: float = 1.0
+    beta_p_lo: float = 0.0  # < 0 means R_lo = 0
+    beta_p_hi: float = 1.0
+    force_diag: int = 1
+    force_sink: int = 0
+    causal: int = 1
+    q_block_offset: int = 0  # global index of query block 0 (in key blocks)
+
+
+FLAG_CENTROID = 1
+FLAG_RESCUE = 2
+FLAG_FORCED = 4
+
+
+# ----------------------------------------------------------------------------
+# Block statistics  [RBS-en, "The Standard Approach and Its Blind Spot"]
+
+
+def block_stats(K: np.ndarray, block_k: int):
+    """Centroid and radius of every key block.
+
+    K: [B, L, Hkv, d] (bf16 bits or float), L a multiple of block_k.
+    c_b = (1/n_b) sum_{k in b} k ;  r_b = max_{k in b} ||k - c_b||_2.
+    Returns centroids [B, Hkv, nKB, d] and radii [B, Hkv, nKB], float64.
+    """
+    B, L, H, d = K.shape
+    assert L % block_k == 0
+    nkb = L // block_k
+    C = np.empty((B, H, nkb, d))
+    R = np.empty((B, H, nkb))
+    for b in range(B):
+        for h in range(H):
+            kb = as_f64(K[b, :, h, :]).reshape(nkb, block_k, d)
+            c = kb.sum(axis=1) / block_k
+            dist = np.sqrt(((kb - c[:, None, :]) ** 2).sum(axis=2))
+            C[b, h] = c
+            R[b, h] = dist.max(axis=1)
+    return C, R
+
+
+# ----------------------------------------------------------------------------
+# Rescue coefficient beta_b  [RBS-en "The Fix"; RBS-id "Dual-Branch Selection"]
+
+
+def quantile_type7(x: np.ndarray, p: float) -> float:
+    """Linear-interpolation sample quantile (Hyndman-Fan type 7)."""
+    xs = np.sort(np.asarray(x, dtype=np.float64).ravel())
+    n = xs.size
+    h = (n - 1) * p
+    lo = int(math.floor(h))
+    hi = min(lo + 1, n - 1)
+    return float(xs[lo] + (h - lo) * (xs[hi] - xs[lo]))
+
+
+def rescue_beta(R: np.ndarray, p: SelectParams):
+    """beta [B, Hkv, nKB] in [0, 1] and the (R_lo, R_hi) range per (batch, KV head).
+
+    RANGE mode: beta_b = clamp((r_b - R_lo) / (R_hi - R_lo), 0, 1) where
+    R_lo, R_hi are the p_lo / p_hi quantiles of the radii of that prompt and
+    KV head (R_lo = 0 when p_lo < 0); a range of (relative) width <= 1e-12
+    gives beta = 1.  CONST mode: beta_b = beta_const.
+    """
+    B, H, nkb = R.shape
+    beta = np.empty_like(R)
+    rng = np.empty((B, H, 2))
+    for b in range(B):
+        for h in range(H):
+            r = R[b, h]
+            if p.beta_mode == 1:
+                beta[b, h] = p.beta_const
+                rng[b, h] = (0.0, 0.0)
+                continue
+            r_lo = 0.0 if p.beta_p_lo < 0 else quantile_type7(r, p.beta_p_lo)
+            r_hi = quantile_type7(r, p.beta_p_hi)
+            rng[b, h] = (r_lo, r_hi)
+            if r_hi - r_lo <= 1e-12 * max(r_hi, 1e-30):
+                beta[b, h] = 1.0
+            else:
+                beta[b, h] = np.clip((r - r_lo) / (r_hi - r_lo), 0.0, 1.0)
+    return beta, rng
+
+
+# ----------------------------------------------------------------------------
+# Query-block representative  [RBS-en "The Fix": the q in q^T c_b]
+
+
+def pooled_queries(Q: np.ndarray, block_q: int):
+    """Mean query of every query block and its Euclidean norm.
+
+    Q: [B, L, Hq, d].  Returns qbar [B, Hq, nQB, d] and qnorm [B, Hq, nQB].
+    """
+    B, L, H, d = Q.shape
+    assert L % block_q == 0
+    nqb = L // block_q
+    qbar = np.empty((B, H, nqb, d))
+    for b in range(B):
+        for h in range(H):
+            qbar[b, h] = as_f64(Q[b, :, h, :]).reshape(nqb, block_q, d).sum(axis=1) / block_q
+    qnorm = np.sqrt((qbar ** 2).sum(axis=-1))
+    return qbar, qnorm
+
+
+# ----------------------------------------------------------------------------
+# Branch scores, per-branch threshold, union  [RBS-en "The Fix"; RBS-id]
+
+
+def keep_count(rho: float, n: int) -> int:
+    """k = ceil(rho * n), at least 1 and at most n (the 1e-9 absorbs rho*n rounding)."""
+    return int(min(n, max(1, math.ceil(rho * n - 1e-9))))
+
+
+def visible_blocks(i: int, nkb: int, p: SelectParams) -> int:
+    """Number of key blocks query block i may select: 0..i+offset when causal, else all."""
+    if p.causal:
+        return min(nkb, i + p.q_block_offset + 1)
+    return nkb
+
+
+def top_k_desc(scores: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k best scores, best first: higher score first, ties to the lower index."""
+    order = np.argsort(-scores, kind="stable")
+    return order[:k]
+
+
+def branch_scores(qbar: np.ndarray, qnorm: np.ndarray, C: np.ndarray, R: np.ndarray, beta: np.ndarray):
+    """Centroid-branch and rescue-branch scores of one (prompt, q head).
+
+    qbar [nQB, d], qnorm [nQB], C [nKB, d], R, beta [nKB] (the q head's KV head).
+    s_c(i, j) = qbar_i . c_j ;  s_r(i, j) = s_c(i, j) + |qbar_i| * r_j * beta_j.
+    """
+    s_c = qbar @ C.T
+    s_r = s_c + qnorm[:, None] * (R * beta)[None, :]
+    return s_c, s_r
+
+
+def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, keep_scores: bool = False):
+    """Per-query-block KV-block lists (CSR), rows ordered (batch, q head, query block).
+
+    For each row: both branches keep their own top-k_i of the visible blocks
+    (k_i = keep_count(rho_branch, n_i)); the row's list is the union of the
+    two kept sets plus the forced diagonal (and block 0 when force_sink),
+    sorted ascending.  flags: bit0 centroid kept, bit1 rescue kept, bit2 forced.
+    Also returns each row's per-branch threshold tau (the k_i-th kept score)
+    and, with keep_scores, the score matrices (for the near-threshold rule).
+    """
+    B, L, Hq, d = Q.shape
+    _, Hkv, nkb, _ = C.shape
+    G = Hq // Hkv
+    beta, _ = rescue_beta(R, p)
+    qbar, qnorm = pooled_queries(Q, p.block_q)
+    nqb = qbar.shape[2]
+    row_ptr = [0]
+    cols, flags = [], []
+    tau = np.zeros((B, Hq, nqb, 2))
+    kept_k = np.zeros((B, Hq, nqb, 2), dtype=np.int64)
+    scores = {} if keep_scores else None
+    for b in range(B):
+        for hq in range(Hq):
+            kvh = hq // G
+            s_c, s_r = branch_scores(qbar[b, hq], qnorm[b, hq], C[b, kvh], R[b, kvh], beta[b, kvh])
+            if keep_scores:
+                scores[(b, hq)] = (s_c, s_r)
+            for i in range(nqb):
+                n = visible_blocks(i, nkb, p)
+                kc = keep_count(p.rho_centroid, n)
+                kr = keep_count(p.rho_rescue, n)
+                top_c = top_k_desc(s_c[i, :n], kc)
+                top_r = top_k_desc(s_r[i, :n], kr)
+                tau[b, hq, i] = (s_c[i, top_c[-1]], s_r[i, top_r[-1]])
+                kept_k[b, hq, i] = (kc, kr)
+                f = np.zeros(nkb, dtype=np.uint8)
+                f[top_c] |= FLAG_CENTROID
+                f[top_r] |= FLAG_RESCUE
+                diag = i + p.q_block_offset
+                if p.force_diag and diag < nkb:
+                    f[diag] |= FLAG_FORCED
+                if p.force_sink:
+                    f[0] |= FLAG_FORCED
+                sel = np.nonzero(f)[0]
+                cols.extend(sel.tolist())
+                flags.extend(f[sel].tolist())
+                row_ptr.append(len(cols))
+    out = {
+        "row_ptr": np.asarray(row_ptr, dtype=np.int64),
+        "col_idx": np.asarray(cols, dtype=np.int64),
+        "flags": np.asarray(flags, dtype=np.uint8),
+        "tau": tau,
+        "k": kept_k,
+        "beta": beta,
+        "qbar": qbar,
+        "qnorm": qnorm,
+    }
+    if keep_scores:
+        out["scores"] = scores
+    return out
+
+
+def list_density(row_ptr: np.ndarray, nqb: int, nkb: int, q_block_offset: int = 0, causal: int = 1) -> float:
+    """Kept-block density: selected (row, block) pairs over visible pairs."""
+    rows = row_ptr.size - 1
+    per_head_visible = sum(min(nkb, i + q_block_offset + 1) if causal else nkb for i in range(nqb))
+    return float(row_ptr[-1]) / (per_head_visible * (rows // nqb))
+
+
+def union_ranks(Q, C, R, p: SelectParams):
+    """For every row: each visible block's better rank over the two branches, and the forced mask.
+
+    rank = position in the branch's best-first order (higher score first, ties
+    to the lower index).  With both branches at the same rho, block j is kept
+    iff min(rank_c, rank_r) < k_i(rho) or j is forced: the same set
+    select_blocks builds.
+    """
+    B, L, Hq, d = Q.shape
+    _, Hkv, nkb, _ = C.shape
+    G = Hq // Hkv
+    beta, _ = rescue_beta(R, p)
+    qbar, qnorm = pooled_queries(Q, p.block_q)
+    nqb = qbar.shape[2]
+    rows = []
+    for b in range(B):
+        for hq in range(Hq):
+            kvh = hq // G
+            s_c, s_r = branch_scores(qbar[b, hq], qnorm[b, hq], C[b, kvh], R[b, kvh], beta[b, kvh])
+            for i in range(nqb):
+                n = visible_blocks(i, nkb, p)
+                rank_c = np.empty(n, dtype=np.int64)
+                rank_c[top_k_desc(s_c[i, :n], n)] = np.arange(n)
+                rank_r = np.empty(n, dtype=np.int64)
+                rank_r[top_k_desc(s_r[i, :n], n)] = np.arange(n)
+                forced = np.zeros(n, dtype=bool)
+                diag = i + p.q_block_offset
+                if p.force_diag and diag < n:
+                    forced[diag] = True
+                if p.force_sink:
+                    forced[0] = True
+                rows.append((np.minimum(rank_c, rank_r), forced))
+    return rows
+
+
+def density_of(rows, rho: float) -> float:
+    """Kept-union density at a shared per-branch rho, from union_ranks output."""
+    kept = visible = 0
+    for best, forced in rows:
+        n = best.size
+        kept += np.count_nonzero((best < keep_count(rho, n)) | forced)
+        visible += n
+    return kept / visible
+
+
+def bisect_rho(Q, C, R, p: SelectParams, target: float, steps: int = 30):
+    """Shared per-branch rho whose kept-union density is closest to ``target``.
+
+    Density is monotone in rho (each branch's top-k sets are nested), so a
+    bisection on [0, 1] converges.  Returns (rho, achieved density).
+    """
+    rows = union_ranks(Q, C, R, p)
+    lo, hi = 0.0, 1.0
+    best = None
+    for _ in range(steps):
+        mid = 0.5 * (lo + hi)
+        dens = density_of(rows, mid)
+        if best is None or abs(dens - target) < abs(best[1] - target):
+            best = (mid, dens)
+        if dens < target:
+            lo = mid
+        else:
+            hi = mid
+    return best
+
+
+# ----------------------------------------------------------------------------
+# List builders: causal-full and Block-attention  [BA 2.1, 2.2, 2.4]
+
+
+def causal_full_lists(batch: int, heads_q: int, nqb: int, q_block_offset: int = 0):
+    """Every causally visible block for every row: j in [0, i + offset]."""
+    row_ptr = [0]
+    cols = []
+    for _ in range(batch * heads_q):
+        for i in range(nqb):
+            cols.extend(range(0, i + q_block_offset + 1))
+            row_ptr.append(len(cols))
+    return np.asarray(row_ptr, dtype=np.int64), np.asarray(cols, dtype=np.int64)
+
+
+def block_attention_lists(seg_start, final_start: int, block: int, batch: int, heads_q: int,
+                          q_first_block: int, q_num_blocks: int):
+    """Block-attention mask as per-query-block lists.
+
+    Segments: passage s covers tokens [seg_start[s], next start); the final
+    block (the user query) starts at ``final_start`` and runs to the end.
+    A query block inside passage s sees the key blocks of passage s up to
+    itself; a query block inside the final block sees every key block up to
+    itself.  Rows cover query blocks q_first_block .. q_first_block +
+    q_num_blocks - 1 (global block indices), for every (batch, q head).
+    """
+    starts = [int(s) for s in seg_start]
+    for s in starts + [final_start]:
+        assert s % block == 0
+    final_blk = final_start // block
+    row_ptr = [0]
+    cols = []
+    for _ in range(batch * heads_q):
+        for gi in range(q_first_block, q_first_block + q_num_blocks):
+            if gi >= final_blk:
+                first = 0
+            else:
+                first = max(s for s in starts if s // block <= gi) // block
+            cols.extend(range(first, gi + 1))
+            row_ptr.append(len(cols))
+    return np.asarray(row_ptr, dtype=np.int64), np.asarray(cols, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# Exact block-sparse attention  [RBS-en "The Fix": exact attention over the
+# selected blocks; standard multi-head / grouped-query attention]
+
+
+def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_offset: int = 0,
+                     scale: float | None = None, causal: int = 1, rows=None):
+    """Softmax attention of each query token over the key tokens of its row's blocks.
+
+    Q [B, Lq, Hq, d]; K, V [B, Lk, Hkv, d]; rows ordered (b, hq, i).  Query
+    token t of row (b, hq, i) sits at position t + q_offset and may see key
+    position s of any listed block when s <= t + q_offset (causal).  The KV
+    head of q head hq is hq // (Hq / Hkv).  Returns O [B, Lq, Hq, d] (NaN for
+    rows not computed) and lse [B, Hq, Lq] = log sum_s exp(scale * q.k_s).
+    ``rows``: optional iterable of row numbers to compute (default: all).
+    """
+    B, Lq, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    G = Hq // Hkv
+    nqb = Lq // block_q
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.full((B, Lq, Hq, d), np.nan)
+    lse = np.full((B, Hq, Lq), np.nan)
+    if rows is None:
+        rows = range(B * Hq * nqb)
+    for row in rows:
+        b, rem = divmod(int(row), Hq * nqb)
+        hq, i = divmod(rem, nqb)
+        kvh = hq // G
+        blocks = col_idx[row_ptr[row]:row_ptr[row + 1]]
+        t0 = i * block_q
+        q = as_f64(Q[b, t0:t0 + block_q, hq, :])
+        if len(blocks) == 0:
+            O[b, t0:t0 + block_q, hq] = 0.0
+            lse[b, hq, t0:t0 + block_q] = -np.inf
+            continue
+        kpos = np.concatenate([np.arange(j * block_k, (j + 1) * block_k) for j in blocks])
+        k = as_f64(K[b, kpos, kvh, :])
+        v = as_f64(V[b, kpos, kvh, :])
+        logits = scale * (q @ k.T)
+        if causal:
+            qpos = np.arange(t0, t0 + block_q) + q_offset
+            logits = np.where(kpos[None, :] <= qpos[:, None], logits, -np.inf)
+        m = logits.max(axis=1, keepdims=True)
+        m = np.where(np.isfinite(m), m, 0.0)
+        w = np.exp(logits - m)
+        z = w.sum(axis=1, keepdims=True)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            O[b, t0:t0 + block_q, hq] = np.where(z > 0, (w @ v) / z, 0.0)
+            lse[b, hq, t0:t0 + block_q] = (np.log(z) + m)[:, 0]
+    return O, lse
+
+
+def dense_causal_attention(Q, K, V, q_offset: int = 0, scale: float | None = None):
+    """Textbook softmax(scale * Q K^T + causal mask) V per q head, full matrices (no blocks).
+
+    Query row t sits at position t + q_offset and sees keys s <= t + q_offset.
+    """
+    B, Lq, Hq, d = Q.shape
+    Lk, Hkv = K.shape[1], K.shape[2]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.empty((B, Lq, Hq, d))
+    mask = np.arange(Lk)[None, :] > (np.arange(Lq)[:, None] + q_offset)
+    for b in range(B):
+        for hq in range(Hq):
+            q = as_f64(Q[b, :, hq, :])
+            k = as_f64(K[b, :, hq // G, :])
+            v = as_f64(V[b, :, hq // G, :])
+            s = scale * (q @ k.T)
+            s[mask] = -np.inf
+            s -= s.max(axis=1, keepdims=True)
+            pmat = np.exp(s)
+            pmat /= pmat.sum(axis=1, keepdims=True)
+            O[b, :, hq] = pmat @ v
+    return O
+
+
+# ----------------------------------------------------------------------------
+# RoPE and position re-encoding  [BA 2.3 Position re-encoding, 2.5 Inference]
+
+
+def rope_inv_freq(d: int, theta: float) -> np.ndarray:
+    """inv_freq_m = theta^(-2m/d), m = 0 .. d/2 - 1."""
+    return theta ** (-2.0 * np.arange(d // 2) / d)
+
+
+def rope_rotate(x: np.ndarray, pos, theta: float, style: int = 0) -> np.ndarray:
+    """Rotate every (pair) of x [B, L, H, d] by the angle pos_t * inv_freq_m.
+
+    style 0 (rotate-half): pairs (m, m + d/2).  style 1 (interleaved): pairs (2m, 2m+1).
+    (a, b) -> (a cos phi - b sin phi, a sin phi + b cos phi).
+    """
+    x = as_f64(x)
+    d = x.shape[-1]
+    phi = np.asarray(pos, dtype=np.float64)[:, None] * rope_inv_freq(d, theta)[None, :]  # [L, d/2]
+    cos = np.cos(phi)[None, :, None, :]
+    sin = np.sin(phi)[None, :, None, :]
+    out = np.empty_like(x)
+    if style == 0:
+        a, b = x[..., : d // 2], x[..., d // 2:]
+        out[..., : d // 2] = a * cos - b * sin
+        out[..., d // 2:] = a * sin + b * cos
+    else:
+        a, b = x[..., 0::2], x[..., 1::2]
+        out[..., 0::2] = a * cos - b * sin
+        out[..., 1::2] = a * sin + b * cos
+    return out
+
+
+def rope_reencode(x: np.ndarray, old_pos, new_pos, theta: float, style: int = 0) -> np.ndarray:
+    """Re-encode keys cached at old_pos to new_pos: reset the rotation to position 0, then rotate to new_pos."""
+    at_zero = rope_rotate(x, -np.asarray(old_pos, dtype=np.float64), theta, style)
+    return rope_rotate(at_zero, new_pos, theta, style)

@@ -1,0 +1,472 @@
+"""Pins for the CPU fp64 oracle: closed forms, library routines, the pages'
+invariants and brute force on tiny inputs.  CPU only.
+
+Each test names what fixes the expected value.  None of them re-types the
+oracle's own formula.
+"""
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rbs_oracle as O
+from workloads import make_block_attention, make_mixture, make_tiny
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_kv(path):
+    out = {}
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k, v = line.split()
+        out[k] = float(v)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Block statistics: closed forms
+
+
+def test_stats_outlier_block_golden():
+    g = _read_kv(os.path.join(GOLDEN, "stats_outlier_block.txt"))
+    n, D = int(g["n"]), g["D"]
+    d = 128
+    a = np.zeros(d)
+    a[:3] = (1.0, -2.0, 0.5)
+    K = np.tile(a, (n, 1))
+    K[17, 7] += D  # the outlier at an arbitrary position inside the block
+    K = K[None, :, None, :]
+    C, R = O.block_stats(K, n)
+    assert C[0, 0, 0, 7] == pytest.approx(g["centroid_coord7"], abs=1e-15)
+    assert C[0, 0, 0, 0] == pytest.approx(g["centroid_coord0"], abs=1e-15)
+    assert C[0, 0, 0, 1] == pytest.approx(g["centroid_coord1"], abs=1e-15)
+    assert C[0, 0, 0, 2] == pytest.approx(g["centroid_coord2"], abs=1e-15)
+    assert R[0, 0, 0] == pytest.approx(g["radius"], abs=1e-12)
+
+
+def test_stats_constant_and_two_point_blocks():
+    rng = np.random.default_rng(1)
+    d, n = 128, 64
+    x, y, z = rng.standard_normal((3, d))
+    K = np.empty((1, 3 * n, 2, d))
+    K[0, :n, 0] = z  # constant block: c = z, r = 0
+    K[0, n:2 * n:2, 0] = x  # two-point block (alternating): c = (x+y)/2, r = |x-y|/2
+    K[0, n + 1:2 * n:2, 0] = y
+    K[0, 2 * n:, 0] = 0.0
+    K[0, :, 1] = K[0, ::-1, 0]  # head 1 = token-reversed head 0 (blocks reversed)
+    C, R = O.block_stats(K, n)
+    np.testing.assert_allclose(C[0, 0, 0], z, atol=1e-14)
+    assert R[0, 0, 0] == pytest.approx(0.0, abs=1e-13)
+    np.testing.assert_allclose(C[0, 0, 1], (x + y) / 2, atol=1e-14)
+    assert R[0, 0, 1] == pytest.approx(np.linalg.norm(x - y) / 2, rel=1e-13)
+    assert R[0, 0, 2] == 0.0
+    np.testing.assert_allclose(C[0, 1, 2], z, atol=1e-14)
+    np.testing.assert_allclose(R[0, 1, ::-1], R[0, 0], atol=1e-13)
+
+
+def test_stats_reads_bf16_bits_exactly():
+    # 1.5 and -0.25 are exact in bf16: bits 0x3FC0 and 0xBE80.
+    bits = np.zeros((1, 2, 1, 128), dtype=np.uint16)
+    bits[0, 0, 0, 0] = 0x3FC0
+    bits[0, 1, 0, 0] = 0xBE80
+    C, R = O.block_stats(bits, 2)
+    assert C[0, 0, 0, 0] == 0.625
+    assert R[0, 0, 0] == 0.875
+
+
+# --------------------------------------------------------------------------
+# beta: quantile vs numpy, closed forms
+
+
+@pytest.mark.parametrize("p", [0.0, 0.1, 0.25, 0.5, 0.9, 1.0])
+def test_quantile_type7_matches_numpy(p):
+    x = np.random.default_rng(2).standard_normal(37)
+    assert O.quantile_type7(x, p) == pytest.approx(float(np.quantile(x, p, method="linear")), abs=1e-15)
+
+
+def test_quantile_type7_hand_values():
+    assert O.quantile_type7(np.array([4.0, 1.0, 3.0, 2.0]), 0.5) == 2.5
+    assert O.quantile_type7(np.array([10.0, 20.0]), 0.25) == 12.5
+
+
+def test_beta_closed_forms():
+    R = np.array([[[1.0, 2.0, 3.0, 5.0]]])
+    b, rng = O.rescue_beta(R, O.SelectParams())
+    np.testing.assert_allclose(b[0, 0], [0.0, 0.25, 0.5, 1.0])
+    assert tuple(rng[0, 0]) == (1.0, 5.0)
+    b, _ = O.rescue_beta(R, O.SelectParams(beta_p_lo=-1.0))
+    np.testing.assert_allclose(b[0, 0], [0.2, 0.4, 0.6, 1.0])
+    # quantiles 0.25 / 0.75 of {1,2,3,5} are 1.75 / 3.5: clamped both ends
+    b, _ = O.rescue_beta(R, O.SelectParams(beta_p_lo=0.25, beta_p_hi=0.75))
+    np.testing.assert_allclose(b[0, 0], [0.0, 0.25 / 1.75, 1.25 / 1.75, 1.0])
+    b, _ = O.rescue_beta(np.full((1, 1, 5), 2.0), O.SelectParams())
+    np.testing.assert_array_equal(b, 1.0)  # degenerate range
+    b, _ = O.rescue_beta(R, O.SelectParams(beta_mode=1, beta_const=0.3))
+    np.testing.assert_array_equal(b, 0.3)
+
+
+def test_beta_is_per_prompt_and_head():
+    R = np.array([[[1.0, 3.0], [10.0, 20.0]], [[0.0, 4.0], [5.0, 5.0]]])
+    b, _ = O.rescue_beta(R, O.SelectParams())
+    np.testing.assert_allclose(b, [[[0, 1], [0, 1]], [[0, 1], [1, 1]]])
+
+
+# --------------------------------------------------------------------------
+# Pooled query: closed forms
+
+
+def test_pooled_queries_closed_forms():
+    d = 128
+    x = np.zeros(d)
+    x[:2] = (3.0, 4.0)
+    Q = np.zeros((1, 8, 2, d))
+    Q[0, :4, 0] = x  # block 0 of head 0: identical rows -> mean x, norm 5
+    Q[0, 4:8:2, 0] = x  # block 1 of head 0: rows x, -x -> mean 0
+    Q[0, 5:8:2, 0] = -x
+    Q[0, :, 1] = np.arange(8)[:, None]  # head 1: mean of 0..3 = 1.5, of 4..7 = 5.5
+    qbar, qn = O.pooled_queries(Q, 4)
+    np.testing.assert_allclose(qbar[0, 0, 0], x)
+    assert qn[0, 0, 0] == pytest.approx(5.0)
+    np.testing.assert_allclose(qbar[0, 0, 1], 0.0)
+    np.testing.assert_allclose(qbar[0, 1, :, 0], [1.5, 5.5])
+    assert qn[0, 1, 1] == pytest.approx(5.5 * math.sqrt(d))
+
+
+# --------------------------------------------------------------------------
+# Cauchy-Schwarz bound with beta = 1 (brute force, tiny inputs)
+
+
+def _tiny(L=1024, Hq=2, Hkv=1, block=64):
+    return make_tiny(L=L, Hq=Hq, Hkv=Hkv, block=block, seed=7)
+
+
+def test_cauchy_schwarz_bound_pooled_and_per_token():
+    inp = _tiny()
+    Q, K = inp["Q"], inp["K"]
+    blk = inp["block"]
+    C, R = O.block_stats(K, blk)
+    p = O.SelectParams(block_q=blk, block_k=blk, beta_mode=1, beta_const=1.0)
+    beta, _ = O.rescue_beta(R, p)
+    qbar, qn = O.pooled_queries(Q, blk)
+    Kf = O.bf16_to_f64(K)
+    Qf = O.bf16_to_f64(Q)
+    nb = C.shape[2]
+    for hq in range(Q.shape[2]):
+        s_c, s_r = O.branch_scores(qbar[0, hq], qn[0, hq], C[0, 0], R[0, 0], beta[0, 0])
+        for j in range(nb):
+            kb = Kf[0, j * blk:(j + 1) * blk, 0]
+            true_max = (qbar[0, hq] @ kb.T).max(axis=1)  # per query block i
+            assert np.all(true_max <= s_r[:, j] + 1e-9)
+            qt = Qf[0, j * blk:(j + 1) * blk, hq]  # a sample of individual tokens
+            per_tok = (qt @ kb.T).max(axis=1)
+            bound = qt @ C[0, 0, j] + np.linalg.norm(qt, axis=1) * R[0, 0, j]
+            assert np.all(per_tok <= bound + 1e-9)
+
+
+def test_cauchy_schwarz_bound_is_tight():
+    # keys c + r*u and c - r*u with u = q/|q|: the max dot product equals the bound.
+    d = 128
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal(d)
+    c = rng.standard_normal(d)
+    r = 2.5
+    u = q / np.linalg.norm(q)
+    K = np.stack([c + r * u, c - r * u] * 2)[None, :, None, :]
+    C, R = O.block_stats(K, 4)
+    assert R[0, 0, 0] == pytest.approx(r, rel=1e-12)
+    s_c, s_r = O.branch_scores(q[None], np.array([np.linalg.norm(q)]), C[0, 0], R[0, 0], np.ones(1))
+    assert s_r[0, 0] == pytest.approx(float((K[0, :, 0] @ q).max()), rel=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Top-k with ties: brute force
+
+
+def test_keep_count_values():
+    assert O.keep_count(0.25, 4) == 1
+    assert O.keep_count(0.25, 5) == 2
+    assert O.keep_count(0.1, 10) == 1
+    assert O.keep_count(1.0, 7) == 7
+    assert O.keep_count(1e-6, 7) == 1
+    assert O.keep_count(0.05, 1024) == 52
+
+
+def test_top_k_matches_brute_force_with_ties():
+    rng = np.random.default_rng(4)
+    for _ in range(200):
+        n = int(rng.integers(1, 9))
+        s = rng.integers(-2, 3, size=n).astype(np.float64)  # many ties
+        k = int(rng.integers(1, n + 1))
+        got = set(O.top_k_desc(s, k).tolist())
+        # brute force: among all k-subsets, the one that dominates every outside element
+        ok = []
+        for sub in itertools.combinations(range(n), k):
+            inside = set(sub)
+            if all((s[a] > s[b]) or (s[a] == s[b] and a < b) for a in inside for b in range(n) if b not in inside):
+                ok.append(inside)
+        assert ok == [got]
+
+
+# --------------------------------------------------------------------------
+# Selection invariants (the pages: independent branch thresholds, masks OR-ed)
+
+
+def _select(inp, **kw):
+    blk = inp["block"]
+    C, R = O.block_stats(inp["K"], blk)
+    p = O.SelectParams(block_q=blk, block_k=blk, **kw)
+    return O.select_blocks(inp["Q"], C, R, p), C, R, p
+
+
+def test_select_branch_sizes_union_and_diag():
+    inp = _tiny()
+    sel, C, R, p = _select(inp, rho_centroid=0.25, rho_rescue=0.25)
+    rp, ci, fl = sel["row_ptr"], sel["col_idx"], sel["flags"]
+    nqb = C.shape[2]
+    for row in range(rp.size - 1):
+        i = row % nqb
+        cols = ci[rp[row]:rp[row + 1]]
+        f = fl[rp[row]:rp[row + 1]]
+        assert np.all(np.diff(cols) > 0)
+        assert cols[-1] == i and f[-1] & O.FLAG_FORCED
+        assert np.all(cols <= i)
+        k = O.keep_count(0.25, i + 1)
+        assert np.count_nonzero(f & O.FLAG_CENTROID) == k
+        assert np.count_nonzero(f & O.FLAG_RESCUE) == k
+        assert np.all(f != 0)
+        assert len(cols) <= min(i + 1, 2 * k + 1)
+
+
+def test_select_beta_zero_reduces_to_centroid_only():
+    inp = _tiny()
+    sel, *_ = _select(inp, rho_centroid=0.25, rho_rescue=0.25, beta_mode=1, beta_const=0.0)
+    fl = sel["flags"]
+    assert np.array_equal((fl & O.FLAG_CENTROID) > 0, (fl & O.FLAG_RESCUE) > 0)
+
+
+def test_select_rho_one_keeps_every_causal_block():
+    inp = _tiny(L=512)
+    sel, C, *_ = _select(inp, rho_centroid=1.0, rho_rescue=1.0)
+    rp, ci = O.causal_full_lists(1, inp["Q"].shape[2], C.shape[2])
+    assert np.array_equal(sel["row_ptr"], rp) and np.array_equal(sel["col_idx"], ci)
+
+
+def test_select_nested_in_rho():
+    inp = _tiny(L=512)
+    small, *_ = _select(inp, rho_centroid=0.1, rho_rescue=0.1)
+    big, *_ = _select(inp, rho_centroid=0.3, rho_rescue=0.3)
+    for row in range(small["row_ptr"].size - 1):
+        a = set(small["col_idx"][small["row_ptr"][row]:small["row_ptr"][row + 1]].tolist())
+        b = set(big["col_idx"][big["row_ptr"][row]:big["row_ptr"][row + 1]].tolist())
+        assert a <= b
+
+
+def test_select_gqa_head_mapping_and_rescue():
+    # Two KV heads of 2 q heads each.  KV head 0 hides one big key in block 3,
+    # KV head 1 in block 5, each aligned with every query of its q heads.  With
+    # beta = 1 and a one-block rescue budget, the rescue branch of q heads 0,1
+    # must pick block 3 and of q heads 2,3 block 5 (for the last query block).
+    d, blk, nb = 128, 16, 8
+    rng = np.random.default_rng(5)
+    Q = np.zeros((1, nb * blk, 4, d))
+    Q[..., 0] = 1.0
+    Q += 0.01 * rng.standard_normal(Q.shape)
+    K = 0.01 * rng.standard_normal((1, nb * blk, 2, d))
+    K[0, 3 * blk + 5, 0, 0] = 40.0
+    K[0, 5 * blk + 2, 1, 0] = 40.0
+    C, R = O.block_stats(K, blk)
+    p = O.SelectParams(block_q=blk, block_k=blk, rho_centroid=1e-6, rho_rescue=1e-6, beta_mode=1,
+                       beta_const=1.0, force_diag=0)
+    sel = O.select_blocks(Q, C, R, p)
+    rp, ci, fl = sel["row_ptr"], sel["col_idx"], sel["flags"]
+    last = [hq * nb + nb - 1 for hq in range(4)]
+    for hq, row in enumerate(last):
+        cols = ci[rp[row]:rp[row + 1]]
+        f = fl[rp[row]:rp[row + 1]]
+        assert cols[f & O.FLAG_RESCUE > 0].tolist() == ([3] if hq < 2 else [5])
+
+
+def test_bisect_rho_hits_density():
+    inp = make_mixture(L=4096, Hq=4, Hkv=2, block=128, seed=11)
+    C, R = O.block_stats(inp["K"], 128)
+    p = O.SelectParams()
+    rho, dens = O.bisect_rho(inp["Q"], C, R, p, 0.25)
+    assert abs(dens - 0.25) < 0.0025 + 1.0 / (4 * 32 * 33 / 2)  # one pair of granularity
+    p.rho_centroid = p.rho_rescue = rho
+    sel = O.select_blocks(inp["Q"], C, R, p)
+    assert O.list_density(sel["row_ptr"], 32, 32) == pytest.approx(dens, abs=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Attention: 100% density == textbook dense causal attention == torch SDPA
+
+
+def _sdpa_ref(Q, K, V, q_offset=0):
+    q = torch.from_numpy(O.bf16_to_f64(Q)).permute(0, 2, 1, 3)
+    k = torch.from_numpy(O.bf16_to_f64(K)).permute(0, 2, 1, 3)
+    v = torch.from_numpy(O.bf16_to_f64(V)).permute(0, 2, 1, 3)
+    G = q.shape[1] // k.shape[1]
+    k = k.repeat_interleave(G, dim=1)
+    v = v.repeat_interleave(G, dim=1)
+    Lq, Lk = q.shape[2], k.shape[2]
+    allowed = torch.arange(Lk)[None, :] <= (torch.arange(Lq)[:, None] + q_offset)
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=allowed)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def test_dense_attention_matches_sdpa_gqa():
+    inp = make_tiny(L=256, Hq=4, Hkv=2, block=64, seed=8)
+    ref = _sdpa_ref(inp["Q"], inp["K"], inp["V"])
+    got = O.dense_causal_attention(inp["Q"], inp["K"], inp["V"])
+    np.testing.assert_allclose(got, ref, atol=1e-12)
+
+
+def test_full_lists_equal_dense_attention_with_offset():
+    inp = make_tiny(L=512, Hq=4, Hkv=2, block=64, seed=9)
+    Q = inp["Q"][:, 256:]  # the last 4 query blocks, at positions 256..511
+    rp, ci = O.causal_full_lists(1, 4, 4, q_block_offset=4)
+    got, lse = O.masked_attention(Q, inp["K"], inp["V"], rp, ci, 64, 64, q_offset=256)
+    ref = _sdpa_ref(Q, inp["K"], inp["V"], q_offset=256)
+    np.testing.assert_allclose(got, ref, atol=1e-12)
+    np.testing.assert_allclose(got, O.dense_causal_attention(Q, inp["K"], inp["V"], q_offset=256), atol=1e-12)
+    # lse against its definition through torch.logsumexp on the masked logits
+    q = O.bf16_to_f64(Q[0, :, 3])
+    k = O.bf16_to_f64(inp["K"][0, :, 1])
+    s = torch.from_numpy(q @ k.T / math.sqrt(128))
+    s[torch.arange(512)[None, :] > torch.arange(256)[:, None] + 256] = -math.inf
+    np.testing.assert_allclose(lse[0, 3], torch.logsumexp(s, dim=1).numpy(), atol=1e-12)
+
+
+def test_masked_attention_hand_cases():
+    d = 128
+    v = np.arange(2 * 1 * d, dtype=np.float64).reshape(1, 2, 1, d)
+    q = np.zeros((1, 2, 1, d))
+    k = np.zeros((1, 2, 1, d))
+    # row 0 (token 0) sees only key 0 -> output v0; token 1 sees two equal logits -> mean
+    O_, lse = O.masked_attention(q, k, v, np.array([0, 1]), np.array([0]), 2, 2)
+    np.testing.assert_allclose(O_[0, 0, 0], v[0, 0, 0])
+    np.testing.assert_allclose(O_[0, 1, 0], v[0, :, 0].mean(axis=0))
+    assert lse[0, 0, 0] == 0.0 and lse[0, 0, 1] == pytest.approx(math.log(2))
+    # an empty list gives zeros and lse = -inf
+    O_, lse = O.masked_attention(q, k, v, np.array([0, 0]), np.array([], dtype=np.int64), 2, 2)
+    assert np.all(O_ == 0) and np.all(lse == -np.inf)
+
+
+# --------------------------------------------------------------------------
+# Block-attention: hand-enumerated lists and the independence invariant
+
+
+def test_block_attention_lists_golden():
+    exp = {}
+    for line in open(os.path.join(GOLDEN, "block_attention_lists_tiny.txt")):
+        if line.strip() and not line.startswith("#"):
+            a, b = line.split(":")
+            exp[int(a)] = [int(x) for x in b.split()]
+    rp, ci = O.block_attention_lists([0, 256], 512, 128, 1, 1, 0, 5)
+    for i in range(5):
+        assert ci[rp[i]:rp[i + 1]].tolist() == exp[i]
+    # rows of the final block only (a final-block pass with a query offset)
+    rp, ci = O.block_attention_lists([0, 256], 512, 128, 1, 1, 4, 1)
+    assert ci.tolist() == exp[4]
+
+
+def test_block_attention_passages_are_independent():
+    inp = make_block_attention(passages=3, passage_len=128, final_len=64, Hq=2, Hkv=1, block=64, seed=12)
+    blk = 64
+    L = inp["Q"].shape[1]
+    rp, ci = O.block_attention_lists(inp["seg_start"], inp["final_start"], blk, 1, 2, 0, L // blk)
+    base, _ = O.masked_attention(inp["Q"], inp["K"], inp["V"], rp, ci, blk, blk)
+    other = make_block_attention(passages=3, passage_len=128, final_len=64, Hq=2, Hkv=1, block=64, seed=13)
+    Q2, K2, V2 = other["Q"].copy(), other["K"].copy(), other["V"].copy()
+    Q2[:, 128:256], K2[:, 128:256], V2[:, 128:256] = inp["Q"][:, 128:256], inp["K"][:, 128:256], inp["V"][:, 128:256]
+    out2, _ = O.masked_attention(Q2, K2, V2, rp, ci, blk, blk)
+    assert np.array_equal(base[:, 128:256], out2[:, 128:256])  # passage 1 unchanged, bit for bit
+    assert not np.allclose(base[:, 384:], out2[:, 384:])  # the final block sees everything
+
+
+# --------------------------------------------------------------------------
+# RoPE: complex-number form, re-encoding == direct encoding, invariants
+
+
+def test_rope_matches_complex_rotation():
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((1, 5, 2, 128))
+    pos = np.array([0, 1, 7, 2048, 33279])
+    theta = 500000.0
+    got = O.rope_rotate(x, pos, theta, 0)
+    freqs = np.power(theta, -np.arange(64) / 64.0)
+    z = (x[..., :64] + 1j * x[..., 64:]) * np.exp(1j * pos[None, :, None, None] * freqs)
+    np.testing.assert_allclose(got[..., :64], z.real, atol=1e-12)
+    np.testing.assert_allclose(got[..., 64:], z.imag, atol=1e-12)
+    got1 = O.rope_rotate(x, pos, theta, 1)
+    z1 = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * pos[None, :, None, None] * freqs)
+    np.testing.assert_allclose(got1[..., 0::2], z1.real, atol=1e-12)
+    np.testing.assert_allclose(got1[..., 1::2], z1.imag, atol=1e-12)
+
+
+@pytest.mark.parametrize("style", [0, 1])
+def test_rope_reencode_equals_direct_encoding(style):
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((1, 6, 3, 128))
+    old = np.array([0, 5, 100, 2047, 3, 0])
+    new = np.array([0, 2053, 30820, 32767, 3, 1])
+    cached = O.rope_rotate(x, old, 500000.0, style)
+    np.testing.assert_allclose(O.rope_reencode(cached, old, new, 500000.0, style),
+                               O.rope_rotate(x, new, 500000.0, style), atol=1e-11)
+    np.testing.assert_allclose(O.rope_reencode(cached, old, old, 500000.0, style), cached, atol=1e-12)
+    pairs = lambda a: a[..., :64] ** 2 + a[..., 64:] ** 2 if style == 0 else a[..., 0::2] ** 2 + a[..., 1::2] ** 2
+    np.testing.assert_allclose(pairs(cached), pairs(x), rtol=1e-12)
+
+
+def test_rope_relative_position_invariance():
+    rng = np.random.default_rng(16)
+    q = rng.standard_normal((1, 1, 1, 128))
+    k = rng.standard_normal((1, 1, 1, 128))
+    dots = []
+    for shift in (0, 37, 32768):
+        qr = O.rope_rotate(q, np.array([shift + 9]), 500000.0)
+        kr = O.rope_rotate(k, np.array([shift + 2]), 500000.0)
+        dots.append(float((qr * kr).sum()))
+    assert dots[1] == pytest.approx(dots[0], abs=1e-10)
+    assert dots[2] == pytest.approx(dots[0], abs=1e-10)
+
+
+# --------------------------------------------------------------------------
+# Planted mistakes: each pin above must fail on a plausible oracle bug.
+
+
+def test_pins_catch_planted_mistakes(monkeypatch):
+    good_scores = O.branch_scores
+
+    def wrong_sign(qbar, qnorm, C, R, beta):
+        s_c, s_r = good_scores(qbar, qnorm, C, R, beta)
+        return s_c, 2 * s_c - s_r  # rescue term subtracted
+    monkeypatch.setattr(O, "branch_scores", wrong_sign)
+    with pytest.raises(AssertionError):
+        test_cauchy_schwarz_bound_pooled_and_per_token()
+    monkeypatch.setattr(O, "branch_scores", good_scores)
+
+    good_stats = O.block_stats
+
+    def radius_from_mean_distance(K, bk):
+        C, R = good_stats(K, bk)
+        return C, R * (bk - 1) / bk  # a "mean distance"-like shrink of the radius
+    monkeypatch.setattr(O, "block_stats", radius_from_mean_distance)
+    with pytest.raises(AssertionError):
+        test_stats_outlier_block_golden()
+    monkeypatch.setattr(O, "block_stats", good_stats)
+
+    good_rot = O.rope_rotate
+
+    def transposed(x, pos, theta, style=0):
+        return good_rot(x, -np.asarray(pos), theta, style)  # rotation the wrong way
+    monkeypatch.setattr(O, "rope_rotate", transposed)
+    with pytest.raises(AssertionError):
+        test_rope_matches_complex_rotation()
