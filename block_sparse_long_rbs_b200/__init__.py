@@ -1,0 +1,234 @@
+"""Block-sparse prefill attention with radius-bounded block selection (RBS)
+and the Block-attention mask, on NVIDIA B200 (sm_100a).
+
+A thin binding over the C ABI of librbs (include/rbs.h): argument
+marshalling only.  Torch tensors supply device memory and the current CUDA
+stream; every step of the computation runs in the library's CUDA kernels.
+Functions carry the same names as the C entry points.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+
+import torch
+
+from ._abi import (  # noqa: F401
+    DEVERR_BLOCK_INDEX,
+    DEVERR_NONCAUSAL,
+    DEVERR_ROW_PTR,
+    DEVERR_TIMEOUT,
+    MAX_KV_BLOCKS,
+    BlockListsC,
+    Bf16Tensor,
+    RbsError,
+    SelectParamsC,
+    check,
+    lib,
+)
+
+__all__ = [
+    "SelectParams", "BlockLists", "rbs_block_stats", "rbs_block_beta", "rbs_pool_queries", "rbs_select",
+    "rbs_select_capacity", "rbs_select_workspace_bytes", "rbs_lists_causal_full", "rbs_lists_block_attention",
+    "bsa_prefill", "rope_reencode", "rbs_get_device_error", "RbsError",
+]
+
+
+@dataclasses.dataclass
+class SelectParams:
+    """Selection parameters (field meanings and defaults as in include/rbs.h)."""
+
+    block_q: int = 128
+    block_k: int = 128
+    rho_centroid: float = 0.05
+    rho_rescue: float = 0.05
+    beta_mode: int = 0
+    beta_const: float = 1.0
+    beta_p_lo: float = 0.0
+    beta_p_hi: float = 1.0
+    force_diag: int = 1
+    force_sink: int = 0
+    causal: int = 1
+    q_block_offset: int = 0
+
+    def c(self) -> SelectParamsC:
+        return SelectParamsC(*[getattr(self, f.name) for f in dataclasses.fields(self)])
+
+
+@dataclasses.dataclass
+class BlockLists:
+    """CSR key-block lists on the device: one row per (batch, q head, query block)."""
+
+    row_ptr: torch.Tensor  # int32 [num_rows + 1]
+    col_idx: torch.Tensor  # int32 [capacity]
+    flags: torch.Tensor | None  # uint8 [capacity]
+    num_rows: int
+
+    def c(self) -> BlockListsC:
+        return BlockListsC(self.row_ptr.data_ptr(), self.col_idx.data_ptr(),
+                           self.flags.data_ptr() if self.flags is not None else None,
+                           self.col_idx.numel(), self.num_rows)
+
+    def nnz(self) -> int:
+        return int(self.row_ptr[-1].item())
+
+    @staticmethod
+    def empty(num_rows: int, capacity: int, device, flags: bool = True) -> "BlockLists":
+        return BlockLists(torch.empty(num_rows + 1, dtype=torch.int32, device=device),
+                          torch.empty(max(1, capacity), dtype=torch.int32, device=device),
+                          torch.empty(max(1, capacity), dtype=torch.uint8, device=device) if flags else None,
+                          num_rows)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _t(x: torch.Tensor, name: str) -> Bf16Tensor:
+    """Describe a [B, L, H, 128] bf16 CUDA tensor (head_dim contiguous) for the C ABI."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if x.dtype != torch.bfloat16 or x.dim() != 4 or x.stride(3) != 1:
+        raise TypeError(f"{name}: expected bf16 [B, L, H, 128] with a contiguous last dimension")
+    B, L, H, D = x.shape
+    return Bf16Tensor(x.data_ptr(), B, L, H, D, x.stride(0), x.stride(1), x.stride(2))
+
+
+def _f32(x: torch.Tensor, name: str) -> int:
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous float32 CUDA tensor")
+    return x.data_ptr()
+
+
+def rbs_block_stats(K: torch.Tensor, block_k: int):
+    """Centroids [B, Hkv, nKB, 128] and radii [B, Hkv, nKB] (fp32) of every key block."""
+    B, L, H, D = K.shape
+    nkb = L // block_k
+    C = torch.empty(B, H, nkb, D, dtype=torch.float32, device=K.device)
+    R = torch.empty(B, H, nkb, dtype=torch.float32, device=K.device)
+    check(lib().rbs_block_stats(ctypes.byref(_t(K, "K")), block_k, C.data_ptr(), R.data_ptr(), _stream()),
+          "rbs_block_stats")
+    return C, R
+
+
+def rbs_block_beta(radii: torch.Tensor, params: SelectParams):
+    """beta [B, Hkv, nKB] and the (R_lo, R_hi) range [B, Hkv, 2] from the radii."""
+    B, H, n = radii.shape
+    beta = torch.empty_like(radii)
+    rng = torch.empty(B, H, 2, dtype=torch.float32, device=radii.device)
+    p = params.c()
+    check(lib().rbs_block_beta(_f32(radii, "radii"), B, H, n, ctypes.byref(p), beta.data_ptr(), rng.data_ptr(),
+                               _stream()), "rbs_block_beta")
+    return beta, rng
+
+
+def rbs_pool_queries(Q: torch.Tensor, block_q: int):
+    """qbar [B, Hq, nQB, 128] and qnorm [B, Hq, nQB] (fp32)."""
+    B, L, H, D = Q.shape
+    nqb = L // block_q
+    qbar = torch.empty(B, H, nqb, D, dtype=torch.float32, device=Q.device)
+    qnorm = torch.empty(B, H, nqb, dtype=torch.float32, device=Q.device)
+    check(lib().rbs_pool_queries(ctypes.byref(_t(Q, "Q")), block_q, qbar.data_ptr(), qnorm.data_ptr(), _stream()),
+          "rbs_pool_queries")
+    return qbar, qnorm
+
+
+def rbs_select_capacity(batch: int, heads_q: int, num_q_blocks: int, num_kv_blocks: int, params: SelectParams) -> int:
+    p = params.c()
+    return int(lib().rbs_select_capacity(batch, heads_q, num_q_blocks, num_kv_blocks, ctypes.byref(p)))
+
+
+def rbs_select_workspace_bytes(batch: int, heads_q: int, num_q_blocks: int, kv_heads: int, num_kv_blocks: int,
+                               params: SelectParams) -> int:
+    p = params.c()
+    return int(lib().rbs_select_workspace_bytes(batch, heads_q, num_q_blocks, kv_heads, num_kv_blocks,
+                                                ctypes.byref(p)))
+
+
+def rbs_select(Q: torch.Tensor, centroids: torch.Tensor, radii: torch.Tensor, params: SelectParams,
+               workspace: torch.Tensor | None = None, out: BlockLists | None = None, beta_out: torch.Tensor | None = None,
+               flags: bool = True) -> BlockLists:
+    """Two-branch selection -> CSR key-block lists (rows = (batch, q head, query block))."""
+    B, L, Hq, _ = Q.shape
+    Hkv, nkb = centroids.shape[1], centroids.shape[2]
+    nqb = L // params.block_q
+    rows = B * Hq * nqb
+    if out is None:
+        out = BlockLists.empty(rows, rbs_select_capacity(B, Hq, nqb, nkb, params), Q.device, flags)
+    if workspace is None:
+        workspace = torch.empty(rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, params), dtype=torch.uint8,
+                                device=Q.device)
+    p = params.c()
+    lc = out.c()
+    check(lib().rbs_select(ctypes.byref(_t(Q, "Q")), _f32(centroids, "centroids"), _f32(radii, "radii"), Hkv, nkb,
+                           ctypes.byref(p), workspace.data_ptr(), workspace.numel(), ctypes.byref(lc),
+                           beta_out.data_ptr() if beta_out is not None else None, _stream()), "rbs_select")
+    return out
+
+
+def rbs_lists_causal_full(batch: int, heads_q: int, num_q_blocks: int, q_block_offset: int = 0, device="cuda",
+                          flags: bool = False) -> BlockLists:
+    """Every causally visible block for every row (the dense reference point)."""
+    nnz = int(lib().rbs_lists_causal_full_nnz(batch, heads_q, num_q_blocks, q_block_offset))
+    out = BlockLists.empty(batch * heads_q * num_q_blocks, nnz, device, flags)
+    lc = out.c()
+    check(lib().rbs_lists_causal_full(batch, heads_q, num_q_blocks, q_block_offset, ctypes.byref(lc), _stream()),
+          "rbs_lists_causal_full")
+    return out
+
+
+def rbs_lists_block_attention(seg_start, final_start: int, block: int, batch: int, heads_q: int, q_first_block: int,
+                              q_num_blocks: int, device="cuda", flags: bool = False) -> BlockLists:
+    """Block-attention mask lists (passages self-attend, the final block sees all)."""
+    seg = (ctypes.c_int32 * len(seg_start))(*[int(s) for s in seg_start])
+    nnz = int(lib().rbs_lists_block_attention_nnz(seg, len(seg_start), final_start, block, batch, heads_q,
+                                                  q_first_block, q_num_blocks))
+    if nnz < 0:
+        raise RbsError(1, "rbs_lists_block_attention_nnz", lib().rbs_last_error().decode())
+    out = BlockLists.empty(batch * heads_q * q_num_blocks, nnz, device, flags)
+    lc = out.c()
+    check(lib().rbs_lists_block_attention(seg, len(seg_start), final_start, block, batch, heads_q, q_first_block,
+                                          q_num_blocks, ctypes.byref(lc), _stream()), "rbs_lists_block_attention")
+    return out
+
+
+def bsa_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, lists: BlockLists, block_q: int = 128,
+                block_k: int = 128, q_offset: int = 0, softmax_scale: float | None = None, causal: bool = True,
+                out: torch.Tensor | None = None, return_lse: bool = False):
+    """Exact softmax attention of every query block over its listed key blocks."""
+    if out is None:
+        out = torch.empty_like(Q)
+    lse = None
+    if return_lse:
+        lse = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], dtype=torch.float32, device=Q.device)
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(Q.shape[-1])
+    lc = lists.c()
+    check(lib().bsa_prefill(ctypes.byref(_t(Q, "Q")), ctypes.byref(_t(K, "K")), ctypes.byref(_t(V, "V")),
+                            ctypes.byref(lc), block_q, block_k, q_offset, scale, 1 if causal else 0,
+                            ctypes.byref(_t(out, "O")), lse.data_ptr() if lse is not None else None, _stream()),
+          "bsa_prefill")
+    return (out, lse) if return_lse else out
+
+
+def rope_reencode(x: torch.Tensor, old_pos: torch.Tensor, new_pos: torch.Tensor, theta: float, rope_style: int = 0,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+    """Move RoPE-encoded vectors from old_pos to new_pos (out may be x for in place)."""
+    if out is None:
+        out = torch.empty_like(x)
+    for name, p in (("old_pos", old_pos), ("new_pos", new_pos)):
+        if not p.is_cuda or p.dtype != torch.int32 or p.numel() != x.shape[1]:
+            raise TypeError(f"{name}: expected int32 CUDA tensor of length {x.shape[1]}")
+    check(lib().rope_reencode(ctypes.byref(_t(x, "x")), ctypes.byref(_t(out, "out")), old_pos.data_ptr(),
+                              new_pos.data_ptr(), theta, rope_style, _stream()), "rope_reencode")
+    return out
+
+
+def rbs_get_device_error() -> int:
+    """Read and clear the library's device error word (synchronises the current stream)."""
+    code = ctypes.c_int32(0)
+    st = lib().rbs_get_device_error(ctypes.byref(code), _stream())
+    if st not in (0, 5):
+        check(st, "rbs_get_device_error")
+    return int(code.value)

@@ -1,0 +1,590 @@
+// librbs: the C ABI declared in include/rbs.h.  Host-side validation,
+// workspace carving, TMA tensor-map encoding and kernel launches.  No call
+// here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "lists.cuh"
+#include "rope.cuh"
+#include "select.cuh"
+#include "stats.cuh"
+
+using namespace rbs;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+rbs_status fail(rbs_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define RBS_REQUIRE(cond, status, ...)       \
+  do {                                       \
+    if (!(cond)) return fail(status, __VA_ARGS__); \
+  } while (0)
+
+rbs_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return RBS_OK;
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sms = 0;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+rbs_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(RBS_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0) return fail(RBS_ERR_UNSUPPORTED, "device %d is sm_%d%d; this build is sm_100a only", dev, major, minor);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  if (!d.attrs_set) {
+    cudaError_t e = cudaSuccess;
+    e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem<128>::kAlloc);
+    e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem<64>::kAlloc);
+    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
+    if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    d.attrs_set = true;
+  }
+  *out = &d;
+  return RBS_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+rbs_status check_tensor(const rbs_bf16_tensor* t, const char* name) {
+  RBS_REQUIRE(t != nullptr && t->data != nullptr, RBS_ERR_INVALID_ARG, "%s: null tensor", name);
+  RBS_REQUIRE(t->batch > 0 && t->seqlen > 0 && t->heads > 0, RBS_ERR_INVALID_ARG, "%s: empty shape", name);
+  RBS_REQUIRE(t->head_dim == RBS_HEAD_DIM, RBS_ERR_UNSUPPORTED, "%s: head_dim %lld != 128", name,
+              static_cast<long long>(t->head_dim));
+  RBS_REQUIRE(aligned16(t->data), RBS_ERR_INVALID_ARG, "%s: base pointer not 16-byte aligned", name);
+  RBS_REQUIRE(t->stride_b > 0 && t->stride_s > 0 && t->stride_h > 0, RBS_ERR_INVALID_ARG, "%s: non-positive stride", name);
+  RBS_REQUIRE(t->stride_b % 8 == 0 && t->stride_s % 8 == 0 && t->stride_h % 8 == 0, RBS_ERR_INVALID_ARG,
+              "%s: strides must be multiples of 8 elements", name);
+  RBS_REQUIRE(t->seqlen < (1ll << 31) && t->heads < (1 << 16) && t->batch < (1 << 16), RBS_ERR_UNSUPPORTED,
+              "%s: shape too large", name);
+  return RBS_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+// 4-D map over [B, L, H, 128] bf16 with a box of `rows` tokens x 64 dims of
+// one head, 128-byte swizzle.  The token and head dimensions are ordered by
+// stride (*seq_inner = 1 when the token stride is the smaller one).
+rbs_status make_tensor_map(const rbs_bf16_tensor* t, int rows, CUtensorMap* map, int* seq_inner) {
+  PFN_encodeTiled enc = encode_fn();
+  if (enc == nullptr) return fail(RBS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const bool si = t->stride_s < t->stride_h;
+  *seq_inner = si ? 1 : 0;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4], estr[4] = {1, 1, 1, 1};
+  dims[0] = RBS_HEAD_DIM;
+  box[0] = 64;
+  if (si) {
+    dims[1] = t->seqlen; strides[0] = t->stride_s * 2; box[1] = rows;
+    dims[2] = t->heads; strides[1] = t->stride_h * 2; box[2] = 1;
+  } else {
+    dims[1] = t->heads; strides[0] = t->stride_h * 2; box[1] = 1;
+    dims[2] = t->seqlen; strides[1] = t->stride_s * 2; box[2] = rows;
+  }
+  dims[3] = t->batch;
+  strides[2] = t->stride_b * 2;
+  box[3] = 1;
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RBS_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return RBS_OK;
+}
+
+int keep_count_host(float rho, int64_t n) {
+  int64_t k = static_cast<int64_t>(std::ceil(static_cast<double>(rho) * static_cast<double>(n) - 1e-4));
+  if (k < 1) k = 1;
+  if (k > n) k = n;
+  return static_cast<int>(k);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct SelectLayout {
+  size_t mask_c, mask_r, counts, qbar, qnorm, beta, total;
+};
+
+SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int64_t nkb) {
+  SelectLayout l{};
+  const int64_t rows = B * Hq * nqb;
+  const int64_t nwords = (nkb + 31) / 32;
+  size_t off = 0;
+  l.mask_c = off; off += align256(rows * nwords * 4);
+  l.mask_r = off; off += align256(rows * nwords * 4);
+  l.counts = off; off += align256(rows * 4);
+  l.qbar = off; off += align256(B * Hq * nqb * RBS_HEAD_DIM * 4);
+  l.qnorm = off; off += align256(B * Hq * nqb * 4);
+  l.beta = off; off += align256(B * Hkv * nkb * 4);
+  l.total = off;
+  return l;
+}
+
+rbs_status check_lists(const rbs_block_lists* out, int64_t rows) {
+  RBS_REQUIRE(out != nullptr && out->row_ptr != nullptr && out->col_idx != nullptr, RBS_ERR_INVALID_ARG,
+              "lists: null pointer");
+  RBS_REQUIRE(out->num_rows == rows, RBS_ERR_INVALID_ARG, "lists: num_rows %d != %lld", out->num_rows,
+              static_cast<long long>(rows));
+  RBS_REQUIRE(out->capacity >= 0 && out->capacity < (1ll << 31), RBS_ERR_UNSUPPORTED, "lists: capacity out of int32 range");
+  return RBS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t rbs_abi_version(void) { return RBS_ABI_VERSION; }
+
+const char* rbs_status_string(rbs_status s) {
+  switch (s) {
+    case RBS_OK: return "ok";
+    case RBS_ERR_INVALID_ARG: return "invalid argument";
+    case RBS_ERR_UNSUPPORTED: return "unsupported";
+    case RBS_ERR_CAPACITY: return "capacity";
+    case RBS_ERR_CUDA: return "cuda error";
+    case RBS_ERR_DEVICE: return "device error";
+  }
+  return "unknown status";
+}
+
+const char* rbs_last_error(void) { return g_last_error; }
+
+void rbs_select_params_default(rbs_select_params* p) {
+  if (p == nullptr) return;
+  p->block_q = 128;
+  p->block_k = 128;
+  p->rho_centroid = 0.05f;
+  p->rho_rescue = 0.05f;
+  p->beta_mode = 0;
+  p->beta_const = 1.0f;
+  p->beta_p_lo = 0.0f;
+  p->beta_p_hi = 1.0f;
+  p->force_diag = 1;
+  p->force_sink = 0;
+  p->causal = 1;
+  p->q_block_offset = 0;
+}
+
+rbs_status rbs_get_device_error(int32_t* code_host, rbs_stream_t stream) {
+  RBS_REQUIRE(code_host != nullptr, RBS_ERR_INVALID_ARG, "null code pointer");
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  const int zero = 0;
+  if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+  *code_host = v;
+  if (v != 0) return fail(RBS_ERR_DEVICE, "device error word 0x%x", v);
+  return RBS_OK;
+}
+
+// ---------------------------------------------------------------------------
+
+rbs_status rbs_block_stats(const rbs_bf16_tensor* K, int32_t block_k, float* centroids, float* radii,
+                           rbs_stream_t stream) {
+  rbs_status st = check_tensor(K, "K");
+  if (st != RBS_OK) return st;
+  RBS_REQUIRE(block_k == 64 || block_k == 128, RBS_ERR_UNSUPPORTED, "block_k must be 64 or 128");
+  RBS_REQUIRE(K->seqlen % block_k == 0, RBS_ERR_UNSUPPORTED, "seqlen %% block_k != 0");
+  RBS_REQUIRE(centroids != nullptr && radii != nullptr, RBS_ERR_INVALID_ARG, "null output");
+  RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
+  DeviceInfo* di;
+  if ((st = device_info(&di)) != RBS_OK) return st;
+  const int nkb = static_cast<int>(K->seqlen / block_k);
+  const dim3 grid(nkb, static_cast<unsigned>(K->heads), static_cast<unsigned>(K->batch));
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K->data);
+  if (block_k == 128)
+    block_stats_kernel<128><<<grid, 128, 0, stream>>>(k, K->stride_b, K->stride_s, K->stride_h, nkb,
+                                                      static_cast<int>(K->heads), centroids, radii);
+  else
+    block_stats_kernel<64><<<grid, 128, 0, stream>>>(k, K->stride_b, K->stride_s, K->stride_h, nkb,
+                                                     static_cast<int>(K->heads), centroids, radii);
+  return check_launch("block_stats_kernel");
+}
+
+rbs_status rbs_block_beta(const float* radii, int64_t batch, int64_t kv_heads, int64_t num_blocks,
+                          const rbs_select_params* p, float* beta, float* radius_range, rbs_stream_t stream) {
+  RBS_REQUIRE(radii != nullptr && beta != nullptr && p != nullptr, RBS_ERR_INVALID_ARG, "null argument");
+  RBS_REQUIRE(batch > 0 && kv_heads > 0 && num_blocks > 0, RBS_ERR_INVALID_ARG, "empty shape");
+  RBS_REQUIRE(num_blocks <= RBS_MAX_KV_BLOCKS, RBS_ERR_UNSUPPORTED, "num_blocks > %d", RBS_MAX_KV_BLOCKS);
+  RBS_REQUIRE(p->beta_mode == 0 || p->beta_mode == 1, RBS_ERR_INVALID_ARG, "beta_mode");
+  RBS_REQUIRE(p->beta_mode == 1 || (p->beta_p_hi >= 0.f && p->beta_p_hi <= 1.f && p->beta_p_lo <= 1.f),
+              RBS_ERR_INVALID_ARG, "beta quantiles out of range");
+  RBS_REQUIRE(kv_heads < 65536 && batch < 65536, RBS_ERR_UNSUPPORTED, "shape too large");
+  DeviceInfo* di;
+  rbs_status st = device_info(&di);
+  if (st != RBS_OK) return st;
+  int n2 = 1;
+  while (n2 < num_blocks) n2 <<= 1;
+  block_beta_kernel<<<dim3(static_cast<unsigned>(kv_heads), static_cast<unsigned>(batch)), 1024, n2 * 4, stream>>>(
+      radii, static_cast<int>(num_blocks), static_cast<int>(kv_heads), p->beta_mode, p->beta_const, p->beta_p_lo,
+      p->beta_p_hi, beta, radius_range);
+  return check_launch("block_beta_kernel");
+}
+
+rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, float* qbar, float* qnorm,
+                            rbs_stream_t stream) {
+  rbs_status st = check_tensor(Q, "Q");
+  if (st != RBS_OK) return st;
+  RBS_REQUIRE(block_q == 64 || block_q == 128, RBS_ERR_UNSUPPORTED, "block_q must be 64 or 128");
+  RBS_REQUIRE(Q->seqlen % block_q == 0, RBS_ERR_UNSUPPORTED, "seqlen %% block_q != 0");
+  RBS_REQUIRE(qbar != nullptr && qnorm != nullptr && aligned16(qbar), RBS_ERR_INVALID_ARG, "bad output");
+  DeviceInfo* di;
+  if ((st = device_info(&di)) != RBS_OK) return st;
+  const int nqb = static_cast<int>(Q->seqlen / block_q);
+  const int Hq = static_cast<int>(Q->heads);
+  const dim3 grid(nqb, (Hq + 3) / 4, static_cast<unsigned>(Q->batch));
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q->data);
+  if (block_q == 128)
+    pool_queries_kernel<128><<<grid, 256, 0, stream>>>(q, Q->stride_b, Q->stride_s, Q->stride_h, Hq, nqb, qbar, qnorm);
+  else
+    pool_queries_kernel<64><<<grid, 256, 0, stream>>>(q, Q->stride_b, Q->stride_s, Q->stride_h, Hq, nqb, qbar, qnorm);
+  return check_launch("pool_queries_kernel");
+}
+
+int64_t rbs_select_capacity(int64_t batch, int64_t heads_q, int64_t num_q_blocks, int64_t num_kv_blocks,
+                            const rbs_select_params* p) {
+  if (p == nullptr || batch <= 0 || heads_q <= 0 || num_q_blocks <= 0 || num_kv_blocks <= 0) return -1;
+  int64_t per_head = 0;
+  for (int64_t i = 0; i < num_q_blocks; ++i) {
+    const int64_t gi = i + p->q_block_offset;
+    const int64_t n = p->causal ? std::min<int64_t>(num_kv_blocks, gi + 1) : num_kv_blocks;
+    if (n <= 0) continue;
+    int64_t c = keep_count_host(p->rho_centroid, n) + keep_count_host(p->rho_rescue, n);
+    c += (p->force_diag && gi < num_kv_blocks) ? 1 : 0;
+    c += p->force_sink ? 1 : 0;
+    per_head += std::min<int64_t>(n, c);
+  }
+  return per_head * batch * heads_q;
+}
+
+size_t rbs_select_workspace_bytes(int64_t batch, int64_t heads_q, int64_t num_q_blocks, int64_t kv_heads,
+                                  int64_t num_kv_blocks, const rbs_select_params* p) {
+  (void)p;
+  if (batch <= 0 || heads_q <= 0 || num_q_blocks <= 0 || kv_heads <= 0 || num_kv_blocks <= 0) return 0;
+  return select_layout(batch, heads_q, num_q_blocks, kv_heads, num_kv_blocks).total;
+}
+
+rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const float* radii, int32_t kv_heads,
+                      int64_t num_kv_blocks, const rbs_select_params* p, void* workspace, size_t workspace_bytes,
+                      rbs_block_lists* out, float* beta_out, rbs_stream_t stream) {
+  rbs_status st = check_tensor(Q, "Q");
+  if (st != RBS_OK) return st;
+  RBS_REQUIRE(p != nullptr && centroids != nullptr && radii != nullptr, RBS_ERR_INVALID_ARG, "null argument");
+  RBS_REQUIRE(p->block_q == p->block_k && (p->block_q == 64 || p->block_q == 128), RBS_ERR_UNSUPPORTED,
+              "block_q must equal block_k, 64 or 128");
+  RBS_REQUIRE(Q->seqlen % p->block_q == 0, RBS_ERR_UNSUPPORTED, "seqlen %% block_q != 0");
+  RBS_REQUIRE(kv_heads > 0 && Q->heads % kv_heads == 0, RBS_ERR_INVALID_ARG, "heads_q %% kv_heads != 0");
+  RBS_REQUIRE(num_kv_blocks > 0 && num_kv_blocks <= RBS_MAX_KV_BLOCKS, RBS_ERR_UNSUPPORTED,
+              "num_kv_blocks must be in [1, %d]", RBS_MAX_KV_BLOCKS);
+  RBS_REQUIRE(p->rho_centroid > 0.f && p->rho_centroid <= 1.f && p->rho_rescue > 0.f && p->rho_rescue <= 1.f,
+              RBS_ERR_INVALID_ARG, "rho must be in (0, 1]");
+  RBS_REQUIRE(p->q_block_offset >= 0, RBS_ERR_INVALID_ARG, "q_block_offset < 0");
+  RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
+  const int64_t B = Q->batch, Hq = Q->heads, nqb = Q->seqlen / p->block_q, nkb = num_kv_blocks;
+  const int64_t rows = B * Hq * nqb;
+  if ((st = check_lists(out, rows)) != RBS_OK) return st;
+  const int64_t cap = rbs_select_capacity(B, Hq, nqb, nkb, p);
+  RBS_REQUIRE(out->capacity >= cap, RBS_ERR_CAPACITY, "list capacity %lld < %lld", static_cast<long long>(out->capacity),
+              static_cast<long long>(cap));
+  const SelectLayout lay = select_layout(B, Hq, nqb, kv_heads, nkb);
+  RBS_REQUIRE(workspace != nullptr && workspace_bytes >= lay.total, RBS_ERR_CAPACITY, "workspace %zu < %zu bytes",
+              workspace_bytes, lay.total);
+  RBS_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, RBS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  DeviceInfo* di;
+  if ((st = device_info(&di)) != RBS_OK) return st;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* beta = beta_out != nullptr ? beta_out : reinterpret_cast<float*>(ws + lay.beta);
+  float* qbar = reinterpret_cast<float*>(ws + lay.qbar);
+  float* qnorm = reinterpret_cast<float*>(ws + lay.qnorm);
+  if ((st = rbs_block_beta(radii, B, kv_heads, nkb, p, beta, nullptr, stream)) != RBS_OK) return st;
+  if ((st = rbs_pool_queries(Q, p->block_q, qbar, qnorm, stream)) != RBS_OK) return st;
+
+  const int G = static_cast<int>(Hq / kv_heads);
+  int R = 1;
+  for (int r = 1; r <= kSelMaxR; ++r)
+    if (G % r == 0) R = r;
+  SelectArgs sa;
+  sa.qbar = qbar;
+  sa.qnorm = qnorm;
+  sa.C = centroids;
+  sa.rad = radii;
+  sa.beta = beta;
+  sa.Hq = static_cast<int>(Hq);
+  sa.Hkv = kv_heads;
+  sa.nqb = static_cast<int>(nqb);
+  sa.nkb = static_cast<int>(nkb);
+  sa.R = R;
+  sa.nwords = static_cast<int>((nkb + 31) / 32);
+  sa.q_block_offset = p->q_block_offset;
+  sa.causal = p->causal;
+  sa.force_diag = p->force_diag;
+  sa.force_sink = p->force_sink;
+  sa.rho_c = p->rho_centroid;
+  sa.rho_r = p->rho_rescue;
+  sa.mask_c = reinterpret_cast<uint32_t*>(ws + lay.mask_c);
+  sa.mask_r = reinterpret_cast<uint32_t*>(ws + lay.mask_r);
+  sa.counts = reinterpret_cast<int*>(ws + lay.counts);
+  const int npad = static_cast<int>((nkb + 31) & ~31ll);
+  const size_t smem = (kSelMaxR * 128 + npad + kSelMaxR * npad + kStageJ * kStagePitch) * sizeof(float);
+  const dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(Hq / R), static_cast<unsigned>(B));
+  if (nkb <= 64) select_rows_kernel<2><<<grid, kSelThreads, smem, stream>>>(sa);
+  else if (nkb <= 256) select_rows_kernel<8><<<grid, kSelThreads, smem, stream>>>(sa);
+  else if (nkb <= 1024) select_rows_kernel<32><<<grid, kSelThreads, smem, stream>>>(sa);
+  else if (nkb <= 2048) select_rows_kernel<64><<<grid, kSelThreads, smem, stream>>>(sa);
+  else select_rows_kernel<128><<<grid, kSelThreads, smem, stream>>>(sa);
+  if ((st = check_launch("select_rows_kernel")) != RBS_OK) return st;
+
+  scan_counts_kernel<<<1, 1024, 0, stream>>>(sa.counts, static_cast<int>(rows), out->row_ptr, out->capacity);
+  if ((st = check_launch("scan_counts_kernel")) != RBS_OK) return st;
+
+  CompactArgs ca;
+  ca.mask_c = sa.mask_c;
+  ca.mask_r = sa.mask_r;
+  ca.row_ptr = out->row_ptr;
+  ca.col_idx = out->col_idx;
+  ca.flags = out->flags;
+  ca.capacity = out->capacity;
+  ca.rows = static_cast<int>(rows);
+  ca.nqb = static_cast<int>(nqb);
+  ca.nkb = static_cast<int>(nkb);
+  ca.nwords = sa.nwords;
+  ca.q_block_offset = p->q_block_offset;
+  ca.force_diag = p->force_diag;
+  ca.force_sink = p->force_sink;
+  compact_lists_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(ca);
+  return check_launch("compact_lists_kernel");
+}
+
+// ---------------------------------------------------------------------------
+
+int64_t rbs_lists_causal_full_nnz(int32_t batch, int32_t heads_q, int32_t num_q_blocks, int32_t q_block_offset) {
+  if (batch <= 0 || heads_q <= 0 || num_q_blocks <= 0 || q_block_offset < 0) return -1;
+  const int64_t n = num_q_blocks;
+  return static_cast<int64_t>(batch) * heads_q * (n * (n - 1) / 2 + n * (q_block_offset + 1));
+}
+
+rbs_status rbs_lists_causal_full(int32_t batch, int32_t heads_q, int32_t num_q_blocks, int32_t q_block_offset,
+                                 rbs_block_lists* out, rbs_stream_t stream) {
+  RBS_REQUIRE(batch > 0 && heads_q > 0 && num_q_blocks > 0 && q_block_offset >= 0, RBS_ERR_INVALID_ARG, "bad shape");
+  const int64_t rows = static_cast<int64_t>(batch) * heads_q * num_q_blocks;
+  rbs_status st = check_lists(out, rows);
+  if (st != RBS_OK) return st;
+  const int64_t nnz = rbs_lists_causal_full_nnz(batch, heads_q, num_q_blocks, q_block_offset);
+  RBS_REQUIRE(out->capacity >= nnz, RBS_ERR_CAPACITY, "list capacity %lld < %lld", static_cast<long long>(out->capacity),
+              static_cast<long long>(nnz));
+  lists_causal_full_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<int>(rows), num_q_blocks, q_block_offset, out->row_ptr, out->col_idx, out->flags);
+  return check_launch("lists_causal_full_kernel");
+}
+
+namespace {
+rbs_status segment_table(const int32_t* seg_start, int32_t num_segments, int32_t final_start, int32_t block,
+                         SegmentTable* t) {
+  RBS_REQUIRE(seg_start != nullptr && num_segments > 0 && num_segments <= RBS_MAX_SEGMENTS, RBS_ERR_INVALID_ARG,
+              "segments: need 1..%d host offsets", RBS_MAX_SEGMENTS);
+  RBS_REQUIRE(block == 64 || block == 128, RBS_ERR_UNSUPPORTED, "block must be 64 or 128");
+  RBS_REQUIRE(seg_start[0] == 0, RBS_ERR_INVALID_ARG, "seg_start[0] must be 0");
+  t->n = num_segments;
+  for (int s = 0; s < num_segments; ++s) {
+    RBS_REQUIRE(seg_start[s] % block == 0, RBS_ERR_UNSUPPORTED, "segment start %d not a multiple of block", seg_start[s]);
+    RBS_REQUIRE(s == 0 || seg_start[s] > seg_start[s - 1], RBS_ERR_INVALID_ARG, "segment starts must ascend");
+    t->start_blk[s] = seg_start[s] / block;
+  }
+  RBS_REQUIRE(final_start % block == 0 && final_start > seg_start[num_segments - 1], RBS_ERR_INVALID_ARG,
+              "final_start must be a block multiple after the last passage");
+  t->final_blk = final_start / block;
+  return RBS_OK;
+}
+
+int64_t ba_prefix_host(const SegmentTable& s, int64_t x) {
+  int64_t tot = 0;
+  for (int p = 0; p < s.n; ++p) {
+    const int64_t a = s.start_blk[p];
+    const int64_t e = p + 1 < s.n ? s.start_blk[p + 1] : s.final_blk;
+    const int64_t m = std::min(std::max(x, a), e) - a;
+    tot += m * (m + 1) / 2;
+  }
+  const int64_t mf = std::max<int64_t>(0, x - s.final_blk);
+  tot += mf * (s.final_blk + 1) + mf * (mf - 1) / 2;
+  return tot;
+}
+}  // namespace
+
+int64_t rbs_lists_block_attention_nnz(const int32_t* seg_start, int32_t num_segments, int32_t final_start,
+                                      int32_t block, int32_t batch, int32_t heads_q, int32_t q_first_block,
+                                      int32_t q_num_blocks) {
+  SegmentTable t;
+  if (segment_table(seg_start, num_segments, final_start, block, &t) != RBS_OK) return -1;
+  if (batch <= 0 || heads_q <= 0 || q_first_block < 0 || q_num_blocks <= 0) return -1;
+  return static_cast<int64_t>(batch) * heads_q *
+         (ba_prefix_host(t, q_first_block + q_num_blocks) - ba_prefix_host(t, q_first_block));
+}
+
+rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t num_segments, int32_t final_start,
+                                     int32_t block, int32_t batch, int32_t heads_q, int32_t q_first_block,
+                                     int32_t q_num_blocks, rbs_block_lists* out, rbs_stream_t stream) {
+  SegmentTable t;
+  rbs_status st = segment_table(seg_start, num_segments, final_start, block, &t);
+  if (st != RBS_OK) return st;
+  RBS_REQUIRE(batch > 0 && heads_q > 0 && q_first_block >= 0 && q_num_blocks > 0, RBS_ERR_INVALID_ARG, "bad shape");
+  const int64_t rows = static_cast<int64_t>(batch) * heads_q * q_num_blocks;
+  if ((st = check_lists(out, rows)) != RBS_OK) return st;
+  const int64_t nnz = rbs_lists_block_attention_nnz(seg_start, num_segments, final_start, block, batch, heads_q,
+                                                    q_first_block, q_num_blocks);
+  RBS_REQUIRE(out->capacity >= nnz, RBS_ERR_CAPACITY, "list capacity %lld < %lld", static_cast<long long>(out->capacity),
+              static_cast<long long>(nnz));
+  lists_block_attention_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      t, static_cast<int>(rows), q_first_block, q_num_blocks, out->row_ptr, out->col_idx, out->flags);
+  return check_launch("lists_block_attention_kernel");
+}
+
+// ---------------------------------------------------------------------------
+
+rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                       const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
+                       float softmax_scale, int32_t causal, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
+  rbs_status st;
+  if ((st = check_tensor(Q, "Q")) != RBS_OK) return st;
+  if ((st = check_tensor(K, "K")) != RBS_OK) return st;
+  if ((st = check_tensor(V, "V")) != RBS_OK) return st;
+  if ((st = check_tensor(O, "O")) != RBS_OK) return st;
+  RBS_REQUIRE(block_q == block_k && (block_q == 64 || block_q == 128), RBS_ERR_UNSUPPORTED,
+              "block_q must equal block_k, 64 or 128");
+  RBS_REQUIRE(K->batch == Q->batch && V->batch == Q->batch && O->batch == Q->batch, RBS_ERR_INVALID_ARG, "batch mismatch");
+  RBS_REQUIRE(K->seqlen == V->seqlen && K->heads == V->heads, RBS_ERR_INVALID_ARG, "K/V shape mismatch");
+  RBS_REQUIRE(O->seqlen == Q->seqlen && O->heads == Q->heads, RBS_ERR_INVALID_ARG, "O shape != Q shape");
+  RBS_REQUIRE(Q->heads % K->heads == 0, RBS_ERR_INVALID_ARG, "heads_q %% heads_kv != 0");
+  RBS_REQUIRE(Q->seqlen % block_q == 0 && K->seqlen % block_k == 0, RBS_ERR_UNSUPPORTED, "seqlen not a block multiple");
+  RBS_REQUIRE(q_offset >= 0 && q_offset % block_k == 0, RBS_ERR_UNSUPPORTED, "q_offset must be a non-negative block multiple");
+  const int64_t nqb = Q->seqlen / block_q;
+  const int64_t rows = Q->batch * Q->heads * nqb;
+  if ((st = check_lists(lists, rows)) != RBS_OK) return st;
+  DeviceInfo* di;
+  if ((st = device_info(&di)) != RBS_OK) return st;
+
+  AttnArgs a;
+  int siq = 0, sik = 0, siv = 0;
+  if ((st = make_tensor_map(Q, block_q, &a.tmQ, &siq)) != RBS_OK) return st;
+  if ((st = make_tensor_map(K, block_k, &a.tmK, &sik)) != RBS_OK) return st;
+  if ((st = make_tensor_map(V, block_k, &a.tmV, &siv)) != RBS_OK) return st;
+  RBS_REQUIRE(siq == 0 && sik == 0 && siv == 0, RBS_ERR_UNSUPPORTED,
+              "Q/K/V must have the head stride no larger than the token stride ([B, L, H, 128] order)");
+  a.row_ptr = lists->row_ptr;
+  a.col_idx = lists->col_idx;
+  a.capacity = lists->capacity;
+  a.O = static_cast<__nv_bfloat16*>(O->data);
+  a.ob = O->stride_b;
+  a.os = O->stride_s;
+  a.oh = O->stride_h;
+  a.lse = lse;
+  a.B = static_cast<int>(Q->batch);
+  a.Hq = static_cast<int>(Q->heads);
+  a.Hkv = static_cast<int>(K->heads);
+  a.nqb = static_cast<int>(nqb);
+  a.nkb = static_cast<int>(K->seqlen / block_k);
+  a.Lq = static_cast<int>(Q->seqlen);
+  a.q_block_off = static_cast<int>(q_offset / block_k);
+  a.causal = causal ? 1 : 0;
+  a.num_rows = static_cast<int>(rows);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(RBS_HEAD_DIM));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const int grid = static_cast<int>(std::min<int64_t>(rows, di->sms));
+  if (block_q == 128)
+    bsa_prefill_kernel<128, 128><<<grid, kAttnThreads, AttnSmem<128>::kAlloc, stream>>>(a);
+  else
+    bsa_prefill_kernel<64, 64><<<grid, kAttnThreads, AttnSmem<64>::kAlloc, stream>>>(a);
+  return check_launch("bsa_prefill_kernel");
+}
+
+// ---------------------------------------------------------------------------
+
+rbs_status rope_reencode(const rbs_bf16_tensor* x_in, rbs_bf16_tensor* x_out, const int32_t* old_pos,
+                         const int32_t* new_pos, float theta, int32_t rope_style, rbs_stream_t stream) {
+  rbs_status st;
+  if ((st = check_tensor(x_in, "x_in")) != RBS_OK) return st;
+  if ((st = check_tensor(x_out, "x_out")) != RBS_OK) return st;
+  RBS_REQUIRE(x_in->batch == x_out->batch && x_in->seqlen == x_out->seqlen && x_in->heads == x_out->heads,
+              RBS_ERR_INVALID_ARG, "x_out shape != x_in shape");
+  RBS_REQUIRE(old_pos != nullptr && new_pos != nullptr, RBS_ERR_INVALID_ARG, "null positions");
+  RBS_REQUIRE(theta > 0.f, RBS_ERR_INVALID_ARG, "theta must be positive");
+  RBS_REQUIRE(rope_style == 0 || rope_style == 1, RBS_ERR_INVALID_ARG, "rope_style must be 0 or 1");
+  const bool alias = x_in->data == x_out->data;
+  RBS_REQUIRE(!alias || (x_in->stride_b == x_out->stride_b && x_in->stride_s == x_out->stride_s &&
+                         x_in->stride_h == x_out->stride_h),
+              RBS_ERR_INVALID_ARG, "in-place re-encoding needs identical strides");
+  DeviceInfo* di;
+  if ((st = device_info(&di)) != RBS_OK) return st;
+  RopeArgs a;
+  a.x = static_cast<const __nv_bfloat16*>(x_in->data);
+  a.y = static_cast<__nv_bfloat16*>(x_out->data);
+  a.xb = x_in->stride_b; a.xs = x_in->stride_s; a.xh = x_in->stride_h;
+  a.yb = x_out->stride_b; a.ys = x_out->stride_s; a.yh = x_out->stride_h;
+  a.old_pos = old_pos;
+  a.new_pos = new_pos;
+  a.L = static_cast<int>(x_in->seqlen);
+  a.H = static_cast<int>(x_in->heads);
+  for (int m = 0; m < 64; ++m)
+    a.inv_freq[m] = std::pow(static_cast<double>(theta), -2.0 * m / static_cast<double>(RBS_HEAD_DIM));
+  const dim3 grid(static_cast<unsigned>((a.L + kRopeTokens - 1) / kRopeTokens), static_cast<unsigned>(x_in->batch));
+  if (rope_style == 0) rope_reencode_kernel<0><<<grid, 256, 0, stream>>>(a);
+  else rope_reencode_kernel<1><<<grid, 256, 0, stream>>>(a);
+  return check_launch("rope_reencode_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,252 @@
+/*
+ * rbs.h -- C ABI of librbs: block-sparse prefill attention with
+ * radius-bounded block selection (RBS) and the Block-attention mask, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources the operations follow (web pages, cited by title and section):
+ *   [RBS-en] "RBS-Attention: How a Geometric Rescue Branch Fixes Sparse
+ *            Prefill for Long-Context LLMs": "The Standard Approach and Its
+ *            Blind Spot" (block centroid and radius), "The Fix: A
+ *            Radius-Adaptive Rescue Branch" (two scoring branches, independent
+ *            thresholds, combined mask, block-sparse attention).
+ *   [RBS-id] "RBS-Attention Bikin Prefill LLM Gede 20x Lebih Cepat, Tanpa
+ *            Training Lagi?": "Dual-Branch Selection: Centroid Base + Rescue
+ *            Branch" (radius distribution per prompt / layer / head).
+ *   [BA]     "Block-Attention for Efficient Prefilling": 2.1 Main idea,
+ *            2.2 Block segmentation, 2.3 Position re-encoding, 2.4 Block
+ *            fine-tune, 2.5 Inference.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer is a DEVICE pointer owned by the caller unless the argument
+ *   says "host".  The library never allocates device memory; calls that need
+ *   scratch take a caller-provided workspace whose size a *_workspace_bytes
+ *   query returns.
+ * - Every call is asynchronous on the given stream (a cudaStream_t; NULL is
+ *   the legacy default stream).  Results are valid once the stream reaches
+ *   the point after the call.
+ * - Host-side validation runs before any launch; a failed check returns its
+ *   status and launches nothing.  A CUDA launch error returns
+ *   RBS_ERR_CUDA.  rbs_last_error() gives a one-line reason for the last
+ *   non-OK status returned on the calling thread.
+ * - A data inconsistency found on the device (a block index out of range, a
+ *   row pointer beyond the list capacity, a pipeline wait that ran out of
+ *   time) never traps: the kernel skips the affected work, records a code in
+ *   the library's device error word and returns.  rbs_get_device_error()
+ *   reads and clears that word.
+ * - Tensors are bf16 [batch, seqlen, heads, head_dim] with head_dim == 128
+ *   contiguous (stride 1) and explicit element strides for the other three
+ *   dimensions; the base pointer and every stride must be 16-byte aligned
+ *   (strides a multiple of 8 elements).
+ * - Block lists ("rows") are CSR with one row per (batch, q head, query
+ *   block), ordered batch-major, then q head, then query block; each row's
+ *   key-block indices are ascending, so a row's diagonal block, when present,
+ *   is its last entry.
+ */
+#ifndef RBS_H_
+#define RBS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RBS_API __attribute__((visibility("default")))
+#else
+#define RBS_API
+#endif
+
+#define RBS_ABI_VERSION 1
+#define RBS_HEAD_DIM 128
+#define RBS_MAX_SEGMENTS 512 /* Block-attention segments per call */
+#define RBS_MAX_KV_BLOCKS 4096 /* key blocks per sequence for rbs_select */
+
+typedef struct CUstream_st* rbs_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  RBS_OK = 0,
+  RBS_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misaligned stride */
+  RBS_ERR_UNSUPPORTED = 2, /* valid but outside what this build implements */
+  RBS_ERR_CAPACITY = 3,    /* output list or workspace too small */
+  RBS_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  RBS_ERR_DEVICE = 5       /* the device error word was set (see below) */
+} rbs_status;
+
+/* Device error word bits (rbs_get_device_error). */
+#define RBS_DEVERR_BLOCK_INDEX 0x1   /* a list entry outside [0, num_kv_blocks) */
+#define RBS_DEVERR_ROW_PTR 0x2       /* row_ptr not monotone or beyond capacity */
+#define RBS_DEVERR_TIMEOUT 0x4       /* a pipeline wait ran out of time */
+#define RBS_DEVERR_NONCAUSAL 0x8     /* a causal row lists a block after its diagonal */
+
+typedef struct {
+  void* data; /* device pointer to the element at [0, 0, 0, 0] */
+  int64_t batch, seqlen, heads, head_dim;
+  int64_t stride_b, stride_s, stride_h; /* in elements; the head_dim stride is 1 */
+} rbs_bf16_tensor;
+
+/*
+ * Selection parameters.  Every point the sources leave open is a field
+ * (defaults from rbs_select_params_default):
+ *   block_q, block_k   query / key block size, 64 or 128, equal (128)
+ *   rho_centroid       centroid branch: keep ceil(rho * n_i) of the n_i
+ *   rho_rescue         rescue branch: same rule, its own rho ([RBS-en] "The
+ *                      Fix": the branches are thresholded independently) (0.05)
+ *   beta_mode          0 = RANGE: beta_b = clamp((r_b - R_lo)/(R_hi - R_lo), 0, 1)
+ *                      with R_lo, R_hi the beta_p_lo / beta_p_hi quantiles
+ *                      (linear interpolation) of the radii of that prompt and
+ *                      KV head ([RBS-id]: per prompt, per head), a degenerate
+ *                      range giving beta = 1; 1 = CONST: beta_b = beta_const (0)
+ *   beta_const         CONST value; 1 gives the Cauchy-Schwarz bound (1.0)
+ *   beta_p_lo/hi       RANGE quantiles; beta_p_lo < 0 means R_lo = 0 (0, 1)
+ *   force_diag         always keep the query block's own (diagonal) key block (1)
+ *   force_sink         always keep key block 0 (0)
+ *   causal             query block i (global index i + q_block_offset) may
+ *                      select key blocks 0 .. i + q_block_offset only (1)
+ *   q_block_offset     global key-block index of query block 0 (0)
+ * Scores are raw dot products (no 1/sqrt(d)); ties between equal scores go
+ * to the lower block index.  Forced blocks do not count toward a branch's k.
+ */
+typedef struct {
+  int32_t block_q, block_k;
+  float rho_centroid, rho_rescue;
+  int32_t beta_mode;
+  float beta_const;
+  float beta_p_lo, beta_p_hi;
+  int32_t force_diag, force_sink, causal;
+  int32_t q_block_offset;
+} rbs_select_params;
+
+/* Per-query-block key-block lists in CSR form (all device memory). */
+typedef struct {
+  int32_t* row_ptr; /* [num_rows + 1]; row r spans col_idx[row_ptr[r] .. row_ptr[r+1]) */
+  int32_t* col_idx; /* [capacity] key-block indices, ascending within a row */
+  uint8_t* flags;   /* [capacity] or NULL: bit0 centroid branch kept the block,
+                       bit1 rescue branch kept it, bit2 forced (diagonal/sink) */
+  int64_t capacity; /* entries col_idx (and flags) can hold */
+  int32_t num_rows; /* batch * heads_q * num_q_blocks */
+} rbs_block_lists;
+
+/* ---- housekeeping ------------------------------------------------------ */
+
+RBS_API int32_t rbs_abi_version(void);
+RBS_API const char* rbs_status_string(rbs_status s);
+/* One-line reason for the last non-OK status returned on this host thread. */
+RBS_API const char* rbs_last_error(void);
+/* Fill *p with the defaults listed above. */
+RBS_API void rbs_select_params_default(rbs_select_params* p);
+/* Read (synchronising the stream) and clear the device error word.
+ * *code_host receives the RBS_DEVERR_* bits; returns RBS_ERR_DEVICE when
+ * any bit was set, RBS_OK otherwise. */
+RBS_API rbs_status rbs_get_device_error(int32_t* code_host, rbs_stream_t stream);
+
+/* ---- block statistics  ([RBS-en] "The Standard Approach and Its Blind Spot")
+ * For every key block b of block_k consecutive tokens of every (batch, KV
+ * head): centroid c_b = mean of the block's keys, radius r_b = max over the
+ * block's keys of ||k - c_b||_2.  fp32 accumulation of the bf16 keys.
+ *   K          [B, L, Hkv, 128] bf16, L a multiple of block_k (64 or 128)
+ *   centroids  out [B, Hkv, L/block_k, 128] fp32, contiguous
+ *   radii      out [B, Hkv, L/block_k] fp32, contiguous
+ */
+RBS_API rbs_status rbs_block_stats(const rbs_bf16_tensor* K, int32_t block_k, float* centroids, float* radii,
+                           rbs_stream_t stream);
+
+/* ---- rescue coefficient  ([RBS-en] "The Fix"; [RBS-id] "Dual-Branch Selection")
+ * beta [B, Hkv, nKB] from radii [B, Hkv, nKB] per p->beta_mode (see the
+ * parameter block above).  radius_range, when not NULL, receives (R_lo, R_hi)
+ * per (batch, KV head) as [B, Hkv, 2] fp32.  nKB <= RBS_MAX_KV_BLOCKS. */
+RBS_API rbs_status rbs_block_beta(const float* radii, int64_t batch, int64_t kv_heads, int64_t num_blocks,
+                          const rbs_select_params* p, float* beta, float* radius_range, rbs_stream_t stream);
+
+/* ---- query-block representative  ([RBS-en] "The Fix": the q of q^T c_b)
+ * qbar [B, Hq, L/block_q, 128] fp32 = mean of each query block's queries;
+ * qnorm [B, Hq, L/block_q] fp32 = ||qbar||_2.  Both contiguous. */
+RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, float* qbar, float* qnorm,
+                            rbs_stream_t stream);
+
+/* ---- selection  ([RBS-en] "The Fix"; [RBS-id] "Dual-Branch Selection")
+ * For every (batch, q head h, query block i), with KV head h / (Hq / Hkv):
+ *   s_c(j) = qbar_i . c_j                      (centroid branch)
+ *   s_r(j) = s_c(j) + ||qbar_i|| * r_j * beta_j  (rescue branch)
+ * over the visible key blocks j (j <= i + q_block_offset when causal); each
+ * branch keeps its own top ceil(rho * n_i) blocks; the row's list is the
+ * union of both kept sets plus the forced blocks, ascending.
+ *   Q            [B, Lq, Hq, 128] bf16, Lq a multiple of block_q
+ *   centroids    [B, Hkv, num_kv_blocks, 128] fp32 (rbs_block_stats)
+ *   radii        [B, Hkv, num_kv_blocks] fp32
+ *   workspace    device scratch of at least rbs_select_workspace_bytes(...)
+ *                bytes, 256-byte aligned; its contents need no initialisation
+ *   out          lists with num_rows = B * Hq * Lq / block_q and capacity >=
+ *                rbs_select_capacity(...); row_ptr, col_idx and flags written
+ *   beta_out     optional [B, Hkv, num_kv_blocks] fp32 copy of beta (or NULL)
+ * Requires Hq % Hkv == 0, num_kv_blocks <= RBS_MAX_KV_BLOCKS. */
+RBS_API int64_t rbs_select_capacity(int64_t batch, int64_t heads_q, int64_t num_q_blocks, int64_t num_kv_blocks,
+                            const rbs_select_params* p);
+RBS_API size_t rbs_select_workspace_bytes(int64_t batch, int64_t heads_q, int64_t num_q_blocks, int64_t kv_heads,
+                                  int64_t num_kv_blocks, const rbs_select_params* p);
+RBS_API rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const float* radii, int32_t kv_heads,
+                      int64_t num_kv_blocks, const rbs_select_params* p, void* workspace, size_t workspace_bytes,
+                      rbs_block_lists* out, float* beta_out, rbs_stream_t stream);
+
+/* ---- list builders (device kernels; no host copies)
+ * Every causally visible block: row (b, h, i) lists 0 .. i + q_block_offset.
+ * Capacity needed: batch * heads_q * sum_i (i + q_block_offset + 1). */
+RBS_API int64_t rbs_lists_causal_full_nnz(int32_t batch, int32_t heads_q, int32_t num_q_blocks, int32_t q_block_offset);
+RBS_API rbs_status rbs_lists_causal_full(int32_t batch, int32_t heads_q, int32_t num_q_blocks, int32_t q_block_offset,
+                                 rbs_block_lists* out, rbs_stream_t stream);
+
+/* Block-attention mask ([BA] 2.1, 2.2, 2.4): passage s covers tokens
+ * [seg_start[s], seg_start[s+1]) (the last passage ends at final_start); the
+ * final block (the user query) covers [final_start, end).  A query block of
+ * passage s lists the key blocks of passage s up to itself; a query block of
+ * the final block lists every key block up to itself.  Rows are query blocks
+ * q_first_block .. q_first_block + q_num_blocks - 1 (global block indices) of
+ * every (batch, q head).  seg_start is a HOST array of num_segments <=
+ * RBS_MAX_SEGMENTS ascending token offsets, seg_start[0] == 0, every offset
+ * and final_start a multiple of block. */
+RBS_API int64_t rbs_lists_block_attention_nnz(const int32_t* seg_start, int32_t num_segments, int32_t final_start,
+                                      int32_t block, int32_t batch, int32_t heads_q, int32_t q_first_block,
+                                      int32_t q_num_blocks);
+RBS_API rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t num_segments, int32_t final_start,
+                                     int32_t block, int32_t batch, int32_t heads_q, int32_t q_first_block,
+                                     int32_t q_num_blocks, rbs_block_lists* out, rbs_stream_t stream);
+
+/* ---- block-sparse prefill attention  ([RBS-en] "The Fix": exact attention over
+ * the selected blocks, standard multi-head / grouped-query attention)
+ * For query token t of row (b, h, i) at position t + q_offset:
+ *   O[b, t, h] = sum_s softmax_s(scale * q_t . k_s) v_s
+ * over the key tokens s of the row's listed blocks, with s <= t + q_offset
+ * when causal; KV head = h / (Hq / Hkv).  bf16 tensor-core products, fp32
+ * accumulation and softmax.
+ *   Q         [B, Lq, Hq, 128] bf16; K, V [B, Lk, Hkv, 128] bf16
+ *   lists     num_rows = B * Hq * Lq / block_q; indices in [0, Lk / block_k)
+ *   block_q == block_k, 64 or 128; q_offset a multiple of block_k
+ *   softmax_scale  <= 0 selects 1/sqrt(128)
+ *   O         out [B, Lq, Hq, 128] bf16 (may not alias Q, K or V)
+ *   lse       optional out [B, Hq, Lq] fp32 = ln sum_s exp(scale q_t.k_s)
+ *             (-inf for an empty row, whose O is 0)
+ * Uses no workspace.  Lists are read, never written. */
+RBS_API rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                       const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
+                       float softmax_scale, int32_t causal, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream);
+
+/* ---- RoPE position re-encoding  ([BA] 2.3 Position re-encoding, 2.5 Inference)
+ * Keys cached with RoPE at old_pos are moved to new_pos: the rotation is reset
+ * to position 0 and applied again at the new position, done as one rotation by
+ * (new_pos - old_pos) * inv_freq_m, inv_freq_m = theta^(-2m/128).  The angle
+ * is formed and reduced in fp64; the rotation is applied in fp32 and rounded
+ * to bf16 once.
+ *   x_in, x_out  [B, L, H, 128] bf16, same shape; x_out may alias x_in
+ *   old_pos, new_pos  [L] int32 token positions (shared by batch and heads)
+ *   rope_style   0 = rotate-half pairs (m, m + 64); 1 = interleaved (2m, 2m+1)
+ * Re-encoding from old_pos = 0 is plain RoPE encoding. */
+RBS_API rbs_status rope_reencode(const rbs_bf16_tensor* x_in, rbs_bf16_tensor* x_out, const int32_t* old_pos,
+                         const int32_t* new_pos, float theta, int32_t rope_style, rbs_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RBS_H_ */

@@ -183,8 +183,13 @@ def pooled_queries(Q: np.ndarray, block_q: int):
 
 
 def keep_count(rho: float, n: int) -> int:
-    """k = ceil(rho * n), at least 1 and at most n (the 1e-9 absorbs rho*n rounding)."""
-    return int(min(n, max(1, math.ceil(rho * n - 1e-9))))
+    """k = ceil(rho * n), at least 1 and at most n.
+
+    rho is a float32 parameter (e.g. float32(0.05) = 0.0500000007...); the
+    1e-4 slack keeps its representation error from adding a block
+    (ceil(20 * float32(0.05)) would otherwise be 2, not 1).
+    """
+    return int(min(n, max(1, math.ceil(rho * n - 1e-4))))
 
 
 def visible_blocks(i: int, nkb: int, p: SelectParams) -> int:

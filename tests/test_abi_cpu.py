@@ -1,0 +1,166 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+header declares, answers the host-only size queries, and rejects bad
+arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_long_rbs_b200 import _abi
+from block_sparse_long_rbs_b200 import SelectParams, BlockLists  # noqa: F401
+from oracle import rbs_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_long_rbs_b200 import build
+    build.build()
+    return _abi.lib()
+
+
+def _declared():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        names += re.findall(r"^RBS_API\s+[\w\s\*]+?\b(\w+)\(", src, flags=re.M)
+    return names
+
+
+def test_header_declares_the_pages_calls():
+    names = set(_declared())
+    for required in ("rbs_block_stats", "rbs_select", "bsa_prefill", "rope_reencode"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_abi.SIGNATURES)
+
+
+def test_housekeeping(L):
+    assert L.rbs_abi_version() == 1
+    assert L.rbs_status_string(0) == b"ok"
+    assert L.rbs_status_string(3) == b"capacity"
+    p = _abi.SelectParamsC()
+    L.rbs_select_params_default(ctypes.byref(p))
+    d = SelectParams()
+    for f in _abi.SelectParamsC._fields_:
+        assert getattr(p, f[0]) == pytest.approx(getattr(d, f[0]))
+
+
+@pytest.mark.parametrize("rho,off,diag,sink", [(0.05, 0, 1, 0), (0.25, 0, 1, 1), (1.0, 3, 0, 0), (0.1, 0, 1, 0)])
+def test_select_capacity_bounds_oracle_rows(L, rho, off, diag, sink):
+    nqb, nkb = 40, 40 + off
+    p = SelectParams(rho_centroid=rho, rho_rescue=rho, force_diag=diag, force_sink=sink, q_block_offset=off)
+    cap = L.rbs_select_capacity(2, 3, nqb, nkb, ctypes.byref(p.c()))
+    rho32 = float(np.float32(rho))
+    expect = 0
+    for i in range(nqb):
+        n = min(nkb, i + off + 1)
+        expect += min(n, 2 * O.keep_count(rho32, n) + diag + sink)
+    assert cap == 6 * expect
+
+
+def test_causal_full_nnz(L):
+    for nqb, off in ((1, 0), (64, 0), (4, 256)):
+        rp, ci = O.causal_full_lists(2, 3, nqb, off)
+        assert L.rbs_lists_causal_full_nnz(2, 3, nqb, off) == ci.size
+
+
+def test_block_attention_nnz_matches_oracle(L):
+    seg = [0, 256, 1024, 1536]
+    arr = (ctypes.c_int32 * 4)(*seg)
+    for first, num in ((0, 13), (12, 1), (3, 9)):
+        rp, ci = O.block_attention_lists(seg, 1536 + 128, 128, 2, 5, first, num)
+        assert L.rbs_lists_block_attention_nnz(arr, 4, 1536 + 128, 128, 2, 5, first, num) == ci.size
+
+
+def test_block_attention_rejects_bad_segments(L):
+    bad = (ctypes.c_int32 * 2)(0, 100)  # not a block multiple
+    assert L.rbs_lists_block_attention_nnz(bad, 2, 512, 128, 1, 1, 0, 4) == -1
+    desc = (ctypes.c_int32 * 2)(128, 256)  # does not start at 0
+    assert L.rbs_lists_block_attention_nnz(desc, 2, 512, 128, 1, 1, 0, 4) == -1
+
+
+def _fake(B=1, Lq=256, H=2, D=128, sb=None, ss=None, sh=None, ptr=0x10000):
+    sh = D if sh is None else sh
+    ss = H * D if ss is None else ss
+    sb = Lq * H * D if sb is None else sb
+    return _abi.Bf16Tensor(ptr, B, Lq, H, D, sb, ss, sh)
+
+
+def test_validation_before_any_launch(L):
+    C = ctypes.c_void_p(0x20000)
+    R = ctypes.c_void_p(0x30000)
+    s = ctypes.c_void_p(0)
+    null = _abi.Bf16Tensor()
+    assert L.rbs_block_stats(ctypes.byref(null), 128, C, R, s) == 1
+    assert L.rbs_block_stats(ctypes.byref(_fake(D=64)), 128, C, R, s) == 2
+    assert L.rbs_block_stats(ctypes.byref(_fake()), 96, C, R, s) == 2
+    assert L.rbs_block_stats(ctypes.byref(_fake(Lq=200)), 128, C, R, s) == 2
+    assert L.rbs_block_stats(ctypes.byref(_fake(ptr=0x10002)), 128, C, R, s) == 1
+    assert L.rbs_block_stats(ctypes.byref(_fake(ss=260)), 128, C, R, s) == 1
+    assert b"strides" in L.rbs_last_error()
+    # valid arguments on a machine without a GPU fail loudly with a CUDA status
+    assert L.rbs_block_stats(ctypes.byref(_fake()), 128, C, R, s) == 4
+
+
+def test_select_rejects_small_capacity_and_workspace(L):
+    p = SelectParams(block_q=64, block_k=64)
+    pc = p.c()
+    q = _fake(Lq=512)
+    rows = 1 * 2 * 8
+    need = L.rbs_select_capacity(1, 2, 8, 8, ctypes.byref(pc))
+    ws = L.rbs_select_workspace_bytes(1, 2, 8, 1, 8, ctypes.byref(pc))
+    assert ws > 0
+    small = _abi.BlockListsC(0x40000, 0x50000, None, need - 1, rows)
+    st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, ws, ctypes.byref(small),
+                      None, None)
+    assert st == 3
+    ok = _abi.BlockListsC(0x40000, 0x50000, None, need, rows)
+    st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, ws - 1, ctypes.byref(ok),
+                      None, None)
+    assert st == 3
+    wrong_rows = _abi.BlockListsC(0x40000, 0x50000, None, need, rows + 1)
+    st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, ws, ctypes.byref(wrong_rows),
+                      None, None)
+    assert st == 1
+    st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 3, 8, ctypes.byref(pc), 0x60000, ws, ctypes.byref(ok),
+                      None, None)
+    assert st == 1  # 2 q heads cannot share 3 KV heads
+
+
+def test_bsa_prefill_validation(L):
+    q = _fake(Lq=256, H=4)
+    k = _fake(Lq=256, H=2)
+    o = _fake(Lq=256, H=4)
+    lists = _abi.BlockListsC(0x40000, 0x50000, None, 100, 1 * 4 * 2)
+    s = ctypes.c_void_p(0)
+    f = L.bsa_prefill
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(lists), 128, 64, 0, 0.0, 1,
+             ctypes.byref(o), None, s) == 2  # block_q != block_k
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(lists), 128, 128, 64, 0.0, 1,
+             ctypes.byref(o), None, s) == 2  # q_offset not a block multiple
+    k3 = _fake(Lq=256, H=3)
+    assert f(ctypes.byref(q), ctypes.byref(k3), ctypes.byref(k3), ctypes.byref(lists), 128, 128, 0, 0.0, 1,
+             ctypes.byref(o), None, s) == 1
+    bad_rows = _abi.BlockListsC(0x40000, 0x50000, None, 100, 7)
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(bad_rows), 128, 128, 0, 0.0, 1,
+             ctypes.byref(o), None, s) == 1
+
+
+def test_rope_validation(L):
+    x = _fake()
+    s = ctypes.c_void_p(0)
+    assert L.rope_reencode(ctypes.byref(x), ctypes.byref(_fake(Lq=128)), 0x1000, 0x2000, 5e5, 0, s) == 1
+    assert L.rope_reencode(ctypes.byref(x), ctypes.byref(x), None, 0x2000, 5e5, 0, s) == 1
+    assert L.rope_reencode(ctypes.byref(x), ctypes.byref(x), 0x1000, 0x2000, 5e5, 2, s) == 1
+    assert L.rope_reencode(ctypes.byref(x), ctypes.byref(x), 0x1000, 0x2000, -1.0, 0, s) == 1

@@ -1,0 +1,101 @@
+"""GPU parity: two-branch selection -> CSR lists, against the oracle's lists.
+
+Lists must match exactly, branch by branch, except for blocks whose oracle
+score lies within 1e-3 * max(1, |tau|) of that branch's threshold tau; those
+are counted.  Each GPU branch must keep exactly k_i blocks, the union must be
+the two branches plus the forced blocks, rows ascending.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_rbs_b200 as rbs
+from helpers import compare_selection, dev
+from oracle import rbs_oracle as O
+from workloads import WORKLOADS, make_inputs, make_mixture, make_tiny
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, block, rho_c, rho_r, **kw):
+    Q, K = inp["Q"], inp["K"]
+    B, L, Hq, _ = Q.shape
+    Hkv = K.shape[2]
+    nqb = L // block
+    nkb = K.shape[1] // block
+    p = rbs.SelectParams(block_q=block, block_k=block, rho_centroid=rho_c, rho_rescue=rho_r, **kw)
+    Cg, Rg = rbs.rbs_block_stats(dev(K), block)
+    lists = rbs.rbs_select(dev(Q), Cg, Rg, p)
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    Co, Ro = O.block_stats(K, block)
+    po = O.SelectParams(block_q=block, block_k=block, rho_centroid=float(np.float32(rho_c)),
+                        rho_rescue=float(np.float32(rho_r)), **{k: (float(np.float32(v)) if isinstance(v, float) else v)
+                                                                for k, v in kw.items()})
+    ora = O.select_blocks(Q, Co, Ro, po, keep_scores=True)
+    return compare_selection(lists, ora, Hq, nqb, nkb)
+
+
+def test_select_tiny_config(cuda_ok):
+    w = WORKLOADS["tiny_rbs_4k"]
+    rep = _run(make_inputs(w), 64, w.rho, w.rho)
+    print("tiny", rep)
+
+
+@pytest.mark.parametrize("beta_mode,const", [(0, 1.0), (1, 1.0), (1, 0.0)])
+def test_select_mixture_small_beta_modes(cuda_ok, beta_mode, const):
+    inp = make_mixture(L=8192, Hq=16, Hkv=2, block=128, seed=201)
+    rep = _run(inp, 128, 0.1, 0.15, beta_mode=beta_mode, beta_const=const)
+    print("mixture8k", beta_mode, const, rep)
+
+
+def test_select_force_sink_batch2_ragged_group(cuda_ok):
+    # batch 2, G = 6 (rows per CTA fall back to 6), sink forced
+    inp = make_mixture(L=4096, Hq=12, Hkv=2, block=128, seed=202, batch=2)
+    rep = _run(inp, 128, 0.2, 0.1, force_sink=1)
+    print("sink", rep)
+
+
+def test_select_noncausal_with_offset(cuda_ok):
+    inp = make_mixture(L=4096, Hq=4, Hkv=1, block=64, seed=203)
+    rep = _run(inp, 64, 0.1, 0.1, causal=0)
+    print("noncausal", rep)
+
+
+def test_select_32k_gqa_config(cuda_ok):
+    w = WORKLOADS["gqa_rbs_32k"]
+    inp = make_inputs(w)
+    Co, Ro = O.block_stats(inp["K"], 128)
+    rho, dens = O.bisect_rho(inp["Q"], Co, Ro, O.SelectParams(), w.density_target)
+    rho32 = float(np.float32(rho))
+    rep = _run(inp, 128, rho32, rho32)
+    print("32k", rho32, dens, rep)
+    assert abs(rep["nnz_gpu"] - rep["nnz_oracle"]) <= rep["centroid"] + rep["rescue"]
+
+
+def test_select_128k_config(cuda_ok):
+    w = WORKLOADS["gqa_rbs_128k"]
+    rep = _run(make_inputs(w), 128, w.rho, w.rho)
+    print("128k", rep)
+
+
+def test_select_deterministic(cuda_ok):
+    inp = make_tiny(L=2048)
+    p = rbs.SelectParams(block_q=64, block_k=64, rho_centroid=0.25, rho_rescue=0.25)
+    Cg, Rg = rbs.rbs_block_stats(dev(inp["K"]), 64)
+    a = rbs.rbs_select(dev(inp["Q"]), Cg, Rg, p)
+    b = rbs.rbs_select(dev(inp["Q"]), Cg, Rg, p)
+    assert torch.equal(a.row_ptr, b.row_ptr)
+    n = a.nnz()
+    assert torch.equal(a.col_idx[:n], b.col_idx[:n]) and torch.equal(a.flags[:n], b.flags[:n])
+
+
+def test_select_rho_one_is_causal_full(cuda_ok):
+    inp = make_tiny(L=1024)
+    p = rbs.SelectParams(block_q=64, block_k=64, rho_centroid=1.0, rho_rescue=1.0)
+    Cg, Rg = rbs.rbs_block_stats(dev(inp["K"]), 64)
+    s = rbs.rbs_select(dev(inp["Q"]), Cg, Rg, p)
+    f = rbs.rbs_lists_causal_full(1, 2, 16, 0)
+    assert torch.equal(s.row_ptr, f.row_ptr)
+    assert torch.equal(s.col_idx[:s.nnz()], f.col_idx[:f.nnz()])

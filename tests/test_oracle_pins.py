@@ -196,6 +196,8 @@ def test_keep_count_values():
     assert O.keep_count(1.0, 7) == 7
     assert O.keep_count(1e-6, 7) == 1
     assert O.keep_count(0.05, 1024) == 52
+    assert O.keep_count(float(np.float32(0.05)), 20) == 1  # float32 rho, exact product 1.0000000149
+    assert O.keep_count(float(np.float32(0.1)), 30) == 3
 
 
 def test_top_k_matches_brute_force_with_ties():
