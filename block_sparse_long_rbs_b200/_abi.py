@@ -18,6 +18,7 @@ STATUS_NAMES = {0: "RBS_OK", 1: "RBS_ERR_INVALID_ARG", 2: "RBS_ERR_UNSUPPORTED",
 DEVERR_BLOCK_INDEX, DEVERR_ROW_PTR, DEVERR_TIMEOUT, DEVERR_NONCAUSAL = 0x1, 0x2, 0x4, 0x8
 MAX_SEGMENTS = 512
 MAX_KV_BLOCKS = 4096
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class Bf16Tensor(ctypes.Structure):
@@ -55,6 +56,7 @@ SIGNATURES = {
     "rbs_select_capacity": (i64, [i64, i64, i64, i64, P(SelectParamsC)]),
     "rbs_select_workspace_bytes": (sz, [i64, i64, i64, i64, i64, P(SelectParamsC)]),
     "rbs_select": (ctypes.c_int, [P(Bf16Tensor), vp, vp, i32, i64, P(SelectParamsC), vp, sz, P(BlockListsC), vp, vp]),
+    "rbs_select_noalloc": (ctypes.c_int, [P(Bf16Tensor), vp, vp, i32, i64, P(SelectParamsC), P(BlockListsC), vp, vp]),
     "rbs_lists_causal_full_nnz": (i64, [i32, i32, i32, i32]),
     "rbs_lists_causal_full": (ctypes.c_int, [i32, i32, i32, i32, P(BlockListsC), vp]),
     "rbs_lists_block_attention_nnz": (i64, [P(i32), i32, i32, i32, i32, i32, i32, i32]),

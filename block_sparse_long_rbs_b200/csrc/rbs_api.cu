@@ -412,6 +412,60 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
 }
 
 // ---------------------------------------------------------------------------
+// Selection without any allocation by the caller.  The scratch that
+// rbs_select normally takes as a workspace is instead a fixed buffer in this
+// library's own device image (RBS_NOALLOC_SCRATCH_BYTES on every device that
+// loads the library, held until the process exits).  Host code cannot use the
+// array's name as a device address, so its address is looked up once per
+// device with that device current and cached.
+
+}  // extern "C"
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[RBS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+rbs_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(RBS_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(RBS_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return RBS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+rbs_status rbs_select_noalloc(const rbs_bf16_tensor* Q, const float* centroids, const float* radii,
+                              int32_t kv_heads, int64_t num_kv_blocks, const rbs_select_params* p,
+                              rbs_block_lists* out, float* beta_out, rbs_stream_t stream) {
+  rbs_status st = check_tensor(Q, "Q");
+  if (st != RBS_OK) return st;
+  RBS_REQUIRE(p != nullptr && (p->block_q == 64 || p->block_q == 128) && Q->seqlen % p->block_q == 0,
+              RBS_ERR_UNSUPPORTED, "block_q must be 64 or 128 and divide seqlen");
+  RBS_REQUIRE(kv_heads > 0 && num_kv_blocks > 0, RBS_ERR_INVALID_ARG, "empty KV shape");
+  const size_t need = rbs_select_workspace_bytes(Q->batch, Q->heads, Q->seqlen / p->block_q, kv_heads,
+                                                 num_kv_blocks, p);
+  RBS_REQUIRE(need > 0 && need <= RBS_NOALLOC_SCRATCH_BYTES, RBS_ERR_CAPACITY,
+              "this selection needs %zu bytes of scratch; the built-in buffer holds %zu (use rbs_select with a "
+              "workspace)", need, static_cast<size_t>(RBS_NOALLOC_SCRATCH_BYTES));
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != RBS_OK) return st;
+  return rbs_select(Q, centroids, radii, kv_heads, num_kv_blocks, p, scratch, RBS_NOALLOC_SCRATCH_BYTES, out,
+                    beta_out, stream);
+}
+
+// ---------------------------------------------------------------------------
 
 int64_t rbs_lists_causal_full_nnz(int32_t batch, int32_t heads_q, int32_t num_q_blocks, int32_t q_block_offset) {
   if (batch <= 0 || heads_q <= 0 || num_q_blocks <= 0 || q_block_offset < 0) return -1;

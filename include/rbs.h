@@ -190,6 +190,30 @@ RBS_API rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, 
                       int64_t num_kv_blocks, const rbs_select_params* p, void* workspace, size_t workspace_bytes,
                       rbs_block_lists* out, float* beta_out, rbs_stream_t stream);
 
+/* ---- selection with no caller-provided scratch
+ * No counterpart in the papers: this is a convenience of the library.  Some
+ * callers cannot hand the library a device workspace -- for example code
+ * running inside a host framework that owns all device memory and forbids raw
+ * allocations, or a serving loop where any allocation could stall other
+ * streams.  This variant of rbs_select allocates nothing: its scratch is a
+ * fixed buffer of RBS_NOALLOC_SCRATCH_BYTES compiled into the library, which
+ * every GPU that loads the library holds until the process exits.
+ * The caller still passes all inputs and outputs (same meaning as
+ * rbs_select).  A selection whose scratch would exceed the buffer
+ * (rbs_select_workspace_bytes > RBS_NOALLOC_SCRATCH_BYTES; the 131072-token,
+ * 32-head, 128-block case needs about 24 MiB) returns RBS_ERR_CAPACITY and
+ * launches nothing.  The first call on each device looks up the buffer's
+ * device address (a CUDA runtime query, no allocation); make that first call
+ * before any stream capture.  All calls on a device share the one buffer:
+ * every scratch region is fully written before it is read, so nothing needs
+ * clearing between calls, but two calls that may overlap on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller. */
+#define RBS_NOALLOC_SCRATCH_BYTES (32u << 20)
+RBS_API rbs_status rbs_select_noalloc(const rbs_bf16_tensor* Q, const float* centroids, const float* radii,
+                                      int32_t kv_heads, int64_t num_kv_blocks, const rbs_select_params* p,
+                                      rbs_block_lists* out, float* beta_out, rbs_stream_t stream);
+
 /* ---- list builders (device kernels; no host copies)
  * Every causally visible block: row (b, h, i) lists 0 .. i + q_block_offset.
  * Capacity needed: batch * heads_q * sum_i (i + q_block_offset + 1). */
