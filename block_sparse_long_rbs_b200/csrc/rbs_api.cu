@@ -79,11 +79,17 @@ rbs_status device_info(DeviceInfo** out) {
                                      AttnSmem<128, kWg128>::kAlloc);
     e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<64, 64, kWg64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      AttnSmem<64, kWg64>::kAlloc);
-    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    e = e ? e : cudaFuncSetAttribute(select_rows_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+#define RBS_SEL_ATTR(KPL)                                                                                  \
+  e = e ? e : cudaFuncSetAttribute(select_rows_kernel<KPL, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                   200 * 1024);                                                              \
+  e = e ? e : cudaFuncSetAttribute(select_rows_kernel<KPL, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                   200 * 1024);
+    RBS_SEL_ATTR(2)
+    RBS_SEL_ATTR(8)
+    RBS_SEL_ATTR(32)
+    RBS_SEL_ATTR(64)
+    RBS_SEL_ATTR(128)
+#undef RBS_SEL_ATTR
     e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
     if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     d.attrs_set = true;
@@ -360,18 +366,17 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* beta = beta_out != nullptr ? beta_out : reinterpret_cast<float*>(ws + lay.beta);
-  float* qbar = reinterpret_cast<float*>(ws + lay.qbar);
-  float* qnorm = reinterpret_cast<float*>(ws + lay.qnorm);
   if ((st = rbs_block_beta(radii, B, kv_heads, nkb, p, beta, nullptr, stream)) != RBS_OK) return st;
-  if ((st = rbs_pool_queries(Q, p->block_q, qbar, qnorm, stream)) != RBS_OK) return st;
 
   const int G = static_cast<int>(Hq / kv_heads);
   int R = 1;
   for (int r = 1; r <= kSelMaxR; ++r)
     if (G % r == 0) R = r;
   SelectArgs sa;
-  sa.qbar = qbar;
-  sa.qnorm = qnorm;
+  sa.Q = static_cast<const __nv_bfloat16*>(Q->data);
+  sa.qb = Q->stride_b;
+  sa.qs = Q->stride_s;
+  sa.qh = Q->stride_h;
   sa.C = centroids;
   sa.rad = radii;
   sa.beta = beta;
@@ -393,11 +398,17 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   const int npad = static_cast<int>((nkb + 31) & ~31ll);
   const size_t smem = (kSelMaxR * 128 + npad + kSelMaxR * npad + kStageJ * kStagePitch) * sizeof(float);
   const dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(Hq / R), static_cast<unsigned>(B));
-  if (nkb <= 64) select_rows_kernel<2><<<grid, kSelThreads, smem, stream>>>(sa);
-  else if (nkb <= 256) select_rows_kernel<8><<<grid, kSelThreads, smem, stream>>>(sa);
-  else if (nkb <= 1024) select_rows_kernel<32><<<grid, kSelThreads, smem, stream>>>(sa);
-  else if (nkb <= 2048) select_rows_kernel<64><<<grid, kSelThreads, smem, stream>>>(sa);
-  else select_rows_kernel<128><<<grid, kSelThreads, smem, stream>>>(sa);
+#define RBS_SEL_LAUNCH(KPL)                                                             \
+  do {                                                                                   \
+    if (p->block_q == 128) select_rows_kernel<KPL, 128><<<grid, kSelThreads, smem, stream>>>(sa); \
+    else select_rows_kernel<KPL, 64><<<grid, kSelThreads, smem, stream>>>(sa);           \
+  } while (0)
+  if (nkb <= 64) RBS_SEL_LAUNCH(2);
+  else if (nkb <= 256) RBS_SEL_LAUNCH(8);
+  else if (nkb <= 1024) RBS_SEL_LAUNCH(32);
+  else if (nkb <= 2048) RBS_SEL_LAUNCH(64);
+  else RBS_SEL_LAUNCH(128);
+#undef RBS_SEL_LAUNCH
   if ((st = check_launch("select_rows_kernel")) != RBS_OK) return st;
 
   scan_counts_kernel<<<1, 1024, 0, stream>>>(sa.counts, static_cast<int>(rows), out->row_ptr, out->capacity);

@@ -8,14 +8,19 @@
 //
 // Kernels:
 //   select_rows_kernel  one CTA per (query block, group of R q heads of one
-//                       KV head, batch).  Scores for all visible blocks are
-//                       computed into shared memory (centroid tiles staged
-//                       through shared memory, 256 blocks x 32 dims at a
-//                       time), then warp w < R finds the exact k-th largest
-//                       score of its row's branch by a 32-step bitwise search
-//                       over order-preserving keys held in registers, breaks
-//                       ties by block index with warp ballots, and emits one
-//                       32-bit mask word per 32 blocks (bit = lane).
+//                       KV head, batch), longest rows (last query blocks)
+//                       first.  The CTA first pools its query block (mean of
+//                       the BQ queries of each of its R heads, streamed from
+//                       HBM with 16-byte loads), then computes the scores of
+//                       all visible blocks into shared memory (centroid tiles
+//                       of 256 blocks x 32 dims staged through shared memory,
+//                       the next tile's loads in flight while one is used),
+//                       then warp w < R finds, for both branches at
+//                       once, the exact k-th largest score of its row by a
+//                       32-step bitwise search over order-preserving keys held
+//                       in registers, breaks ties by block index with warp
+//                       ballots, and emits one 32-bit mask word per 32 blocks
+//                       (bit = lane).
 //   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr.
 //   compact_lists_kernel one warp per row turns mask words into ascending
 //                       block indices and per-entry branch flags.
@@ -26,8 +31,8 @@
 namespace rbs {
 
 struct SelectArgs {
-  const float* qbar;   // [B, Hq, nqb, 128]
-  const float* qnorm;  // [B, Hq, nqb]
+  const __nv_bfloat16* Q;  // [B, Lq, Hq, 128]
+  int64_t qb, qs, qh;      // element strides
   const float* C;      // [B, Hkv, nkb, 128]
   const float* rad;    // [B, Hkv, nkb]
   const float* beta;   // [B, Hkv, nkb]
@@ -41,7 +46,7 @@ struct SelectArgs {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelMaxR = 8;
-constexpr int kStageJ = 256;  // key blocks per staged centroid tile
+constexpr int kStageJ = 256;  // key blocks per staged centroid tile (one per thread)
 constexpr int kStageD = 32;   // dims per staged centroid tile
 constexpr int kStagePitch = kStageD + 1;
 
@@ -57,47 +62,107 @@ __device__ __forceinline__ int keep_count(float rho, int n) {
   return k < 1 ? 1 : (k > n ? n : k);
 }
 
-// Exact top-k of the warp's keys (key 0 = not a candidate; k <= #candidates):
-// returns, per lane, the mask words this lane owns (word t is owned by lane
+// Exact top-k of the warp's keys for two branches at once (key 0 = not a
+// candidate; k <= #candidates).  The k-th largest key T is built bit by bit
+// from the top (the largest T with at least k keys >= T); keys above T are
+// kept, and of the keys equal to T the ones with the lowest block index.
+// Returns, per lane, the mask words this lane owns (word t is owned by lane
 // t % 32) with bit `lane` of word t set iff block 32t + lane is kept.
 template <int KPL>
-__device__ __forceinline__ void warp_topk_words(const uint32_t (&key)[KPL], int k, int lane,
-                                                uint32_t (&own)[(KPL + 31) / 32]) {
-  uint32_t T = 0;
+__device__ __forceinline__ void warp_topk2(const uint32_t (&kc)[KPL], const uint32_t (&kr)[KPL], int k_c, int k_r,
+                                           int lane, uint32_t (&own_c)[(KPL + 31) / 32],
+                                           uint32_t (&own_r)[(KPL + 31) / 32]) {
+  uint32_t Tc = 0, Tr = 0;
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    int cnt = 0;
+    const uint32_t cc = Tc | (1u << bit), cr = Tr | (1u << bit);
+    int nc2[2] = {0, 0}, nr2[2] = {0, 0};  // two partial counts per branch (shorter add chains)
 #pragma unroll
-    for (int t = 0; t < KPL; ++t) cnt += key[t] >= cand ? 1 : 0;
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= k) T = cand;
+    for (int t = 0; t < KPL; ++t) {
+      nc2[t & 1] += kc[t] >= cc ? 1 : 0;
+      nr2[t & 1] += kr[t] >= cr ? 1 : 0;
+    }
+    const int nc = __reduce_add_sync(0xffffffffu, nc2[0] + nc2[1]);
+    const int nr = __reduce_add_sync(0xffffffffu, nr2[0] + nr2[1]);
+    if (nc >= k_c) Tc = cc;
+    if (nr >= k_r) Tr = cr;
   }
-  int gt = 0;
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) gt += key[t] > T ? 1 : 0;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const int need = k - gt;  // ties at T to keep, lowest block index first
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int base = 0;
-#pragma unroll
-  for (int t = 0; t < (KPL + 31) / 32; ++t) own[t] = 0;
+  int gc = 0, gr = 0;
 #pragma unroll
   for (int t = 0; t < KPL; ++t) {
-    const bool tie = key[t] == T;
-    const uint32_t bal = __ballot_sync(0xffffffffu, tie);
-    const int rank = base + __popc(bal & lt_mask);
-    const bool sel = key[t] > T || (tie && rank < need);
-    const uint32_t word = __ballot_sync(0xffffffffu, sel);
-    if (lane == (t & 31)) own[t >> 5] = word;
-    base += __popc(bal);
+    gc += kc[t] > Tc ? 1 : 0;
+    gr += kr[t] > Tr ? 1 : 0;
+  }
+  const int need_c = k_c - __reduce_add_sync(0xffffffffu, gc);  // ties at T to keep, lowest index first
+  const int need_r = k_r - __reduce_add_sync(0xffffffffu, gr);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base_c = 0, base_r = 0;
+#pragma unroll
+  for (int t = 0; t < (KPL + 31) / 32; ++t) own_c[t] = own_r[t] = 0;
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    const bool tie_c = kc[t] == Tc, tie_r = kr[t] == Tr;
+    const uint32_t bc = __ballot_sync(0xffffffffu, tie_c), br = __ballot_sync(0xffffffffu, tie_r);
+    const bool sel_c = kc[t] > Tc || (tie_c && base_c + __popc(bc & lt_mask) < need_c);
+    const bool sel_r = kr[t] > Tr || (tie_r && base_r + __popc(br & lt_mask) < need_r);
+    const uint32_t wc = __ballot_sync(0xffffffffu, sel_c), wr = __ballot_sync(0xffffffffu, sel_r);
+    if (lane == (t & 31)) {
+      own_c[t >> 5] = wc;
+      own_r[t >> 5] = wr;
+    }
+    base_c += __popc(bc);
+    base_r += __popc(br);
   }
 }
 
-template <int KPL>
+// Both branches' top-k of one row (warp-wide) -> mask words and the row's
+// union count.  Keys hold KP slots per lane (block 32t + lane in slot t); the
+// row's mask words cover all nwords <= (KPMAX + 31) / 32 * 32 words.
+template <int KP, int KPMAX>
+__device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float* sc, const float* rb,
+                                                const float* qn, int warp, int lane, int hq0, int b, int i, int gi,
+                                                int n, int npad) {
+  const int hq = hq0 + warp;
+  const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
+  const float qnv = qn[warp];
+  constexpr int NO = (KP + 31) / 32;
+  uint32_t own_c[NO], own_r[NO];
+  {
+    uint32_t kc[KP], kr[KP];
+#pragma unroll
+    for (int t = 0; t < KP; ++t) {
+      const int j = 32 * t + lane;
+      const float sv = j < n ? sc[warp * npad + j] : 0.f;
+      kc[t] = j < n ? order_key(sv) : 0u;
+      kr[t] = j < n ? order_key(fmaf(qnv, rb[j], sv)) : 0u;
+    }
+    warp_topk2<KP>(kc, kr, keep_count(a.rho_c, n), keep_count(a.rho_r, n), lane, own_c, own_r);
+  }
+  int cnt = 0;
+  constexpr int NW = (KPMAX + 31) / 32;  // mask words this lane may own
+#pragma unroll
+  for (int q = 0; q < NW; ++q) {
+    const int t = 32 * q + lane;
+    if (t < a.nwords) {
+      const uint32_t wc = (q < NO && t < KP) ? own_c[q < NO ? q : 0] : 0u;
+      const uint32_t wr = (q < NO && t < KP) ? own_r[q < NO ? q : 0] : 0u;
+      uint32_t f = 0;
+      if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
+      if (a.force_sink && t == 0) f |= 1u;
+      cnt += __popc(wc | wr | f);
+      a.mask_c[row * a.nwords + t] = wc;
+      a.mask_r[row * a.nwords + t] = wr;
+    }
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) a.counts[row] = cnt;
+}
+
+template <int KPL, int BQ>
 __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
-  const int i = blockIdx.x, hblk = blockIdx.y, b = blockIdx.z;
+  const int i = a.nqb - 1 - static_cast<int>(blockIdx.x);  // longest rows first
+  const int hblk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = a.R;
   const int G = a.Hq / a.Hkv;
@@ -107,62 +172,121 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
   const int n = a.causal ? min(a.nkb, gi + 1) : a.nkb;
   const int npad = (a.nkb + 31) & ~31;
 
-  float* qs = sm;                         // [R][128]
+  float* qs = sm;                         // [R][128] pooled queries
   float* rb = qs + kSelMaxR * 128;        // [npad]  r_j * beta_j
   float* sc = rb + npad;                  // [R][npad] centroid-branch scores
-  float* cs = sc + kSelMaxR * npad;       // [kStageJ][kStagePitch]
+  float* cs = sc + kSelMaxR * npad;       // [kStageJ][kStagePitch]; first holds pooling partial sums
   __shared__ float qn[kSelMaxR];
 
   const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
-  for (int idx = tid; idx < R * 128; idx += kSelThreads) {
-    const int h = idx >> 7, d = idx & 127;
-    qs[idx] = a.qbar[(static_cast<int64_t>(b * a.Hq + hq0 + h) * a.nqb + i) * 128 + d];
-  }
-  if (tid < R) qn[tid] = a.qnorm[static_cast<int64_t>(b * a.Hq + hq0 + tid) * a.nqb + i];
   for (int j = tid; j < n; j += kSelThreads) rb[j] = a.rad[kv_off + j] * a.beta[kv_off + j];
 
-  // ---- scores s_c for j < n
-  const float* Cb = a.C + kv_off * 128;
-  for (int j0 = 0; j0 < n; j0 += kStageJ) {
-    const int jn = min(kStageJ, n - j0);
-    float acc[kSelMaxR];
+  // ---- pooled query of each of the R heads: mean of the BQ queries of block i.
+  // Thread (rg, col): 16-byte chunk col % 16 of head col / 16, rows rg, rg + RG, ...
+  {
+    const int cols = R * 16;
+    const int RG = kSelThreads / cols;
+    const int col = tid % cols, rg = tid / cols;
+    float acc[8];
 #pragma unroll
-    for (int h = 0; h < kSelMaxR; ++h) acc[h] = 0.f;
-    for (int d0 = 0; d0 < 128; d0 += kStageD) {
-      __syncthreads();
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    if (rg < RG) {
+      const char* base = reinterpret_cast<const char*>(a.Q + b * a.qb + static_cast<int64_t>(i) * BQ * a.qs +
+                                                       (hq0 + col / 16) * a.qh) + (col % 16) * 16;
+      for (int r0 = rg; r0 < BQ; r0 += 8 * RG) {
+        uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < (kStageJ * kStageD / 4) / kSelThreads; ++u) {
-        const int idx = tid + kSelThreads * u;
-        const int jl = idx >> 3, d4 = idx & 7;
-        if (jl < jn) {
-          const float4 v = *reinterpret_cast<const float4*>(Cb + static_cast<int64_t>(j0 + jl) * 128 + d0 + 4 * d4);
-          float* dst = cs + jl * kStagePitch + 4 * d4;
-          dst[0] = v.x;
-          dst[1] = v.y;
-          dst[2] = v.z;
-          dst[3] = v.w;
+        for (int u = 0; u < 8; ++u) {
+          const int row = r0 + u * RG;
+          v[u] = row < BQ ? ldg_stream(base + static_cast<int64_t>(row) * a.qs * 2) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] += bf16lo(w[q]);
+            acc[2 * q + 1] += bf16hi(w[q]);
+          }
         }
       }
-      __syncthreads();
-      if (tid < jn) {
-        const float* crow = cs + tid * kStagePitch;
-#pragma unroll 4
-        for (int d = 0; d < kStageD; d += 4) {
-          const float c0 = crow[d], c1 = crow[d + 1], c2 = crow[d + 2], c3 = crow[d + 3];
 #pragma unroll
-          for (int h = 0; h < kSelMaxR; ++h) {
-            if (h < R) {
-              const float4 q = *reinterpret_cast<const float4*>(qs + h * 128 + d0 + d);
-              acc[h] = fmaf(q.x, c0, acc[h]);
-              acc[h] = fmaf(q.y, c1, acc[h]);
-              acc[h] = fmaf(q.z, c2, acc[h]);
-              acc[h] = fmaf(q.w, c3, acc[h]);
-            }
+      for (int e = 0; e < 8; ++e) cs[rg * (R * 128) + col * 8 + e] = acc[e];
+    }
+    __syncthreads();
+    for (int o = tid; o < R * 128; o += kSelThreads) {
+      float sum = 0.f;
+      for (int g2 = 0; g2 < RG; ++g2) sum += cs[g2 * (R * 128) + o];
+      qs[o] = sum * (1.0f / BQ);
+    }
+    __syncthreads();
+    if (warp < R) {
+      float s2 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s2 = fmaf(qs[warp * 128 + lane + 32 * e], qs[warp * 128 + lane + 32 * e], s2);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      if (lane == 0) qn[warp] = sqrtf(s2);
+    }
+  }
+
+  // ---- scores s_c for j < n: thread t owns block j0 + t of each 256-block tile.
+  // Stage (j-tile, 32-dim slice) k's global loads are issued while stage k-1
+  // is being used.
+  const float* Cb = a.C + kv_off * 128;
+  const int nstages = ((n + kStageJ - 1) / kStageJ) * (128 / kStageD);
+  constexpr int kLoads = (kStageJ * kStageD / 4) / kSelThreads;  // float4 per thread per stage
+  float4 pre[kLoads];
+  auto load_stage = [&](int st) {
+    const int j0 = (st / (128 / kStageD)) * kStageJ, d0 = (st % (128 / kStageD)) * kStageD;
+    const int jn = min(kStageJ, n - j0);
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+      const int idx = tid + kSelThreads * u;
+      const int jl = idx >> 3, d4 = idx & 7;
+      pre[u] = jl < jn ? *reinterpret_cast<const float4*>(Cb + static_cast<int64_t>(j0 + jl) * 128 + d0 + 4 * d4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  float acc[kSelMaxR];
+  load_stage(0);
+  for (int st = 0; st < nstages; ++st) {
+    const int j0 = (st / (128 / kStageD)) * kStageJ, d0 = (st % (128 / kStageD)) * kStageD;
+    const int jn = min(kStageJ, n - j0);
+    if (d0 == 0) {
+#pragma unroll
+      for (int h = 0; h < kSelMaxR; ++h) acc[h] = 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+      const int idx = tid + kSelThreads * u;
+      float* dst = cs + (idx >> 3) * kStagePitch + 4 * (idx & 7);
+      dst[0] = pre[u].x;
+      dst[1] = pre[u].y;
+      dst[2] = pre[u].z;
+      dst[3] = pre[u].w;
+    }
+    __syncthreads();
+    if (st + 1 < nstages) load_stage(st + 1);
+    if (tid < jn) {
+      const float* crow = cs + tid * kStagePitch;
+#pragma unroll 4
+      for (int d = 0; d < kStageD; d += 4) {
+        const float c0 = crow[d], c1 = crow[d + 1], c2 = crow[d + 2], c3 = crow[d + 3];
+#pragma unroll
+        for (int h = 0; h < kSelMaxR; ++h) {
+          if (h < R) {
+            const float4 q = *reinterpret_cast<const float4*>(qs + h * 128 + d0 + d);
+            acc[h] = fmaf(q.x, c0, acc[h]);
+            acc[h] = fmaf(q.y, c1, acc[h]);
+            acc[h] = fmaf(q.z, c2, acc[h]);
+            acc[h] = fmaf(q.w, c3, acc[h]);
           }
         }
       }
     }
-    if (tid < jn) {
+    if (d0 + kStageD == 128 && tid < jn) {
 #pragma unroll
       for (int h = 0; h < kSelMaxR; ++h)
         if (h < R) sc[h * npad + j0 + tid] = acc[h];
@@ -170,58 +294,30 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
   }
   __syncthreads();
 
-  // ---- per-branch top-k, one warp per row
+  // ---- per-branch top-k (both branches together), one warp per row, with
+  // as few key slots per lane as this row needs
   if (warp < R) {
-    const int hq = hq0 + warp;
-    const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
-    const float qnv = qn[warp];
-    constexpr int NO = (KPL + 31) / 32;
-    uint32_t own_c[NO], own_r[NO];
-    {
-      uint32_t key[KPL];
-#pragma unroll
-      for (int t = 0; t < KPL; ++t) {
-        const int j = 32 * t + lane;
-        key[t] = j < n ? order_key(sc[warp * npad + j]) : 0u;
-      }
-      warp_topk_words<KPL>(key, keep_count(a.rho_c, n), lane, own_c);
-    }
-    {
-      uint32_t key[KPL];
-#pragma unroll
-      for (int t = 0; t < KPL; ++t) {
-        const int j = 32 * t + lane;
-        key[t] = j < n ? order_key(fmaf(qnv, rb[j], sc[warp * npad + j])) : 0u;
-      }
-      warp_topk_words<KPL>(key, keep_count(a.rho_r, n), lane, own_r);
-    }
-    int cnt = 0;
-#pragma unroll
-    for (int q = 0; q < NO; ++q) {
-      const int t = 32 * q + lane;
-      if (t < a.nwords) {
-        uint32_t f = 0;
-        if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
-        if (a.force_sink && t == 0) f |= 1u;
-        cnt += __popc(own_c[q] | own_r[q] | f);
-        a.mask_c[row * a.nwords + t] = own_c[q];
-        a.mask_r[row * a.nwords + t] = own_r[q];
-      }
-    }
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (lane == 0) a.counts[row] = cnt;
+    if (KPL > 8 && n <= 64) select_topk_row<2, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad);
+    else if (KPL > 8 && n <= 256) select_topk_row<8, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad);
+    else select_topk_row<KPL, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad);
   }
 }
 
-// Exclusive scan of per-row counts into row_ptr (one CTA of 1024 threads).
+// Exclusive scan of per-row counts into row_ptr (one CTA of 1024 threads;
+// each thread owns a contiguous run of rows, read and written 4 at a time).
 __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict__ counts, int rows,
                                                            int* __restrict__ row_ptr, int64_t capacity) {
   __shared__ long long wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (rows + 1023) / 1024;
+  const int per = ((rows + 1023) / 1024 + 3) & ~3;  // multiple of 4
   const int s0 = min(rows, tid * per), s1 = min(rows, s0 + per);
   long long local = 0;
-  for (int r = s0; r < s1; ++r) local += counts[r];
+  int r = s0;
+  for (; r + 4 <= s1; r += 4) {
+    const int4 c4 = *reinterpret_cast<const int4*>(counts + r);
+    local += static_cast<long long>(c4.x) + c4.y + c4.z + c4.w;
+  }
+  for (; r < s1; ++r) local += counts[r];
   long long incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -242,7 +338,18 @@ __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict
   }
   __syncthreads();
   long long run = wsum[warp] + incl - local;
-  for (int r = s0; r < s1; ++r) {
+  r = s0;
+  for (; r + 4 <= s1; r += 4) {
+    const int4 c4 = *reinterpret_cast<const int4*>(counts + r);
+    int4 o;
+    o.x = static_cast<int>(run);
+    o.y = static_cast<int>(run += c4.x);
+    o.z = static_cast<int>(run += c4.y);
+    o.w = static_cast<int>(run += c4.z);
+    run += c4.w;
+    *reinterpret_cast<int4*>(row_ptr + r) = o;
+  }
+  for (; r < s1; ++r) {
     row_ptr[r] = static_cast<int>(run);
     run += counts[r];
   }
