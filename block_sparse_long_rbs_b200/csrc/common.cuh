@@ -93,15 +93,17 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // Time limit for any pipeline wait (normal waits last microseconds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Wait for the phase with the given parity to complete, spinning on the
-// non-suspending probe.  Returns false, with *abort set, if the wait ran past
-// the time limit or another role of the CTA already aborted.
+// Wait for the phase with the given parity to complete.  try_wait suspends
+// the waiting thread inside the hardware until the phase completes (or a short
+// system limit passes), so waiting warps do not take issue slots from the
+// warps sharing their scheduler.  Returns false, with *abort set, if the wait
+// ran past the time limit or another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_test_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort = 1;

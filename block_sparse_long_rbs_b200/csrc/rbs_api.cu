@@ -20,15 +20,7 @@
 
 using namespace rbs;
 
-// Softmax warpgroups of the 128-block attention kernel (2 or 4).
-#ifndef RBS_ATTN_WG
-#define RBS_ATTN_WG 2
-#endif
-
 namespace {
-
-constexpr int kWg128 = RBS_ATTN_WG;
-constexpr int kWg64 = 2;
 
 thread_local char g_last_error[512] = "";
 
@@ -75,10 +67,10 @@ rbs_status device_info(DeviceInfo** out) {
   }
   if (!d.attrs_set) {
     cudaError_t e = cudaSuccess;
-    e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<128, 128, kWg128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     AttnSmem<128, kWg128>::kAlloc);
-    e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<64, 64, kWg64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     AttnSmem<64, kWg64>::kAlloc);
+    e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     AttnSmem<128>::kAlloc);
+    e = e ? e : cudaFuncSetAttribute(bsa_prefill_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     AttnSmem<64>::kAlloc);
 #define RBS_SEL_ATTR(KPL)                                                                                  \
   e = e ? e : cudaFuncSetAttribute(select_rows_kernel<KPL, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                                    200 * 1024);                                                              \
@@ -594,15 +586,12 @@ rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const
   if ((st = device_info(&di)) != RBS_OK) return st;
 
   AttnArgs a;
-  int sik = 0, siv = 0;
+  int siq = 0, sik = 0, siv = 0;
+  if ((st = make_tensor_map(Q, block_q, &a.tmQ, &siq)) != RBS_OK) return st;
   if ((st = make_tensor_map(K, block_k, &a.tmK, &sik)) != RBS_OK) return st;
   if ((st = make_tensor_map(V, block_k, &a.tmV, &siv)) != RBS_OK) return st;
-  RBS_REQUIRE(sik == 0 && siv == 0, RBS_ERR_UNSUPPORTED,
-              "K/V must have the head stride no larger than the token stride ([B, L, H, 128] order)");
-  a.Q = static_cast<const __nv_bfloat16*>(Q->data);
-  a.qb = Q->stride_b;
-  a.qs = Q->stride_s;
-  a.qh = Q->stride_h;
+  RBS_REQUIRE(siq == 0 && sik == 0 && siv == 0, RBS_ERR_UNSUPPORTED,
+              "Q/K/V must have the head stride no larger than the token stride ([B, L, H, 128] order)");
   a.row_ptr = lists->row_ptr;
   a.col_idx = lists->col_idx;
   a.capacity = lists->capacity;
@@ -624,9 +613,9 @@ rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const
   a.scale_log2 = scale * 1.4426950408889634f;
   const int grid = static_cast<int>(std::min<int64_t>(rows, di->sms));
   if (block_q == 128)
-    bsa_prefill_kernel<128, 128, kWg128><<<grid, attn_threads(kWg128), AttnSmem<128, kWg128>::kAlloc, stream>>>(a);
+    bsa_prefill_kernel<128, 128><<<grid, kAttnThreads, AttnSmem<128>::kAlloc, stream>>>(a);
   else
-    bsa_prefill_kernel<64, 64, kWg64><<<grid, attn_threads(kWg64), AttnSmem<64, kWg64>::kAlloc, stream>>>(a);
+    bsa_prefill_kernel<64, 64><<<grid, kAttnThreads, AttnSmem<64>::kAlloc, stream>>>(a);
   return check_launch("bsa_prefill_kernel");
 }
 

@@ -244,7 +244,9 @@ RBS_API rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t n
  * over the key tokens s of the row's listed blocks, with s <= t + q_offset
  * when causal; KV head = h / (Hq / Hkv).  bf16 tensor-core products, fp32
  * accumulation and softmax.
- *   Q         [B, Lq, Hq, 128] bf16; K, V [B, Lk, Hkv, 128] bf16
+ *   Q         [B, Lq, Hq, 128] bf16; K, V [B, Lk, Hkv, 128] bf16; each with
+ *             stride_h <= stride_s (heads inside tokens, as in a packed QKV
+ *             projection; else RBS_ERR_UNSUPPORTED)
  *   lists     num_rows = B * Hq * Lq / block_q; indices in [0, Lk / block_k)
  *   block_q == block_k, 64 or 128; q_offset a multiple of block_k
  *   softmax_scale  <= 0 selects 1/sqrt(128)
