@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
     }
   } else if (warp == 10) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp runs the loop; one elected lane issues each tcgen05 instruction
       constexpr uint32_t idS = idesc_bf16_f32(128, BK, 0, 0);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
       // Descriptors are built once; a buffer or k-step only adds its
@@ -272,39 +272,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       bool ok = true;
       for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
         const int qb = item & 1, n = x.n;
-        if (!mbar_wait(bar(kBarQFull + qb), (item >> 1) & 1, abort_flag)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarQFull + qb), (item >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint64_t qd = qdesc0 + qb * kQUnits;
         auto issue_s = [&](int t) -> bool {
           const int st = t & 1, s = kit % kNS;
-          if (!mbar_wait(bar(kBarKFull + s), (kit / kNS) & 1, abort_flag)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarKFull + s), (kit / kNS) & 1, abort_flag))) return false;
           tc_fence_after();
           const uint64_t kd = kdesc0 + s * kStageUnits;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 2, offk = (kk >> 2) * kKHalf + (kk & 3) * 2;
-            umma_ss(tmem + L::col_s(st), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
+            umma_ss_warp(tmem + L::col_s(st), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
           }
-          umma_commit(bar(kBarSFull + st));
-          umma_commit(bar(kBarKEmpty + s));
-          if (t == n - 1) umma_commit(bar(kBarQEmpty + qb));
+          umma_commit_warp(bar(kBarSFull + st));
+          umma_commit_warp(bar(kBarKEmpty + s));
+          if (t == n - 1) umma_commit_warp(bar(kBarQEmpty + qb));
           ++kit;
           return true;
         };
         auto issue_pv = [&](int t) -> bool {
           const int st = t & 1, s = vit % kNS;
           const bool first = t < 2;  // first tile of this stream in the row
-          if (!mbar_wait(bar(kBarPFull + st), nP[st] & 1, abort_flag)) return false;
-          if (!mbar_wait(bar(kBarVFull + s), (vit / kNS) & 1, abort_flag)) return false;
-          if (first && item > 0 && !mbar_wait(bar(kBarOEmpty + st), (item - 1) & 1, abort_flag)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPFull + st), nP[st] & 1, abort_flag))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarVFull + s), (vit / kNS) & 1, abort_flag))) return false;
+          if (first && item > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(kBarOEmpty + st), (item - 1) & 1, abort_flag))) return false;
           tc_fence_after();
           const uint64_t vd = vdesc0 + s * kStageUnits;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma_ts(tmem + L::col_o(st), tmem + L::col_s(st) + kk * 8, vd + kk * (2048 >> 4), idPV,
+            umma_ts_warp(tmem + L::col_o(st), tmem + L::col_s(st) + kk * 8, vd + kk * (2048 >> 4), idPV,
                     (first && kk == 0) ? 0u : 1u);
-          umma_commit(bar(kBarVEmpty + s));
-          if (t >= n - 2) umma_commit(bar(kBarOFull + st));  // the stream's last tile of this row
+          umma_commit_warp(bar(kBarVEmpty + s));
+          if (t >= n - 2) umma_commit_warp(bar(kBarOFull + st));  // the stream's last tile of this row
           ++vit;
           ++nP[st];
           return true;
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         ++item;
       }
       // drain all outstanding tensor-core work before TMEM is freed
-      umma_commit(bar(kBarDrain));
+      umma_commit_warp(bar(kBarDrain));
       mbar_drain(bar(kBarDrain), 0);
     }
   } else {
