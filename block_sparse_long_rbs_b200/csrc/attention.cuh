@@ -7,37 +7,41 @@
 // order.  Persistent CTAs take non-empty work items round-robin in an order
 // that starts with the last query blocks (the longest causal rows).
 //
-// Two softmax streams.  The row's key tiles alternate between stream A
-// (tiles 0, 2, 4, ...) and stream B (tiles 1, 3, 5, ...).  Each stream keeps
-// its own S tile (P is written back over it), its own O accumulator and its
-// own running max and sum, and the two partial results are merged exactly in
-// the epilogue:  O = (O_A 2^(m_A-m) + O_B 2^(m_B-m)) / (l_A 2^(m_A-m) + l_B 2^(m_B-m)).
-// While one stream's softmax runs, the tensor core works on the other's
-// tiles, so neither waits for the other.
+// One softmax pipeline with three S buffers in TMEM.  While the softmax
+// warps work on tile t, the tensor core computes S for tiles t+1 and t+2 and
+// accumulates P_{t-1} V_{t-1}, so the tensor core and the softmax overlap
+// without either waiting on the other's latency.
 //
-// Roles (352 threads):
-//   warps 0-3  softmax of stream A, warps 4-7 softmax of stream B: thread r
-//              owns query row r (TMEM lane r) of its stream's tiles.  Pass 1
-//              reads the S row from TMEM for the row maximum; the running max
-//              is lazily updated (O rescaled in TMEM only when it grows by
-//              more than 2^8; the final normalisation uses the same max, so
-//              the result is exact); pass 2 re-reads S and writes
-//              P = exp2(S*c - m) as packed bf16 pairs over the S columns
-//              (3 of every 8 element pairs on the FMA pipe, see exp2_fma2,
-//              the rest on the SFU).  In the epilogue warpgroup g merges and
-//              writes dims [64g, 64g+64) of every output row.
+// Roles (384 threads):
+//   warps 0-7  softmax: warp w owns query rows 32(w%4) .. 32(w%4)+31 (its
+//              TMEM lane quarter) and the S columns of half w/4 of every key
+//              tile.  Pass 1 reads its half row of S into registers and takes
+//              the half-row maximum; the two warps of a lane quarter exchange
+//              their maxima through shared memory (an mbarrier per quarter).
+//              The running max is lazily updated (O rescaled in TMEM only when
+//              it grows by more than 2^8; the final normalisation uses the same
+//              max, so the result is exact).  Pass 2 forms
+//              P = exp2(S*c - m) from the registers (3 of every 8 element pairs
+//              on the FMA pipe, see exp2_fma2, the rest on the SFU) and writes
+//              it as packed bf16 pairs over the first quarter of its own S
+//              columns.  In the epilogue the two warps of a quarter add their
+//              row sums and each writes 64 of the 128 output dims.
 //   warp 8     Q and K producer, warp 9 V producer (one thread each): TMA
 //              loads of the Q tile (double-buffered) and of the K_j / V_j
 //              tiles gathered by block index (4-D tensor maps over
 //              [B, L, H, 128], 128B swizzle, no multicast) into 2-deep K and
 //              V rings; list indices fetched one tile ahead.
-//   warp 10    TMEM allocator and MMA issuer (one thread):
-//                S_t  = Q K_t^T  into stream (t&1)'s S   A = Q (smem), B = K_t (smem)
-//                O   += P_t V_t  into stream (t&1)'s O   A = P (TMEM), B = V_t (MN-major smem)
-//              issue order S_0, S_1, PV_0, S_2, PV_1, S_3, ...; S_{t+2} is
-//              issued after PV_t, which reads P_t from the same columns (the
-//              tensor core executes one thread's MMAs in order).
-// TMEM columns: S_A [0, BK), O_A [128, 256), S_B [256, 256+BK), O_B [384, 512).
+//   warp 10    TMEM allocator and S issuer, warp 11 PV issuer (each warp runs
+//              its loop; one elected lane issues):
+//                S_g  = Q K_g^T  into S buffer g%3    A = Q (smem), B = K_g (smem)
+//                O   += P_g V_g                        A = P (TMEM), B = V_g (MN-major smem)
+//              over the CTA's tiles g = 0, 1, 2, ... of all its rows in
+//              sequence.  S_{g+3} overwrites P_g, so the S issuer waits for
+//              PV_g to complete; otherwise the two issuers run independently,
+//              so each one's waits and commits overlap the other's MMAs.
+//              The K and V producers refill a ring stage when the S (PV)
+//              barrier of the tile that used it completes.
+// TMEM columns: S buffers [0, BK), [128, 128+BK), [256, 256+BK); O [384, 512).
 //
 // Every mbarrier wait is bounded; on a timeout all roles unwind, in-flight
 // TMA loads and MMAs are drained (bounded), TMEM is freed, and the device
@@ -62,7 +66,7 @@ struct AttnArgs {
   float scale_log2;
 };
 
-constexpr int kAttnThreads = 352;
+constexpr int kAttnThreads = 384;
 constexpr int kNS = 2;  // K and V ring depth
 
 // Software base-2 exponential of two values at once, on the FMA pipe:
@@ -97,14 +101,15 @@ struct AttnSmem {
   static constexpr int kQ = 0;                   // two Q buffers
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kNS * kKVBytes;
-  static constexpr int kX = kV + kNS * kKVBytes;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
-  static constexpr int kBar = kX + 2 * 2 * 2 * 128 * 4;
+  static constexpr int kX = kV + kNS * kKVBytes;  // float [2 exchange parity][2 halves][128 rows]
+  static constexpr int kBar = kX + 2 * 2 * 128 * 4;
   static constexpr int kBarBytes = 256;
   static constexpr int kTotal = kBar + kBarBytes;
   static constexpr int kAlloc = kTotal + 1024;  // slack to align the base to 1024
   static constexpr uint32_t kTmemCols = 512;
-  __host__ __device__ static constexpr uint32_t col_s(int st) { return st * 256; }
-  __host__ __device__ static constexpr uint32_t col_o(int st) { return st * 256 + 128; }
+  static constexpr int kSBufs = 3;
+  __host__ __device__ static constexpr uint32_t col_s(int buf) { return buf * 128; }
+  static constexpr uint32_t kColO = 384;
 };
 
 // barrier slots (8 bytes each)
@@ -112,16 +117,15 @@ enum : int {
   kBarQFull = 0,                 // + buffer (2)
   kBarQEmpty = kBarQFull + 2,    // + buffer (2)
   kBarKFull = kBarQEmpty + 2,    // + stage
-  kBarKEmpty = kBarKFull + kNS,  // + stage
-  kBarVFull = kBarKEmpty + kNS,  // + stage
-  kBarVEmpty = kBarVFull + kNS,  // + stage
-  kBarSFull = kBarVEmpty + kNS,  // + stream
-  kBarPFull = kBarSFull + 2,     // + stream
-  kBarOFull = kBarPFull + 2,     // + stream
-  kBarOEmpty = kBarOFull + 2,    // + stream
-  kBarX = kBarOEmpty + 2,
-  kBarDrain = kBarX + 1,
-  kNumBars = kBarDrain + 1
+  kBarVFull = kBarKFull + kNS,   // + stage
+  kBarSFull = kBarVFull + kNS,   // + S buffer (3)
+  kBarPFull = kBarSFull + 3,     // + S buffer (3)
+  kBarPVDone = kBarPFull + 3,    // + tile index mod 4: one phase per fourth PV
+  kBarOFull = kBarPVDone + 4,    // one phase per row
+  kBarOEmpty = kBarOFull + 1,    // one phase per row
+  kBarX = kBarOEmpty + 1,        // + lane quarter (4): the two warps' exchanges
+  kBarDrain = kBarX + 4,         // + issuer (2)
+  kNumBars = kBarDrain + 2
 };
 static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
 
@@ -161,7 +165,7 @@ __device__ __forceinline__ Work next_work(const AttnArgs& a, int w) {
 template <int BQ, int BK>
 __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __grid_constant__ AttnArgs a) {
   using L = AttnSmem<BK>;
-  constexpr int kStreamWarps = 4;  // softmax warps per stream; their barriers count one arrival per warp
+  constexpr int kSoftmaxWarps = 8;  // barriers the softmax warps complete count one arrival per warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -180,19 +184,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarQFull + s), 1);
       mbar_init(bar(kBarQEmpty + s), 1);
-      mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarPFull + s), kStreamWarps);
-      mbar_init(bar(kBarOFull + s), 1);
-      mbar_init(bar(kBarOEmpty + s), 2 * kStreamWarps);
     }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarVEmpty + s), 1);
     }
-    mbar_init(bar(kBarX), 2 * kStreamWarps);
-    mbar_init(bar(kBarDrain), 1);
+    for (int s = 0; s < L::kSBufs; ++s) {
+      mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarPFull + s), kSoftmaxWarps);
+    }
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kBarPVDone + s), 1);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOEmpty), kSoftmaxWarps);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(kBarX + q), 2);
+    mbar_init(bar(kBarDrain + 0), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,7 +224,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       const CUtensorMap* map = isK ? &a.tmK : &a.tmV;
       const uint32_t ring = isK ? sK : sV;
       const int full0 = isK ? kBarKFull : kBarVFull;
-      const int empty0 = isK ? kBarKEmpty : kBarVEmpty;
       tma_prefetch_desc(map);
       if (isK) tma_prefetch_desc(&a.tmQ);
       uint32_t nf = 0, nq = 0;  // ring fills, Q fills issued
@@ -239,7 +244,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           if (t + 1 < x.n) j_next = __ldg(a.col_idx + x.beg + t + 1);
           if (j < 0 || j >= a.nkb) j = 0;
           const int s = nf % kNS;
-          if (nf >= kNS && !mbar_wait(bar(empty0 + s), ((nf / kNS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          // the stage's previous tile, nf - kNS, must be consumed: its S (for
+          // K) or PV (for V) is complete.  Neither barrier can move past that
+          // phase before this load lands, so the parity is unambiguous.
+          if (nf >= kNS) {
+            const uint32_t prev = nf - kNS;
+            const bool done = isK ? mbar_wait(bar(kBarSFull + prev % 3), (prev / 3) & 1, abort_flag)
+                                  : mbar_wait(bar(kBarPVDone + (prev & 3)), (prev >> 2) & 1, abort_flag);
+            if (!done) { ok = false; break; }
+          }
           mbar_arrive_expect_tx(bar(full0 + s), BK * 256);
           tma_load_4d(ring + s * L::kKVBytes, map, bar(full0 + s), 0, kvh, j * BK, x.b);
           tma_load_4d(ring + s * L::kKVBytes + BK * 128, map, bar(full0 + s), 64, kvh, j * BK, x.b);
@@ -255,9 +268,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         for (uint32_t s = 0; s < 2; ++s)
           if (s < nq) mbar_drain(bar(kBarQFull + s), ((nq - s + 1) / 2 - 1) & 1);
     }
-  } else if (warp == 10) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 10 || warp == 11) {
+    // ------------------------------------------------------------ S issuer / PV issuer
     {  // the whole warp runs the loop; one elected lane issues each tcgen05 instruction
+      const bool isS = warp == 10;
       constexpr uint32_t idS = idesc_bf16_f32(128, BK, 0, 0);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
       // Descriptors are built once; a buffer or k-step only adds its
@@ -268,64 +282,78 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       const uint64_t vdesc0 = smem_desc(sV, BK * 128, 1024, kLayoutSW128);
       constexpr uint32_t kQUnits = L::kQBytes >> 4, kStageUnits = L::kKVBytes >> 4;
       constexpr uint32_t kQHalf = (128 * 128) >> 4, kKHalf = (BK * 128) >> 4;
-      uint32_t kit = 0, vit = 0, item = 0, nP[2] = {0, 0};
+      constexpr int kStepsHalf = BK / 32;  // K16 steps per half of a key tile
+      auto wait = [&](int k, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar(k), parity, abort_flag)); };
+      // Each issuer walks the CTA's (row, tile) sequence: g counts tiles over
+      // all rows, it rows.
+      Work x = next_work(a, blockIdx.x);
+      int t = 0;
+      uint32_t g = 0, it = 0;
       bool ok = true;
-      for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
-        const int qb = item & 1, n = x.n;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarQFull + qb), (item >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint64_t qd = qdesc0 + qb * kQUnits;
-        auto issue_s = [&](int t) -> bool {
-          const int st = t & 1, s = kit % kNS;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarKFull + s), (kit / kNS) & 1, abort_flag))) return false;
+      for (; ok && x.w < a.num_rows; ++g) {
+        const int b = g % L::kSBufs, s = g % kNS;
+        if (isS) {
+          const int qb = it & 1;
+          if (t == 0 && !wait(kBarQFull + qb, (it >> 1) & 1)) break;
+          if (!wait(kBarKFull + s, (g / kNS) & 1)) break;
+          // S_g overwrites P_{g-3}: PV_{g-3} must be complete.  The next phase
+          // of that barrier is PV_{g+1}, which needs S_{g+1}: not yet issued.
+          if (g >= L::kSBufs && !wait(kBarPVDone + ((g - 3) & 3), ((g - 3) >> 2) & 1)) break;
           tc_fence_after();
-          const uint64_t kd = kdesc0 + s * kStageUnits;
+          const uint64_t qd = qdesc0 + qb * kQUnits, kd = kdesc0 + s * kStageUnits;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 2, offk = (kk >> 2) * kKHalf + (kk & 3) * 2;
-            umma_ss_warp(tmem + L::col_s(st), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
+            umma_ss_warp(tmem + L::col_s(b), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
           }
-          umma_commit_warp(bar(kBarSFull + st));
-          umma_commit_warp(bar(kBarKEmpty + s));
-          if (t == n - 1) umma_commit_warp(bar(kBarQEmpty + qb));
-          ++kit;
-          return true;
-        };
-        auto issue_pv = [&](int t) -> bool {
-          const int st = t & 1, s = vit % kNS;
-          const bool first = t < 2;  // first tile of this stream in the row
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPFull + st), nP[st] & 1, abort_flag))) return false;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarVFull + s), (vit / kNS) & 1, abort_flag))) return false;
-          if (first && item > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(kBarOEmpty + st), (item - 1) & 1, abort_flag))) return false;
+          umma_commit_warp(bar(kBarSFull + b));
+          if (t == x.n - 1) umma_commit_warp(bar(kBarQEmpty + qb));
+        } else {
+          if (!wait(kBarPFull + b, (g / L::kSBufs) & 1)) break;
+          if (!wait(kBarVFull + s, (g / kNS) & 1)) break;
+          if (t == 0 && it > 0 && !wait(kBarOEmpty, (it - 1) & 1)) break;
           tc_fence_after();
           const uint64_t vd = vdesc0 + s * kStageUnits;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_ts_warp(tmem + L::col_o(st), tmem + L::col_s(st) + kk * 8, vd + kk * (2048 >> 4), idPV,
-                    (first && kk == 0) ? 0u : 1u);
-          umma_commit_warp(bar(kBarVEmpty + s));
-          if (t >= n - 2) umma_commit_warp(bar(kBarOFull + st));  // the stream's last tile of this row
-          ++vit;
-          ++nP[st];
-          return true;
-        };
-        ok = issue_s(0) && (n < 2 || issue_s(1));
-        for (int t = 0; t < n && ok; ++t) ok = issue_pv(t) && (t + 2 >= n || issue_s(t + 2));
-        ++item;
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // P of key half kk / kStepsHalf sits at the start of that half's S columns
+            const uint32_t pcol = L::col_s(b) + (kk / kStepsHalf) * (BK / 2) + (kk % kStepsHalf) * 8;
+            umma_ts_warp(tmem + L::kColO, tmem + pcol, vd + kk * (2048 >> 4), idPV, (t == 0 && kk == 0) ? 0u : 1u);
+          }
+          umma_commit_warp(bar(kBarPVDone + (g & 3)));
+          if (t == x.n - 1) umma_commit_warp(bar(kBarOFull));
+        }
+        if (++t == x.n) {
+          x = next_work(a, x.w + gridDim.x);
+          t = 0;
+          ++it;
+        }
       }
-      // drain all outstanding tensor-core work before TMEM is freed
-      umma_commit_warp(bar(kBarDrain));
-      mbar_drain(bar(kBarDrain), 0);
+      // drain this issuer's outstanding tensor-core work before TMEM is freed
+      umma_commit_warp(bar(kBarDrain + (isS ? 0 : 1)));
+      mbar_drain(bar(kBarDrain + (isS ? 0 : 1)), 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax streams (warps 0-7)
-    const int st = warp >> 2;  // stream: tiles st, st + 2, ...; epilogue dims [64 st, 64 st + 64)
-    const int r = tid & 127;   // query row within the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    constexpr int kHalf = BK / 2;  // S columns per warp
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c = a.scale_log2;
     auto warp_arrive = [&](int k) {
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(k));
+    };
+    // exchange one value per row with the other warp of this lane quarter
+    uint32_t nx = 0;
+    auto exchange = [&](float v, float& other) -> bool {
+      float* xb = xch + (nx & 1) * 256;  // [2 halves][128 rows]
+      xb[hf * 128 + r] = v;
+      warp_arrive(kBarX + quarter);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarX + quarter), nx & 1, abort_flag))) return false;
+      other = xb[(hf ^ 1) * 128 + r];
+      ++nx;
+      return true;
     };
 
     // rows with no (or a corrupt) list: zeros and LSE = -inf, no pipeline
@@ -354,57 +382,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       }
     }
 
-    uint32_t nS = 0, nO[2] = {0, 0}, item = 0;
+    uint32_t g = 0, item = 0;  // tiles and rows processed by this CTA
     bool ok = true;
     for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
       const int n = x.n;
       const int gi = x.i + a.q_block_off;
-      float m_used = -INFINITY;  // this stream's running max, in log2 units (score * c)
-      float2 l2 = make_float2(0.f, 0.f);
-      int j_next = st < n ? __ldg(a.col_idx + x.beg + st) : 0;
-      for (int t = st; t < n; t += 2) {
+      float m_used = -INFINITY;  // running max, in log2 units (score * c)
+      float2 l2 = make_float2(0.f, 0.f);  // this warp's half of the row sum
+      int j_next = __ldg(a.col_idx + x.beg);
+      for (int t = 0; t < n; ++t, ++g) {
         const int j = j_next;
-        if (t + 2 < n) j_next = __ldg(a.col_idx + x.beg + t + 2);
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + st), nS & 1, abort_flag))) { ok = false; break; }
-        ++nS;
+        if (t + 1 < n) j_next = __ldg(a.col_idx + x.beg + t + 1);
+        const int b = g % L::kSBufs;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + b), (g / L::kSBufs) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
         const bool bad = j < 0 || j >= a.nkb;
         const bool dead = bad || (a.causal && j > gi);
         const bool diag = a.causal && j == gi;
-        if (dead && r == 0) raise_error(bad ? RBS_DEVERR_BLOCK_INDEX : RBS_DEVERR_NONCAUSAL);
-        // tile column c is masked when c > r (diagonal block) or always (dead block)
-        auto mask64 = [&](uint32_t(&v)[2][32], int base) {
-          if (dead || diag) {
+        if (dead && r == 0 && hf == 0) raise_error(bad ? RBS_DEVERR_BLOCK_INDEX : RBS_DEVERR_NONCAUSAL);
+        // pass 1: this warp's half row of S into registers, masked; its maximum
+        const uint32_t scol = L::col_s(b) + hf * kHalf;
+        uint32_t v[kHalf / 32][32];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int lim = dead ? -1 : r - (base + 32 * q);
+        for (int q = 0; q < kHalf / 32; ++q) tmem_ld32(lane_base + scol + 32 * q, v[q]);
+        tmem_wait_ld();
+        if (dead || diag) {
+          // tile column hf * kHalf + 32 q + e is masked when it is above the diagonal (or always)
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (e > lim) v[q][e] = __float_as_uint(-INFINITY);
-            }
-          }
-        };
-        // pass 1: the row maximum, 64 columns at a time
-        float mx = -INFINITY;
+          for (int q = 0; q < kHalf / 32; ++q) {
+            const int lim = dead ? -1 : r - (hf * kHalf + 32 * q);
 #pragma unroll
-        for (int h64 = 0; h64 < BK / 64; ++h64) {
-          uint32_t v[2][32];
-          tmem_ld32(lane_base + L::col_s(st) + 64 * h64, v[0]);
-          tmem_ld32(lane_base + L::col_s(st) + 64 * h64 + 32, v[1]);
-          tmem_wait_ld();
-          mask64(v, 64 * h64);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            float m0 = __uint_as_float(v[q][0]);
-#pragma unroll
-            for (int e = 1; e < 31; e += 2) m0 = fmax3(m0, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
-            mx = fmax3(mx, m0, __uint_as_float(v[q][31]));
+            for (int e = 0; e < 32; ++e)
+              if (e > lim) v[q][e] = __float_as_uint(-INFINITY);
           }
         }
-        const float m_new = fmaxf(m_used, mx * c);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kHalf / 32; ++q) {
+          float m0 = __uint_as_float(v[q][0]);
+#pragma unroll
+          for (int e = 1; e < 31; e += 2) m0 = fmax3(m0, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
+          mx = fmax3(mx, m0, __uint_as_float(v[q][31]));
+        }
+        float mo;
+        if (!exchange(mx, mo)) { ok = false; break; }
+        const float m_new = fmaxf(m_used, fmaxf(mx, mo) * c);
         float factor = 1.f;
         bool rescale = false;
-        if (t < 2) {
+        if (t == 0) {
           m_used = m_new;
         } else if (m_new - m_used > 8.f) {
           factor = ptx_exp2(m_used - m_new);
@@ -414,84 +439,71 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         const float m_exp = m_used == -INFINITY ? 0.f : m_used;
         l2.x *= factor;
         l2.y *= factor;
-        // this stream's previous PV is complete (S_t was issued after it): O is stable
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t v[32];
-            tmem_ld32(lane_base + L::col_o(st) + 32 * q, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * factor);
-            tmem_st32(lane_base + L::col_o(st) + 32 * q, v);
-          }
-        }
-        // pass 2: P = exp2(s*c - m), 64 columns at a time, written as packed
-        // bf16 pairs over S columns this thread has already consumed
+        // pass 2: P = exp2(s*c - m) from the registers, written as packed bf16
+        // pairs over the first kHalf/2 of this warp's S columns (already read)
         const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_exp, -m_exp);
         float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        uint32_t pw[kHalf / 2];
 #pragma unroll
-        for (int h64 = 0; h64 < BK / 64; ++h64) {
-          uint32_t v[2][32];
-          tmem_ld32(lane_base + L::col_s(st) + 64 * h64, v[0]);
-          tmem_ld32(lane_base + L::col_s(st) + 64 * h64 + 32, v[1]);
-          tmem_wait_ld();
-          mask64(v, 64 * h64);
-          uint32_t pw[32];
-#pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const float2 sv = make_float2(__uint_as_float(v[e >> 5][e & 31]), __uint_as_float(v[e >> 5][(e & 31) + 1]));
-            const float2 arg = ffma2(sv, c2, nm2);
-            const int pi = (e >> 1) & 7;  // pairs 1, 4 and 6 of every 8 on the FMA pipe
-            const float2 p = (pi == 1 || pi == 4 || pi == 6) ? exp2_fma2(arg)
-                                                               : make_float2(ptx_exp2(arg.x), ptx_exp2(arg.y));
-            acc[(e >> 1) & 1] = fadd2(acc[(e >> 1) & 1], p);
-            pw[e >> 1] = pack_bf16x2(p.x, p.y);
-          }
-          tmem_st32(lane_base + L::col_s(st) + 32 * h64, pw);
+        for (int e = 0; e < kHalf; e += 2) {
+          const float2 sv = make_float2(__uint_as_float(v[e >> 5][e & 31]), __uint_as_float(v[e >> 5][(e & 31) + 1]));
+          const float2 arg = ffma2(sv, c2, nm2);
+          const int pi = (e >> 1) & 7;  // pairs 1, 4 and 6 of every 8 on the FMA pipe
+          const float2 p = (pi == 1 || pi == 4 || pi == 6) ? exp2_fma2(arg)
+                                                             : make_float2(ptx_exp2(arg.x), ptx_exp2(arg.y));
+          acc[(e >> 1) & 1] = fadd2(acc[(e >> 1) & 1], p);
+          pw[e >> 1] = pack_bf16x2(p.x, p.y);
+        }
+        if constexpr (kHalf == 64) {
+          tmem_st32(lane_base + scol, pw);
+        } else {
+          tmem_st16(lane_base + scol, pw);
         }
         l2 = fadd2(l2, fadd2(acc[0], acc[1]));
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O is scaled after P is formed, so the wait below overlaps the
+          // exponentials.  O must hold every earlier tile's product first.
+          // The next phase of PV_{g-1}'s barrier is PV_{g+3}, which cannot
+          // start before this tile's P is complete.
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPVDone + ((g - 1) & 3)), ((g - 1) >> 2) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + L::kColO + 64 * hf + 32 * q, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(lane_base + L::kColO + 64 * hf + 32 * q, o);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
-        warp_arrive(kBarPFull + st);
+        warp_arrive(kBarPFull + b);
       }
       if (!ok) break;
 
-      // ---- epilogue: merge the two streams, O / l -> bf16, LSE
-      float* xb = xch + (item & 1) * 512;  // [2 streams][m, l][128 rows]
-      xb[st * 256 + r] = m_used;
-      xb[st * 256 + 128 + r] = l2.x + l2.y;
-      warp_arrive(kBarX);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarX), item & 1, abort_flag))) { ok = false; break; }
-      const bool hasB = n > 1;  // stream B has tiles only when the row has two or more
-      const float mA = xb[r], lA = xb[128 + r];
-      const float mB = hasB ? xb[256 + r] : -INFINITY, lB = hasB ? xb[384 + r] : 0.f;
-      const float m = fmaxf(mA, mB);
-      const float wA = lA > 0.f ? ptx_exp2(mA - m) : 0.f;
-      const float wB = lB > 0.f ? ptx_exp2(mB - m) : 0.f;
-      const float lt = lA * wA + lB * wB;
+      // ---- epilogue: O / l -> bf16 (this warp: dims [64 hf, 64 hf + 64)), LSE
+      const float lh = l2.x + l2.y;
+      float lo;
+      if (!exchange(lh, lo)) { ok = false; break; }
+      const float lt = lh + lo;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      bool okw = mbar_wait(bar(kBarOFull + 0), nO[0] & 1, abort_flag);
-      if (hasB && okw) okw = mbar_wait(bar(kBarOFull + 1), nO[1] & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
-      ++nO[0];
-      if (hasB) ++nO[1];
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarOFull), item & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       const int64_t qrow = static_cast<int64_t>(x.i) * BQ + r;
-      uint4* dst = reinterpret_cast<uint4*>(a.O + x.b * a.ob + qrow * a.os + x.h * a.oh) + 8 * st;
-      const float sa = wA * inv, sb = wB * inv;
+      uint4* dst = reinterpret_cast<uint4*>(a.O + x.b * a.ob + qrow * a.os + x.h * a.oh) + 8 * hf;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        uint32_t va[32], vb[32];
-        tmem_ld32(lane_base + L::col_o(0) + 64 * st + 32 * q, va);
-        if (hasB) tmem_ld32(lane_base + L::col_o(1) + 64 * st + 32 * q, vb);
+        uint32_t va[32];
+        tmem_ld32(lane_base + L::kColO + 64 * hf + 32 * q, va);
         tmem_wait_ld();
         float o[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          o[e] = __uint_as_float(va[e]) * sa;
-          if (hasB) o[e] = fmaf(__uint_as_float(vb[e]), sb, o[e]);
-        }
+        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(va[e]) * inv;
         if (r < BQ) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -500,13 +512,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
                                         pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
         }
       }
-      if (st == 0 && a.lse != nullptr && r < BQ) {
+      if (hf == 0 && a.lse != nullptr && r < BQ) {
         a.lse[(static_cast<int64_t>(x.b) * a.Hq + x.h) * a.Lq + qrow] =
-            lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+            lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
       }
       tc_fence_before();
-      warp_arrive(kBarOEmpty + 0);
-      warp_arrive(kBarOEmpty + 1);
+      warp_arrive(kBarOEmpty);
       ++item;
     }
   }
