@@ -11,8 +11,9 @@ Prints ONE JSON line (rank 0).  `value` = effective TFLOP/s of the whole step
 max-over-ranks step time.  Also reported: attention-only ms and TFLOP/s,
 selection ms, stats ms, the attention kernel's roofline, clocks, an
 end-to-end number through the same calls with host buffers, the Block-
-attention RAG flow (cache build, RoPE re-encoding, final block) and the CPU
-oracle baseline.
+attention RAG flow (cache build, RoPE re-encoding, final block), a density
+sweep at 64K (selection and attention time at 2-100% kept density) and the
+CPU oracle baseline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 N > 1 runs under torchrun: every rank processes its own prompt (weak
@@ -42,6 +43,9 @@ WORKLOAD = "gqa_rbs_128k"
 BLOCK = 128
 HEAD_DIM = 128
 FLOP_PER_PAIR = 4 * BLOCK * BLOCK * HEAD_DIM  # QK^T and PV on one 128x128 block pair
+# kernels one step launches: block stats; beta, scoring + top-k, scan, compaction; attention
+LAUNCHES_PER_STEP = 6
+SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
 
 
 def load_peaks():
@@ -252,7 +256,7 @@ def run_ours(args, ws, rank):
                              "frac_hbm": round(select_bytes / (select_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)},
         },
         "clocks": clocks,
-        "gpu_launches": args.steps * 7,
+        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
     }
     if args.e2e:
         out["e2e"] = e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn=None, ctx=dict(
@@ -265,6 +269,8 @@ def run_ours(args, ws, rank):
     torch.cuda.empty_cache()
     if args.block_attention and rank == 0:
         out["block_attention"] = block_attention_measure(rbs, peaks)
+    if args.density_sweep and rank == 0:
+        out["density_sweep"] = density_sweep_measure(rbs, peaks)
     if args.cpu_baseline and rank == 0:
         out["cpu_baseline"] = cpu_baseline(Qh, Kh, Vh, w, budget_s=args.cpu_budget)
     return out
@@ -393,6 +399,83 @@ def block_attention_measure(rbs, peaks):
     return res
 
 
+def _time_ms(fn, reps: int, warm: int = 2) -> float:
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def density_sweep_measure(rbs, peaks):
+    """Selection and attention time against the kept-union density at 64K
+    tokens (32 q / 8 KV heads, the compact/dispersed key mixture).  For each
+    target density one rho, shared by both branches, is found by bisection on
+    [0, 1] (the kept sets are nested in rho, so the density is monotone) until
+    the achieved density is within 0.25 percentage points; 100% is rho = 1."""
+    import torch
+    w = WORKLOADS["density_sweep_64k"]
+    inp = make_inputs(w)
+    Q, K, V = to_dev(inp["Q"]), to_dev(inp["K"]), to_dev(inp["V"])
+    B, L, Hq, _ = Q.shape
+    Hkv = K.shape[2]
+    nqb = nkb = L // BLOCK
+    C, R = rbs.rbs_block_stats(K, BLOCK)
+    p_full = rbs.SelectParams(block_q=BLOCK, block_k=BLOCK, rho_centroid=1.0, rho_rescue=1.0)
+    lists = rbs.BlockLists.empty(B * Hq * nqb, rbs.rbs_select_capacity(B, Hq, nqb, nkb, p_full), "cuda")
+    wsb = torch.empty(rbs.rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, p_full), dtype=torch.uint8, device="cuda")
+    visible = B * Hq * nqb * (nqb + 1) // 2
+    O = torch.empty_like(Q)
+
+    def select(rho):
+        p = rbs.SelectParams(block_q=BLOCK, block_k=BLOCK, rho_centroid=rho, rho_rescue=rho)
+        rbs.rbs_select(Q, C, R, p, workspace=wsb, out=lists)
+
+    def density(rho):
+        select(rho)
+        return lists.nnz() / visible
+
+    rows = []
+    for target in SWEEP_TARGETS:
+        if target >= 1.0:
+            rho, dens = 1.0, density(1.0)
+        else:
+            lo, hi = 0.0, 1.0
+            rho, dens = hi, 1.0
+            for _ in range(30):
+                mid = float(np.float32(0.5 * (lo + hi)))
+                dens = density(mid)
+                rho = mid
+                if abs(dens - target) <= 0.0025:
+                    break
+                if dens < target:
+                    lo = mid
+                else:
+                    hi = mid
+        select(rho)
+        nnz = lists.nnz()
+        sel_ms = _time_ms(lambda: select(rho), 5)
+        attn_ms = _time_ms(lambda: rbs.bsa_prefill(Q, K, V, lists, BLOCK, BLOCK, out=O), 3 if target >= 0.5 else 5)
+        tflops = nnz * FLOP_PER_PAIR / (attn_ms * 1e-3) / 1e12
+        rows.append({"target": target, "rho": rho, "density": round(nnz / visible, 5), "pairs": nnz,
+                     "select_ms": round(sel_ms, 4), "attn_ms": round(attn_ms, 4), "attn_tflops": round(tflops, 1),
+                     "attn_frac_peak": round(tflops / peaks["bf16_tflops_sustained"], 4)})
+    assert rbs.rbs_get_device_error() == 0
+    dense_ms = rows[-1]["attn_ms"]
+    for r in rows:
+        r["speedup_vs_dense"] = round(dense_ms / (r["attn_ms"] + r["select_ms"]), 2)
+    return {"workload": "density_sweep_64k: L=65536, 32 q / 8 KV heads, 128x128 blocks, causal", "rows": rows}
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (rank 0, N=1 semantics)
 
@@ -481,6 +564,7 @@ def main():
     ap.add_argument("--no-dense", dest="dense", action="store_false")
     ap.add_argument("--no-block-attention", dest="block_attention", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-density-sweep", dest="density_sweep", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--seq-len", type=int, default=None,

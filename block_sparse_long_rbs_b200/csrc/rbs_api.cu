@@ -163,7 +163,7 @@ int keep_count_host(float rho, int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct SelectLayout {
-  size_t mask_c, mask_r, counts, qbar, qnorm, beta, total;
+  size_t mask_c, mask_r, counts, beta, total;
 };
 
 SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int64_t nkb) {
@@ -174,8 +174,6 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
   l.mask_c = off; off += align256(rows * nwords * 4);
   l.mask_r = off; off += align256(rows * nwords * 4);
   l.counts = off; off += align256(rows * 4);
-  l.qbar = off; off += align256(B * Hq * nqb * RBS_HEAD_DIM * 4);
-  l.qnorm = off; off += align256(B * Hq * nqb * 4);
   l.beta = off; off += align256(B * Hkv * nkb * 4);
   l.total = off;
   return l;
