@@ -115,51 +115,162 @@ __device__ __forceinline__ void warp_topk2(const uint32_t (&kc)[KPL], const uint
   }
 }
 
+// Exact top-k of both branches by pruning, for k <= 64 (key(t) = this
+// lane's key in slot t, block 32 t + lane, read from shared memory).  Each
+// lane's two largest keys form a 64-key subset of the row.  L is the largest
+// key with its low 16 bits clear such that at least k keys of the subset are
+// >= L; it is at most the subset's k-th largest key, hence at most the row's
+// k-th largest key T, so every key >= T is a candidate (key >= L).  When at
+// most 64 keys are candidates they are compacted in ascending block order
+// into shared memory, T is found among them by a bitwise search (the largest
+// T with at least k candidates >= T), the keys above T are kept and of the
+// ties at T the lowest block indices, and the kept blocks are OR-ed into
+// words[0, nwords) (cleared first).  Returns false, having written nothing
+// the caller uses, when k > 64 or more than 64 keys of a branch are
+// candidates (many near-equal keys); the caller then runs the full search.
+// Both branches advance together so their reduction chains overlap.
+// Warp-uniform.
+template <int KP, typename KeyC, typename KeyR>
+__device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_c, int k_r, int lane, int nwords,
+                                                  uint32_t* scratch, uint32_t* words_c, uint32_t* words_r) {
+  if (k_c > 64 || k_r > 64) return false;
+  uint32_t* ck_c = scratch;  // candidate keys [64] and blocks [64] of each branch
+  int* ci_c = reinterpret_cast<int*>(scratch + 64);
+  uint32_t* ck_r = scratch + 128;
+  int* ci_r = reinterpret_cast<int*>(scratch + 192);
+  uint32_t c1 = 0, c2 = 0, r1 = 0, r2 = 0;  // this lane's two largest keys per branch
+#pragma unroll 4
+  for (int t = 0; t < KP; ++t) {
+    const uint32_t uc = key_c(t), ur = key_r(t);
+    c2 = max(c2, min(c1, uc));
+    c1 = max(c1, uc);
+    r2 = max(r2, min(r1, ur));
+    r1 = max(r1, ur);
+  }
+  // The subset holds at least k keys that are not absent (rows interleave
+  // blocks over the lanes), and a present key is >= 2^16, so L > 0 and no
+  // absent slot (key 0) becomes a candidate.
+  uint32_t Lc = 0, Lr = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 16; --bit) {
+    const uint32_t xc = Lc | (1u << bit), xr = Lr | (1u << bit);
+    const int nc = __reduce_add_sync(0xffffffffu, (c1 >= xc ? 1 : 0) + (c2 >= xc ? 1 : 0));
+    const int nr = __reduce_add_sync(0xffffffffu, (r1 >= xr ? 1 : 0) + (r2 >= xr ? 1 : 0));
+    if (nc >= k_c) Lc = xc;
+    if (nr >= k_r) Lr = xr;
+  }
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base_c = 0, base_r = 0;
+#pragma unroll 4
+  for (int t = 0; t < KP; ++t) {
+    const uint32_t uc = key_c(t), ur = key_r(t);
+    const bool cand_c = uc >= Lc, cand_r = ur >= Lr;
+    const uint32_t bc = __ballot_sync(0xffffffffu, cand_c), br = __ballot_sync(0xffffffffu, cand_r);
+    const int pc = base_c + __popc(bc & lt_mask), pr = base_r + __popc(br & lt_mask);
+    if (cand_c && pc < 64) {
+      ck_c[pc] = uc;
+      ci_c[pc] = 32 * t + lane;
+    }
+    if (cand_r && pr < 64) {
+      ck_r[pr] = ur;
+      ci_r[pr] = 32 * t + lane;
+    }
+    base_c += __popc(bc);
+    base_r += __popc(br);
+  }
+  if (base_c > 64 || base_r > 64) return false;
+  __syncwarp();
+  const uint32_t a0 = lane < base_c ? ck_c[lane] : 0u, a1 = lane + 32 < base_c ? ck_c[lane + 32] : 0u;
+  const uint32_t b0 = lane < base_r ? ck_r[lane] : 0u, b1 = lane + 32 < base_r ? ck_r[lane + 32] : 0u;
+  const int ia0 = lane < base_c ? ci_c[lane] : 0, ia1 = lane + 32 < base_c ? ci_c[lane + 32] : 0;
+  const int ib0 = lane < base_r ? ci_r[lane] : 0, ib1 = lane + 32 < base_r ? ci_r[lane + 32] : 0;
+  uint32_t Tc = 0, Tr = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t xc = Tc | (1u << bit), xr = Tr | (1u << bit);
+    const int nc = __reduce_add_sync(0xffffffffu, (a0 >= xc ? 1 : 0) + (a1 >= xc ? 1 : 0));
+    const int nr = __reduce_add_sync(0xffffffffu, (b0 >= xr ? 1 : 0) + (b1 >= xr ? 1 : 0));
+    if (nc >= k_c) Tc = xc;
+    if (nr >= k_r) Tr = xr;
+  }
+  // candidate position p (= lane, lane + 32) is in ascending block order, so
+  // a tie's rank is the number of ties at lower positions
+  const int need_c = k_c - __reduce_add_sync(0xffffffffu, (a0 > Tc ? 1 : 0) + (a1 > Tc ? 1 : 0));
+  const int need_r = k_r - __reduce_add_sync(0xffffffffu, (b0 > Tr ? 1 : 0) + (b1 > Tr ? 1 : 0));
+  const bool ta0 = a0 == Tc, ta1 = a1 == Tc, tb0 = b0 == Tr, tb1 = b1 == Tr;
+  const uint32_t ba0 = __ballot_sync(0xffffffffu, ta0), ba1 = __ballot_sync(0xffffffffu, ta1);
+  const uint32_t bb0 = __ballot_sync(0xffffffffu, tb0), bb1 = __ballot_sync(0xffffffffu, tb1);
+  const bool sa0 = a0 > Tc || (ta0 && __popc(ba0 & lt_mask) < need_c);
+  const bool sa1 = a1 > Tc || (ta1 && __popc(ba0) + __popc(ba1 & lt_mask) < need_c);
+  const bool sb0 = b0 > Tr || (tb0 && __popc(bb0 & lt_mask) < need_r);
+  const bool sb1 = b1 > Tr || (tb1 && __popc(bb0) + __popc(bb1 & lt_mask) < need_r);
+  for (int w = lane; w < nwords; w += 32) words_c[w] = words_r[w] = 0u;
+  __syncwarp();
+  if (sa0) atomicOr(&words_c[ia0 >> 5], 1u << (ia0 & 31));
+  if (sa1) atomicOr(&words_c[ia1 >> 5], 1u << (ia1 & 31));
+  if (sb0) atomicOr(&words_r[ib0 >> 5], 1u << (ib0 & 31));
+  if (sb1) atomicOr(&words_r[ib1 >> 5], 1u << (ib1 & 31));
+  __syncwarp();
+  return true;
+}
+
 // Both branches' top-k of one row (warp-wide) -> mask words and the row's
 // union count.  Keys hold KP slots per lane (block 32t + lane in slot t); the
 // row's mask words cover all nwords <= (KPMAX + 31) / 32 * 32 words.
 template <int KP, int KPMAX>
 __device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float* sc, const float* rb,
                                                 const float* qn, int warp, int lane, int hq0, int b, int i, int gi,
-                                                int n, int npad) {
+                                                int n, int npad, uint32_t* scratch) {
   const int hq = hq0 + warp;
   const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
   const float qnv = qn[warp];
-  constexpr int NO = (KP + 31) / 32;
-  uint32_t own_c[NO], own_r[NO];
-  {
+  // per-warp scratch: candidates of both branches [256], mask words of both branches
+  uint32_t* words_c = scratch + 256;
+  uint32_t* words_r = words_c + a.nwords;
+  const float* srow = sc + warp * npad;
+  auto key_c = [&](int t) -> uint32_t {
+    const int j = 32 * t + lane;
+    return j < n ? order_key(srow[j]) : 0u;
+  };
+  auto key_r = [&](int t) -> uint32_t {
+    const int j = 32 * t + lane;
+    return j < n ? order_key(fmaf(qnv, rb[j], srow[j])) : 0u;
+  };
+  const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
+  const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, scratch, words_c, words_r);
+  if (!done) {
     uint32_t kc[KP], kr[KP];
 #pragma unroll
     for (int t = 0; t < KP; ++t) {
-      const int j = 32 * t + lane;
-      const float sv = j < n ? sc[warp * npad + j] : 0.f;
-      kc[t] = j < n ? order_key(sv) : 0u;
-      kr[t] = j < n ? order_key(fmaf(qnv, rb[j], sv)) : 0u;
+      kc[t] = key_c(t);
+      kr[t] = key_r(t);
     }
-    warp_topk2<KP>(kc, kr, keep_count(a.rho_c, n), keep_count(a.rho_r, n), lane, own_c, own_r);
+    constexpr int NO = (KP + 31) / 32;
+    uint32_t own_c[NO], own_r[NO];
+    warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
+    for (int w = lane; w < a.nwords; w += 32) {
+      const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
+      words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+      words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+    }
+    __syncwarp();
   }
   int cnt = 0;
-  constexpr int NW = (KPMAX + 31) / 32;  // mask words this lane may own
-#pragma unroll
-  for (int q = 0; q < NW; ++q) {
-    const int t = 32 * q + lane;
-    if (t < a.nwords) {
-      const uint32_t wc = (q < NO && t < KP) ? own_c[q < NO ? q : 0] : 0u;
-      const uint32_t wr = (q < NO && t < KP) ? own_r[q < NO ? q : 0] : 0u;
-      uint32_t f = 0;
-      if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
-      if (a.force_sink && t == 0) f |= 1u;
-      cnt += __popc(wc | wr | f);
-      a.mask_c[row * a.nwords + t] = wc;
-      a.mask_r[row * a.nwords + t] = wr;
-    }
+  for (int t = lane; t < a.nwords; t += 32) {
+    const uint32_t wc = words_c[t], wr = words_r[t];
+    uint32_t f = 0;
+    if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
+    if (a.force_sink && t == 0) f |= 1u;
+    cnt += __popc(wc | wr | f);
+    a.mask_c[row * a.nwords + t] = wc;
+    a.mask_r[row * a.nwords + t] = wr;
   }
   cnt = __reduce_add_sync(0xffffffffu, cnt);
   if (lane == 0) a.counts[row] = cnt;
 }
 
 template <int KPL, int BQ>
-__global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads, KPL <= 32 ? 3 : 1) select_rows_kernel(SelectArgs a) {
   extern __shared__ __align__(16) float sm[];
   const int i = a.nqb - 1 - static_cast<int>(blockIdx.x);  // longest rows first
   const int hblk = blockIdx.y, b = blockIdx.z;
@@ -172,7 +283,7 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
   const int n = a.causal ? min(a.nkb, gi + 1) : a.nkb;
   const int npad = (a.nkb + 31) & ~31;
 
-  float* qs = sm;                         // [R][128] pooled queries
+  float* qs = sm;                         // [128][8] pooled queries, dim-major (heads >= R are 0)
   float* rb = qs + kSelMaxR * 128;        // [npad]  r_j * beta_j
   float* sc = rb + npad;                  // [R][npad] centroid-branch scores
   float* cs = sc + kSelMaxR * npad;       // [kStageJ][kStagePitch]; first holds pooling partial sums
@@ -214,16 +325,21 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
       for (int e = 0; e < 8; ++e) cs[rg * (R * 128) + col * 8 + e] = acc[e];
     }
     __syncthreads();
-    for (int o = tid; o < R * 128; o += kSelThreads) {
+    for (int o = tid; o < kSelMaxR * 128; o += kSelThreads) {
+      const int h = o >> 7, d = o & 127;  // o = h * 128 + d, the pooling sums' order
       float sum = 0.f;
-      for (int g2 = 0; g2 < RG; ++g2) sum += cs[g2 * (R * 128) + o];
-      qs[o] = sum * (1.0f / BQ);
+      if (h < R)
+        for (int g2 = 0; g2 < RG; ++g2) sum += cs[g2 * (R * 128) + o];
+      qs[d * kSelMaxR + h] = sum * (1.0f / BQ);
     }
     __syncthreads();
     if (warp < R) {
       float s2 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s2 = fmaf(qs[warp * 128 + lane + 32 * e], qs[warp * 128 + lane + 32 * e], s2);
+      for (int e = 0; e < 4; ++e) {
+        const float v = qs[(lane + 32 * e) * kSelMaxR + warp];
+        s2 = fmaf(v, v, s2);
+      }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
       if (lane == 0) qn[warp] = sqrtf(s2);
@@ -248,14 +364,16 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
-  float acc[kSelMaxR];
+  // four head pairs per thread, accumulated with paired FMAs (the heads of a
+  // pair share the centroid value)
+  float2 acc[kSelMaxR / 2];
   load_stage(0);
   for (int st = 0; st < nstages; ++st) {
     const int j0 = (st / (128 / kStageD)) * kStageJ, d0 = (st % (128 / kStageD)) * kStageD;
     const int jn = min(kStageJ, n - j0);
     if (d0 == 0) {
 #pragma unroll
-      for (int h = 0; h < kSelMaxR; ++h) acc[h] = 0.f;
+      for (int h = 0; h < kSelMaxR / 2; ++h) acc[h] = make_float2(0.f, 0.f);
     }
     __syncthreads();
 #pragma unroll
@@ -271,25 +389,32 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
     if (st + 1 < nstages) load_stage(st + 1);
     if (tid < jn) {
       const float* crow = cs + tid * kStagePitch;
-#pragma unroll 4
-      for (int d = 0; d < kStageD; d += 4) {
-        const float c0 = crow[d], c1 = crow[d + 1], c2 = crow[d + 2], c3 = crow[d + 3];
-#pragma unroll
-        for (int h = 0; h < kSelMaxR; ++h) {
-          if (h < R) {
-            const float4 q = *reinterpret_cast<const float4*>(qs + h * 128 + d0 + d);
-            acc[h] = fmaf(q.x, c0, acc[h]);
-            acc[h] = fmaf(q.y, c1, acc[h]);
-            acc[h] = fmaf(q.z, c2, acc[h]);
-            acc[h] = fmaf(q.w, c3, acc[h]);
-          }
+      const float* qd = qs + d0 * kSelMaxR;
+      if (R > 4) {
+#pragma unroll 8
+        for (int d = 0; d < kStageD; ++d) {
+          const float2 cc = make_float2(crow[d], crow[d]);
+          const float4 qa = *reinterpret_cast<const float4*>(qd + d * kSelMaxR);
+          const float4 qb = *reinterpret_cast<const float4*>(qd + d * kSelMaxR + 4);
+          acc[0] = ffma2(make_float2(qa.x, qa.y), cc, acc[0]);
+          acc[1] = ffma2(make_float2(qa.z, qa.w), cc, acc[1]);
+          acc[2] = ffma2(make_float2(qb.x, qb.y), cc, acc[2]);
+          acc[3] = ffma2(make_float2(qb.z, qb.w), cc, acc[3]);
+        }
+      } else {
+#pragma unroll 8
+        for (int d = 0; d < kStageD; ++d) {
+          const float2 cc = make_float2(crow[d], crow[d]);
+          const float4 qa = *reinterpret_cast<const float4*>(qd + d * kSelMaxR);
+          acc[0] = ffma2(make_float2(qa.x, qa.y), cc, acc[0]);
+          acc[1] = ffma2(make_float2(qa.z, qa.w), cc, acc[1]);
         }
       }
     }
     if (d0 + kStageD == 128 && tid < jn) {
 #pragma unroll
       for (int h = 0; h < kSelMaxR; ++h)
-        if (h < R) sc[h * npad + j0 + tid] = acc[h];
+        if (h < R) sc[h * npad + j0 + tid] = (h & 1) ? acc[h >> 1].y : acc[h >> 1].x;
     }
   }
   __syncthreads();
@@ -297,9 +422,11 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(SelectArgs a) 
   // ---- per-branch top-k (both branches together), one warp per row, with
   // as few key slots per lane as this row needs
   if (warp < R) {
-    if (KPL > 8 && n <= 64) select_topk_row<2, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad);
-    else if (KPL > 8 && n <= 256) select_topk_row<8, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad);
-    else select_topk_row<KPL, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad);
+    // the staging area is free after the scores: per-warp top-k scratch
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(cs) + warp * (256 + 2 * a.nwords);
+    if (KPL > 8 && n <= 64) select_topk_row<2, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad, scratch);
+    else if (KPL > 8 && n <= 256) select_topk_row<8, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad, scratch);
+    else select_topk_row<KPL, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad, scratch);
   }
 }
 
