@@ -7,25 +7,32 @@
 // order.  Persistent CTAs take non-empty work items round-robin in an order
 // that starts with the last query blocks (the longest causal rows).
 //
-// One softmax pipeline with three S buffers in TMEM.  While the softmax
-// warps work on tile t, the tensor core computes S for tiles t+1 and t+2 and
-// accumulates P_{t-1} V_{t-1}, so the tensor core and the softmax overlap
-// without either waiting on the other's latency.
+// One softmax pipeline with two S buffers in TMEM.  While the softmax warps
+// work on tile t, the tensor core computes S for tile t+1 and accumulates
+// P_{t-1} V_{t-1}, so the tensor core and the softmax overlap without either
+// waiting on the other's latency.
+//
+// Each key tile is split into two column halves, and each half has its own
+// softmax state: running max m_h, row sum l_h and accumulator
+// O_h = sum over tiles of P_h V_h (the P and V rows of that half's keys).
+// The two halves are merged exactly once per row, in the epilogue:
+//   O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)),
+// so the two warps that share a query row never wait for each other inside
+// the key loop.
 //
 // Roles (384 threads):
 //   warps 0-7  softmax: warp w owns query rows 32(w%4) .. 32(w%4)+31 (its
-//              TMEM lane quarter) and the S columns of half w/4 of every key
-//              tile.  Pass 1 reads its half row of S into registers and takes
-//              the half-row maximum; the two warps of a lane quarter exchange
-//              their maxima through shared memory (an mbarrier per quarter).
-//              The running max is lazily updated (O rescaled in TMEM only when
-//              it grows by more than 2^8; the final normalisation uses the same
-//              max, so the result is exact).  Pass 2 forms
-//              P = exp2(S*c - m) from the registers (3 of every 8 element pairs
-//              on the FMA pipe, see exp2_fma2, the rest on the SFU) and writes
-//              it as packed bf16 pairs over the first quarter of its own S
-//              columns.  In the epilogue the two warps of a quarter add their
-//              row sums and each writes 64 of the 128 output dims.
+//              TMEM lane quarter) and column half h = w/4 of every key tile.
+//              Pass 1 reads its half row of S into registers and takes its
+//              maximum; the running max is lazily updated (O_h rescaled in
+//              TMEM only when it grows by more than 2^8; the final
+//              normalisation uses the same max, so the result is exact).
+//              Pass 2 forms P = exp2(S*c - m_h) from the registers (3 of every
+//              8 element pairs on the FMA pipe, see exp2_fma2, the rest on the
+//              SFU) and writes it as packed bf16 pairs over the first quarter
+//              of its own S columns.  In the epilogue the two warps of a
+//              quarter exchange (m_h, l_h) and each writes 64 of the 128
+//              output dims from both accumulators.
 //   warp 8     Q and K producer, warp 9 V producer (one thread each): TMA
 //              loads of the Q tile (double-buffered) and of the K_j / V_j
 //              tiles gathered by block index (4-D tensor maps over
@@ -33,15 +40,15 @@
 //              V rings; list indices fetched one tile ahead.
 //   warp 10    TMEM allocator and S issuer, warp 11 PV issuer (each warp runs
 //              its loop; one elected lane issues):
-//                S_g  = Q K_g^T  into S buffer g%3    A = Q (smem), B = K_g (smem)
-//                O   += P_g V_g                        A = P (TMEM), B = V_g (MN-major smem)
+//                S_g   = Q K_g^T      into S buffer g%2  A = Q (smem), B = K_g (smem)
+//                O_h  += P_g,h V_g,h  for h = 0, 1       A = P (TMEM), B = V_g (MN-major smem)
 //              over the CTA's tiles g = 0, 1, 2, ... of all its rows in
-//              sequence.  S_{g+3} overwrites P_g, so the S issuer waits for
+//              sequence.  S_{g+2} overwrites P_g, so the S issuer waits for
 //              PV_g to complete; otherwise the two issuers run independently,
 //              so each one's waits and commits overlap the other's MMAs.
 //              The K and V producers refill a ring stage when the S (PV)
 //              barrier of the tile that used it completes.
-// TMEM columns: S buffers [0, BK), [128, 128+BK), [256, 256+BK); O [384, 512).
+// TMEM columns: S buffers [0, BK), [128, 128+BK); O_0 [256, 384), O_1 [384, 512).
 //
 // Every mbarrier wait is bounded; on a timeout all roles unwind, in-flight
 // TMA loads and MMAs are drained (bounded), TMEM is freed, and the device
@@ -101,15 +108,15 @@ struct AttnSmem {
   static constexpr int kQ = 0;                   // two Q buffers
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kNS * kKVBytes;
-  static constexpr int kX = kV + kNS * kKVBytes;  // float [2 exchange parity][2 halves][128 rows]
-  static constexpr int kBar = kX + 2 * 2 * 128 * 4;
+  static constexpr int kX = kV + kNS * kKVBytes;  // float [2 exchange parity][2 halves][(m, l)][128 rows]
+  static constexpr int kBar = kX + 2 * 2 * 2 * 128 * 4;
   static constexpr int kBarBytes = 256;
   static constexpr int kTotal = kBar + kBarBytes;
   static constexpr int kAlloc = kTotal + 1024;  // slack to align the base to 1024
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kSBufs = 3;
+  static constexpr int kSBufs = 2;
   __host__ __device__ static constexpr uint32_t col_s(int buf) { return buf * 128; }
-  static constexpr uint32_t kColO = 384;
+  __host__ __device__ static constexpr uint32_t col_o(int half) { return 256 + half * 128; }
 };
 
 // barrier slots (8 bytes each)
@@ -118,9 +125,9 @@ enum : int {
   kBarQEmpty = kBarQFull + 2,    // + buffer (2)
   kBarKFull = kBarQEmpty + 2,    // + stage
   kBarVFull = kBarKFull + kNS,   // + stage
-  kBarSFull = kBarVFull + kNS,   // + S buffer (3)
-  kBarPFull = kBarSFull + 3,     // + S buffer (3)
-  kBarPVDone = kBarPFull + 3,    // + tile index mod 4: one phase per fourth PV
+  kBarSFull = kBarVFull + kNS,   // + S buffer (2)
+  kBarPFull = kBarSFull + 2,     // + S buffer (2)
+  kBarPVDone = kBarPFull + 2,    // + tile index mod 4: one phase per fourth PV
   kBarOFull = kBarPVDone + 4,    // one phase per row
   kBarOEmpty = kBarOFull + 1,    // one phase per row
   kBarX = kBarOEmpty + 1,        // + lane quarter (4): the two warps' exchanges
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           // phase before this load lands, so the parity is unambiguous.
           if (nf >= kNS) {
             const uint32_t prev = nf - kNS;
-            const bool done = isK ? mbar_wait(bar(kBarSFull + prev % 3), (prev / 3) & 1, abort_flag)
+            const bool done = isK ? mbar_wait(bar(kBarSFull + prev % L::kSBufs), (prev / L::kSBufs) & 1, abort_flag)
                                   : mbar_wait(bar(kBarPVDone + (prev & 3)), (prev >> 2) & 1, abort_flag);
             if (!done) { ok = false; break; }
           }
@@ -296,9 +303,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           const int qb = it & 1;
           if (t == 0 && !wait(kBarQFull + qb, (it >> 1) & 1)) break;
           if (!wait(kBarKFull + s, (g / kNS) & 1)) break;
-          // S_g overwrites P_{g-3}: PV_{g-3} must be complete.  The next phase
-          // of that barrier is PV_{g+1}, which needs S_{g+1}: not yet issued.
-          if (g >= L::kSBufs && !wait(kBarPVDone + ((g - 3) & 3), ((g - 3) >> 2) & 1)) break;
+          // S_g overwrites P_{g-2}: PV_{g-2} must be complete.  The next phase
+          // of that barrier is PV_{g+2}, which needs S_{g+2}: not yet issued.
+          if (g >= L::kSBufs && !wait(kBarPVDone + ((g - 2) & 3), ((g - 2) >> 2) & 1)) break;
           tc_fence_after();
           const uint64_t qd = qdesc0 + qb * kQUnits, kd = kdesc0 + s * kStageUnits;
 #pragma unroll
@@ -316,9 +323,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           const uint64_t vd = vdesc0 + s * kStageUnits;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            // P of key half kk / kStepsHalf sits at the start of that half's S columns
-            const uint32_t pcol = L::col_s(b) + (kk / kStepsHalf) * (BK / 2) + (kk % kStepsHalf) * 8;
-            umma_ts_warp(tmem + L::kColO, tmem + pcol, vd + kk * (2048 >> 4), idPV, (t == 0 && kk == 0) ? 0u : 1u);
+            // key half h = kk / kStepsHalf: its P sits at the start of that
+            // half's S columns and accumulates into O_h
+            const int h = kk / kStepsHalf;
+            const uint32_t pcol = L::col_s(b) + h * (BK / 2) + (kk % kStepsHalf) * 8;
+            umma_ts_warp(tmem + L::col_o(h), tmem + pcol, vd + kk * (2048 >> 4), idPV,
+                         (t == 0 && kk % kStepsHalf == 0) ? 0u : 1u);
           }
           umma_commit_warp(bar(kBarPVDone + (g & 3)));
           if (t == x.n - 1) umma_commit_warp(bar(kBarOFull));
@@ -344,14 +354,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(k));
     };
-    // exchange one value per row with the other warp of this lane quarter
+    // exchange (m, l) of each row with the other warp of this lane quarter
     uint32_t nx = 0;
-    auto exchange = [&](float v, float& other) -> bool {
-      float* xb = xch + (nx & 1) * 256;  // [2 halves][128 rows]
-      xb[hf * 128 + r] = v;
+    auto exchange = [&](float m, float l, float& mo, float& lo) -> bool {
+      float* xb = xch + (nx & 1) * 512;  // [2 halves][(m, l)][128 rows]
+      xb[hf * 256 + r] = m;
+      xb[hf * 256 + 128 + r] = l;
       warp_arrive(kBarX + quarter);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarX + quarter), nx & 1, abort_flag))) return false;
-      other = xb[(hf ^ 1) * 128 + r];
+      mo = xb[(hf ^ 1) * 256 + r];
+      lo = xb[(hf ^ 1) * 256 + 128 + r];
       ++nx;
       return true;
     };
@@ -387,8 +399,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
     for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
       const int n = x.n;
       const int gi = x.i + a.q_block_off;
-      float m_used = -INFINITY;  // running max, in log2 units (score * c)
-      float2 l2 = make_float2(0.f, 0.f);  // this warp's half of the row sum
+      float m_used = -INFINITY;  // this half's running max, in log2 units (score * c)
+      float2 l2 = make_float2(0.f, 0.f);  // this half's row sum
       int j_next = __ldg(a.col_idx + x.beg);
       for (int t = 0; t < n; ++t, ++g) {
         const int j = j_next;
@@ -424,9 +436,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           for (int e = 1; e < 31; e += 2) m0 = fmax3(m0, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
           mx = fmax3(mx, m0, __uint_as_float(v[q][31]));
         }
-        float mo;
-        if (!exchange(mx, mo)) { ok = false; break; }
-        const float m_new = fmaxf(m_used, fmaxf(mx, mo) * c);
+        const float m_new = fmaxf(m_used, mx * c);
         float factor = 1.f;
         bool rescale = false;
         if (t == 0) {
@@ -471,13 +481,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           }
           tc_fence_after();
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          for (int q = 0; q < 4; ++q) {
             uint32_t o[32];
-            tmem_ld32(lane_base + L::kColO + 64 * hf + 32 * q, o);
+            tmem_ld32(lane_base + L::col_o(hf) + 32 * q, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(lane_base + L::kColO + 64 * hf + 32 * q, o);
+            tmem_st32(lane_base + L::col_o(hf) + 32 * q, o);
           }
         }
         tmem_wait_st();
@@ -486,24 +496,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       }
       if (!ok) break;
 
-      // ---- epilogue: O / l -> bf16 (this warp: dims [64 hf, 64 hf + 64)), LSE
+      // ---- epilogue: merge the halves, O / l -> bf16 (this warp: dims
+      // [64 hf, 64 hf + 64) of both accumulators), LSE
       const float lh = l2.x + l2.y;
-      float lo;
-      if (!exchange(lh, lo)) { ok = false; break; }
-      const float lt = lh + lo;
+      float mo, lo;
+      if (!exchange(m_used, lh, mo, lo)) { ok = false; break; }
+      const float m0 = hf == 0 ? m_used : mo, l0 = hf == 0 ? lh : lo;
+      const float m1 = hf == 0 ? mo : m_used, l1 = hf == 0 ? lo : lh;
+      const float m = fmaxf(m0, m1);
+      const float w0 = l0 > 0.f ? ptx_exp2(m0 - m) : 0.f;
+      const float w1 = l1 > 0.f ? ptx_exp2(m1 - m) : 0.f;
+      const float lt = l0 * w0 + l1 * w1;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float s0 = w0 * inv, s1 = w1 * inv;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarOFull), item & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       const int64_t qrow = static_cast<int64_t>(x.i) * BQ + r;
       uint4* dst = reinterpret_cast<uint4*>(a.O + x.b * a.ob + qrow * a.os + x.h * a.oh) + 8 * hf;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        uint32_t va[32];
-        tmem_ld32(lane_base + L::kColO + 64 * hf + 32 * q, va);
+        uint32_t va[32], vb[32];
+        tmem_ld32(lane_base + L::col_o(0) + 64 * hf + 32 * q, va);
+        tmem_ld32(lane_base + L::col_o(1) + 64 * hf + 32 * q, vb);
         tmem_wait_ld();
         float o[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(va[e]) * inv;
+        for (int e = 0; e < 32; ++e) o[e] = fmaf(__uint_as_float(vb[e]), s1, __uint_as_float(va[e]) * s0);
         if (r < BQ) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -514,7 +532,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       }
       if (hf == 0 && a.lse != nullptr && r < BQ) {
         a.lse[(static_cast<int64_t>(x.b) * a.Hq + x.h) * a.Lq + qrow] =
-            lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+            lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
       }
       tc_fence_before();
       warp_arrive(kBarOEmpty);
