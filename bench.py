@@ -258,6 +258,9 @@ def run_ours(args, ws, rank):
         "clocks": clocks,
         "gpu_launches": args.steps * LAUNCHES_PER_STEP,
     }
+    if args.isolated:
+        out["kernels"]["isolated"] = isolated_bandwidth_measure(
+            rbs, lib, tK, tQ, C, R, pc, lc, ws_buf, Hkv, nkb, stats_bytes, select_bytes, peaks)
     if args.e2e:
         out["e2e"] = e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn=None, ctx=dict(
             C=C, R=R, lists=lists, ws_buf=ws_buf, pc=pc, lc=lc, Hkv=Hkv, nkb=nkb, flops=flops, ws=ws))
@@ -274,6 +277,44 @@ def run_ours(args, ws, rank):
     if args.cpu_baseline and rank == 0:
         out["cpu_baseline"] = cpu_baseline(Qh, Kh, Vh, w, budget_s=args.cpu_budget)
     return out
+
+
+def isolated_bandwidth_measure(rbs, lib, tK, tQ, C, R, pc, lc, ws_buf, Hkv, nkb, stats_bytes, select_bytes, peaks):
+    """The bandwidth-bound kernels timed alone: before each launch a 512 MB
+    read fills L2 with clean lines, so the kernel pays neither for L2 hits on
+    its own input nor for writing back another kernel's dirty output (inside
+    the step, stats runs right after attention has written 1 GiB of O)."""
+    import ctypes
+    import torch
+    from block_sparse_long_rbs_b200 import _stream
+    flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
+    sink = torch.empty(1, dtype=torch.float32, device="cuda")
+
+    def stats():
+        rbs.check(lib.rbs_block_stats(ctypes.byref(tK), BLOCK, C.data_ptr(), R.data_ptr(), _stream()), "stats")
+
+    def select():
+        rbs.check(lib.rbs_select(ctypes.byref(tQ), C.data_ptr(), R.data_ptr(), Hkv, nkb, ctypes.byref(pc),
+                                 ws_buf.data_ptr(), ws_buf.numel(), ctypes.byref(lc), None, _stream()), "select")
+
+    res = {}
+    for name, fn, byt in (("block_stats", stats, stats_bytes), ("select_total", select, select_bytes)):
+        times = []
+        for _ in range(12):
+            sink.copy_(flush.sum().view(1))
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times[2:])
+        gbs = byt / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    res["note"] = "each launch after a 512 MB read (clean L2); median of 10"
+    del flush
+    return res
 
 
 def e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn, ctx):
@@ -372,19 +413,24 @@ def block_attention_measure(rbs, peaks):
         "final_block": lambda: rbs.bsa_prefill(Qf, Kg, V, final_lists, BLOCK, BLOCK, q_offset=P * PL, out=Of),
     }
     res = {}
+    flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
+    sink = torch.empty(1, dtype=torch.float32, device="cuda")
     for name, fn in parts.items():
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        reps = 20
-        a.record()
-        for _ in range(reps):
+        times = []
+        for _ in range(12):
+            sink.copy_(flush.sum().view(1))  # clean L2 before each launch (the cache is 64 MiB)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
             fn()
-        b.record()
-        torch.cuda.synchronize()
-        res[name] = {"ms": round(a.elapsed_time(b) / reps, 4)}
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        res[name] = {"ms": round(statistics.median(times[2:]), 4)}
+    del flush
     assert rbs.rbs_get_device_error() == 0
     rope_bytes = 2 * L * w.heads_kv * HEAD_DIM * 2
     gbs = rope_bytes / (res["rope_reencode"]["ms"] * 1e-3) / 1e9
@@ -565,6 +611,7 @@ def main():
     ap.add_argument("--no-block-attention", dest="block_attention", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-density-sweep", dest="density_sweep", action="store_false")
+    ap.add_argument("--no-isolated", dest="isolated", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--seq-len", type=int, default=None,
