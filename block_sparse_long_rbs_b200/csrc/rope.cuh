@@ -48,16 +48,43 @@ template <int STYLE>
 __global__ void __launch_bounds__(256) rope_reencode_kernel(const __grid_constant__ RopeArgs a) {
   __shared__ float cs[kRopeTokens][64];
   __shared__ float sn[kRopeTokens][64];
+  __shared__ double inv[64];
   const int t0 = blockIdx.x * kRopeTokens, b = blockIdx.y, tid = threadIdx.x;
-  for (int k = tid; k < kRopeTokens * 64; k += blockDim.x) {
-    const int tl = k >> 6, m = k & 63, t = t0 + tl;
-    double sv = 0.0, cv = 1.0;
-    if (t < a.L) {
-      const double phi = static_cast<double>(a.new_pos[t] - a.old_pos[t]) * a.inv_freq[m];
-      sincos(phi, &sv, &cv);
+  // the frequency table to shared memory with uniform (non-divergent) reads of
+  // the parameter block
+  if (tid < 64) {
+    double f = 0.0;
+#pragma unroll
+    for (int m = 0; m < 64; ++m)
+      if (m == tid) f = a.inv_freq[m];
+    inv[tid] = f;
+  }
+  // When every token of the CTA moves by the same offset (a passage moved as
+  // a whole), one sine/cosine per m serves all of them.
+  const int tme = t0 + tid % kRopeTokens;
+  const int d0 = a.new_pos[t0] - a.old_pos[t0];
+  const bool uniform = __syncthreads_and(tme >= a.L || a.new_pos[tme] - a.old_pos[tme] == d0);
+  if (uniform) {
+    if (tid < 64) {
+      double sv, cv;
+      sincos(static_cast<double>(d0) * inv[tid], &sv, &cv);
+#pragma unroll
+      for (int tl = 0; tl < kRopeTokens; ++tl) {
+        cs[tl][tid] = static_cast<float>(cv);
+        sn[tl][tid] = static_cast<float>(sv);
+      }
     }
-    cs[tl][m] = static_cast<float>(cv);
-    sn[tl][m] = static_cast<float>(sv);
+  } else {
+    for (int k = tid; k < kRopeTokens * 64; k += blockDim.x) {
+      const int tl = k >> 6, m = k & 63, t = t0 + tl;
+      double sv = 0.0, cv = 1.0;
+      if (t < a.L) {
+        const double phi = static_cast<double>(a.new_pos[t] - a.old_pos[t]) * inv[m];
+        sincos(phi, &sv, &cv);
+      }
+      cs[tl][m] = static_cast<float>(cv);
+      sn[tl][m] = static_cast<float>(sv);
+    }
   }
   __syncthreads();
   constexpr int CPH = STYLE == 0 ? 8 : 16;  // tasks per head
