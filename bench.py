@@ -261,6 +261,10 @@ def run_ours(args, ws, rank):
     if args.isolated:
         out["kernels"]["isolated"] = isolated_bandwidth_measure(
             rbs, lib, tK, tQ, C, R, pc, lc, ws_buf, Hkv, nkb, stats_bytes, select_bytes, peaks)
+    if args.selector_quality and rank == 0:
+        out["selector_quality"] = {
+            WORKLOAD: selector_quality_measure(rbs, Q, C, R, lists, inp["plants"], B, Hq, nqb, nkb, w.rho),
+            "tiny_rbs_4k": tiny_selector_quality(rbs)}
     if args.e2e:
         out["e2e"] = e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn=None, ctx=dict(
             C=C, R=R, lists=lists, ws_buf=ws_buf, pc=pc, lc=lc, Hkv=Hkv, nkb=nkb, flops=flops, ws=ws))
@@ -277,6 +281,83 @@ def run_ours(args, ws, rank):
     if args.cpu_baseline and rank == 0:
         out["cpu_baseline"] = cpu_baseline(Qh, Kh, Vh, w, budget_s=args.cpu_budget)
     return out
+
+
+def _lists_host(lists):
+    nnz = lists.nnz()
+    return lists.row_ptr.cpu().numpy().astype(np.int64), lists.col_idx[:nnz].cpu().numpy()
+
+
+def _plant_recall(rp, ci, plants, Hq, nqb, block=BLOCK):
+    """Fraction of planted keys whose key block is listed for the planted query's row."""
+    hit = 0
+    for (b, _h, j, _pos_k, q_head, q_tok) in plants:
+        row = (b * Hq + q_head) * nqb + q_tok // block
+        seg = ci[rp[row]:rp[row + 1]]
+        k = np.searchsorted(seg, j)
+        hit += int(k < seg.size and seg[k] == j)
+    return hit / max(1, len(plants))
+
+
+def selector_quality_measure(rbs, Q, C, R, lists, plants, B, Hq, nqb, nkb, rho, block=BLOCK):
+    """Selector diagnostics on the benchmark prompt (no number in the sources
+    to compare with; reported, not pinned): recall of the planted keys' blocks
+    by the two-branch selection, the same recall for centroid-only selection
+    (beta = 0, so the rescue branch repeats the centroid branch) at the same
+    kept density (its rho found by bisection), and the share of kept entries
+    that only the rescue branch chose."""
+    import torch
+    rp, ci = _lists_host(lists)
+    visible = B * Hq * nqb * (nqb + 1) // 2
+    dens_rbs = ci.size / visible
+    flags = lists.flags[:ci.size].cpu().numpy() if lists.flags is not None else None
+    rescue_only = float(np.mean(flags == 2)) if flags is not None else None
+    recall_rbs = _plant_recall(rp, ci, plants, Hq, nqb, block)
+    p_full = rbs.SelectParams(block_q=block, block_k=block, rho_centroid=1.0, rho_rescue=1.0)
+    cap = rbs.rbs_select_capacity(B, Hq, nqb, nkb, p_full)
+    out = rbs.BlockLists.empty(B * Hq * nqb, cap, "cuda")
+    wsb = torch.empty(rbs.rbs_select_workspace_bytes(B, Hq, nqb, C.shape[1], nkb, p_full), dtype=torch.uint8,
+                      device="cuda")
+
+    def centroid_only(r):
+        p = rbs.SelectParams(block_q=block, block_k=block, rho_centroid=r, rho_rescue=r, beta_mode=1, beta_const=0.0)
+        rbs.rbs_select(Q, C, R, p, workspace=wsb, out=out)
+        return out.nnz() / visible
+
+    lo, hi, r = 0.0, 1.0, rho
+    for _ in range(30):
+        r = float(np.float32(0.5 * (lo + hi)))
+        d = centroid_only(r)
+        if abs(d - dens_rbs) <= 0.0025:
+            break
+        if d < dens_rbs:
+            lo = r
+        else:
+            hi = r
+    dens_c = centroid_only(r)
+    rp2, ci2 = _lists_host(out)
+    recall_c = _plant_recall(rp2, ci2, plants, Hq, nqb, block)
+    assert rbs.rbs_get_device_error() == 0
+    return {"planted_keys": len(plants), "rbs": {"rho_per_branch": rho, "density": round(dens_rbs, 5),
+                                                 "planted_block_recall": round(recall_rbs, 4),
+                                                 "rescue_only_share": None if rescue_only is None else round(rescue_only, 4)},
+            "centroid_only_equal_density": {"rho": r, "density": round(dens_c, 5),
+                                            "planted_block_recall": round(recall_c, 4)},
+            "note": "diagnostic: the sources print no value for these"}
+
+
+def tiny_selector_quality(rbs):
+    """The same diagnostics on the tiny workload (4K tokens, 64-token blocks,
+    rho = 0.25 per branch, one planted key in every 16th key block)."""
+    wt = WORKLOADS["tiny_rbs_4k"]
+    it = make_inputs(wt)
+    Qt, Kt = to_dev(it["Q"]), to_dev(it["K"])
+    B, L, Hq, _ = Qt.shape
+    nb = L // wt.block
+    Ct, Rt = rbs.rbs_block_stats(Kt, wt.block)
+    p = rbs.SelectParams(block_q=wt.block, block_k=wt.block, rho_centroid=wt.rho, rho_rescue=wt.rho)
+    lt = rbs.rbs_select(Qt, Ct, Rt, p)
+    return selector_quality_measure(rbs, Qt, Ct, Rt, lt, it["plants"], B, Hq, nb, nb, wt.rho, wt.block)
 
 
 def isolated_bandwidth_measure(rbs, lib, tK, tQ, C, R, pc, lc, ws_buf, Hkv, nkb, stats_bytes, select_bytes, peaks):
@@ -612,6 +693,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-density-sweep", dest="density_sweep", action="store_false")
     ap.add_argument("--no-isolated", dest="isolated", action="store_false")
+    ap.add_argument("--no-selector-quality", dest="selector_quality", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--seq-len", type=int, default=None,

@@ -1,0 +1,24 @@
+"""Host-side helpers of bench.py (no GPU): the planted-key recall count."""
+
+import numpy as np
+
+import bench
+
+
+def test_plant_recall_counts_listed_blocks():
+    # 1 batch, 2 q heads, 4 query blocks of 128 tokens: rows are (head, query block)
+    Hq, nqb = 2, 4
+    lists = {0: [0], 1: [0, 1], 2: [1, 2], 3: [0, 3], 4: [0], 5: [1], 6: [0, 2], 7: [3]}
+    rp = np.zeros(Hq * nqb + 1, dtype=np.int64)
+    ci = []
+    for row in range(Hq * nqb):
+        ci += lists[row]
+        rp[row + 1] = len(ci)
+    ci = np.array(ci, dtype=np.int32)
+    # plants: (b, kv head, key block, key pos, q head, query token)
+    plants = [(0, 0, 2, 300, 0, 2 * 128 + 5),   # row 2 lists block 2: hit
+              (0, 0, 1, 200, 1, 3 * 128 + 1),   # row 7 lists only block 3: miss
+              (0, 0, 0, 10, 1, 2 * 128 + 64),   # row 6 lists block 0: hit
+              (0, 0, 2, 290, 0, 3 * 128 + 9)]   # row 3 lists blocks 0, 3: miss
+    assert bench._plant_recall(rp, ci, plants, Hq, nqb) == 0.5
+    assert bench._plant_recall(rp, ci, [], Hq, nqb) == 0.0
