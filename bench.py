@@ -264,7 +264,8 @@ def run_ours(args, ws, rank):
     if args.selector_quality and rank == 0:
         out["selector_quality"] = {
             WORKLOAD: selector_quality_measure(rbs, Q, C, R, lists, inp["plants"], B, Hq, nqb, nkb, w.rho),
-            "tiny_rbs_4k": tiny_selector_quality(rbs)}
+            "tiny_rbs_4k": tiny_selector_quality(rbs),
+            "mixture_8k": mixture_selector_quality(rbs)}
     if args.e2e:
         out["e2e"] = e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn=None, ctx=dict(
             C=C, R=R, lists=lists, ws_buf=ws_buf, pc=pc, lc=lc, Hkv=Hkv, nkb=nkb, flops=flops, ws=ws))
@@ -357,7 +358,59 @@ def tiny_selector_quality(rbs):
     Ct, Rt = rbs.rbs_block_stats(Kt, wt.block)
     p = rbs.SelectParams(block_q=wt.block, block_k=wt.block, rho_centroid=wt.rho, rho_rescue=wt.rho)
     lt = rbs.rbs_select(Qt, Ct, Rt, p)
-    return selector_quality_measure(rbs, Qt, Ct, Rt, lt, it["plants"], B, Hq, nb, nb, wt.rho, wt.block)
+    res = selector_quality_measure(rbs, Qt, Ct, Rt, lt, it["plants"], B, Hq, nb, nb, wt.rho, wt.block)
+    res["top5pct_attention_blocks_by_radius_quintile"] = radius_quintile_share(Qt, to_dev(it["K"]), Rt, wt.block)
+    return res
+
+
+def mixture_selector_quality(rbs):
+    """The diagnostics, with the attention-mass quintiles, on the benchmark's
+    compact/dispersed key mixture at a size where dense attention is cheap:
+    8192 tokens, 8 q / 1 KV head, 128-token blocks, rho = 0.05 per branch."""
+    from workloads import make_mixture
+    it = make_mixture(8192, 8, 1, BLOCK, seed=WORKLOADS[WORKLOAD].seed)
+    Qt, Kt = to_dev(it["Q"]), to_dev(it["K"])
+    B, L, Hq, _ = Qt.shape
+    nb = L // BLOCK
+    Ct, Rt = rbs.rbs_block_stats(Kt, BLOCK)
+    rho = WORKLOADS[WORKLOAD].rho
+    lt = rbs.rbs_select(Qt, Ct, Rt, rbs.SelectParams(block_q=BLOCK, block_k=BLOCK, rho_centroid=rho, rho_rescue=rho))
+    res = selector_quality_measure(rbs, Qt, Ct, Rt, lt, it["plants"], B, Hq, nb, nb, rho)
+    res["top5pct_attention_blocks_by_radius_quintile"] = radius_quintile_share(Qt, Kt, Rt, BLOCK)
+    return res
+
+
+def radius_quintile_share(Q, K, R, block):
+    """Of the 5% of causally visible (query block, key block) pairs that carry
+    the most attention mass (dense causal softmax attention, mass of a pair =
+    the block's summed probability averaged over the query block's tokens),
+    the share whose key block lies in each quintile of that KV head's block
+    radii (smallest radii first).  Equal shares (0.2 each) would mean the
+    radius says nothing about where attention mass sits."""
+    import torch
+    B, L, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    G = Hq // Hkv
+    nb = L // block
+    tri = torch.ones(L, L, dtype=torch.bool, device=Q.device).tril()
+    vis = torch.ones(nb, nb, dtype=torch.bool, device=Q.device).tril()
+    masses, quint = [], []
+    for b in range(B):
+        for hq in range(Hq):
+            kvh = hq // G
+            s = (Q[b, :, hq].float() @ K[b, :, kvh].float().T) / math.sqrt(d)
+            prob = torch.softmax(s.masked_fill(~tri, float("-inf")), dim=1)
+            mass = prob.view(nb, block, nb, block).sum(3).mean(1)  # [query block, key block]
+            r = R[b, kvh]
+            edges = torch.quantile(r, torch.tensor([0.2, 0.4, 0.6, 0.8], device=r.device))
+            q = torch.bucketize(r, edges)  # 0..4 per key block
+            masses.append(mass[vis])
+            quint.append(q.expand(nb, nb)[vis])
+    m = torch.cat(masses)
+    qv = torch.cat(quint)
+    top = m >= torch.quantile(m, 0.95)
+    counts = torch.bincount(qv[top], minlength=5).float()
+    return [round(float(c), 4) for c in (counts / counts.sum()).tolist()]
 
 
 def isolated_bandwidth_measure(rbs, lib, tK, tQ, C, R, pc, lc, ws_buf, Hkv, nkb, stats_bytes, select_bytes, peaks):

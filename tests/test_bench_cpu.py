@@ -22,3 +22,15 @@ def test_plant_recall_counts_listed_blocks():
               (0, 0, 2, 290, 0, 3 * 128 + 9)]   # row 3 lists blocks 0, 3: miss
     assert bench._plant_recall(rp, ci, plants, Hq, nqb) == 0.5
     assert bench._plant_recall(rp, ci, [], Hq, nqb) == 0.0
+
+
+def test_radius_quintile_share_is_a_distribution():
+    import torch
+    g = torch.Generator().manual_seed(5)
+    Q = torch.randn(1, 512, 2, 128, generator=g)
+    K = torch.randn(1, 512, 1, 128, generator=g)
+    R = torch.rand(1, 1, 8, generator=g)
+    share = bench.radius_quintile_share(Q, K, R, 64)
+    assert len(share) == 5
+    assert abs(sum(share) - 1.0) < 1e-3
+    assert all(0.0 <= x <= 1.0 for x in share)
