@@ -120,24 +120,34 @@ def dist_setup():
     return ws, rank, local
 
 
-def barrier_max(x: float, ws: int) -> float:
+def _reduce(x: float, ws: int, op: str) -> float:
+    """x reduced over all ranks (max or sum); the identity at ws == 1.  The
+    tensor lives where the process group's backend needs it (CUDA for NCCL,
+    host memory for gloo)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def barrier_max(x: float, ws: int) -> float:
+    return _reduce(x, ws, "max")
 
 
 def barrier_sum(x: float, ws: int) -> float:
-    if ws == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(x, ws, "sum")
+
+
+def aggregate(step_ms: float, flops: float, ws: int) -> tuple[float, float, float]:
+    """Whole-job figures of a weak-scaling run: the slowest rank's step time,
+    the FLOPs of all ranks, and the job's TFLOP/s = all FLOPs / slowest time."""
+    ms = barrier_max(step_ms, ws)
+    total = barrier_sum(flops, ws)
+    return ms, total, total / (ms * 1e-3) / 1e12
 
 
 def sync_all(ws: int):
@@ -225,9 +235,7 @@ def run_ours(args, ws, rank):
     stats_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     select_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    step_ms = barrier_max(total_ms / args.steps, ws)
-    all_flops = barrier_sum(float(flops), ws)
-    value = all_flops / (step_ms * 1e-3) / 1e12
+    step_ms, all_flops, value = aggregate(total_ms / args.steps, float(flops), ws)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
 
