@@ -83,6 +83,12 @@ class SelectParams:
     force_sink: int = 0
     causal: int = 1
     q_block_offset: int = 0  # global index of query block 0 (in key blocks)
+    # threshold rule per branch: 0 = TOPK_FRACTION (keep the top k_i), 1 =
+    # MAX_RELATIVE (keep every visible block scoring at least the row's
+    # maximum minus delta, no ranking)
+    threshold_mode: int = 0
+    delta_centroid: float = 0.0
+    delta_rescue: float = 0.0
 
 
 FLAG_CENTROID = 1
@@ -225,6 +231,13 @@ def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, 
     sorted ascending.  flags: bit0 centroid kept, bit1 rescue kept, bit2 forced.
     Also returns each row's per-branch threshold tau (the k_i-th kept score)
     and, with keep_scores, the score matrices (for the near-threshold rule).
+
+    threshold_mode 1 replaces each branch's top-k by a threshold relative to
+    the row maximum, tau = max_j s(i, j) - delta_branch: every visible block
+    with s >= tau is kept (the max-based dynamic thresholding [RBS-en] "How
+    This Fits Into the Broader Sparse Attention Landscape" describes as an
+    alternative to ranking, with the rescue branch layered on it).  k then
+    reports the kept count.
     """
     B, L, Hq, d = Q.shape
     _, Hkv, nkb, _ = C.shape
@@ -245,11 +258,19 @@ def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, 
                 scores[(b, hq)] = (s_c, s_r)
             for i in range(nqb):
                 n = visible_blocks(i, nkb, p)
-                kc = keep_count(p.rho_centroid, n)
-                kr = keep_count(p.rho_rescue, n)
-                top_c = top_k_desc(s_c[i, :n], kc)
-                top_r = top_k_desc(s_r[i, :n], kr)
-                tau[b, hq, i] = (s_c[i, top_c[-1]], s_r[i, top_r[-1]])
+                if p.threshold_mode == 1:
+                    t_c = s_c[i, :n].max() - p.delta_centroid
+                    t_r = s_r[i, :n].max() - p.delta_rescue
+                    top_c = np.nonzero(s_c[i, :n] >= t_c)[0]
+                    top_r = np.nonzero(s_r[i, :n] >= t_r)[0]
+                    kc, kr = top_c.size, top_r.size
+                    tau[b, hq, i] = (t_c, t_r)
+                else:
+                    kc = keep_count(p.rho_centroid, n)
+                    kr = keep_count(p.rho_rescue, n)
+                    top_c = top_k_desc(s_c[i, :n], kc)
+                    top_r = top_k_desc(s_r[i, :n], kr)
+                    tau[b, hq, i] = (s_c[i, top_c[-1]], s_r[i, top_r[-1]])
                 kept_k[b, hq, i] = (kc, kr)
                 f = np.zeros(nkb, dtype=np.uint8)
                 f[top_c] |= FLAG_CENTROID

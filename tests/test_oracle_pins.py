@@ -472,3 +472,55 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "rope_rotate", transposed)
     with pytest.raises(AssertionError):
         test_rope_matches_complex_rotation()
+
+
+# ---- max-relative threshold mode ([RBS-en] "How This Fits Into the Broader
+# Sparse Attention Landscape": thresholding against the row maximum, no sort)
+
+
+def test_max_relative_hand_built_scores():
+    # Every key of block j is v_j * e_0 (radius 0, so both branches score
+    # v_j); every query is e_0, so s(i, j) = v_j exactly.
+    d, blk, nb = 128, 16, 6
+    v = np.array([1.0, 5.0, 4.5, 2.0, 4.9, 0.5])
+    K = np.zeros((1, nb * blk, 1, d))
+    for j in range(nb):
+        K[0, j * blk:(j + 1) * blk, 0, 0] = v[j]
+    Q = np.zeros((1, nb * blk, 1, d))
+    Q[..., 0] = 1.0
+    C, R = O.block_stats(K, blk)
+    assert np.allclose(R, 0.0)
+    p = O.SelectParams(block_q=blk, block_k=blk, threshold_mode=1, delta_centroid=0.55, delta_rescue=0.15,
+                       force_diag=0)
+    sel = O.select_blocks(Q, C, R, p)
+    rp, ci, fl = sel["row_ptr"], sel["col_idx"], sel["flags"]
+    # row i sees blocks 0..i; centroid keeps v_j >= max - 0.55, rescue v_j >= max - 0.15
+    want_c = {0: [0], 1: [1], 2: [1, 2], 3: [1, 2], 4: [1, 2, 4], 5: [1, 2, 4]}
+    want_r = {0: [0], 1: [1], 2: [1], 3: [1], 4: [1, 4], 5: [1, 4]}
+    for i in range(nb):
+        cols = ci[rp[i]:rp[i + 1]]
+        f = fl[rp[i]:rp[i + 1]]
+        assert cols[(f & O.FLAG_CENTROID) > 0].tolist() == want_c[i]
+        assert cols[(f & O.FLAG_RESCUE) > 0].tolist() == want_r[i]
+        assert sel["k"][0, 0, i].tolist() == [len(want_c[i]), len(want_r[i])]
+
+
+def test_max_relative_zero_delta_is_top1_and_infinite_delta_is_full():
+    inp = _tiny(L=512)
+    top1, *_ = _select(inp, rho_centroid=1e-6, rho_rescue=1e-6)  # k = 1 per branch
+    zero, *_ = _select(inp, threshold_mode=1, delta_centroid=0.0, delta_rescue=0.0)
+    assert np.array_equal(top1["row_ptr"], zero["row_ptr"]) and np.array_equal(top1["col_idx"], zero["col_idx"])
+    assert np.array_equal(top1["flags"], zero["flags"])
+    full, C, *_ = _select(inp, threshold_mode=1, delta_centroid=np.inf, delta_rescue=np.inf)
+    rp, ci = O.causal_full_lists(1, inp["Q"].shape[2], C.shape[2])
+    assert np.array_equal(full["row_ptr"], rp) and np.array_equal(full["col_idx"], ci)
+
+
+def test_max_relative_nested_in_delta():
+    inp = _tiny(L=512)
+    small, *_ = _select(inp, threshold_mode=1, delta_centroid=5.0, delta_rescue=5.0)
+    big, *_ = _select(inp, threshold_mode=1, delta_centroid=20.0, delta_rescue=20.0)
+    for row in range(small["row_ptr"].size - 1):
+        a = set(small["col_idx"][small["row_ptr"][row]:small["row_ptr"][row + 1]].tolist())
+        b = set(big["col_idx"][big["row_ptr"][row]:big["row_ptr"][row + 1]].tolist())
+        assert a <= b
