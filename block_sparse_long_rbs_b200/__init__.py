@@ -52,6 +52,9 @@ class SelectParams:
     force_sink: int = 0
     causal: int = 1
     q_block_offset: int = 0
+    threshold_mode: int = 0  # 0 = top-k fraction, 1 = within delta of the row maximum
+    delta_centroid: float = 0.0
+    delta_rescue: float = 0.0
 
     def c(self) -> SelectParamsC:
         return SelectParamsC(*[getattr(self, f.name) for f in dataclasses.fields(self)])

@@ -31,7 +31,8 @@ class SelectParamsC(ctypes.Structure):
     _fields_ = [("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32), ("rho_centroid", ctypes.c_float),
                 ("rho_rescue", ctypes.c_float), ("beta_mode", ctypes.c_int32), ("beta_const", ctypes.c_float),
                 ("beta_p_lo", ctypes.c_float), ("beta_p_hi", ctypes.c_float), ("force_diag", ctypes.c_int32),
-                ("force_sink", ctypes.c_int32), ("causal", ctypes.c_int32), ("q_block_offset", ctypes.c_int32)]
+                ("force_sink", ctypes.c_int32), ("causal", ctypes.c_int32), ("q_block_offset", ctypes.c_int32),
+                ("threshold_mode", ctypes.c_int32), ("delta_centroid", ctypes.c_float), ("delta_rescue", ctypes.c_float)]
 
 
 class BlockListsC(ctypes.Structure):

@@ -222,6 +222,9 @@ void rbs_select_params_default(rbs_select_params* p) {
   p->force_sink = 0;
   p->causal = 1;
   p->q_block_offset = 0;
+  p->threshold_mode = 0;
+  p->delta_centroid = 0.0f;
+  p->delta_rescue = 0.0f;
 }
 
 rbs_status rbs_get_device_error(int32_t* code_host, rbs_stream_t stream) {
@@ -310,7 +313,9 @@ int64_t rbs_select_capacity(int64_t batch, int64_t heads_q, int64_t num_q_blocks
     const int64_t gi = i + p->q_block_offset;
     const int64_t n = p->causal ? std::min<int64_t>(num_kv_blocks, gi + 1) : num_kv_blocks;
     if (n <= 0) continue;
-    int64_t c = keep_count_host(p->rho_centroid, n) + keep_count_host(p->rho_rescue, n);
+    // MAX_RELATIVE keeps an unbounded number: every visible block may be kept
+    int64_t c = p->threshold_mode == 1 ? n
+                                       : keep_count_host(p->rho_centroid, n) + keep_count_host(p->rho_rescue, n);
     c += (p->force_diag && gi < num_kv_blocks) ? 1 : 0;
     c += p->force_sink ? 1 : 0;
     per_head += std::min<int64_t>(n, c);
@@ -337,8 +342,12 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   RBS_REQUIRE(kv_heads > 0 && Q->heads % kv_heads == 0, RBS_ERR_INVALID_ARG, "heads_q %% kv_heads != 0");
   RBS_REQUIRE(num_kv_blocks > 0 && num_kv_blocks <= RBS_MAX_KV_BLOCKS, RBS_ERR_UNSUPPORTED,
               "num_kv_blocks must be in [1, %d]", RBS_MAX_KV_BLOCKS);
-  RBS_REQUIRE(p->rho_centroid > 0.f && p->rho_centroid <= 1.f && p->rho_rescue > 0.f && p->rho_rescue <= 1.f,
+  RBS_REQUIRE(p->threshold_mode == 0 || p->threshold_mode == 1, RBS_ERR_INVALID_ARG, "threshold_mode must be 0 or 1");
+  RBS_REQUIRE(p->threshold_mode == 1 ||
+                  (p->rho_centroid > 0.f && p->rho_centroid <= 1.f && p->rho_rescue > 0.f && p->rho_rescue <= 1.f),
               RBS_ERR_INVALID_ARG, "rho must be in (0, 1]");
+  RBS_REQUIRE(p->threshold_mode == 0 || (p->delta_centroid >= 0.f && p->delta_rescue >= 0.f),
+              RBS_ERR_INVALID_ARG, "delta must be >= 0 (and not NaN)");
   RBS_REQUIRE(p->q_block_offset >= 0, RBS_ERR_INVALID_ARG, "q_block_offset < 0");
   RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
   const int64_t B = Q->batch, Hq = Q->heads, nqb = Q->seqlen / p->block_q, nkb = num_kv_blocks;
@@ -380,6 +389,9 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   sa.causal = p->causal;
   sa.force_diag = p->force_diag;
   sa.force_sink = p->force_sink;
+  sa.threshold_mode = p->threshold_mode;
+  sa.delta_c = p->delta_centroid;
+  sa.delta_r = p->delta_rescue;
   sa.rho_c = p->rho_centroid;
   sa.rho_r = p->rho_rescue;
   sa.mask_c = reinterpret_cast<uint32_t*>(ws + lay.mask_c);

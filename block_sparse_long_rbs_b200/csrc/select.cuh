@@ -39,6 +39,8 @@ struct SelectArgs {
   int Hq, Hkv, nqb, nkb, R, nwords;
   int q_block_offset, causal, force_diag, force_sink;
   float rho_c, rho_r;
+  int threshold_mode;    // 0 = top-k fraction, 1 = within delta of the row maximum
+  float delta_c, delta_r;
   uint32_t* mask_c;  // [rows, nwords]
   uint32_t* mask_r;  // [rows, nwords]
   int* counts;       // [rows]
@@ -236,24 +238,54 @@ __device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float
     const int j = 32 * t + lane;
     return j < n ? order_key(fmaf(qnv, rb[j], srow[j])) : 0u;
   };
-  const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
-  const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, scratch, words_c, words_r);
-  if (!done) {
-    uint32_t kc[KP], kr[KP];
-#pragma unroll
-    for (int t = 0; t < KP; ++t) {
-      kc[t] = key_c(t);
-      kr[t] = key_r(t);
+  if (a.threshold_mode == 1) {
+    // Each branch keeps every visible block scoring at least its row maximum
+    // minus delta; the threshold is formed in fp32 from the maximum score.
+    float mc = -INFINITY, mr = -INFINITY;
+    for (int j = lane; j < n; j += 32) {
+      mc = fmaxf(mc, srow[j]);
+      mr = fmaxf(mr, fmaf(qnv, rb[j], srow[j]));
     }
-    constexpr int NO = (KP + 31) / 32;
-    uint32_t own_c[NO], own_r[NO];
-    warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+      mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+    }
+    const uint32_t tc = order_key(mc - a.delta_c), tr = order_key(mr - a.delta_r);
     for (int w = lane; w < a.nwords; w += 32) {
-      const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
-      words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
-      words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+      uint32_t wc = 0, wr = 0;
+      for (int bit = 0; bit < 32; ++bit) {
+        const int j = 32 * w + bit;
+        if (j < n) {
+          const float sv = srow[j];
+          if (order_key(sv) >= tc) wc |= 1u << bit;
+          if (order_key(fmaf(qnv, rb[j], sv)) >= tr) wr |= 1u << bit;
+        }
+      }
+      words_c[w] = wc;
+      words_r[w] = wr;
     }
     __syncwarp();
+  } else {
+    const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
+    const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, scratch, words_c, words_r);
+    if (!done) {
+      uint32_t kc[KP], kr[KP];
+#pragma unroll
+      for (int t = 0; t < KP; ++t) {
+        kc[t] = key_c(t);
+        kr[t] = key_r(t);
+      }
+      constexpr int NO = (KP + 31) / 32;
+      uint32_t own_c[NO], own_r[NO];
+      warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
+      for (int w = lane; w < a.nwords; w += 32) {
+        const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
+        words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+        words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+      }
+      __syncwarp();
+    }
   }
   int cnt = 0;
   for (int t = lane; t < a.nwords; t += 32) {

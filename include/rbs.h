@@ -59,7 +59,7 @@ extern "C" {
 #define RBS_API
 #endif
 
-#define RBS_ABI_VERSION 1
+#define RBS_ABI_VERSION 2
 #define RBS_HEAD_DIM 128
 #define RBS_MAX_SEGMENTS 512 /* Block-attention segments per call */
 #define RBS_MAX_KV_BLOCKS 4096 /* key blocks per sequence for rbs_select */
@@ -106,6 +106,14 @@ typedef struct {
  *   causal             query block i (global index i + q_block_offset) may
  *                      select key blocks 0 .. i + q_block_offset only (1)
  *   q_block_offset     global key-block index of query block 0 (0)
+ *   threshold_mode     0 = TOPK_FRACTION: each branch keeps its top
+ *                      ceil(rho * n_i) as above; 1 = MAX_RELATIVE: each branch
+ *                      keeps every visible block whose score is at least the
+ *                      row's maximum score minus delta_centroid / delta_rescue
+ *                      (no ranking; [RBS-en] "How This Fits Into the Broader
+ *                      Sparse Attention Landscape") (0)
+ *   delta_centroid, delta_rescue  MAX_RELATIVE margins in raw score units,
+ *                      >= 0 (0, 0)
  * Scores are raw dot products (no 1/sqrt(d)); ties between equal scores go
  * to the lower block index.  Forced blocks do not count toward a branch's k.
  */
@@ -117,6 +125,8 @@ typedef struct {
   float beta_p_lo, beta_p_hi;
   int32_t force_diag, force_sink, causal;
   int32_t q_block_offset;
+  int32_t threshold_mode;
+  float delta_centroid, delta_rescue;
 } rbs_select_params;
 
 /* Per-query-block key-block lists in CSR form (all device memory). */
@@ -171,7 +181,8 @@ RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, f
  *   s_c(j) = qbar_i . c_j                      (centroid branch)
  *   s_r(j) = s_c(j) + ||qbar_i|| * r_j * beta_j  (rescue branch)
  * over the visible key blocks j (j <= i + q_block_offset when causal); each
- * branch keeps its own top ceil(rho * n_i) blocks; the row's list is the
+ * branch keeps its own top ceil(rho * n_i) blocks (or, in MAX_RELATIVE mode,
+ * the blocks within its delta of the row maximum); the row's list is the
  * union of both kept sets plus the forced blocks, ascending.
  *   Q            [B, Lq, Hq, 128] bf16, Lq a multiple of block_q
  *   centroids    [B, Hkv, num_kv_blocks, 128] fp32 (rbs_block_stats)

@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_housekeeping(L):
-    assert L.rbs_abi_version() == 1
+    assert L.rbs_abi_version() == 2
     assert L.rbs_status_string(0) == b"ok"
     assert L.rbs_status_string(3) == b"capacity"
     p = _abi.SelectParamsC()
@@ -164,3 +164,27 @@ def test_rope_validation(L):
     assert L.rope_reencode(ctypes.byref(x), ctypes.byref(x), None, 0x2000, 5e5, 0, s) == 1
     assert L.rope_reencode(ctypes.byref(x), ctypes.byref(x), 0x1000, 0x2000, 5e5, 2, s) == 1
     assert L.rope_reencode(ctypes.byref(x), ctypes.byref(x), 0x1000, 0x2000, -1.0, 0, s) == 1
+
+
+def test_max_relative_capacity_is_every_visible_block(L):
+    p = SelectParams(threshold_mode=1, delta_centroid=1.0, delta_rescue=2.0)
+    cap = L.rbs_select_capacity(1, 2, 16, 16, ctypes.byref(p.c()))
+    assert cap == 2 * sum(i + 1 for i in range(16))
+
+
+def test_select_rejects_bad_threshold_fields(L):
+    q = _fake(Lq=512)
+    rows = 1 * 2 * 8
+    ok = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, rows)
+    for kw in ({"threshold_mode": 2}, {"threshold_mode": 1, "delta_centroid": -1.0},
+               {"threshold_mode": 1, "delta_rescue": float("nan")}):
+        pc = SelectParams(block_q=64, block_k=64, **kw).c()
+        st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, 1 << 20,
+                          ctypes.byref(ok), None, None)
+        assert st == 1, kw
+    # MAX_RELATIVE ignores rho (it may be zero)
+    pc = SelectParams(block_q=64, block_k=64, rho_centroid=0.0, rho_rescue=0.0, threshold_mode=1,
+                      delta_centroid=1.0, delta_rescue=1.0).c()
+    st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, 1 << 20,
+                      ctypes.byref(ok), None, None)
+    assert st == 4  # past validation: no GPU here

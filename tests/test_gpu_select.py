@@ -34,7 +34,7 @@ def _run(inp, block, rho_c, rho_r, **kw):
                         rho_rescue=float(np.float32(rho_r)), **{k: (float(np.float32(v)) if isinstance(v, float) else v)
                                                                 for k, v in kw.items()})
     ora = O.select_blocks(Q, Co, Ro, po, keep_scores=True)
-    return compare_selection(lists, ora, Hq, nqb, nkb)
+    return compare_selection(lists, ora, Hq, nqb, nkb, exact_k=kw.get("threshold_mode", 0) == 0)
 
 
 def test_select_tiny_config(cuda_ok):
@@ -99,3 +99,16 @@ def test_select_rho_one_is_causal_full(cuda_ok):
     f = rbs.rbs_lists_causal_full(1, 2, 16, 0)
     assert torch.equal(s.row_ptr, f.row_ptr)
     assert torch.equal(s.col_idx[:s.nnz()], f.col_idx[:f.nnz()])
+
+
+@pytest.mark.parametrize("dc,dr", [(0.1, 0.5), (0.5, 2.0)])
+def test_select_max_relative_tiny(cuda_ok, dc, dr):
+    w = WORKLOADS["tiny_rbs_4k"]
+    rep = _run(make_inputs(w), 64, w.rho, w.rho, threshold_mode=1, delta_centroid=dc, delta_rescue=dr)
+    print("max-relative tiny", dc, dr, rep)
+
+
+def test_select_max_relative_mixture_gqa(cuda_ok):
+    inp = make_mixture(L=8192, Hq=16, Hkv=2, block=128, seed=201)
+    rep = _run(inp, 128, 0.05, 0.05, threshold_mode=1, delta_centroid=0.5, delta_rescue=2.0)
+    print("max-relative mixture", rep)
