@@ -5,7 +5,8 @@
 // Work item = one list row (batch b, q head h, query block i): a 128-row
 // query tile (BQ valid rows) against the row's listed key blocks, in list
 // order.  Persistent CTAs take non-empty work items round-robin in an order
-// that starts with the last query blocks (the longest causal rows).
+// that keeps one KV head's rows together and, within it, starts with the last
+// query blocks (the longest causal rows).
 //
 // One softmax pipeline with two S buffers in TMEM.  While the softmax warps
 // work on tile t, the tensor core computes S for tile t+1 and accumulates
@@ -136,13 +137,19 @@ enum : int {
 };
 static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
 
+// Work order: batch entry, then KV head, then query block from the last (the
+// longest causal rows first), then the G q heads sharing that KV head.  The
+// CTAs working at the same time therefore read the K/V tiles of one KV head,
+// which fit in L2 (64 MiB for 131072 tokens), instead of every head's.
 __device__ __forceinline__ void decode_work(const AttnArgs& a, int w, int& b, int& h, int& i, int& row) {
-  const int bh_count = a.B * a.Hq;
-  i = a.nqb - 1 - w / bh_count;
-  const int bh = w % bh_count;
-  b = bh / a.Hq;
-  h = bh % a.Hq;
-  row = bh * a.nqb + i;
+  const int G = a.Hq / a.Hkv;
+  const int per_b = a.Hq * a.nqb, per_kvh = G * a.nqb;
+  b = w / per_b;
+  const int rem = w % per_b;
+  const int kvh = rem / per_kvh, r2 = rem % per_kvh;
+  i = a.nqb - 1 - r2 / G;
+  h = kvh * G + r2 % G;
+  row = (b * a.Hq + h) * a.nqb + i;
 }
 
 // Row extent with validation (identical in every role): -1 for a corrupt row.
