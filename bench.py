@@ -46,6 +46,24 @@ FLOP_PER_PAIR = 4 * BLOCK * BLOCK * HEAD_DIM  # QK^T and PV on one 128x128 block
 # kernels one step launches: block stats; beta, scoring + top-k, scan, compaction; attention
 LAUNCHES_PER_STEP = 6
 SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
+# DRAM traffic of one 131072-token attention launch (dram__bytes_read.sum +
+# dram__bytes_write.sum, one single-pass ncu capture of the default workload;
+# profiles/launches_gqa_rbs_128k.md gives the command), valid for the kernel
+# sources with this digest; any other build reports null.
+ATTN_TRAFFIC_BYTES = 3.25e9 + 1.04e9
+ATTN_TRAFFIC_SOURCES = ("block_sparse_long_rbs_b200/csrc/attention.cuh", "block_sparse_long_rbs_b200/csrc/common.cuh")
+ATTN_TRAFFIC_DIGEST = "6d0eecb19f62cd80"
+
+
+def attn_traffic(seq_len: int):
+    import hashlib
+    if seq_len != WORKLOADS[WORKLOAD].seqlen:
+        return None
+    h = hashlib.sha256()
+    for f in ATTN_TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return ATTN_TRAFFIC_BYTES if h.hexdigest()[:16] == ATTN_TRAFFIC_DIGEST else None
 
 
 def load_peaks():
@@ -255,7 +273,7 @@ def run_ours(args, ws, rank):
         "selected_tflop": round(flops / 1e12, 4),
         "causal_exact_tflop": round((flops - diag_half) / 1e12, 4),
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(attn_tflops / peak, 4), "traffic": None,
+                     "frac": round(attn_tflops / peak, 4), "traffic": attn_traffic(L),
                      "kernel": "bsa_prefill_kernel<128,128>", "peak_kind": f"bf16 sustained ({peaks['source']})"},
         "kernels": {
             "block_stats": {"ms": round(stats_ms, 4), "gbs": round(stats_bytes / (stats_ms * 1e-3) / 1e9, 1),
