@@ -478,8 +478,12 @@ def isolated_bandwidth_measure(rbs, lib, tK, tQ, C, R, pc, lc, ws_buf, Hkv, nkb,
 
 
 def e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn, ctx):
-    """Same step through the same calls, with the inputs copied from pinned host
-    memory and the output copied back inside the timed region."""
+    """Same step through the same calls, with every step's inputs copied from
+    pinned host memory and its output O copied back inside the timed region.
+    Steps are pipelined over two device buffer sets and three streams (host
+    to device, compute, device to host), so step k's compute overlaps step
+    k+1's input copy and step k-1's output copy; the time is from the first
+    input copy's start to the last output copy's end."""
     import ctypes
     import torch
     from block_sparse_long_rbs_b200 import _stream, _t
@@ -487,40 +491,64 @@ def e2e_measure(args, rbs, lib, Qh, Kh, Vh, step_fn, ctx):
     Kp = torch.from_numpy(Kh.view(np.int16)).view(torch.bfloat16).pin_memory()
     Vp = torch.from_numpy(Vh.view(np.int16)).view(torch.bfloat16).pin_memory()
     Op = torch.empty_like(Qp).pin_memory()
-    Qd, Kd, Vd = torch.empty_like(Qp, device="cuda"), torch.empty_like(Kp, device="cuda"), torch.empty_like(Vp, device="cuda")
-    Od = torch.empty_like(Qd)
-    tQ, tK, tV, tO = _t(Qd, "Q"), _t(Kd, "K"), _t(Vd, "V"), _t(Od, "O")
+    bufs = []
+    for _ in range(2):
+        Qd, Kd, Vd = (torch.empty_like(Qp, device="cuda"), torch.empty_like(Kp, device="cuda"),
+                      torch.empty_like(Vp, device="cuda"))
+        Od = torch.empty_like(Qd)
+        bufs.append((Qd, Kd, Vd, Od, _t(Qd, "Q"), _t(Kd, "K"), _t(Vd, "V"), _t(Od, "O")))
     C, R, ws_buf, pc, lc = ctx["C"], ctx["R"], ctx["ws_buf"], ctx["pc"], ctx["lc"]
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {}
 
-    def step():
-        s = _stream()
-        Qd.copy_(Qp, non_blocking=True)
-        Kd.copy_(Kp, non_blocking=True)
-        Vd.copy_(Vp, non_blocking=True)
-        rbs.check(lib.rbs_block_stats(ctypes.byref(tK), BLOCK, C.data_ptr(), R.data_ptr(), s), "stats")
-        rbs.check(lib.rbs_select(ctypes.byref(tQ), C.data_ptr(), R.data_ptr(), ctx["Hkv"], ctx["nkb"],
-                                 ctypes.byref(pc), ws_buf.data_ptr(), ws_buf.numel(), ctypes.byref(lc), None, s), "select")
-        rbs.check(lib.bsa_prefill(ctypes.byref(tQ), ctypes.byref(tK), ctypes.byref(tV), ctypes.byref(lc), BLOCK, BLOCK,
-                                  0, 1.0 / math.sqrt(HEAD_DIM), 1, ctypes.byref(tO), None, s), "attn")
-        Op.copy_(Od, non_blocking=True)
+    def step(k):
+        Qd, Kd, Vd, Od, tQ, tK, tV, tO = bufs[k % 2]
+        ev[k] = [torch.cuda.Event() for _ in range(3)]  # inputs in, computed, output out
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(ev[k - 2][1])  # step k-2 no longer reads this buffer set
+            Qd.copy_(Qp, non_blocking=True)
+            Kd.copy_(Kp, non_blocking=True)
+            Vd.copy_(Vp, non_blocking=True)
+            ev[k][0].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev[k][0])
+            if k >= 2:
+                s_cmp.wait_event(ev[k - 2][2])  # step k-2's O has been copied out
+            s = _stream()
+            rbs.check(lib.rbs_block_stats(ctypes.byref(tK), BLOCK, C.data_ptr(), R.data_ptr(), s), "stats")
+            rbs.check(lib.rbs_select(ctypes.byref(tQ), C.data_ptr(), R.data_ptr(), ctx["Hkv"], ctx["nkb"],
+                                     ctypes.byref(pc), ws_buf.data_ptr(), ws_buf.numel(), ctypes.byref(lc), None, s),
+                      "select")
+            rbs.check(lib.bsa_prefill(ctypes.byref(tQ), ctypes.byref(tK), ctypes.byref(tV), ctypes.byref(lc), BLOCK,
+                                      BLOCK, 0, 1.0 / math.sqrt(HEAD_DIM), 1, ctypes.byref(tO), None, s), "attn")
+            ev[k][1].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev[k][1])
+            Op.copy_(Od, non_blocking=True)
+            ev[k][2].record(s_out)
 
     steps = max(3, min(args.steps, 10))
-    for _ in range(2):
-        step()
+    for k in range(2):
+        step(k)
+    torch.cuda.synchronize()
     sync_all(ctx["ws"])
+    ev.clear()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        step()
-    b.record()
+    a.record(s_in)
+    for k in range(steps):
+        step(k)
+    b.record(s_out)
     torch.cuda.synchronize()
     sync_all(ctx["ws"])
     ms = barrier_max(a.elapsed_time(b) / steps, ctx["ws"])
     flops = barrier_sum(float(ctx["flops"]), ctx["ws"])
+    del bufs
+    torch.cuda.empty_cache()
     return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": int(Qh.nbytes + Kh.nbytes + Vh.nbytes), "d2h_bytes_per_step": int(Qh.nbytes),
-            "steps": steps}
+            "steps": steps, "pipelined": "2 buffer sets, separate copy-in / compute / copy-out streams"}
 
 
 def dense_measure(rbs, Q, K, V, B, Hq, nqb, peak):
