@@ -66,6 +66,14 @@ def attn_traffic(seq_len: int):
     return ATTN_TRAFFIC_BYTES if h.hexdigest()[:16] == ATTN_TRAFFIC_DIGEST else None
 
 
+def bench_config(L: int, B: int, ws: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": f"{WORKLOAD}: L={L}, 32 q / 4 KV heads, head_dim 128, 128x128 blocks, causal, "
+                        f"rho=0.05 per branch", "batch": B, "seq_len": L,
+            "parallelism": "one prompt per GPU, no collective" if ws > 1 else "single GPU",
+            "l2": "inputs larger than L2 (Q 1 GiB, K and V 128 MiB each); no flush"}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -264,10 +272,7 @@ def run_ours(args, ws, rank):
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded compact/dispersed key mixture, planted keys)",
-        "config": {"workload": f"{WORKLOAD}: L={L}, 32 q / 4 KV heads, head_dim 128, 128x128 blocks, causal, "
-                               f"rho=0.05 per branch", "batch": B, "seq_len": L,
-                   "parallelism": "one prompt per GPU, no collective" if ws > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (Q 1 GiB, K and V 128 MiB each); no flush"},
+        "config": bench_config(L, B, ws),
         "attn_ms": round(attn_ms, 4), "attn_tflops": round(attn_tflops, 2), "select_ms": round(select_ms, 4),
         "stats_ms": round(stats_ms, 4), "nnz_pairs": nnz, "density": round(nnz / visible, 5),
         "selected_tflop": round(flops / 1e12, 4),
@@ -781,8 +786,7 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded compact/dispersed key mixture, planted keys)",
-            "config": {"workload": f"{WORKLOAD}: L=131072, 32 q / 4 KV heads, head_dim 128, 128x128 blocks, causal, "
-                                   f"rho=0.05 per branch", "batch": 1, "seq_len": 131072},
+            "config": bench_config(WORKLOADS[WORKLOAD].seqlen, 1, 1),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
                              "sample": base["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
