@@ -73,9 +73,9 @@ rbs_status device_info(DeviceInfo** out) {
                                      AttnSmem<64>::kAlloc);
 #define RBS_SEL_ATTR(KPL)                                                                                  \
   e = e ? e : cudaFuncSetAttribute(select_rows_kernel<KPL, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                   200 * 1024);                                                              \
+                                   static_cast<int>(sel_smem_bytes(RBS_MAX_KV_BLOCKS)));                     \
   e = e ? e : cudaFuncSetAttribute(select_rows_kernel<KPL, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                   200 * 1024);
+                                   static_cast<int>(sel_smem_bytes(RBS_MAX_KV_BLOCKS)));
     RBS_SEL_ATTR(2)
     RBS_SEL_ATTR(8)
     RBS_SEL_ATTR(32)
@@ -148,6 +148,35 @@ rbs_status make_tensor_map(const rbs_bf16_tensor* t, int rows, CUtensorMap* map,
   box[3] = 1;
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RBS_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return RBS_OK;
+}
+
+// 4-D map over [B, L, H, 128] bf16 for the selection's pooling: a box of
+// 64 dims x R heads x kPoolRows tokens, no swizzle (the token and head
+// dimensions ordered by stride as above).
+rbs_status make_pool_tensor_map(const rbs_bf16_tensor* t, int R, CUtensorMap* map, int* seq_inner) {
+  PFN_encodeTiled enc = encode_fn();
+  if (enc == nullptr) return fail(RBS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const bool si = t->stride_s < t->stride_h;
+  *seq_inner = si ? 1 : 0;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4], estr[4] = {1, 1, 1, 1};
+  dims[0] = RBS_HEAD_DIM;
+  box[0] = 64;
+  if (si) {
+    dims[1] = t->seqlen; strides[0] = t->stride_s * 2; box[1] = kPoolRows;
+    dims[2] = t->heads; strides[1] = t->stride_h * 2; box[2] = R;
+  } else {
+    dims[1] = t->heads; strides[0] = t->stride_h * 2; box[1] = R;
+    dims[2] = t->seqlen; strides[1] = t->stride_s * 2; box[2] = kPoolRows;
+  }
+  dims[3] = t->batch;
+  strides[2] = t->stride_b * 2;
+  box[3] = 1;
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(RBS_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return RBS_OK;
@@ -371,16 +400,18 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   int R = 1;
   for (int r = 1; r <= kSelMaxR; ++r)
     if (G % r == 0) R = r;
+  CUtensorMap qmap;
+  int seq_inner = 0;
+  if ((st = make_pool_tensor_map(Q, R, &qmap, &seq_inner)) != RBS_OK) return st;
   SelectArgs sa;
-  sa.Q = static_cast<const __nv_bfloat16*>(Q->data);
-  sa.qb = Q->stride_b;
-  sa.qs = Q->stride_s;
-  sa.qh = Q->stride_h;
   sa.C = centroids;
   sa.rad = radii;
   sa.beta = beta;
+  sa.B = static_cast<int>(B);
   sa.Hq = static_cast<int>(Hq);
   sa.Hkv = kv_heads;
+  sa.items = static_cast<int>(B * nqb * (Hq / R));
+  sa.seq_inner = seq_inner;
   sa.nqb = static_cast<int>(nqb);
   sa.nkb = static_cast<int>(nkb);
   sa.R = R;
@@ -398,20 +429,26 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   sa.mask_r = reinterpret_cast<uint32_t*>(ws + lay.mask_r);
   sa.counts = reinterpret_cast<int*>(ws + lay.counts);
   const int npad = static_cast<int>((nkb + 31) & ~31ll);
-  const size_t smem = (kSelMaxR * 128 + npad + kSelMaxR * npad + kStageJ * kStagePitch) * sizeof(float);
-  const dim3 grid(static_cast<unsigned>(nqb), static_cast<unsigned>(Hq / R), static_cast<unsigned>(B));
-#define RBS_SEL_LAUNCH(KPL)                                                             \
-  do {                                                                                   \
-    if (p->block_q == 128) select_rows_kernel<KPL, 128><<<grid, kSelThreads, smem, stream>>>(sa); \
-    else select_rows_kernel<KPL, 64><<<grid, kSelThreads, smem, stream>>>(sa);           \
-  } while (0)
+  const size_t smem = sel_smem_bytes(npad);
+  // persistent: as many CTAs as fit on the device at once, each walking the
+  // work items with a stride of the grid
+  auto launch = [&](auto kern) -> rbs_status {
+    int per_sm = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSelThreads, smem);
+    if (e != cudaSuccess || per_sm < 1) return fail(RBS_ERR_CUDA, "select_rows_kernel does not fit on an SM");
+    const int grid = static_cast<int>(std::min<int64_t>(sa.items, static_cast<int64_t>(per_sm) * di->sms));
+    kern<<<grid, kSelThreads, smem, stream>>>(qmap, sa);
+    return check_launch("select_rows_kernel");
+  };
+#define RBS_SEL_LAUNCH(KPL) \
+  st = p->block_q == 128 ? launch(select_rows_kernel<KPL, 128>) : launch(select_rows_kernel<KPL, 64>)
   if (nkb <= 64) RBS_SEL_LAUNCH(2);
   else if (nkb <= 256) RBS_SEL_LAUNCH(8);
   else if (nkb <= 1024) RBS_SEL_LAUNCH(32);
   else if (nkb <= 2048) RBS_SEL_LAUNCH(64);
   else RBS_SEL_LAUNCH(128);
 #undef RBS_SEL_LAUNCH
-  if ((st = check_launch("select_rows_kernel")) != RBS_OK) return st;
+  if (st != RBS_OK) return st;
 
   scan_counts_kernel<<<1, 1024, 0, stream>>>(sa.counts, static_cast<int>(rows), out->row_ptr, out->capacity);
   if ((st = check_launch("scan_counts_kernel")) != RBS_OK) return st;

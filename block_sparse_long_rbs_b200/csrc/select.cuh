@@ -7,20 +7,22 @@
 // blocks, and the rows are compacted into CSR lists.
 //
 // Kernels:
-//   select_rows_kernel  one CTA per (query block, group of R q heads of one
-//                       KV head, batch), longest rows (last query blocks)
-//                       first.  The CTA first pools its query block (mean of
-//                       the BQ queries of each of its R heads, streamed from
-//                       HBM with 16-byte loads), then computes the scores of
-//                       all visible blocks into shared memory (centroid tiles
-//                       of 256 blocks x 32 dims staged through shared memory,
-//                       the next tile's loads in flight while one is used),
-//                       then warp w < R finds, for both branches at
-//                       once, the exact k-th largest score of its row by a
-//                       32-step bitwise search over order-preserving keys held
-//                       in registers, breaks ties by block index with warp
-//                       ballots, and emits one 32-bit mask word per 32 blocks
-//                       (bit = lane).
+//   select_rows_kernel  persistent: CTA c walks the work items (query block
+//                       i, group of R q heads of one KV head, batch) c,
+//                       c + grid, ... in longest-row-first order.  Warps 8-9
+//                       pool the NEXT item's query block (mean of its BQ
+//                       queries per head) out of a TMA-fed ring of 8-row
+//                       chunks while warps 0-7 work on the current item:
+//                       centroid tiles of 512 blocks x 16 dims are staged
+//                       through shared memory (16-byte chunks swizzled so
+//                       both the stores and the row reads are conflict-free),
+//                       every thread forms the fp32 dot products of two
+//                       blocks with all R pooled queries, and then warp
+//                       w < R finds both branches' exact top-k of its row
+//                       (a pruned search over order-preserving keys, with a
+//                       full 32-step bitwise search as the fallback), breaks
+//                       ties by block index with warp ballots, and emits one
+//                       32-bit mask word per 32 blocks.
 //   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr.
 //   compact_lists_kernel one warp per row turns mask words into ascending
 //                       block indices and per-entry branch flags.
@@ -31,12 +33,12 @@
 namespace rbs {
 
 struct SelectArgs {
-  const __nv_bfloat16* Q;  // [B, Lq, Hq, 128]
-  int64_t qb, qs, qh;      // element strides
   const float* C;      // [B, Hkv, nkb, 128]
   const float* rad;    // [B, Hkv, nkb]
   const float* beta;   // [B, Hkv, nkb]
-  int Hq, Hkv, nqb, nkb, R, nwords;
+  int B, Hq, Hkv, nqb, nkb, R, nwords;
+  int items;           // B * nqb * (Hq / R)
+  int seq_inner;       // 1 when Q's token stride is smaller than its head stride
   int q_block_offset, causal, force_diag, force_sink;
   float rho_c, rho_r;
   int threshold_mode;    // 0 = top-k fraction, 1 = within delta of the row maximum
@@ -46,11 +48,36 @@ struct SelectArgs {
   int* counts;       // [rows]
 };
 
-constexpr int kSelThreads = 256;
+constexpr int kSelComputeThreads = 256;  // warps 0-7: scores and top-k
+constexpr int kSelPoolThreads = 64;      // warps 8-9: pooling of the next item
+constexpr int kSelThreads = kSelComputeThreads + kSelPoolThreads;
 constexpr int kSelMaxR = 8;
-constexpr int kStageJ = 256;  // key blocks per staged centroid tile (one per thread)
-constexpr int kStageD = 32;   // dims per staged centroid tile
-constexpr int kStagePitch = kStageD + 1;
+constexpr int kStageJ = 512;   // key blocks per staged centroid tile (two per compute thread)
+constexpr int kStageD = 16;    // dims per staged tile: 64-byte rows of four 16-byte chunks
+constexpr int kPoolRows = 8;   // query rows per TMA chunk
+constexpr int kPoolStages = 2;
+constexpr int kPoolChunkBytes = kPoolRows * kSelMaxR * 128 * 2;  // the largest chunk (R = 8)
+constexpr int kTopkCap = 128;  // candidates per branch in the pruned top-k (four per lane)
+
+// Dynamic shared memory of select_rows_kernel, in bytes from a 128-byte
+// aligned base: the chunk ring, the centroid staging tile (reused as top-k
+// scratch), two buffers of pooled queries [128][8], then r*beta [npad] and
+// the centroid-branch scores [8][npad].
+constexpr int kSelOffCs = kPoolStages * kPoolChunkBytes;
+constexpr int kSelOffQs = kSelOffCs + kStageJ * kStageD * 4;
+constexpr int kSelOffRb = kSelOffQs + 2 * 128 * kSelMaxR * 4;
+__host__ __device__ constexpr size_t sel_smem_bytes(int npad) {
+  return static_cast<size_t>(kSelOffRb) + static_cast<size_t>(1 + kSelMaxR) * npad * 4;
+}
+// top-k scratch of one warp: candidate keys and blocks of both branches,
+// then both branches' mask words
+__host__ __device__ constexpr int sel_topk_scratch_words(int nwords) { return 4 * kTopkCap + 2 * nwords; }
+static_assert(kSelComputeThreads / 32 * sel_topk_scratch_words(RBS_MAX_KV_BLOCKS / 32) * 4 <= kStageJ * kStageD * 4,
+              "top-k scratch must fit in the staging tile");
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -117,50 +144,57 @@ __device__ __forceinline__ void warp_topk2(const uint32_t (&kc)[KPL], const uint
   }
 }
 
+// Insert x into the descending list (t0 >= t1 >= t2 >= t3).
+__device__ __forceinline__ void top4_insert(uint32_t& t0, uint32_t& t1, uint32_t& t2, uint32_t& t3, uint32_t x) {
+  const uint32_t y0 = min(t0, x);
+  t0 = max(t0, x);
+  const uint32_t y1 = min(t1, y0);
+  t1 = max(t1, y0);
+  const uint32_t y2 = min(t2, y1);
+  t2 = max(t2, y1);
+  t3 = max(t3, y2);
+}
+
 // Exact top-k of both branches by pruning, for k <= 64 (key(t) = this
-// lane's key in slot t, block 32 t + lane, read from shared memory).  Each
-// lane's two largest keys form a 64-key subset of the row.  L is the largest
-// key with its low 16 bits clear such that at least k keys of the subset are
-// >= L; it is at most the subset's k-th largest key, hence at most the row's
-// k-th largest key T, so every key >= T is a candidate (key >= L).  When at
-// most 64 keys are candidates they are compacted in ascending block order
-// into shared memory, T is found among them by a bitwise search (the largest
-// T with at least k candidates >= T), the keys above T are kept and of the
-// ties at T the lowest block indices, and the kept blocks are OR-ed into
-// words[0, nwords) (cleared first).  Returns false, having written nothing
-// the caller uses, when k > 64 or more than 64 keys of a branch are
-// candidates (many near-equal keys); the caller then runs the full search.
-// Both branches advance together so their reduction chains overlap.
+// lane's key in slot t, block 32 t + lane, 0 for an absent slot).  Each lane
+// keeps its four largest keys per branch; that subset of the row holds at
+// least k present keys (all of them when n <= 128, 128 otherwise), so its
+// k-th largest key, rounded down to 24 bits (L), is at most the row's k-th
+// largest key T, and every key >= T is a candidate (key >= L).  When at most
+// kTopkCap keys of each branch are candidates they are compacted in
+// ascending block order into shared memory, T is found among them by a
+// bitwise search (the largest T with at least k candidates >= T), the keys
+// above T are kept and of the ties at T the lowest block indices, and the
+// kept blocks are OR-ed into words[0, nwords) (cleared first).  Returns
+// false, having written nothing the caller uses, when k > 64 or a branch has
+// more candidates (many near-equal keys); the caller then runs the full
+// search.  Both branches advance together so their reduction chains overlap.
 // Warp-uniform.
 template <int KP, typename KeyC, typename KeyR>
 __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_c, int k_r, int lane, int nwords,
                                                   uint32_t* scratch, uint32_t* words_c, uint32_t* words_r) {
   if (k_c > 64 || k_r > 64) return false;
-  uint32_t* ck_c = scratch;  // candidate keys [64] and blocks [64] of each branch
-  int* ci_c = reinterpret_cast<int*>(scratch + 64);
-  uint32_t* ck_r = scratch + 128;
-  int* ci_r = reinterpret_cast<int*>(scratch + 192);
-  uint32_t c1 = 0, c2 = 0, r1 = 0, r2 = 0;  // this lane's two largest keys per branch
+  uint32_t* ck_c = scratch;  // candidate keys and blocks of each branch
+  int* ci_c = reinterpret_cast<int*>(scratch + kTopkCap);
+  uint32_t* ck_r = scratch + 2 * kTopkCap;
+  int* ci_r = reinterpret_cast<int*>(scratch + 3 * kTopkCap);
+  uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0, r0 = 0, r1 = 0, r2 = 0, r3 = 0;
 #pragma unroll 4
   for (int t = 0; t < KP; ++t) {
-    const uint32_t uc = key_c(t), ur = key_r(t);
-    c2 = max(c2, min(c1, uc));
-    c1 = max(c1, uc);
-    r2 = max(r2, min(r1, ur));
-    r1 = max(r1, ur);
+    top4_insert(c0, c1, c2, c3, key_c(t));
+    top4_insert(r0, r1, r2, r3, key_r(t));
   }
-  // The subset holds at least k keys that are not absent (rows interleave
-  // blocks over the lanes), and a present key is >= 2^16, so L > 0 and no
-  // absent slot (key 0) becomes a candidate.
   uint32_t Lc = 0, Lr = 0;
 #pragma unroll 1
-  for (int bit = 31; bit >= 16; --bit) {
+  for (int bit = 31; bit >= 8; --bit) {
     const uint32_t xc = Lc | (1u << bit), xr = Lr | (1u << bit);
-    const int nc = __reduce_add_sync(0xffffffffu, (c1 >= xc ? 1 : 0) + (c2 >= xc ? 1 : 0));
-    const int nr = __reduce_add_sync(0xffffffffu, (r1 >= xr ? 1 : 0) + (r2 >= xr ? 1 : 0));
+    const int nc = __reduce_add_sync(0xffffffffu, (c0 >= xc) + (c1 >= xc) + (c2 >= xc) + (c3 >= xc));
+    const int nr = __reduce_add_sync(0xffffffffu, (r0 >= xr) + (r1 >= xr) + (r2 >= xr) + (r3 >= xr));
     if (nc >= k_c) Lc = xc;
     if (nr >= k_r) Lr = xr;
   }
+  // Every float's key but one NaN pattern is >= 256, so L > 0 and no absent
+  // slot (key 0) becomes a candidate.
   const uint32_t lt_mask = (1u << lane) - 1u;
   int base_c = 0, base_r = 0;
 #pragma unroll 4
@@ -169,49 +203,57 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
     const bool cand_c = uc >= Lc, cand_r = ur >= Lr;
     const uint32_t bc = __ballot_sync(0xffffffffu, cand_c), br = __ballot_sync(0xffffffffu, cand_r);
     const int pc = base_c + __popc(bc & lt_mask), pr = base_r + __popc(br & lt_mask);
-    if (cand_c && pc < 64) {
+    if (cand_c && pc < kTopkCap) {
       ck_c[pc] = uc;
       ci_c[pc] = 32 * t + lane;
     }
-    if (cand_r && pr < 64) {
+    if (cand_r && pr < kTopkCap) {
       ck_r[pr] = ur;
       ci_r[pr] = 32 * t + lane;
     }
     base_c += __popc(bc);
     base_r += __popc(br);
   }
-  if (base_c > 64 || base_r > 64) return false;
+  if (base_c > kTopkCap || base_r > kTopkCap) return false;
   __syncwarp();
-  const uint32_t a0 = lane < base_c ? ck_c[lane] : 0u, a1 = lane + 32 < base_c ? ck_c[lane + 32] : 0u;
-  const uint32_t b0 = lane < base_r ? ck_r[lane] : 0u, b1 = lane + 32 < base_r ? ck_r[lane + 32] : 0u;
-  const int ia0 = lane < base_c ? ci_c[lane] : 0, ia1 = lane + 32 < base_c ? ci_c[lane + 32] : 0;
-  const int ib0 = lane < base_r ? ci_r[lane] : 0, ib1 = lane + 32 < base_r ? ci_r[lane + 32] : 0;
+  // candidate position p = lane + 32 s holds slot s of this lane (0 = none)
+  uint32_t a[4], bk[4];
+  int ia[4], ib[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int p = lane + 32 * s;
+    a[s] = p < base_c ? ck_c[p] : 0u;
+    ia[s] = p < base_c ? ci_c[p] : 0;
+    bk[s] = p < base_r ? ck_r[p] : 0u;
+    ib[s] = p < base_r ? ci_r[p] : 0;
+  }
   uint32_t Tc = 0, Tr = 0;
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t xc = Tc | (1u << bit), xr = Tr | (1u << bit);
-    const int nc = __reduce_add_sync(0xffffffffu, (a0 >= xc ? 1 : 0) + (a1 >= xc ? 1 : 0));
-    const int nr = __reduce_add_sync(0xffffffffu, (b0 >= xr ? 1 : 0) + (b1 >= xr ? 1 : 0));
+    const int nc = __reduce_add_sync(0xffffffffu, (a[0] >= xc) + (a[1] >= xc) + (a[2] >= xc) + (a[3] >= xc));
+    const int nr = __reduce_add_sync(0xffffffffu, (bk[0] >= xr) + (bk[1] >= xr) + (bk[2] >= xr) + (bk[3] >= xr));
     if (nc >= k_c) Tc = xc;
     if (nr >= k_r) Tr = xr;
   }
-  // candidate position p (= lane, lane + 32) is in ascending block order, so
-  // a tie's rank is the number of ties at lower positions
-  const int need_c = k_c - __reduce_add_sync(0xffffffffu, (a0 > Tc ? 1 : 0) + (a1 > Tc ? 1 : 0));
-  const int need_r = k_r - __reduce_add_sync(0xffffffffu, (b0 > Tr ? 1 : 0) + (b1 > Tr ? 1 : 0));
-  const bool ta0 = a0 == Tc, ta1 = a1 == Tc, tb0 = b0 == Tr, tb1 = b1 == Tr;
-  const uint32_t ba0 = __ballot_sync(0xffffffffu, ta0), ba1 = __ballot_sync(0xffffffffu, ta1);
-  const uint32_t bb0 = __ballot_sync(0xffffffffu, tb0), bb1 = __ballot_sync(0xffffffffu, tb1);
-  const bool sa0 = a0 > Tc || (ta0 && __popc(ba0 & lt_mask) < need_c);
-  const bool sa1 = a1 > Tc || (ta1 && __popc(ba0) + __popc(ba1 & lt_mask) < need_c);
-  const bool sb0 = b0 > Tr || (tb0 && __popc(bb0 & lt_mask) < need_r);
-  const bool sb1 = b1 > Tr || (tb1 && __popc(bb0) + __popc(bb1 & lt_mask) < need_r);
+  const int need_c = k_c - __reduce_add_sync(0xffffffffu, (a[0] > Tc) + (a[1] > Tc) + (a[2] > Tc) + (a[3] > Tc));
+  const int need_r = k_r - __reduce_add_sync(0xffffffffu, (bk[0] > Tr) + (bk[1] > Tr) + (bk[2] > Tr) + (bk[3] > Tr));
   for (int w = lane; w < nwords; w += 32) words_c[w] = words_r[w] = 0u;
   __syncwarp();
-  if (sa0) atomicOr(&words_c[ia0 >> 5], 1u << (ia0 & 31));
-  if (sa1) atomicOr(&words_c[ia1 >> 5], 1u << (ia1 & 31));
-  if (sb0) atomicOr(&words_r[ib0 >> 5], 1u << (ib0 & 31));
-  if (sb1) atomicOr(&words_r[ib1 >> 5], 1u << (ib1 & 31));
+  // positions ascend with the block index, so a tie's rank is the number of
+  // ties at lower positions
+  int rank_c = 0, rank_r = 0;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const bool tc = a[s] == Tc, tr = bk[s] == Tr;
+    const uint32_t bc = __ballot_sync(0xffffffffu, tc), br = __ballot_sync(0xffffffffu, tr);
+    const bool sc = a[s] > Tc || (tc && rank_c + __popc(bc & lt_mask) < need_c);
+    const bool sr = bk[s] > Tr || (tr && rank_r + __popc(br & lt_mask) < need_r);
+    if (sc) atomicOr(&words_c[ia[s] >> 5], 1u << (ia[s] & 31));
+    if (sr) atomicOr(&words_r[ib[s] >> 5], 1u << (ib[s] & 31));
+    rank_c += __popc(bc);
+    rank_r += __popc(br);
+  }
   __syncwarp();
   return true;
 }
@@ -220,14 +262,12 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
 // union count.  Keys hold KP slots per lane (block 32t + lane in slot t); the
 // row's mask words cover all nwords <= (KPMAX + 31) / 32 * 32 words.
 template <int KP, int KPMAX>
-__device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float* sc, const float* rb,
-                                                const float* qn, int warp, int lane, int hq0, int b, int i, int gi,
-                                                int n, int npad, uint32_t* scratch) {
+__device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float* sc, const float* rb, float qnv,
+                                                int warp, int lane, int hq0, int b, int i, int gi, int n, int npad,
+                                                uint32_t* scratch) {
   const int hq = hq0 + warp;
   const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
-  const float qnv = qn[warp];
-  // per-warp scratch: candidates of both branches [256], mask words of both branches
-  uint32_t* words_c = scratch + 256;
+  uint32_t* words_c = scratch + 4 * kTopkCap;
   uint32_t* words_r = words_c + a.nwords;
   const float* srow = sc + warp * npad;
   auto key_c = [&](int t) -> uint32_t {
@@ -301,164 +341,255 @@ __device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float
   if (lane == 0) a.counts[row] = cnt;
 }
 
+// Work item w -> (batch, query block, first q head): longest rows first.
+__device__ __forceinline__ void sel_item(const SelectArgs& a, int w, int& b, int& i, int& hq0) {
+  const int nh = a.Hq / a.R;
+  const int per_i = a.B * nh;
+  i = a.nqb - 1 - w / per_i;
+  const int rem = w % per_i;
+  b = rem / nh;
+  hq0 = (rem % nh) * a.R;
+}
+
+// Dot products of one 16-dim slice of the staged tile with the pooled
+// queries: NP head pairs, the thread's block jA and, when TWO, jB = jA + 256.
+template <int NP, bool TWO>
+__device__ __forceinline__ void score_slice(const float* cs, const float* qd, int jA, float2 (&accA)[4],
+                                            float2 (&accB)[4]) {
+  const int jB = jA + 256;
+  const float* rowA = cs + jA * kStageD;
+  const float* rowB = cs + jB * kStageD;
+  const int swA = (jA >> 1) & 3, swB = (jB >> 1) & 3;
+#pragma unroll
+  for (int dq = 0; dq < kStageD / 4; ++dq) {
+    const float4 cA = *reinterpret_cast<const float4*>(rowA + 4 * (dq ^ swA));
+    float4 cB = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (TWO) cB = *reinterpret_cast<const float4*>(rowB + 4 * (dq ^ swB));
+    const float ca[4] = {cA.x, cA.y, cA.z, cA.w}, cb[4] = {cB.x, cB.y, cB.z, cB.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float* q = qd + (4 * dq + e) * kSelMaxR;
+      const float4 q0 = *reinterpret_cast<const float4*>(q);
+      const float2 xa = make_float2(ca[e], ca[e]), xb = make_float2(cb[e], cb[e]);
+      accA[0] = ffma2(make_float2(q0.x, q0.y), xa, accA[0]);
+      accA[1] = ffma2(make_float2(q0.z, q0.w), xa, accA[1]);
+      if (TWO) {
+        accB[0] = ffma2(make_float2(q0.x, q0.y), xb, accB[0]);
+        accB[1] = ffma2(make_float2(q0.z, q0.w), xb, accB[1]);
+      }
+      if (NP > 2) {
+        const float4 q1 = *reinterpret_cast<const float4*>(q + 4);
+        accA[2] = ffma2(make_float2(q1.x, q1.y), xa, accA[2]);
+        accA[3] = ffma2(make_float2(q1.z, q1.w), xa, accA[3]);
+        if (TWO) {
+          accB[2] = ffma2(make_float2(q1.x, q1.y), xb, accB[2]);
+          accB[3] = ffma2(make_float2(q1.z, q1.w), xb, accB[3]);
+        }
+      }
+    }
+  }
+}
+
 template <int KPL, int BQ>
-__global__ void __launch_bounds__(kSelThreads, KPL <= 32 ? 3 : 1) select_rows_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) float sm[];
-  const int i = a.nqb - 1 - static_cast<int>(blockIdx.x);  // longest rows first
-  const int hblk = blockIdx.y, b = blockIdx.z;
+__global__ void __launch_bounds__(kSelThreads, KPL <= 32 ? 2 : 1)
+    select_rows_kernel(const __grid_constant__ CUtensorMap qmap, SelectArgs a) {
+  extern __shared__ __align__(128) uint8_t sel_smem[];
+  __shared__ __align__(8) uint64_t full_bar[kPoolStages];
+  __shared__ float qn_s[2][kSelMaxR];
+  __shared__ int abort_flag;
+  uint8_t* qring = sel_smem;
+  float* cs = reinterpret_cast<float*>(sel_smem + kSelOffCs);
+  float* qs_all = reinterpret_cast<float*>(sel_smem + kSelOffQs);  // [2][128 dims][8 heads]
+  const int npad = (a.nkb + 31) & ~31;
+  float* rb = reinterpret_cast<float*>(sel_smem + kSelOffRb);  // [npad]  r_j * beta_j
+  float* sc = rb + npad;                                        // [8][npad] centroid-branch scores
+
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = a.R;
   const int G = a.Hq / a.Hkv;
-  const int hq0 = hblk * R;
-  const int kvh = hq0 / G;
-  const int gi = i + a.q_block_offset;
-  const int n = a.causal ? min(a.nkb, gi + 1) : a.nkb;
-  const int npad = (a.nkb + 31) & ~31;
+  const int nitems = a.items > static_cast<int>(blockIdx.x)
+                         ? (a.items - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                         : 0;
+  constexpr int kChunks = BQ / kPoolRows;
 
-  float* qs = sm;                         // [128][8] pooled queries, dim-major (heads >= R are 0)
-  float* rb = qs + kSelMaxR * 128;        // [npad]  r_j * beta_j
-  float* sc = rb + npad;                  // [R][npad] centroid-branch scores
-  float* cs = sc + kSelMaxR * npad;       // [kStageJ][kStagePitch]; first holds pooling partial sums
-  __shared__ float qn[kSelMaxR];
+  if (tid == 0) {
+    for (int s = 0; s < kPoolStages; ++s) mbar_init(smem_u32(&full_bar[s]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int o = tid; o < 2 * 128 * kSelMaxR; o += kSelThreads) qs_all[o] = 0.f;  // heads >= R stay 0
+  __syncthreads();
 
-  const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
-  for (int j = tid; j < n; j += kSelThreads) rb[j] = a.rad[kv_off + j] * a.beta[kv_off + j];
-
-  // ---- pooled query of each of the R heads: mean of the BQ queries of block i.
-  // Thread (rg, col): 16-byte chunk col % 16 of head col / 16, rows rg, rg + RG, ...
-  {
-    const int cols = R * 16;
-    const int RG = kSelThreads / cols;
-    const int col = tid % cols, rg = tid / cols;
-    float acc[8];
+  if (warp >= kSelComputeThreads / 32) {
+    // ===== pooling warps: item k's query block, while item k - 1 is scored.
+    // Chunk g = k * kChunks + c holds rows c * 8 .. c * 8 + 7 of item k's
+    // query block for its R heads, d 0-63 then d 64-127, in stage g % 2.
+    const int ptid = tid - kSelComputeThreads;
+    const int h = ptid >> 3, dq = ptid & 7;  // head, 16-dim group of this thread
+    const int total = nitems * kChunks;
+    const uint32_t chunk_bytes = static_cast<uint32_t>(kPoolRows * R * 128 * 2);
+    int issued = 0;
+    auto issue = [&](int g) {
+      const int k = g / kChunks, c = g % kChunks;
+      int b, i, hq0;
+      sel_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, i, hq0);
+      const int s = g % kPoolStages;
+      const uint32_t bar = smem_u32(&full_bar[s]);
+      const uint32_t dst = smem_u32(qring + s * kPoolChunkBytes);
+      const int row0 = i * BQ + c * kPoolRows;
+      const int c1 = a.seq_inner ? row0 : hq0, c2 = a.seq_inner ? hq0 : row0;
+      mbar_arrive_expect_tx(bar, chunk_bytes);
+      tma_load_4d(dst, &qmap, bar, 0, c1, c2, b);
+      tma_load_4d(dst + chunk_bytes / 2, &qmap, bar, 64, c1, c2, b);
+      issued = g + 1;
+    };
+    if (ptid == 0) {
+      tma_prefetch_desc(&qmap);
+      for (int g = 0; g < kPoolStages && g < total; ++g) issue(g);
+    }
+    // element offset of this thread's 16 dims of row r: [half][row][head][64]
+    // for token-major Q, [half][head][row][64] for head-major Q.  Threads of
+    // the upper half read their two 16-byte pieces in the other order, so a
+    // quarter warp covers all banks.
+    const int hoff = (dq >> 2) * (kPoolRows * R * 64) + (a.seq_inner ? h * kPoolRows * 64 : h * 64) + (dq & 3) * 16;
+    const int rstride = a.seq_inner ? 64 : R * 64;
+    const int p0 = (dq >> 2) * 8, p1 = 8 - p0;  // element offsets of the two pieces, in reading order
+    for (int k = 0; k < nitems; ++k) {
+      float acc[16];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    if (rg < RG) {
-      const char* base = reinterpret_cast<const char*>(a.Q + b * a.qb + static_cast<int64_t>(i) * BQ * a.qs +
-                                                       (hq0 + col / 16) * a.qh) + (col % 16) * 16;
-      for (int r0 = rg; r0 < BQ; r0 += 8 * RG) {
-        uint4 v[8];
+      for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+      for (int c = 0; c < kChunks; ++c) {
+        const int g = k * kChunks + c, s = g % kPoolStages;
+        const bool ok = mbar_wait(smem_u32(&full_bar[s]), static_cast<uint32_t>((g / kPoolStages) & 1), &abort_flag);
+        if (ok && h < R) {
+          const __nv_bfloat16* chunk = reinterpret_cast<const __nv_bfloat16*>(qring + s * kPoolChunkBytes) + hoff;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int row = r0 + u * RG;
-          v[u] = row < BQ ? ldg_stream(base + static_cast<int64_t>(row) * a.qs * 2) : make_uint4(0, 0, 0, 0);
+          for (int r = 0; r < kPoolRows; ++r) {
+            const uint4 v0 = *reinterpret_cast<const uint4*>(chunk + r * rstride + p0);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(chunk + r * rstride + p1);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              acc[2 * q] += bf16lo(w[q]);
+              acc[2 * q + 1] += bf16hi(w[q]);
+            }
+          }
         }
+        named_bar_sync(2, kSelPoolThreads);  // stage s is free
+        if (ptid == 0 && g + kPoolStages < total && !abort_flag) issue(g + kPoolStages);
+      }
+      float* qs = qs_all + (k & 1) * 128 * kSelMaxR;
+      float s2 = 0.f;
+      if (h < R) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        for (int e = 0; e < 16; ++e) {
+          // acc[e] is dim 16 dq + e of the first piece read, then the second
+          const int d = 16 * dq + (e < 8 ? p0 : p1) + (e & 7);
+          const float m = acc[e] * (1.0f / BQ);
+          qs[d * kSelMaxR + h] = m;
+          s2 = fmaf(m, m, s2);
+        }
+      }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            acc[2 * q] += bf16lo(w[q]);
-            acc[2 * q + 1] += bf16hi(w[q]);
+      for (int o = 4; o >= 1; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);  // the 8 threads of head h
+      if (dq == 0 && h < R) qn_s[k & 1][h] = sqrtf(s2);
+      __syncthreads();  // item k pooled; item k - 1 scored
+    }
+    __syncthreads();  // the last item scored
+    if (ptid == 0 && abort_flag) {
+      // after a timeout, wait (bounded) for the chunks still in flight
+      for (int g = issued - kPoolStages; g < issued; ++g)
+        if (g >= 0) mbar_drain(smem_u32(&full_bar[g % kPoolStages]), static_cast<uint32_t>((g / kPoolStages) & 1));
+    }
+    return;
+  }
+
+  // ===== scoring and top-k warps
+  __syncthreads();  // item 0 pooled
+  constexpr int kSlices = 128 / kStageD;
+  constexpr int kLoads = kStageJ * kStageD / 4 / kSelComputeThreads;  // float4 per thread per stage
+  for (int k = 0; k < nitems; ++k) {
+    int b, i, hq0;
+    sel_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, i, hq0);
+    const int kvh = hq0 / G;
+    const int gi = i + a.q_block_offset;
+    const int n = a.causal ? min(a.nkb, gi + 1) : a.nkb;
+    const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
+    const float* qs = qs_all + (k & 1) * 128 * kSelMaxR;
+    for (int j = tid; j < n; j += kSelComputeThreads) rb[j] = a.rad[kv_off + j] * a.beta[kv_off + j];
+
+    // ---- s_c for j < n: tile of 512 blocks x 16 dims per stage; thread t
+    // owns blocks j0 + t and j0 + t + 256.  Stage st + 1's global loads are
+    // in flight while stage st is used.
+    const float* Cb = a.C + kv_off * 128;
+    const int nstages = ((n + kStageJ - 1) / kStageJ) * kSlices;
+    float4 pre[kLoads];
+    auto load_stage = [&](int st) {
+      const int j0 = (st / kSlices) * kStageJ, d0 = (st % kSlices) * kStageD;
+      const int jn = min(kStageJ, n - j0);
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int idx = tid + kSelComputeThreads * u;
+        const int jl = idx >> 2, q4 = idx & 3;
+        pre[u] = jl < jn ? *reinterpret_cast<const float4*>(Cb + static_cast<int64_t>(j0 + jl) * 128 + d0 + 4 * q4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    float2 accA[4], accB[4];
+    load_stage(0);
+    for (int st = 0; st < nstages; ++st) {
+      const int j0 = (st / kSlices) * kStageJ, d0 = (st % kSlices) * kStageD;
+      const int jn = min(kStageJ, n - j0);
+      if (d0 == 0) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) accA[p] = accB[p] = make_float2(0.f, 0.f);
+      }
+      named_bar_sync(1, kSelComputeThreads);  // the previous stage is consumed
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int idx = tid + kSelComputeThreads * u;
+        const int jl = idx >> 2, q4 = idx & 3;
+        *reinterpret_cast<float4*>(cs + jl * kStageD + 4 * (q4 ^ ((jl >> 1) & 3))) = pre[u];
+      }
+      named_bar_sync(1, kSelComputeThreads);  // this stage is visible
+      if (st + 1 < nstages) load_stage(st + 1);
+      const float* qd = qs + d0 * kSelMaxR;
+      if (tid < jn) {
+        if (jn > 256) {
+          if (R > 4) score_slice<4, true>(cs, qd, tid, accA, accB);
+          else score_slice<2, true>(cs, qd, tid, accA, accB);
+        } else {
+          if (R > 4) score_slice<4, false>(cs, qd, tid, accA, accB);
+          else score_slice<2, false>(cs, qd, tid, accA, accB);
+        }
+      }
+      if (d0 + kStageD == 128) {
+#pragma unroll
+        for (int hh = 0; hh < kSelMaxR; ++hh) {
+          if (hh < R) {
+            const float va = (hh & 1) ? accA[hh >> 1].y : accA[hh >> 1].x;
+            const float vb = (hh & 1) ? accB[hh >> 1].y : accB[hh >> 1].x;
+            if (tid < jn) sc[hh * npad + j0 + tid] = va;
+            if (tid + 256 < jn) sc[hh * npad + j0 + tid + 256] = vb;
           }
         }
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) cs[rg * (R * 128) + col * 8 + e] = acc[e];
     }
-    __syncthreads();
-    for (int o = tid; o < kSelMaxR * 128; o += kSelThreads) {
-      const int h = o >> 7, d = o & 127;  // o = h * 128 + d, the pooling sums' order
-      float sum = 0.f;
-      if (h < R)
-        for (int g2 = 0; g2 < RG; ++g2) sum += cs[g2 * (R * 128) + o];
-      qs[d * kSelMaxR + h] = sum * (1.0f / BQ);
-    }
-    __syncthreads();
+    named_bar_sync(1, kSelComputeThreads);  // scores complete; the staging tile is free
+
+    // ---- per-branch top-k (both branches together), one warp per row, with
+    // as few key slots per lane as this row needs
     if (warp < R) {
-      float s2 = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float v = qs[(lane + 32 * e) * kSelMaxR + warp];
-        s2 = fmaf(v, v, s2);
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-      if (lane == 0) qn[warp] = sqrtf(s2);
+      uint32_t* scratch = reinterpret_cast<uint32_t*>(cs) + warp * sel_topk_scratch_words(a.nwords);
+      const float qnv = qn_s[k & 1][warp];
+      if (KPL > 2 && n <= 64) select_topk_row<2, KPL>(a, sc, rb, qnv, warp, lane, hq0, b, i, gi, n, npad, scratch);
+      else if (KPL > 8 && n <= 256) select_topk_row<8, KPL>(a, sc, rb, qnv, warp, lane, hq0, b, i, gi, n, npad, scratch);
+      else if (KPL > 16 && n <= 512) select_topk_row<16, KPL>(a, sc, rb, qnv, warp, lane, hq0, b, i, gi, n, npad, scratch);
+      else if (KPL > 32 && n <= 1024) select_topk_row<32, KPL>(a, sc, rb, qnv, warp, lane, hq0, b, i, gi, n, npad, scratch);
+      else if (KPL > 64 && n <= 2048) select_topk_row<64, KPL>(a, sc, rb, qnv, warp, lane, hq0, b, i, gi, n, npad, scratch);
+      else select_topk_row<KPL, KPL>(a, sc, rb, qnv, warp, lane, hq0, b, i, gi, n, npad, scratch);
     }
-  }
-
-  // ---- scores s_c for j < n: thread t owns block j0 + t of each 256-block tile.
-  // Stage (j-tile, 32-dim slice) k's global loads are issued while stage k-1
-  // is being used.
-  const float* Cb = a.C + kv_off * 128;
-  const int nstages = ((n + kStageJ - 1) / kStageJ) * (128 / kStageD);
-  constexpr int kLoads = (kStageJ * kStageD / 4) / kSelThreads;  // float4 per thread per stage
-  float4 pre[kLoads];
-  auto load_stage = [&](int st) {
-    const int j0 = (st / (128 / kStageD)) * kStageJ, d0 = (st % (128 / kStageD)) * kStageD;
-    const int jn = min(kStageJ, n - j0);
-#pragma unroll
-    for (int u = 0; u < kLoads; ++u) {
-      const int idx = tid + kSelThreads * u;
-      const int jl = idx >> 3, d4 = idx & 7;
-      pre[u] = jl < jn ? *reinterpret_cast<const float4*>(Cb + static_cast<int64_t>(j0 + jl) * 128 + d0 + 4 * d4)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  // four head pairs per thread, accumulated with paired FMAs (the heads of a
-  // pair share the centroid value)
-  float2 acc[kSelMaxR / 2];
-  load_stage(0);
-  for (int st = 0; st < nstages; ++st) {
-    const int j0 = (st / (128 / kStageD)) * kStageJ, d0 = (st % (128 / kStageD)) * kStageD;
-    const int jn = min(kStageJ, n - j0);
-    if (d0 == 0) {
-#pragma unroll
-      for (int h = 0; h < kSelMaxR / 2; ++h) acc[h] = make_float2(0.f, 0.f);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < kLoads; ++u) {
-      const int idx = tid + kSelThreads * u;
-      float* dst = cs + (idx >> 3) * kStagePitch + 4 * (idx & 7);
-      dst[0] = pre[u].x;
-      dst[1] = pre[u].y;
-      dst[2] = pre[u].z;
-      dst[3] = pre[u].w;
-    }
-    __syncthreads();
-    if (st + 1 < nstages) load_stage(st + 1);
-    if (tid < jn) {
-      const float* crow = cs + tid * kStagePitch;
-      const float* qd = qs + d0 * kSelMaxR;
-      if (R > 4) {
-#pragma unroll 8
-        for (int d = 0; d < kStageD; ++d) {
-          const float2 cc = make_float2(crow[d], crow[d]);
-          const float4 qa = *reinterpret_cast<const float4*>(qd + d * kSelMaxR);
-          const float4 qb = *reinterpret_cast<const float4*>(qd + d * kSelMaxR + 4);
-          acc[0] = ffma2(make_float2(qa.x, qa.y), cc, acc[0]);
-          acc[1] = ffma2(make_float2(qa.z, qa.w), cc, acc[1]);
-          acc[2] = ffma2(make_float2(qb.x, qb.y), cc, acc[2]);
-          acc[3] = ffma2(make_float2(qb.z, qb.w), cc, acc[3]);
-        }
-      } else {
-#pragma unroll 8
-        for (int d = 0; d < kStageD; ++d) {
-          const float2 cc = make_float2(crow[d], crow[d]);
-          const float4 qa = *reinterpret_cast<const float4*>(qd + d * kSelMaxR);
-          acc[0] = ffma2(make_float2(qa.x, qa.y), cc, acc[0]);
-          acc[1] = ffma2(make_float2(qa.z, qa.w), cc, acc[1]);
-        }
-      }
-    }
-    if (d0 + kStageD == 128 && tid < jn) {
-#pragma unroll
-      for (int h = 0; h < kSelMaxR; ++h)
-        if (h < R) sc[h * npad + j0 + tid] = (h & 1) ? acc[h >> 1].y : acc[h >> 1].x;
-    }
-  }
-  __syncthreads();
-
-  // ---- per-branch top-k (both branches together), one warp per row, with
-  // as few key slots per lane as this row needs
-  if (warp < R) {
-    // the staging area is free after the scores: per-warp top-k scratch
-    uint32_t* scratch = reinterpret_cast<uint32_t*>(cs) + warp * (256 + 2 * a.nwords);
-    if (KPL > 8 && n <= 64) select_topk_row<2, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad, scratch);
-    else if (KPL > 8 && n <= 256) select_topk_row<8, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad, scratch);
-    else select_topk_row<KPL, KPL>(a, sc, rb, qn, warp, lane, hq0, b, i, gi, n, npad, scratch);
+    __syncthreads();  // item k done; item k + 1 pooled
   }
 }
 
