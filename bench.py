@@ -12,8 +12,9 @@ max-over-ranks step time.  Also reported: attention-only ms and TFLOP/s,
 selection ms, stats ms, the attention kernel's roofline, clocks, an
 end-to-end number through the same calls with host buffers, the Block-
 attention RAG flow (cache build, RoPE re-encoding, final block), a density
-sweep at 64K (selection and attention time at 2-100% kept density) and the
-CPU oracle baseline.
+sweep at 64K (selection and attention time at 2-100% kept density), the same
+prompt with KV-group lists (one list per KV head shared by its q heads) and
+the CPU oracle baseline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 N > 1 runs under torchrun: every rank processes its own prompt (weak
@@ -50,9 +51,9 @@ SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
 # dram__bytes_write.sum, one single-pass ncu capture of the default workload;
 # profiles/launches_gqa_rbs_128k.md gives the command), valid for the kernel
 # sources with this digest; any other build reports null.
-ATTN_TRAFFIC_BYTES = 3.25e9 + 1.04e9
+ATTN_TRAFFIC_BYTES = 3.234e9 + 1.038e9
 ATTN_TRAFFIC_SOURCES = ("block_sparse_long_rbs_b200/csrc/attention.cuh", "block_sparse_long_rbs_b200/csrc/common.cuh")
-ATTN_TRAFFIC_DIGEST = "6d0eecb19f62cd80"
+ATTN_TRAFFIC_DIGEST = "de2dc7480fe2059f"
 
 
 def attn_traffic(seq_len: int):
@@ -304,6 +305,8 @@ def run_ours(args, ws, rank):
         out["dense"] = dense_measure(rbs, Q, K, V, B, Hq, nqb, peak)
         out["dense"]["speedup_attn_only"] = round(out["dense"]["ms"] / attn_ms, 2)
         out["dense"]["speedup_with_selection"] = round(out["dense"]["ms"] / (attn_ms + select_ms + stats_ms), 2)
+    if args.group_lists and rank == 0:
+        out["kv_group_lists"] = group_lists_measure(rbs, Q, K, V, C, R, w.rho, B, Hq, Hkv, nqb, nkb, nnz, peak)
     del Q, K, V, O
     torch.cuda.empty_cache()
     if args.block_attention and rank == 0:
@@ -638,6 +641,34 @@ def block_attention_measure(rbs, peaks):
     return res
 
 
+def group_lists_measure(rbs, Q, K, V, C, R, rho, B, Hq, Hkv, nqb, nkb, nnz_heads, peak):
+    """KV-group lists (one list per KV head, the union of its q heads'):
+    selection and attention time on the same prompt, and how many more block
+    pairs the shared lists make every q head compute."""
+    import torch
+    G = Hq // Hkv
+    p = rbs.SelectParams(block_q=BLOCK, block_k=BLOCK, rho_centroid=rho, rho_rescue=rho, list_mode=1)
+    lists = rbs.BlockLists.empty(B * Hkv * nqb, rbs.rbs_select_capacity(B, Hq, nqb, nkb, p), "cuda")
+    ws_buf = torch.empty(rbs.rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, p), dtype=torch.uint8, device="cuda")
+    sel = lambda: rbs.rbs_select(Q, C, R, p, workspace=ws_buf, out=lists)
+    sel()
+    O = torch.empty_like(Q)
+    att = lambda: rbs.bsa_prefill(Q, K, V, lists, BLOCK, BLOCK, out=O)
+    att()
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    nnz = lists.nnz()
+    sel_ms = _time_ms(sel, 10)
+    att_ms = _time_ms(att, 5)
+    flops = G * nnz * FLOP_PER_PAIR  # every q head computes its group's whole list
+    visible = B * Hq * nqb * (nqb + 1) // 2
+    del O
+    return {"select_ms": round(sel_ms, 4), "attn_ms": round(att_ms, 4), "list_entries": nnz,
+            "pairs_per_q_head_total": G * nnz, "pairs_vs_per_head_lists": round(G * nnz / nnz_heads, 3),
+            "density": round(G * nnz / visible, 5), "attn_tflops": round(flops / (att_ms * 1e-3) / 1e12, 2),
+            "frac_of_peak": round(flops / (att_ms * 1e-3) / 1e12 / peak, 4)}
+
+
 def _time_ms(fn, reps: int, warm: int = 2) -> float:
     import torch
     for _ in range(warm):
@@ -805,6 +836,7 @@ def main():
     ap.add_argument("--no-density-sweep", dest="density_sweep", action="store_false")
     ap.add_argument("--no-isolated", dest="isolated", action="store_false")
     ap.add_argument("--no-selector-quality", dest="selector_quality", action="store_false")
+    ap.add_argument("--no-group-lists", dest="group_lists", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--seq-len", type=int, default=None,

@@ -55,6 +55,7 @@ class SelectParams:
     threshold_mode: int = 0  # 0 = top-k fraction, 1 = within delta of the row maximum
     delta_centroid: float = 0.0
     delta_rescue: float = 0.0
+    list_mode: int = 0  # 0 = one list per q head, 1 = one per KV head (union of its q heads)
 
     def c(self) -> SelectParamsC:
         return SelectParamsC(*[getattr(self, f.name) for f in dataclasses.fields(self)])
@@ -153,11 +154,12 @@ def rbs_select_workspace_bytes(batch: int, heads_q: int, num_q_blocks: int, kv_h
 def rbs_select(Q: torch.Tensor, centroids: torch.Tensor, radii: torch.Tensor, params: SelectParams,
                workspace: torch.Tensor | None = None, out: BlockLists | None = None, beta_out: torch.Tensor | None = None,
                flags: bool = True) -> BlockLists:
-    """Two-branch selection -> CSR key-block lists (rows = (batch, q head, query block))."""
+    """Two-branch selection -> CSR key-block lists, rows = (batch, q head, query block), or
+    (batch, KV head, query block) when params.list_mode == 1."""
     B, L, Hq, _ = Q.shape
     Hkv, nkb = centroids.shape[1], centroids.shape[2]
     nqb = L // params.block_q
-    rows = B * Hq * nqb
+    rows = B * (Hkv if params.list_mode == 1 else Hq) * nqb
     if out is None:
         out = BlockLists.empty(rows, rbs_select_capacity(B, Hq, nqb, nkb, params), Q.device, flags)
     if workspace is None:

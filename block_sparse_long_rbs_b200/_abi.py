@@ -32,7 +32,8 @@ class SelectParamsC(ctypes.Structure):
                 ("rho_rescue", ctypes.c_float), ("beta_mode", ctypes.c_int32), ("beta_const", ctypes.c_float),
                 ("beta_p_lo", ctypes.c_float), ("beta_p_hi", ctypes.c_float), ("force_diag", ctypes.c_int32),
                 ("force_sink", ctypes.c_int32), ("causal", ctypes.c_int32), ("q_block_offset", ctypes.c_int32),
-                ("threshold_mode", ctypes.c_int32), ("delta_centroid", ctypes.c_float), ("delta_rescue", ctypes.c_float)]
+                ("threshold_mode", ctypes.c_int32), ("delta_centroid", ctypes.c_float), ("delta_rescue", ctypes.c_float),
+                ("list_mode", ctypes.c_int32)]
 
 
 class BlockListsC(ctypes.Structure):
@@ -74,6 +75,7 @@ class RbsError(RuntimeError):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
 
 
+ABI_VERSION = 3  # RBS_ABI_VERSION of include/rbs.h that these structures match
 _lib = None
 
 
@@ -88,6 +90,9 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        if L.rbs_abi_version() != ABI_VERSION:
+            raise ImportError(f"{LIB_PATH} has ABI version {L.rbs_abi_version()}, this binding expects {ABI_VERSION}; "
+                              "rebuild it with python -m block_sparse_long_rbs_b200.build")
         _lib = L
     return _lib
 

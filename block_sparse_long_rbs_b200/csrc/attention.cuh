@@ -70,7 +70,8 @@ struct AttnArgs {
   int64_t ob, os, oh;
   float* lse;
   int B, Hq, Hkv, nqb, nkb, Lq;
-  int q_block_off, causal, num_rows;
+  int q_block_off, causal, num_rows;  // num_rows: work items, B * Hq * nqb
+  int group_lists;  // 1: list row (b, KV head, i) serves every q head of the KV head
   float scale_log2;
 };
 
@@ -149,7 +150,7 @@ __device__ __forceinline__ void decode_work(const AttnArgs& a, int w, int& b, in
   const int kvh = rem / per_kvh, r2 = rem % per_kvh;
   i = a.nqb - 1 - r2 / G;
   h = kvh * G + r2 % G;
-  row = (b * a.Hq + h) * a.nqb + i;
+  row = (a.group_lists ? b * a.Hkv + kvh : b * a.Hq + h) * a.nqb + i;
 }
 
 // Row extent with validation (identical in every role): -1 for a corrupt row.

@@ -254,6 +254,7 @@ void rbs_select_params_default(rbs_select_params* p) {
   p->threshold_mode = 0;
   p->delta_centroid = 0.0f;
   p->delta_rescue = 0.0f;
+  p->list_mode = 0;
 }
 
 rbs_status rbs_get_device_error(int32_t* code_host, rbs_stream_t stream) {
@@ -378,10 +379,12 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   RBS_REQUIRE(p->threshold_mode == 0 || (p->delta_centroid >= 0.f && p->delta_rescue >= 0.f),
               RBS_ERR_INVALID_ARG, "delta must be >= 0 (and not NaN)");
   RBS_REQUIRE(p->q_block_offset >= 0, RBS_ERR_INVALID_ARG, "q_block_offset < 0");
+  RBS_REQUIRE(p->list_mode == 0 || p->list_mode == 1, RBS_ERR_INVALID_ARG, "list_mode must be 0 or 1");
   RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
   const int64_t B = Q->batch, Hq = Q->heads, nqb = Q->seqlen / p->block_q, nkb = num_kv_blocks;
-  const int64_t rows = B * Hq * nqb;
-  if ((st = check_lists(out, rows)) != RBS_OK) return st;
+  const int64_t rows = B * Hq * nqb;                                       // one per q head
+  const int64_t list_rows = p->list_mode == 1 ? B * kv_heads * nqb : rows;  // rows of the output lists
+  if ((st = check_lists(out, list_rows)) != RBS_OK) return st;
   const int64_t cap = rbs_select_capacity(B, Hq, nqb, nkb, p);
   RBS_REQUIRE(out->capacity >= cap, RBS_ERR_CAPACITY, "list capacity %lld < %lld", static_cast<long long>(out->capacity),
               static_cast<long long>(cap));
@@ -450,9 +453,6 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
 #undef RBS_SEL_LAUNCH
   if (st != RBS_OK) return st;
 
-  scan_counts_kernel<<<1, 1024, 0, stream>>>(sa.counts, static_cast<int>(rows), out->row_ptr, out->capacity);
-  if ((st = check_launch("scan_counts_kernel")) != RBS_OK) return st;
-
   CompactArgs ca;
   ca.mask_c = sa.mask_c;
   ca.mask_r = sa.mask_r;
@@ -460,14 +460,26 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   ca.col_idx = out->col_idx;
   ca.flags = out->flags;
   ca.capacity = out->capacity;
-  ca.rows = static_cast<int>(rows);
+  ca.rows = static_cast<int>(list_rows);
   ca.nqb = static_cast<int>(nqb);
   ca.nkb = static_cast<int>(nkb);
   ca.nwords = sa.nwords;
   ca.q_block_offset = p->q_block_offset;
   ca.force_diag = p->force_diag;
   ca.force_sink = p->force_sink;
-  compact_lists_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(ca);
+  ca.Hq = static_cast<int>(Hq);
+  ca.Hl = p->list_mode == 1 ? kv_heads : static_cast<int>(Hq);
+  ca.glist = p->list_mode == 1 ? G : 1;
+  const unsigned list_grid = static_cast<unsigned>((list_rows + 7) / 8);
+  if (p->list_mode == 1) {
+    // the per-head counts written by the selection are replaced by the
+    // counts of the group unions (list_rows <= rows entries)
+    group_counts_kernel<<<list_grid, 256, 0, stream>>>(ca, sa.counts);
+    if ((st = check_launch("group_counts_kernel")) != RBS_OK) return st;
+  }
+  scan_counts_kernel<<<1, 1024, 0, stream>>>(sa.counts, static_cast<int>(list_rows), out->row_ptr, out->capacity);
+  if ((st = check_launch("scan_counts_kernel")) != RBS_OK) return st;
+  compact_lists_kernel<<<list_grid, 256, 0, stream>>>(ca);
   return check_launch("compact_lists_kernel");
 }
 
@@ -627,8 +639,10 @@ rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const
   RBS_REQUIRE(Q->seqlen % block_q == 0 && K->seqlen % block_k == 0, RBS_ERR_UNSUPPORTED, "seqlen not a block multiple");
   RBS_REQUIRE(q_offset >= 0 && q_offset % block_k == 0, RBS_ERR_UNSUPPORTED, "q_offset must be a non-negative block multiple");
   const int64_t nqb = Q->seqlen / block_q;
-  const int64_t rows = Q->batch * Q->heads * nqb;
-  if ((st = check_lists(lists, rows)) != RBS_OK) return st;
+  const int64_t rows = Q->batch * Q->heads * nqb;  // work items: one per (batch, q head, query block)
+  // one list per q head, or one per KV head shared by its q heads
+  const bool group_lists = lists != nullptr && Q->heads != K->heads && lists->num_rows == Q->batch * K->heads * nqb;
+  if ((st = check_lists(lists, group_lists ? Q->batch * K->heads * nqb : rows)) != RBS_OK) return st;
   DeviceInfo* di;
   if ((st = device_info(&di)) != RBS_OK) return st;
 
@@ -656,6 +670,7 @@ rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const
   a.q_block_off = static_cast<int>(q_offset / block_k);
   a.causal = causal ? 1 : 0;
   a.num_rows = static_cast<int>(rows);
+  a.group_lists = group_lists ? 1 : 0;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(RBS_HEAD_DIM));
   a.scale_log2 = scale * 1.4426950408889634f;
   const int grid = static_cast<int>(std::min<int64_t>(rows, di->sms));

@@ -23,9 +23,12 @@
 //                       full 32-step bitwise search as the fallback), breaks
 //                       ties by block index with warp ballots, and emits one
 //                       32-bit mask word per 32 blocks.
+//   group_counts_kernel (KV_GROUP lists) one warp per (batch, KV head, query
+//                       block) counts the union of its q heads' masks.
 //   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr.
-//   compact_lists_kernel one warp per row turns mask words into ascending
-//                       block indices and per-entry branch flags.
+//   compact_lists_kernel one warp per list row turns mask words (OR-ed over
+//                       the q heads of a KV_GROUP row) into ascending block
+//                       indices and per-entry branch flags.
 #pragma once
 
 #include "common.cuh"
@@ -650,35 +653,72 @@ __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict
 }
 
 struct CompactArgs {
-  const uint32_t* mask_c;
+  const uint32_t* mask_c;  // [B * Hq * nqb, nwords], one row per q head
   const uint32_t* mask_r;
   const int* row_ptr;
   int32_t* col_idx;
   uint8_t* flags;
   int64_t capacity;
   int rows, nqb, nkb, nwords, q_block_offset, force_diag, force_sink;
+  int Hq, Hl, glist;  // list row (b, hl, i) = union of q heads hl * glist .. + glist - 1
 };
+
+// Forced-block bits of mask word t of a row whose global query block is gi.
+__device__ __forceinline__ uint32_t forced_word(int t, int gi, int nkb, int force_diag, int force_sink) {
+  uint32_t f = 0;
+  if (force_diag && gi < nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
+  if (force_sink && t == 0) f |= 1u;
+  return f;
+}
+
+// Mask word t of list row (b, hl, i): the OR over the row's q heads.
+__device__ __forceinline__ void list_row_word(const CompactArgs& a, int b, int hl, int i, int t, uint32_t& c,
+                                              uint32_t& r) {
+  c = r = 0;
+  for (int hh = 0; hh < a.glist; ++hh) {
+    const int64_t m = ((static_cast<int64_t>(b) * a.Hq + hl * a.glist + hh) * a.nqb + i) * a.nwords + t;
+    c |= a.mask_c[m];
+    r |= a.mask_r[m];
+  }
+}
+
+// KV_GROUP lists: the entry count of every list row (b, g, i).
+__global__ void __launch_bounds__(256) group_counts_kernel(CompactArgs a, int* __restrict__ counts) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= a.rows) return;
+  const int i = row % a.nqb, bh = row / a.nqb;
+  const int b = bh / a.Hl, hl = bh % a.Hl;
+  const int gi = i + a.q_block_offset;
+  int cnt = 0;
+  for (int t = lane; t < a.nwords; t += 32) {
+    uint32_t c, r;
+    list_row_word(a, b, hl, i, t, c, r);
+    cnt += __popc(c | r | forced_word(t, gi, a.nkb, a.force_diag, a.force_sink));
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) counts[row] = cnt;
+}
 
 __global__ void __launch_bounds__(256) compact_lists_kernel(CompactArgs a) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= a.rows) return;
-  const int gi = row % a.nqb + a.q_block_offset;
+  const int i = row % a.nqb, bh = row / a.nqb;
+  const int b = bh / a.Hl, hl = bh % a.Hl;
+  const int gi = i + a.q_block_offset;
   const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
   if (beg < 0 || end < beg || end > a.capacity) {
     if (lane == 0) raise_error(RBS_DEVERR_ROW_PTR);
     return;
   }
   int run = beg;
-  const int64_t mbase = static_cast<int64_t>(row) * a.nwords;
   for (int w0 = 0; w0 < a.nwords; w0 += 32) {
     const int t = w0 + lane;
     uint32_t c = 0, r = 0, f = 0;
     if (t < a.nwords) {
-      c = a.mask_c[mbase + t];
-      r = a.mask_r[mbase + t];
-      if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
-      if (a.force_sink && t == 0) f |= 1u;
+      list_row_word(a, b, hl, i, t, c, r);
+      f = forced_word(t, gi, a.nkb, a.force_diag, a.force_sink);
     }
     uint32_t u = c | r | f;
     const int cnt = __popc(u);

@@ -59,7 +59,7 @@ extern "C" {
 #define RBS_API
 #endif
 
-#define RBS_ABI_VERSION 2
+#define RBS_ABI_VERSION 3
 #define RBS_HEAD_DIM 128
 #define RBS_MAX_SEGMENTS 512 /* Block-attention segments per call */
 #define RBS_MAX_KV_BLOCKS 4096 /* key blocks per sequence for rbs_select */
@@ -114,6 +114,14 @@ typedef struct {
  *                      Sparse Attention Landscape") (0)
  *   delta_centroid, delta_rescue  MAX_RELATIVE margins in raw score units,
  *                      >= 0 (0, 0)
+ *   list_mode          0 = PER_HEAD: one list per (batch, q head, query
+ *                      block); 1 = KV_GROUP: one list per (batch, KV head,
+ *                      query block), the union of the lists of the Hq / Hkv
+ *                      q heads that share the KV head, so that those heads
+ *                      attend to the same key blocks (grouped-query attention,
+ *                      [RBS-en] "How This Fits Into the Broader Sparse
+ *                      Attention Landscape"; shared key blocks across queries,
+ *                      [QUILT] Abstract) (0)
  * Scores are raw dot products (no 1/sqrt(d)); ties between equal scores go
  * to the lower block index.  Forced blocks do not count toward a branch's k.
  */
@@ -127,6 +135,7 @@ typedef struct {
   int32_t q_block_offset;
   int32_t threshold_mode;
   float delta_centroid, delta_rescue;
+  int32_t list_mode;
 } rbs_select_params;
 
 /* Per-query-block key-block lists in CSR form (all device memory). */
@@ -134,9 +143,13 @@ typedef struct {
   int32_t* row_ptr; /* [num_rows + 1]; row r spans col_idx[row_ptr[r] .. row_ptr[r+1]) */
   int32_t* col_idx; /* [capacity] key-block indices, ascending within a row */
   uint8_t* flags;   /* [capacity] or NULL: bit0 centroid branch kept the block,
-                       bit1 rescue branch kept it, bit2 forced (diagonal/sink) */
+                       bit1 rescue branch kept it, bit2 forced (diagonal/sink);
+                       in KV_GROUP lists a bit is set when it holds for any
+                       q head of the group */
   int64_t capacity; /* entries col_idx (and flags) can hold */
-  int32_t num_rows; /* batch * heads_q * num_q_blocks */
+  int32_t num_rows; /* batch * heads * num_q_blocks, rows ordered (batch, head,
+                       query block); heads = heads_q (one list per q head) or
+                       heads_kv (one list per KV head, shared by its q heads) */
 } rbs_block_lists;
 
 /* ---- housekeeping ------------------------------------------------------ */
@@ -189,8 +202,10 @@ RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, f
  *   radii        [B, Hkv, num_kv_blocks] fp32
  *   workspace    device scratch of at least rbs_select_workspace_bytes(...)
  *                bytes, 256-byte aligned; its contents need no initialisation
- *   out          lists with num_rows = B * Hq * Lq / block_q and capacity >=
- *                rbs_select_capacity(...); row_ptr, col_idx and flags written
+ *   out          lists with num_rows = B * Hq * Lq / block_q (B * Hkv * Lq /
+ *                block_q when list_mode is KV_GROUP) and capacity >=
+ *                rbs_select_capacity(...), which bounds both modes;
+ *                row_ptr, col_idx and flags written
  *   beta_out     optional [B, Hkv, num_kv_blocks] fp32 copy of beta (or NULL)
  * Requires Hq % Hkv == 0, num_kv_blocks <= RBS_MAX_KV_BLOCKS. */
 RBS_API int64_t rbs_select_capacity(int64_t batch, int64_t heads_q, int64_t num_q_blocks, int64_t num_kv_blocks,
@@ -258,7 +273,9 @@ RBS_API rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t n
  *   Q         [B, Lq, Hq, 128] bf16; K, V [B, Lk, Hkv, 128] bf16; each with
  *             stride_h <= stride_s (heads inside tokens, as in a packed QKV
  *             projection; else RBS_ERR_UNSUPPORTED)
- *   lists     num_rows = B * Hq * Lq / block_q; indices in [0, Lk / block_k)
+ *   lists     num_rows = B * Hq * Lq / block_q (row (b, h, i) serves q head
+ *             h) or B * Hkv * Lq / block_q (row (b, g, i) serves every q
+ *             head of KV head g); indices in [0, Lk / block_k)
  *   block_q == block_k, 64 or 128; q_offset a multiple of block_k
  *   softmax_scale  <= 0 selects 1/sqrt(128)
  *   O         out [B, Lq, Hq, 128] bf16 (may not alias Q, K or V)

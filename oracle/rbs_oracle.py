@@ -89,6 +89,10 @@ class SelectParams:
     threshold_mode: int = 0
     delta_centroid: float = 0.0
     delta_rescue: float = 0.0
+    # list layout: 0 = one list per (batch, q head, query block); 1 = one list
+    # per (batch, KV head, query block), the union of the lists of the q heads
+    # that share the KV head (they then attend to the same key blocks)
+    list_mode: int = 0
 
 
 FLAG_CENTROID = 1
@@ -238,6 +242,13 @@ def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, 
     This Fits Into the Broader Sparse Attention Landscape" describes as an
     alternative to ranking, with the rescue branch layered on it).  k then
     reports the kept count.
+
+    list_mode 1 returns one list per (batch, KV head, query block) instead:
+    the union of the lists of the G = Hq / Hkv q heads of that KV head, each
+    entry's flags the OR of those heads' flags (grouped-query attention with
+    the key blocks shared by the group, [RBS-en] "How This Fits Into the
+    Broader Sparse Attention Landscape"; sharing selected KV entries across
+    queries, [QUILT] Abstract).  tau and k stay per q head.
     """
     B, L, Hq, d = Q.shape
     _, Hkv, nkb, _ = C.shape
@@ -284,6 +295,8 @@ def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, 
                 cols.extend(sel.tolist())
                 flags.extend(f[sel].tolist())
                 row_ptr.append(len(cols))
+    if p.list_mode == 1:
+        row_ptr, cols, flags = group_union_lists(row_ptr, cols, flags, B, Hq, Hkv, nqb, nkb)
     out = {
         "row_ptr": np.asarray(row_ptr, dtype=np.int64),
         "col_idx": np.asarray(cols, dtype=np.int64),
@@ -297,6 +310,26 @@ def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, 
     if keep_scores:
         out["scores"] = scores
     return out
+
+
+def group_union_lists(row_ptr, cols, flags, B: int, Hq: int, Hkv: int, nqb: int, nkb: int):
+    """Per-q-head CSR rows (b, hq, i) -> per-KV-head rows (b, g, i): the set union
+    of the rows of q heads g*G .. g*G + G - 1, ascending, flags OR-ed."""
+    G = Hq // Hkv
+    out_ptr, out_cols, out_flags = [0], [], []
+    for b in range(B):
+        for g in range(Hkv):
+            for i in range(nqb):
+                f = np.zeros(nkb, dtype=np.uint8)
+                for hq in range(g * G, (g + 1) * G):
+                    r = (b * Hq + hq) * nqb + i
+                    for e in range(row_ptr[r], row_ptr[r + 1]):
+                        f[cols[e]] |= flags[e]
+                sel = np.nonzero(f)[0]
+                out_cols.extend(sel.tolist())
+                out_flags.extend(f[sel].tolist())
+                out_ptr.append(len(out_cols))
+    return out_ptr, out_cols, out_flags
 
 
 def list_density(row_ptr: np.ndarray, nqb: int, nkb: int, q_block_offset: int = 0, causal: int = 1) -> float:
@@ -424,12 +457,15 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
                      scale: float | None = None, causal: int = 1, rows=None):
     """Softmax attention of each query token over the key tokens of its row's blocks.
 
-    Q [B, Lq, Hq, d]; K, V [B, Lk, Hkv, d]; rows ordered (b, hq, i).  Query
-    token t of row (b, hq, i) sits at position t + q_offset and may see key
+    Q [B, Lq, Hq, d]; K, V [B, Lk, Hkv, d].  The lists hold one row per
+    (b, hq, i), or, when they have B * Hkv * nqb rows (Hkv < Hq), one row per
+    (b, KV head, i) that every q head of the KV head uses.  Query token t of
+    query block i of q head hq sits at position t + q_offset and may see key
     position s of any listed block when s <= t + q_offset (causal).  The KV
     head of q head hq is hq // (Hq / Hkv).  Returns O [B, Lq, Hq, d] (NaN for
     rows not computed) and lse [B, Hq, Lq] = log sum_s exp(scale * q.k_s).
-    ``rows``: optional iterable of row numbers to compute (default: all).
+    ``rows``: optional iterable of (b, hq, i) numbers (b * Hq + hq) * nqb + i
+    to compute (default: all).
     """
     B, Lq, Hq, d = Q.shape
     Hkv = K.shape[2]
@@ -439,13 +475,15 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
         scale = 1.0 / math.sqrt(d)
     O = np.full((B, Lq, Hq, d), np.nan)
     lse = np.full((B, Hq, Lq), np.nan)
+    group_lists = Hkv < Hq and len(row_ptr) - 1 == B * Hkv * nqb
     if rows is None:
         rows = range(B * Hq * nqb)
     for row in rows:
         b, rem = divmod(int(row), Hq * nqb)
         hq, i = divmod(rem, nqb)
         kvh = hq // G
-        blocks = col_idx[row_ptr[row]:row_ptr[row + 1]]
+        lrow = (b * Hkv + kvh) * nqb + i if group_lists else row
+        blocks = col_idx[row_ptr[lrow]:row_ptr[lrow + 1]]
         t0 = i * block_q
         q = as_f64(Q[b, t0:t0 + block_q, hq, :])
         if len(blocks) == 0:

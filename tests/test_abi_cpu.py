@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_housekeeping(L):
-    assert L.rbs_abi_version() == 2
+    assert L.rbs_abi_version() == 3
     assert L.rbs_status_string(0) == b"ok"
     assert L.rbs_status_string(3) == b"capacity"
     p = _abi.SelectParamsC()
@@ -188,3 +188,32 @@ def test_select_rejects_bad_threshold_fields(L):
     st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, 1 << 20,
                       ctypes.byref(ok), None, None)
     assert st == 4  # past validation: no GPU here
+
+
+def test_kv_group_lists_validation(L):
+    """KV_GROUP lists have one row per (batch, KV head, query block); both entry
+    points take exactly that row count in that mode (and reject others)."""
+    s = ctypes.c_void_p(0)
+    q = _fake(Lq=512, H=4)  # 4 q heads, 64-token blocks -> 8 query blocks
+    group = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, 1 * 2 * 8)  # 2 KV heads
+    per_head = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, 1 * 4 * 8)
+    pc = SelectParams(block_q=64, block_k=64, list_mode=1).c()
+    sel = lambda lists, p: L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 2, 8, ctypes.byref(p), 0x60000, 1 << 24,
+                                        ctypes.byref(lists), None, None)
+    assert sel(per_head, pc) == 1
+    assert sel(group, pc) == 4  # past validation: no GPU here
+    assert sel(group, SelectParams(block_q=64, block_k=64).c()) == 1  # per-head mode wants 32 rows
+    assert sel(group, SelectParams(block_q=64, block_k=64, list_mode=2).c()) == 1
+    # capacity of the per-head lists bounds the group unions: sum_g min(n, G x) <= G sum min(n, x)
+    p1 = SelectParams(block_q=64, block_k=64, list_mode=1)
+    assert L.rbs_select_capacity(1, 4, 8, 8, ctypes.byref(p1.c())) == L.rbs_select_capacity(
+        1, 4, 8, 8, ctypes.byref(SelectParams(block_q=64, block_k=64).c()))
+    k = _fake(Lq=512, H=2)
+    o = _fake(Lq=512, H=4)
+    f = L.bsa_prefill
+    for lists in (group, per_head):
+        assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(lists), 64, 64, 0, 0.0, 1,
+                 ctypes.byref(o), None, s) == 4  # both shapes pass validation
+    odd = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, 1 * 3 * 8)
+    assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(odd), 64, 64, 0, 0.0, 1,
+             ctypes.byref(o), None, s) == 1

@@ -524,3 +524,118 @@ def test_max_relative_nested_in_delta():
         a = set(small["col_idx"][small["row_ptr"][row]:small["row_ptr"][row + 1]].tolist())
         b = set(big["col_idx"][big["row_ptr"][row]:big["row_ptr"][row + 1]].tolist())
         assert a <= b
+
+
+# --------------------------------------------------------------------------
+# KV-group lists (one list per KV head, shared by its q heads)
+
+
+def _rows_as_sets(sel):
+    rp, ci = sel["row_ptr"], sel["col_idx"]
+    return [set(ci[rp[r]:rp[r + 1]].tolist()) for r in range(rp.size - 1)]
+
+
+def test_group_lists_with_one_head_per_group_are_the_head_lists():
+    # Hq == Hkv: every group is a single q head, so the union is that head's list
+    inp = make_mixture(L=2048, Hq=2, Hkv=2, block=128, seed=21)
+    C, R = O.block_stats(inp["K"], 128)
+    kw = dict(block_q=128, block_k=128, rho_centroid=0.2, rho_rescue=0.2)
+    a = O.select_blocks(inp["Q"], C, R, O.SelectParams(**kw))
+    b = O.select_blocks(inp["Q"], C, R, O.SelectParams(list_mode=1, **kw))
+    for key in ("row_ptr", "col_idx", "flags"):
+        assert np.array_equal(a[key], b[key])
+
+
+def test_group_lists_are_the_set_union_of_their_heads():
+    # 4 q heads on 2 KV heads, 2 batch entries: group row (b, g, i) must be
+    # exactly the set union of rows (b, 2g, i) and (b, 2g + 1, i), with each
+    # entry's flags the OR of the heads' flags for that block
+    inp = make_mixture(L=2048, Hq=4, Hkv=2, block=128, seed=22, batch=2)
+    C, R = O.block_stats(inp["K"], 128)
+    kw = dict(block_q=128, block_k=128, rho_centroid=0.15, rho_rescue=0.15, force_sink=1)
+    per = O.select_blocks(inp["Q"], C, R, O.SelectParams(**kw))
+    grp = O.select_blocks(inp["Q"], C, R, O.SelectParams(list_mode=1, **kw))
+    nqb, B, Hq, Hkv = 16, 2, 4, 2
+    assert grp["row_ptr"].size - 1 == B * Hkv * nqb
+    hs, gs = _rows_as_sets(per), _rows_as_sets(grp)
+    grew = 0
+    for b in range(B):
+        for g in range(Hkv):
+            for i in range(nqb):
+                heads = [hs[(b * Hq + hq) * nqb + i] for hq in (2 * g, 2 * g + 1)]
+                row = (b * Hkv + g) * nqb + i
+                assert gs[row] == heads[0] | heads[1]
+                grew += len(gs[row]) > max(len(h) for h in heads)
+                e0, e1 = grp["row_ptr"][row], grp["row_ptr"][row + 1]
+                assert np.all(np.diff(grp["col_idx"][e0:e1]) > 0)
+                for e in range(e0, e1):
+                    j, want = int(grp["col_idx"][e]), 0
+                    for hq in (2 * g, 2 * g + 1):
+                        r = (b * Hq + hq) * nqb + i
+                        hit = np.nonzero(per["col_idx"][per["row_ptr"][r]:per["row_ptr"][r + 1]] == j)[0]
+                        if hit.size:
+                            want |= int(per["flags"][per["row_ptr"][r] + hit[0]])
+                    assert int(grp["flags"][e]) == want
+    assert grew > 0  # the heads of a group do select different blocks here
+
+
+def test_group_lists_attention_is_per_head_attention_on_the_shared_row():
+    # attention with one list per KV head equals attention with per-q-head
+    # lists in which every q head carries its group's list
+    inp = make_mixture(L=1024, Hq=4, Hkv=2, block=128, seed=23)
+    C, R = O.block_stats(inp["K"], 128)
+    grp = O.select_blocks(inp["Q"], C, R, O.SelectParams(block_q=128, block_k=128, rho_centroid=0.2,
+                                                          rho_rescue=0.2, list_mode=1))
+    nqb, Hq, G = 8, 4, 2
+    rp, ci = [0], []
+    for hq in range(Hq):
+        for i in range(nqb):
+            r = (hq // G) * nqb + i
+            ci.extend(grp["col_idx"][grp["row_ptr"][r]:grp["row_ptr"][r + 1]].tolist())
+            rp.append(len(ci))
+    rows = [0, 7, 9, 14, 21, 31]
+    Og, lg = O.masked_attention(inp["Q"], inp["K"], inp["V"], grp["row_ptr"], grp["col_idx"], 128, 128, rows=rows)
+    Oe, le = O.masked_attention(inp["Q"], inp["K"], inp["V"], np.asarray(rp), np.asarray(ci), 128, 128, rows=rows)
+    for row in rows:
+        hq, i = divmod(row, nqb)
+        t = slice(i * 128, (i + 1) * 128)
+        assert np.array_equal(Og[0, t, hq], Oe[0, t, hq])
+        assert np.array_equal(lg[0, hq, t], le[0, hq, t])
+    # and the q heads of one group really differ in their queries: same list, different outputs
+    assert not np.allclose(Og[0, 7 * 128:8 * 128, 0], Og[0, 7 * 128:8 * 128, 1])
+
+
+def test_group_pins_catch_planted_mistakes(monkeypatch):
+    good_union = O.group_union_lists
+
+    def interleaved_groups(row_ptr, cols, flags, B, Hq, Hkv, nqb, nkb):
+        # q head hq assigned to group hq % Hkv instead of hq // (Hq / Hkv)
+        perm = [hq for g in range(Hkv) for hq in range(g, Hq, Hkv)]
+        rp, ci, fl = [0], [], []
+        for b in range(B):
+            for hq in perm:
+                for i in range(nqb):
+                    r = (b * Hq + hq) * nqb + i
+                    ci.extend(cols[row_ptr[r]:row_ptr[r + 1]])
+                    fl.extend(flags[row_ptr[r]:row_ptr[r + 1]])
+                    rp.append(len(ci))
+        return good_union(rp, ci, fl, B, Hq, Hkv, nqb, nkb)
+    monkeypatch.setattr(O, "group_union_lists", interleaved_groups)
+    with pytest.raises(AssertionError):
+        test_group_lists_are_the_set_union_of_their_heads()
+    monkeypatch.setattr(O, "group_union_lists", good_union)
+
+    good_attn = O.masked_attention
+
+    def per_head_rows_only(Q, K, V, row_ptr, col_idx, *a, **kw):
+        # a group row read as if it were per-head: q head hq takes row hq * nqb + i
+        B, Lq, Hq, _ = Q.shape
+        nqb = Lq // a[0]
+        rows_in = len(row_ptr) - 1
+        if rows_in == B * Hq * nqb:
+            return good_attn(Q, K, V, row_ptr, col_idx, *a, **kw)
+        rp = list(row_ptr) + [row_ptr[-1]] * (B * Hq * nqb - rows_in)
+        return good_attn(Q, K, V, np.asarray(rp), col_idx, *a, **kw)
+    monkeypatch.setattr(O, "masked_attention", per_head_rows_only)
+    with pytest.raises(AssertionError):
+        test_group_lists_attention_is_per_head_attention_on_the_shared_row()
