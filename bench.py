@@ -13,8 +13,9 @@ selection ms, stats ms, the attention kernel's roofline, clocks, an
 end-to-end number through the same calls with host buffers, the Block-
 attention RAG flow (cache build, RoPE re-encoding, final block), a density
 sweep at 64K (selection and attention time at 2-100% kept density), the same
-prompt with KV-group lists (one list per KV head shared by its q heads) and
-the CPU oracle baseline.
+prompt with KV-group lists (one list per KV head shared by its q heads), the
+same lists with the rescue blocks' contribution weighted by 0.5, and the CPU
+oracle baseline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 N > 1 runs under torchrun: every rank processes its own prompt (weak
@@ -51,9 +52,9 @@ SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
 # dram__bytes_write.sum, one single-pass ncu capture of the default workload;
 # profiles/launches_gqa_rbs_128k.md gives the command), valid for the kernel
 # sources with this digest; any other build reports null.
-ATTN_TRAFFIC_BYTES = 3.234e9 + 1.038e9
+ATTN_TRAFFIC_BYTES = 3.345e9 + 1.039e9
 ATTN_TRAFFIC_SOURCES = ("block_sparse_long_rbs_b200/csrc/attention.cuh", "block_sparse_long_rbs_b200/csrc/common.cuh")
-ATTN_TRAFFIC_DIGEST = "de2dc7480fe2059f"
+ATTN_TRAFFIC_DIGEST = "af8b21ab5100c5b2"
 
 
 def attn_traffic(seq_len: int):
@@ -305,6 +306,8 @@ def run_ours(args, ws, rank):
         out["dense"] = dense_measure(rbs, Q, K, V, B, Hq, nqb, peak)
         out["dense"]["speedup_attn_only"] = round(out["dense"]["ms"] / attn_ms, 2)
         out["dense"]["speedup_with_selection"] = round(out["dense"]["ms"] / (attn_ms + select_ms + stats_ms), 2)
+    if args.rescue_weighted and rank == 0:
+        out["rescue_weighted"] = rescue_weighted_measure(rbs, Q, K, V, lists, flops, attn_ms, peak)
     if args.group_lists and rank == 0:
         out["kv_group_lists"] = group_lists_measure(rbs, Q, K, V, C, R, w.rho, B, Hq, Hkv, nqb, nkb, nnz, peak)
     del Q, K, V, O
@@ -641,6 +644,22 @@ def block_attention_measure(rbs, peaks):
     return res
 
 
+def rescue_weighted_measure(rbs, Q, K, V, lists, flops, attn_ms, peak, weight: float = 0.5):
+    """The same prompt and lists with the rescue-only blocks' softmax mass scaled
+    by `weight` (one pass: a log2(weight) offset on those tiles' logits)."""
+    import torch
+    O = torch.empty_like(Q)
+    fn = lambda: rbs.bsa_prefill_rescue_weighted(Q, K, V, lists, weight, BLOCK, BLOCK, out=O)
+    fn()
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    ms = _time_ms(fn, 5)
+    del O
+    return {"weight": weight, "attn_ms": round(ms, 4), "attn_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "frac_of_peak": round(flops / (ms * 1e-3) / 1e12 / peak, 4),
+            "vs_unweighted_step_attn": round(ms / attn_ms, 4)}
+
+
 def group_lists_measure(rbs, Q, K, V, C, R, rho, B, Hq, Hkv, nqb, nkb, nnz_heads, peak):
     """KV-group lists (one list per KV head, the union of its q heads'):
     selection and attention time on the same prompt, and how many more block
@@ -837,6 +856,7 @@ def main():
     ap.add_argument("--no-isolated", dest="isolated", action="store_false")
     ap.add_argument("--no-selector-quality", dest="selector_quality", action="store_false")
     ap.add_argument("--no-group-lists", dest="group_lists", action="store_false")
+    ap.add_argument("--no-rescue-weighted", dest="rescue_weighted", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--seq-len", type=int, default=None,

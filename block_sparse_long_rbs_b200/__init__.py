@@ -217,6 +217,26 @@ def bsa_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, lists: BlockL
     return (out, lse) if return_lse else out
 
 
+def bsa_prefill_rescue_weighted(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, lists: BlockLists,
+                                rescue_weight: float, block_q: int = 128, block_k: int = 128, q_offset: int = 0,
+                                softmax_scale: float | None = None, causal: bool = True,
+                                out: torch.Tensor | None = None, return_lse: bool = False):
+    """bsa_prefill with the rescue-only blocks' softmax mass scaled by rescue_weight
+    (the lists' flags say which entries those are)."""
+    if out is None:
+        out = torch.empty_like(Q)
+    lse = None
+    if return_lse:
+        lse = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], dtype=torch.float32, device=Q.device)
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(Q.shape[-1])
+    lc = lists.c()
+    check(lib().bsa_prefill_rescue_weighted(
+        ctypes.byref(_t(Q, "Q")), ctypes.byref(_t(K, "K")), ctypes.byref(_t(V, "V")), ctypes.byref(lc), block_q,
+        block_k, q_offset, scale, 1 if causal else 0, float(rescue_weight), ctypes.byref(_t(out, "O")),
+        lse.data_ptr() if lse is not None else None, _stream()), "bsa_prefill_rescue_weighted")
+    return (out, lse) if return_lse else out
+
+
 def rope_reencode(x: torch.Tensor, old_pos: torch.Tensor, new_pos: torch.Tensor, theta: float, rope_style: int = 0,
                   out: torch.Tensor | None = None) -> torch.Tensor:
     """Move RoPE-encoded vectors from old_pos to new_pos (out may be x for in place)."""

@@ -65,6 +65,8 @@ SIGNATURES = {
     "rbs_lists_block_attention": (ctypes.c_int, [P(i32), i32, i32, i32, i32, i32, i32, i32, P(BlockListsC), vp]),
     "bsa_prefill": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), P(Bf16Tensor), P(BlockListsC), i32, i32, i64, f32,
                                    i32, P(Bf16Tensor), vp, vp]),
+    "bsa_prefill_rescue_weighted": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), P(Bf16Tensor), P(BlockListsC), i32,
+                                                   i32, i64, f32, i32, f32, P(Bf16Tensor), vp, vp]),
     "rope_reencode": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), vp, vp, f32, i32, vp]),
 }
 

@@ -28,6 +28,9 @@
 //              maximum; the running max is lazily updated (O_h rescaled in
 //              TMEM only when it grows by more than 2^8; the final
 //              normalisation uses the same max, so the result is exact).
+//              A tile of a rescue-only block whose contribution is weighted
+//              by w has log2(w) added to its scaled scores (max and
+//              exponentials alike), which weights its softmax mass by w.
 //              Pass 2 forms P = exp2(S*c - m_h) from the registers (3 of every
 //              8 element pairs on the FMA pipe, see exp2_fma2, the rest on the
 //              SFU) and writes it as packed bf16 pairs over the first quarter
@@ -72,6 +75,11 @@ struct AttnArgs {
   int B, Hq, Hkv, nqb, nkb, Lq;
   int q_block_off, causal, num_rows;  // num_rows: work items, B * Hq * nqb
   int group_lists;  // 1: list row (b, KV head, i) serves every q head of the KV head
+  // rescue blocks weighted by w: entries whose flags are exactly "rescue
+  // branch only" get log2(w) added to their logits (in log2 units); flags is
+  // null when every block has weight 1
+  const uint8_t* flags;
+  float rescue_bias;
   float scale_log2;
 };
 
@@ -410,9 +418,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       float m_used = -INFINITY;  // this half's running max, in log2 units (score * c)
       float2 l2 = make_float2(0.f, 0.f);  // this half's row sum
       int j_next = __ldg(a.col_idx + x.beg);
+      int f_next = a.flags != nullptr ? __ldg(a.flags + x.beg) : 0;
       for (int t = 0; t < n; ++t, ++g) {
         const int j = j_next;
-        if (t + 1 < n) j_next = __ldg(a.col_idx + x.beg + t + 1);
+        // log2 weight of this tile: log2(w) for a rescue-only block, else 0
+        const float bias = (f_next & 7) == 2 ? a.rescue_bias : 0.f;
+        if (t + 1 < n) {
+          j_next = __ldg(a.col_idx + x.beg + t + 1);
+          if (a.flags != nullptr) f_next = __ldg(a.flags + x.beg + t + 1);
+        }
         const int b = g % L::kSBufs;
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + b), (g / L::kSBufs) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
@@ -444,7 +458,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           for (int e = 1; e < 31; e += 2) m0 = fmax3(m0, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
           mx = fmax3(mx, m0, __uint_as_float(v[q][31]));
         }
-        const float m_new = fmaxf(m_used, mx * c);
+        const float m_new = fmaxf(m_used, fmaf(mx, c, bias));
         float factor = 1.f;
         bool rescale = false;
         if (t == 0) {
@@ -459,7 +473,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         l2.y *= factor;
         // pass 2: P = exp2(s*c - m) from the registers, written as packed bf16
         // pairs over the first kHalf/2 of this warp's S columns (already read)
-        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_exp, -m_exp);
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(bias - m_exp, bias - m_exp);
         float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         uint32_t pw[kHalf / 2];
 #pragma unroll

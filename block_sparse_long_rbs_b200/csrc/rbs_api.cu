@@ -622,9 +622,16 @@ rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t num_segme
 
 // ---------------------------------------------------------------------------
 
-rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
-                       const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
-                       float softmax_scale, int32_t causal, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// bsa_prefill and its rescue-weighted form: flags == nullptr gives every
+// block weight 1; otherwise rescue-only entries get log2(w) = rescue_bias.
+rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                      const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
+                      float softmax_scale, int32_t causal, const uint8_t* flags, float rescue_bias,
+                      rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
   rbs_status st;
   if ((st = check_tensor(Q, "Q")) != RBS_OK) return st;
   if ((st = check_tensor(K, "K")) != RBS_OK) return st;
@@ -671,6 +678,8 @@ rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const
   a.causal = causal ? 1 : 0;
   a.num_rows = static_cast<int>(rows);
   a.group_lists = group_lists ? 1 : 0;
+  a.flags = flags;
+  a.rescue_bias = rescue_bias;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(RBS_HEAD_DIM));
   a.scale_log2 = scale * 1.4426950408889634f;
   const int grid = static_cast<int>(std::min<int64_t>(rows, di->sms));
@@ -679,6 +688,31 @@ rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const
   else
     bsa_prefill_kernel<64, 64><<<grid, kAttnThreads, AttnSmem<64>::kAlloc, stream>>>(a);
   return check_launch("bsa_prefill_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                       const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
+                       float softmax_scale, int32_t causal, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
+  return launch_bsa(Q, K, V, lists, block_q, block_k, q_offset, softmax_scale, causal, nullptr, 0.f, O, lse, stream);
+}
+
+rbs_status bsa_prefill_rescue_weighted(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                                       const rbs_block_lists* lists, int32_t block_q, int32_t block_k,
+                                       int64_t q_offset, float softmax_scale, int32_t causal, float rescue_weight,
+                                       rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
+  RBS_REQUIRE(rescue_weight >= 0.f && std::isfinite(rescue_weight), RBS_ERR_INVALID_ARG,
+              "rescue_weight must be finite and >= 0");
+  if (rescue_weight == 1.f)
+    return launch_bsa(Q, K, V, lists, block_q, block_k, q_offset, softmax_scale, causal, nullptr, 0.f, O, lse, stream);
+  RBS_REQUIRE(lists != nullptr && lists->flags != nullptr, RBS_ERR_INVALID_ARG,
+              "rescue weighting needs the lists' branch flags");
+  const float bias = rescue_weight > 0.f ? std::log2(rescue_weight) : -INFINITY;
+  return launch_bsa(Q, K, V, lists, block_q, block_k, q_offset, softmax_scale, causal, lists->flags, bias, O, lse,
+                    stream);
 }
 
 // ---------------------------------------------------------------------------

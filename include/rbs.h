@@ -286,6 +286,27 @@ RBS_API rbs_status bsa_prefill(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* 
                        const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
                        float softmax_scale, int32_t causal, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream);
 
+/* ---- rescue blocks with a controlled contribution  ([RBS-id] "Dual-Branch
+ * Selection": regular blocks through the block-sparse pass, rescue blocks
+ * handled separately, their contribution controllable)
+ * A list entry is a rescue block when its flags have the rescue bit and
+ * neither the centroid nor the forced bit; every other entry is regular.  With
+ * x_s = scale * q_t . k_s and w = rescue_weight:
+ *   O[b, t, h] = (sum_{s regular} e^{x_s} v_s + w sum_{s rescue} e^{x_s} v_s)
+ *              / (sum_{s regular} e^{x_s}     + w sum_{s rescue} e^{x_s})
+ * i.e. the regular and the rescue partial attentions merged with the rescue
+ * partial's softmax mass scaled by w; lse = ln of that denominator (-inf and
+ * O = 0 when it is 0).  w = 1 is bsa_prefill; w = 0 keeps the regular blocks
+ * only.  Arguments, layouts and errors as bsa_prefill, plus:
+ *   rescue_weight  finite, >= 0 (else RBS_ERR_INVALID_ARG)
+ *   lists->flags   required unless rescue_weight == 1 (else RBS_ERR_INVALID_ARG)
+ * One pass: the kernel adds log2(w) to the scaled scores of the rescue
+ * blocks' tiles, which weights their softmax mass by w. */
+RBS_API rbs_status bsa_prefill_rescue_weighted(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K,
+                                       const rbs_bf16_tensor* V, const rbs_block_lists* lists, int32_t block_q,
+                                       int32_t block_k, int64_t q_offset, float softmax_scale, int32_t causal,
+                                       float rescue_weight, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream);
+
 /* ---- RoPE position re-encoding  ([BA] 2.3 Position re-encoding, 2.5 Inference)
  * Keys cached with RoPE at old_pos are moved to new_pos: the rotation is reset
  * to position 0 and applied again at the new position, done as one rotation by

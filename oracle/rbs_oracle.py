@@ -507,6 +507,59 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
     return O, lse
 
 
+def split_regular_rescue(row_ptr, col_idx, flags):
+    """Split lists into the regular blocks (kept by the centroid branch, or
+    forced) and the rescue blocks (kept by the rescue branch alone), each in
+    CSR form over the same rows ([RBS-id] "Dual-Branch Selection": regular
+    blocks go through the standard block-sparse pass, rescue blocks are
+    handled separately).  Entries without any flag count as regular."""
+    reg_ptr, reg_idx, res_ptr, res_idx = [0], [], [0], []
+    for r in range(len(row_ptr) - 1):
+        for e in range(row_ptr[r], row_ptr[r + 1]):
+            f = int(flags[e])
+            rescue_only = (f & FLAG_RESCUE) and not (f & (FLAG_CENTROID | FLAG_FORCED))
+            (res_idx if rescue_only else reg_idx).append(int(col_idx[e]))
+        reg_ptr.append(len(reg_idx))
+        res_ptr.append(len(res_idx))
+    as_arr = lambda x: np.asarray(x, dtype=np.int64)
+    return as_arr(reg_ptr), as_arr(reg_idx), as_arr(res_ptr), as_arr(res_idx)
+
+
+def rescue_weighted_attention(Q, K, V, row_ptr, col_idx, flags, rescue_weight: float, block_q: int, block_k: int,
+                              q_offset: int = 0, scale: float | None = None, causal: int = 1, rows=None):
+    """Attention with the rescue blocks handled separately and their contribution
+    scaled by rescue_weight (gamma >= 0) ([RBS-id] "Dual-Branch Selection": the
+    rescue blocks' contribution can be controlled precisely).
+
+    The regular blocks and the rescue blocks are each attended on their own
+    (softmax partials O_reg, lse_reg and O_res, lse_res), and the partials are
+    merged with the rescue partial's softmax mass multiplied by gamma:
+      Z = exp(lse_reg) + gamma exp(lse_res)
+      O = (exp(lse_reg) O_reg + gamma exp(lse_res) O_res) / Z,  lse = log Z.
+    gamma = 1 is attention over the union of both sets; gamma = 0 is attention
+    over the regular blocks alone.  A row with Z = 0 gives O = 0, lse = -inf.
+    Arguments as masked_attention, plus the lists' flags.
+    """
+    reg_ptr, reg_idx, res_ptr, res_idx = split_regular_rescue(row_ptr, col_idx, flags)
+    Oa, la = masked_attention(Q, K, V, reg_ptr, reg_idx, block_q, block_k, q_offset, scale, causal, rows)
+    Ob, lb = masked_attention(Q, K, V, res_ptr, res_idx, block_q, block_k, q_offset, scale, causal, rows)
+    m = np.maximum(la, lb)
+    m = np.where(np.isfinite(m), m, 0.0)
+    with np.errstate(invalid="ignore", over="ignore"):
+        wa = np.where(np.isfinite(la), np.exp(la - m), 0.0)
+        wb = np.where(np.isfinite(lb), rescue_weight * np.exp(lb - m), 0.0)
+        z = wa + wb
+        Oa0 = np.where(np.isfinite(la)[..., None].transpose(0, 2, 1, 3), Oa, 0.0)
+        Ob0 = np.where(np.isfinite(lb)[..., None].transpose(0, 2, 1, 3), Ob, 0.0)
+        wa_t, wb_t, z_t = (x.transpose(0, 2, 1)[..., None] for x in (wa, wb, z))
+        O = np.where(z_t > 0, (wa_t * Oa0 + wb_t * Ob0) / np.where(z_t > 0, z_t, 1.0), 0.0)
+        lse = np.where(z > 0, np.log(np.where(z > 0, z, 1.0)) + m, -np.inf)
+    nan_rows = np.isnan(la)  # rows not computed stay NaN
+    O = np.where(nan_rows.transpose(0, 2, 1)[..., None], np.nan, O)
+    lse = np.where(nan_rows, np.nan, lse)
+    return O, lse
+
+
 def dense_causal_attention(Q, K, V, q_offset: int = 0, scale: float | None = None):
     """Textbook softmax(scale * Q K^T + causal mask) V per q head, full matrices (no blocks).
 

@@ -639,3 +639,121 @@ def test_group_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "masked_attention", per_head_rows_only)
     with pytest.raises(AssertionError):
         test_group_lists_attention_is_per_head_attention_on_the_shared_row()
+
+
+# --------------------------------------------------------------------------
+# Rescue blocks handled separately with a weighted contribution
+# ([RBS-id] "Dual-Branch Selection")
+
+
+def _weighted_case(seed=31):
+    inp = make_mixture(L=1024, Hq=2, Hkv=1, block=128, seed=seed)
+    C, R = O.block_stats(inp["K"], 128)
+    sel = O.select_blocks(inp["Q"], C, R, O.SelectParams(block_q=128, block_k=128, rho_centroid=0.2,
+                                                          rho_rescue=0.3))
+    return inp, sel
+
+
+def _filtered(sel, keep):
+    rp, ci, fl = sel["row_ptr"], sel["col_idx"], sel["flags"]
+    out_p, out_c = [0], []
+    for r in range(rp.size - 1):
+        out_c.extend(int(ci[e]) for e in range(rp[r], rp[r + 1]) if keep(int(fl[e])))
+        out_p.append(len(out_c))
+    return np.asarray(out_p), np.asarray(out_c, dtype=np.int64)
+
+
+def test_rescue_weight_one_is_union_attention_and_zero_is_regular_only():
+    inp, sel = _weighted_case()
+    args = (inp["Q"], inp["K"], inp["V"])
+    rescue_rows = 0
+    for r in range(sel["row_ptr"].size - 1):
+        f = sel["flags"][sel["row_ptr"][r]:sel["row_ptr"][r + 1]]
+        rescue_rows += bool(np.any(f == O.FLAG_RESCUE))
+    assert rescue_rows >= 4  # the case exercises rescue-only blocks
+    W1, l1 = O.rescue_weighted_attention(*args, sel["row_ptr"], sel["col_idx"], sel["flags"], 1.0, 128, 128)
+    U, lu = O.masked_attention(*args, sel["row_ptr"], sel["col_idx"], 128, 128)
+    np.testing.assert_allclose(W1, U, atol=1e-12)
+    np.testing.assert_allclose(l1, lu, atol=1e-12)
+    W0, l0 = O.rescue_weighted_attention(*args, sel["row_ptr"], sel["col_idx"], sel["flags"], 0.0, 128, 128)
+    rp, ci = _filtered(sel, lambda f: bool(f & (O.FLAG_CENTROID | O.FLAG_FORCED)))
+    G0, lg0 = O.masked_attention(*args, rp, ci, 128, 128)
+    np.testing.assert_allclose(W0, G0, atol=1e-12)
+    np.testing.assert_allclose(l0, lg0, atol=1e-12)
+    assert not np.allclose(W0, U, atol=1e-6)
+
+
+def test_rescue_weight_closed_form_two_keys():
+    # one query token at position 1 sees key 0 (a rescue-only block) and key 1
+    # (its forced diagonal block), blocks of one token: the output is the
+    # two-term weighted softmax (e^{s1} v1 + g e^{s0} v0) / (e^{s1} + g e^{s0})
+    rng = np.random.default_rng(32)
+    d = 128
+    Q = rng.standard_normal((1, 2, 1, d))
+    K = rng.standard_normal((1, 2, 1, d))
+    V = rng.standard_normal((1, 2, 1, d))
+    rp = np.array([0, 1, 3])
+    ci = np.array([0, 0, 1])
+    fl = np.array([O.FLAG_FORCED, O.FLAG_RESCUE, O.FLAG_FORCED], dtype=np.uint8)
+    for g in (0.0, 0.3, 1.0, 7.5):
+        W, lse = O.rescue_weighted_attention(Q, K, V, rp, ci, fl, g, 1, 1)
+        s0 = float(Q[0, 1, 0] @ K[0, 0, 0]) / math.sqrt(d)
+        s1 = float(Q[0, 1, 0] @ K[0, 1, 0]) / math.sqrt(d)
+        z = math.exp(s1) + g * math.exp(s0)
+        want = (math.exp(s1) * V[0, 1, 0] + g * math.exp(s0) * V[0, 0, 0]) / z
+        np.testing.assert_allclose(W[0, 1, 0], want, rtol=1e-12, atol=1e-13)
+        assert lse[0, 0, 1] == pytest.approx(math.log(z), abs=1e-12)
+        np.testing.assert_allclose(W[0, 0, 0], V[0, 0, 0], atol=1e-15)  # row 0: its diagonal key only
+
+
+def test_rescue_weight_large_limit_is_rescue_only_attention():
+    inp, sel = _weighted_case(seed=33)
+    args = (inp["Q"], inp["K"], inp["V"])
+    rp, ci = _filtered(sel, lambda f: f == O.FLAG_RESCUE)
+    Wb, _ = O.rescue_weighted_attention(*args, sel["row_ptr"], sel["col_idx"], sel["flags"], 1e30, 128, 128)
+    Rb, lrb = O.masked_attention(*args, rp, ci, 128, 128)
+    nqb = 8
+    for row in range(rp.size - 1):
+        if rp[row + 1] == rp[row]:
+            continue
+        hq, i = divmod(row, nqb)
+        t = slice(i * 128, (i + 1) * 128)
+        np.testing.assert_allclose(Wb[0, t, hq], Rb[0, t, hq], atol=1e-9)
+
+
+def test_rescue_weight_pins_catch_planted_mistakes(monkeypatch):
+    good = O.split_regular_rescue
+
+    def forced_as_rescue(row_ptr, col_idx, flags):
+        # a forced block that the rescue branch also kept treated as rescue
+        fl = [O.FLAG_RESCUE if (int(f) & O.FLAG_RESCUE and not int(f) & O.FLAG_CENTROID) else int(f) for f in flags]
+        return good(row_ptr, col_idx, fl)
+    monkeypatch.setattr(O, "split_regular_rescue", forced_as_rescue)
+    with pytest.raises(AssertionError):
+        test_rescue_weight_closed_form_two_keys_forced_and_rescue()
+    monkeypatch.setattr(O, "split_regular_rescue", good)
+
+    def swapped(row_ptr, col_idx, flags):  # the weight lands on the regular partial instead
+        reg_p, reg_i, res_p, res_i = good(row_ptr, col_idx, flags)
+        return res_p, res_i, reg_p, reg_i
+    monkeypatch.setattr(O, "split_regular_rescue", swapped)
+    with pytest.raises(AssertionError):
+        test_rescue_weight_closed_form_two_keys()
+
+
+def test_rescue_weight_closed_form_two_keys_forced_and_rescue():
+    # a block both forced and kept by the rescue branch is regular: its weight
+    # does not depend on gamma
+    rng = np.random.default_rng(34)
+    d = 128
+    Q = rng.standard_normal((1, 2, 1, d))
+    K = rng.standard_normal((1, 2, 1, d))
+    V = rng.standard_normal((1, 2, 1, d))
+    rp = np.array([0, 1, 3])
+    ci = np.array([0, 0, 1])
+    fl = np.array([O.FLAG_FORCED, O.FLAG_RESCUE, O.FLAG_FORCED | O.FLAG_RESCUE], dtype=np.uint8)
+    a, _ = O.rescue_weighted_attention(Q, K, V, rp, ci, fl, 0.25, 1, 1)
+    s0 = float(Q[0, 1, 0] @ K[0, 0, 0]) / math.sqrt(d)
+    s1 = float(Q[0, 1, 0] @ K[0, 1, 0]) / math.sqrt(d)
+    want = (math.exp(s1) * V[0, 1, 0] + 0.25 * math.exp(s0) * V[0, 0, 0]) / (math.exp(s1) + 0.25 * math.exp(s0))
+    np.testing.assert_allclose(a[0, 1, 0], want, rtol=1e-12, atol=1e-13)
