@@ -109,7 +109,7 @@ def _f32(x: torch.Tensor, name: str) -> int:
 def rbs_block_stats(K: torch.Tensor, block_k: int):
     """Centroids [B, Hkv, nKB, 128] and radii [B, Hkv, nKB] (fp32) of every key block."""
     B, L, H, D = K.shape
-    nkb = L // block_k
+    nkb = -(-L // block_k)  # a last, partial block holds the remaining keys
     C = torch.empty(B, H, nkb, D, dtype=torch.float32, device=K.device)
     R = torch.empty(B, H, nkb, dtype=torch.float32, device=K.device)
     check(lib().rbs_block_stats(ctypes.byref(_t(K, "K")), block_k, C.data_ptr(), R.data_ptr(), _stream()),
@@ -131,7 +131,7 @@ def rbs_block_beta(radii: torch.Tensor, params: SelectParams):
 def rbs_pool_queries(Q: torch.Tensor, block_q: int):
     """qbar [B, Hq, nQB, 128] and qnorm [B, Hq, nQB] (fp32)."""
     B, L, H, D = Q.shape
-    nqb = L // block_q
+    nqb = -(-L // block_q)
     qbar = torch.empty(B, H, nqb, D, dtype=torch.float32, device=Q.device)
     qnorm = torch.empty(B, H, nqb, dtype=torch.float32, device=Q.device)
     check(lib().rbs_pool_queries(ctypes.byref(_t(Q, "Q")), block_q, qbar.data_ptr(), qnorm.data_ptr(), _stream()),
@@ -158,7 +158,7 @@ def rbs_select(Q: torch.Tensor, centroids: torch.Tensor, radii: torch.Tensor, pa
     (batch, KV head, query block) when params.list_mode == 1."""
     B, L, Hq, _ = Q.shape
     Hkv, nkb = centroids.shape[1], centroids.shape[2]
-    nqb = L // params.block_q
+    nqb = -(-L // params.block_q)
     rows = B * (Hkv if params.list_mode == 1 else Hq) * nqb
     if out is None:
         out = BlockLists.empty(rows, rbs_select_capacity(B, Hq, nqb, nkb, params), Q.device, flags)

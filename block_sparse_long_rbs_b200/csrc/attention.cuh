@@ -73,6 +73,7 @@ struct AttnArgs {
   int64_t ob, os, oh;
   float* lse;
   int B, Hq, Hkv, nqb, nkb, Lq;
+  int k_tail;  // keys in the last key block (BK unless Lk is not a block multiple)
   int q_block_off, causal, num_rows;  // num_rows: work items, B * Hq * nqb
   int group_lists;  // 1: list row (b, KV head, i) serves every q head of the KV head
   // rescue blocks weighted by w: entries whose flags are exactly "rescue
@@ -402,11 +403,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         const int ei = __shfl_sync(0xffffffffu, i, src);
         for (int k = lane; k < BQ * 16; k += 32) {
           const int64_t qrow = static_cast<int64_t>(ei) * BQ + (k >> 4);
-          reinterpret_cast<uint4*>(a.O + eb * a.ob + qrow * a.os + eh * a.oh)[k & 15] = make_uint4(0, 0, 0, 0);
+          if (qrow < a.Lq)
+            reinterpret_cast<uint4*>(a.O + eb * a.ob + qrow * a.os + eh * a.oh)[k & 15] = make_uint4(0, 0, 0, 0);
         }
         if (a.lse != nullptr)
           for (int k = lane; k < BQ; k += 32)
-            a.lse[(static_cast<int64_t>(eb) * a.Hq + eh) * a.Lq + static_cast<int64_t>(ei) * BQ + k] = -INFINITY;
+            if (static_cast<int64_t>(ei) * BQ + k < a.Lq)
+              a.lse[(static_cast<int64_t>(eb) * a.Hq + eh) * a.Lq + static_cast<int64_t>(ei) * BQ + k] = -INFINITY;
       }
     }
 
@@ -433,6 +436,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         const bool bad = j < 0 || j >= a.nkb;
         const bool dead = bad || (a.causal && j > gi);
         const bool diag = a.causal && j == gi;
+        const bool tail = j == a.nkb - 1 && a.k_tail < BK;  // keys past Lk were loaded as zeros
         if (dead && r == 0 && hf == 0) raise_error(bad ? RBS_DEVERR_BLOCK_INDEX : RBS_DEVERR_NONCAUSAL);
         // pass 1: this warp's half row of S into registers, masked; its maximum
         const uint32_t scol = L::col_s(b) + hf * kHalf;
@@ -440,11 +444,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
 #pragma unroll
         for (int q = 0; q < kHalf / 32; ++q) tmem_ld32(lane_base + scol + 32 * q, v[q]);
         tmem_wait_ld();
-        if (dead || diag) {
-          // tile column hf * kHalf + 32 q + e is masked when it is above the diagonal (or always)
+        if (dead || diag || tail) {
+          // tile column hf * kHalf + 32 q + e is masked when it is above the
+          // diagonal, past the last key, or always (a dead tile)
 #pragma unroll
           for (int q = 0; q < kHalf / 32; ++q) {
-            const int lim = dead ? -1 : r - (hf * kHalf + 32 * q);
+            const int col0 = hf * kHalf + 32 * q;
+            int lim = dead ? -1 : BK;
+            if (diag) lim = min(lim, r - col0);
+            if (tail) lim = min(lim, a.k_tail - 1 - col0);
 #pragma unroll
             for (int e = 0; e < 32; ++e)
               if (e > lim) v[q][e] = __float_as_uint(-INFINITY);
@@ -544,7 +552,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         float o[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = fmaf(__uint_as_float(vb[e]), s1, __uint_as_float(va[e]) * s0);
-        if (r < BQ) {
+        if (r < BQ && qrow < a.Lq) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             dst[4 * q + k] = make_uint4(pack_bf16x2(o[8 * k], o[8 * k + 1]), pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
@@ -552,7 +560,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
                                         pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
         }
       }
-      if (hf == 0 && a.lse != nullptr && r < BQ) {
+      if (hf == 0 && a.lse != nullptr && r < BQ && qrow < a.Lq) {
         a.lse[(static_cast<int64_t>(x.b) * a.Hq + x.h) * a.Lq + qrow] =
             lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
       }

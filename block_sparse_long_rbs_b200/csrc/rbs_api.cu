@@ -278,20 +278,20 @@ rbs_status rbs_block_stats(const rbs_bf16_tensor* K, int32_t block_k, float* cen
   rbs_status st = check_tensor(K, "K");
   if (st != RBS_OK) return st;
   RBS_REQUIRE(block_k == 64 || block_k == 128, RBS_ERR_UNSUPPORTED, "block_k must be 64 or 128");
-  RBS_REQUIRE(K->seqlen % block_k == 0, RBS_ERR_UNSUPPORTED, "seqlen %% block_k != 0");
   RBS_REQUIRE(centroids != nullptr && radii != nullptr, RBS_ERR_INVALID_ARG, "null output");
   RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
   DeviceInfo* di;
   if ((st = device_info(&di)) != RBS_OK) return st;
-  const int nkb = static_cast<int>(K->seqlen / block_k);
+  const int nkb = static_cast<int>((K->seqlen + block_k - 1) / block_k);
+  const int L = static_cast<int>(K->seqlen);
   const dim3 grid(nkb, static_cast<unsigned>(K->heads), static_cast<unsigned>(K->batch));
   const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K->data);
   if (block_k == 128)
     block_stats_kernel<128><<<grid, 128, 0, stream>>>(k, K->stride_b, K->stride_s, K->stride_h, nkb,
-                                                      static_cast<int>(K->heads), centroids, radii);
+                                                      static_cast<int>(K->heads), L, centroids, radii);
   else
     block_stats_kernel<64><<<grid, 128, 0, stream>>>(k, K->stride_b, K->stride_s, K->stride_h, nkb,
-                                                     static_cast<int>(K->heads), centroids, radii);
+                                                     static_cast<int>(K->heads), L, centroids, radii);
   return check_launch("block_stats_kernel");
 }
 
@@ -320,18 +320,20 @@ rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, float* qb
   rbs_status st = check_tensor(Q, "Q");
   if (st != RBS_OK) return st;
   RBS_REQUIRE(block_q == 64 || block_q == 128, RBS_ERR_UNSUPPORTED, "block_q must be 64 or 128");
-  RBS_REQUIRE(Q->seqlen % block_q == 0, RBS_ERR_UNSUPPORTED, "seqlen %% block_q != 0");
   RBS_REQUIRE(qbar != nullptr && qnorm != nullptr && aligned16(qbar), RBS_ERR_INVALID_ARG, "bad output");
   DeviceInfo* di;
   if ((st = device_info(&di)) != RBS_OK) return st;
-  const int nqb = static_cast<int>(Q->seqlen / block_q);
+  const int nqb = static_cast<int>((Q->seqlen + block_q - 1) / block_q);
+  const int L = static_cast<int>(Q->seqlen);
   const int Hq = static_cast<int>(Q->heads);
   const dim3 grid(nqb, (Hq + 3) / 4, static_cast<unsigned>(Q->batch));
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q->data);
   if (block_q == 128)
-    pool_queries_kernel<128><<<grid, 256, 0, stream>>>(q, Q->stride_b, Q->stride_s, Q->stride_h, Hq, nqb, qbar, qnorm);
+    pool_queries_kernel<128><<<grid, 256, 0, stream>>>(q, Q->stride_b, Q->stride_s, Q->stride_h, Hq, nqb, L, qbar,
+                                                       qnorm);
   else
-    pool_queries_kernel<64><<<grid, 256, 0, stream>>>(q, Q->stride_b, Q->stride_s, Q->stride_h, Hq, nqb, qbar, qnorm);
+    pool_queries_kernel<64><<<grid, 256, 0, stream>>>(q, Q->stride_b, Q->stride_s, Q->stride_h, Hq, nqb, L, qbar,
+                                                      qnorm);
   return check_launch("pool_queries_kernel");
 }
 
@@ -368,7 +370,6 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   RBS_REQUIRE(p != nullptr && centroids != nullptr && radii != nullptr, RBS_ERR_INVALID_ARG, "null argument");
   RBS_REQUIRE(p->block_q == p->block_k && (p->block_q == 64 || p->block_q == 128), RBS_ERR_UNSUPPORTED,
               "block_q must equal block_k, 64 or 128");
-  RBS_REQUIRE(Q->seqlen % p->block_q == 0, RBS_ERR_UNSUPPORTED, "seqlen %% block_q != 0");
   RBS_REQUIRE(kv_heads > 0 && Q->heads % kv_heads == 0, RBS_ERR_INVALID_ARG, "heads_q %% kv_heads != 0");
   RBS_REQUIRE(num_kv_blocks > 0 && num_kv_blocks <= RBS_MAX_KV_BLOCKS, RBS_ERR_UNSUPPORTED,
               "num_kv_blocks must be in [1, %d]", RBS_MAX_KV_BLOCKS);
@@ -381,7 +382,7 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   RBS_REQUIRE(p->q_block_offset >= 0, RBS_ERR_INVALID_ARG, "q_block_offset < 0");
   RBS_REQUIRE(p->list_mode == 0 || p->list_mode == 1, RBS_ERR_INVALID_ARG, "list_mode must be 0 or 1");
   RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
-  const int64_t B = Q->batch, Hq = Q->heads, nqb = Q->seqlen / p->block_q, nkb = num_kv_blocks;
+  const int64_t B = Q->batch, Hq = Q->heads, nqb = (Q->seqlen + p->block_q - 1) / p->block_q, nkb = num_kv_blocks;
   const int64_t rows = B * Hq * nqb;                                       // one per q head
   const int64_t list_rows = p->list_mode == 1 ? B * kv_heads * nqb : rows;  // rows of the output lists
   if ((st = check_lists(out, list_rows)) != RBS_OK) return st;
@@ -414,6 +415,7 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   sa.Hq = static_cast<int>(Hq);
   sa.Hkv = kv_heads;
   sa.items = static_cast<int>(B * nqb * (Hq / R));
+  sa.Lq = static_cast<int>(Q->seqlen);
   sa.seq_inner = seq_inner;
   sa.nqb = static_cast<int>(nqb);
   sa.nkb = static_cast<int>(nkb);
@@ -523,10 +525,10 @@ rbs_status rbs_select_noalloc(const rbs_bf16_tensor* Q, const float* centroids, 
                               rbs_block_lists* out, float* beta_out, rbs_stream_t stream) {
   rbs_status st = check_tensor(Q, "Q");
   if (st != RBS_OK) return st;
-  RBS_REQUIRE(p != nullptr && (p->block_q == 64 || p->block_q == 128) && Q->seqlen % p->block_q == 0,
-              RBS_ERR_UNSUPPORTED, "block_q must be 64 or 128 and divide seqlen");
+  RBS_REQUIRE(p != nullptr && (p->block_q == 64 || p->block_q == 128), RBS_ERR_UNSUPPORTED,
+              "block_q must be 64 or 128");
   RBS_REQUIRE(kv_heads > 0 && num_kv_blocks > 0, RBS_ERR_INVALID_ARG, "empty KV shape");
-  const size_t need = rbs_select_workspace_bytes(Q->batch, Q->heads, Q->seqlen / p->block_q, kv_heads,
+  const size_t need = rbs_select_workspace_bytes(Q->batch, Q->heads, (Q->seqlen + p->block_q - 1) / p->block_q, kv_heads,
                                                  num_kv_blocks, p);
   RBS_REQUIRE(need > 0 && need <= RBS_NOALLOC_SCRATCH_BYTES, RBS_ERR_CAPACITY,
               "this selection needs %zu bytes of scratch; the built-in buffer holds %zu (use rbs_select with a "
@@ -643,9 +645,8 @@ rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const 
   RBS_REQUIRE(K->seqlen == V->seqlen && K->heads == V->heads, RBS_ERR_INVALID_ARG, "K/V shape mismatch");
   RBS_REQUIRE(O->seqlen == Q->seqlen && O->heads == Q->heads, RBS_ERR_INVALID_ARG, "O shape != Q shape");
   RBS_REQUIRE(Q->heads % K->heads == 0, RBS_ERR_INVALID_ARG, "heads_q %% heads_kv != 0");
-  RBS_REQUIRE(Q->seqlen % block_q == 0 && K->seqlen % block_k == 0, RBS_ERR_UNSUPPORTED, "seqlen not a block multiple");
   RBS_REQUIRE(q_offset >= 0 && q_offset % block_k == 0, RBS_ERR_UNSUPPORTED, "q_offset must be a non-negative block multiple");
-  const int64_t nqb = Q->seqlen / block_q;
+  const int64_t nqb = (Q->seqlen + block_q - 1) / block_q;
   const int64_t rows = Q->batch * Q->heads * nqb;  // work items: one per (batch, q head, query block)
   // one list per q head, or one per KV head shared by its q heads
   const bool group_lists = lists != nullptr && Q->heads != K->heads && lists->num_rows == Q->batch * K->heads * nqb;
@@ -672,7 +673,8 @@ rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const 
   a.Hq = static_cast<int>(Q->heads);
   a.Hkv = static_cast<int>(K->heads);
   a.nqb = static_cast<int>(nqb);
-  a.nkb = static_cast<int>(K->seqlen / block_k);
+  a.nkb = static_cast<int>((K->seqlen + block_k - 1) / block_k);
+  a.k_tail = static_cast<int>(K->seqlen - static_cast<int64_t>(a.nkb - 1) * block_k);
   a.Lq = static_cast<int>(Q->seqlen);
   a.q_block_off = static_cast<int>(q_offset / block_k);
   a.causal = causal ? 1 : 0;

@@ -41,6 +41,7 @@ struct SelectArgs {
   const float* beta;   // [B, Hkv, nkb]
   int B, Hq, Hkv, nqb, nkb, R, nwords;
   int items;           // B * nqb * (Hq / R)
+  int Lq;              // query tokens; the last query block holds Lq - (nqb - 1) BQ of them
   int seq_inner;       // 1 when Q's token stride is smaller than its head stride
   int q_block_offset, causal, force_diag, force_sink;
   float rho_c, rho_r;
@@ -482,13 +483,17 @@ __global__ void __launch_bounds__(kSelThreads, KPL <= 32 ? 2 : 1)
         if (ptid == 0 && g + kPoolStages < total && !abort_flag) issue(g + kPoolStages);
       }
       float* qs = qs_all + (k & 1) * 128 * kSelMaxR;
+      int ib, ii, ih;
+      sel_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), ib, ii, ih);
+      const int nq = min(BQ, a.Lq - ii * BQ);  // rows past Lq were loaded as zeros
+      const float inv_n = nq == BQ ? 1.0f / BQ : 1.0f / nq;
       float s2 = 0.f;
       if (h < R) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           // acc[e] is dim 16 dq + e of the first piece read, then the second
           const int d = 16 * dq + (e < 8 ? p0 : p1) + (e & 7);
-          const float m = acc[e] * (1.0f / BQ);
+          const float m = acc[e] * inv_n;
           qs[d * kSelMaxR + h] = m;
           s2 = fmaf(m, m, s2);
         }

@@ -1,6 +1,8 @@
 // Key-block statistics ([RBS-en] "The Standard Approach and Its Blind
 // Spot"): centroid c_b = mean of the block's keys, radius r_b = max over the
-// block's keys of ||k - c_b||_2.
+// block's keys of ||k - c_b||_2.  When the sequence length L is not a block
+// multiple the last block holds the L - (nkb - 1) BK remaining keys (n_b of
+// them), and its mean and maximum run over those keys only.
 //
 // One 128-thread CTA per (key block, KV head, batch).  The block's BK key
 // rows (256 bytes each) are read once with 16-byte streaming loads and kept
@@ -16,10 +18,11 @@ namespace rbs {
 
 template <int BK>
 __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* __restrict__ K, int64_t sb,
-                                                          int64_t ss, int64_t sh, int nkb, int H,
+                                                          int64_t ss, int64_t sh, int nkb, int H, int L,
                                                           float* __restrict__ C, float* __restrict__ R) {
   constexpr int RPT = BK / 8;  // rows per thread
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nb = min(BK, L - j * BK);  // keys in this block
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int chunk = tid & 15;
   const int rgrp = tid >> 4;
@@ -31,7 +34,8 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
                      chunk * 16;
   uint4 v[RPT];
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) v[r] = ldg_stream(base + static_cast<int64_t>(rgrp + 8 * r) * ss * 2);
+  for (int r = 0; r < RPT; ++r)
+    v[r] = rgrp + 8 * r < nb ? ldg_stream(base + static_cast<int64_t>(rgrp + 8 * r) * ss * 2) : make_uint4(0, 0, 0, 0);
 
   float acc[8];
 #pragma unroll
@@ -53,7 +57,7 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
     for (int e = 0; e < 8; ++e) part[warp][chunk * 8 + e] = acc[e];
   }
   __syncthreads();
-  const float c = ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) * (1.0f / BK);
+  const float c = ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) * (nb == BK ? 1.0f / BK : 1.0f / nb);
   cen[tid] = c;
   C[(static_cast<int64_t>(b * H + h) * nkb + j) * RBS_HEAD_DIM + tid] = c;
   __syncthreads();
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
     // the 16 lanes of a row share (lane >> 4)
 #pragma unroll
     for (int o = 8; o >= 1; o >>= 1) d2 += __shfl_xor_sync(0xffffffffu, d2, o);
-    m = fmaxf(m, d2);
+    if (rgrp + 8 * r < nb) m = fmaxf(m, d2);
   }
   m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
   if (lane == 0) wmax[warp] = m;
@@ -161,17 +165,20 @@ __global__ void __launch_bounds__(1024) block_beta_kernel(const float* __restric
 }
 
 // ---------------------------------------------------------------------------
-// Query-block representative: qbar = mean of the block's BQ queries and its
+// Query-block representative: qbar = mean of the block's BQ queries (of the
+// remaining L - (nqb - 1) BQ queries for a last, partial block) and its
 // norm.  One 256-thread CTA per (query block, group of 4 q heads, batch):
 // thread t owns 16-byte chunk (t % 16) of head (t / 16) % 4 and rows
 // (t / 64) + 4r.  Deterministic reduction order.
 
 template <int BQ>
 __global__ void __launch_bounds__(256) pool_queries_kernel(const __nv_bfloat16* __restrict__ Q, int64_t sb,
-                                                           int64_t ss, int64_t sh, int Hq, int nqb,
+                                                           int64_t ss, int64_t sh, int Hq, int nqb, int L,
                                                            float* __restrict__ qbar, float* __restrict__ qnorm) {
   constexpr int RPT = BQ / 4;
   const int i = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+  const int nq = min(BQ, L - i * BQ);  // queries in this block
+  const float inv_n = nq == BQ ? 1.0f / BQ : 1.0f / nq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int col = tid & 63;
   const int hl = col >> 4, chunk = col & 15, rg = tid >> 6;
@@ -189,7 +196,9 @@ __global__ void __launch_bounds__(256) pool_queries_kernel(const __nv_bfloat16* 
     for (int r0 = 0; r0 < RPT; r0 += 8) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = ldg_stream(base + static_cast<int64_t>(rg + 4 * (r0 + u)) * ss * 2);
+      for (int u = 0; u < 8; ++u)
+        v[u] = rg + 4 * (r0 + u) < nq ? ldg_stream(base + static_cast<int64_t>(rg + 4 * (r0 + u)) * ss * 2)
+                                      : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -207,8 +216,8 @@ __global__ void __launch_bounds__(256) pool_queries_kernel(const __nv_bfloat16* 
   // thread t produces outputs 2t, 2t+1 (head t / 64, elements 2(t % 64) ..)
   const int o = 2 * tid;
   const int oh = tid >> 6;
-  const float m0 = ((part[0][o] + part[1][o]) + (part[2][o] + part[3][o])) * (1.0f / BQ);
-  const float m1 = ((part[0][o + 1] + part[1][o + 1]) + (part[2][o + 1] + part[3][o + 1])) * (1.0f / BQ);
+  const float m0 = ((part[0][o] + part[1][o]) + (part[2][o] + part[3][o])) * inv_n;
+  const float m1 = ((part[0][o + 1] + part[1][o + 1]) + (part[2][o + 1] + part[3][o + 1])) * inv_n;
   float s2 = m0 * m0 + m1 * m1;
 #pragma unroll
   for (int w = 16; w >= 1; w >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, w);

@@ -168,10 +168,12 @@ RBS_API rbs_status rbs_get_device_error(int32_t* code_host, rbs_stream_t stream)
 /* ---- block statistics  ([RBS-en] "The Standard Approach and Its Blind Spot")
  * For every key block b of block_k consecutive tokens of every (batch, KV
  * head): centroid c_b = mean of the block's keys, radius r_b = max over the
- * block's keys of ||k - c_b||_2.  fp32 accumulation of the bf16 keys.
- *   K          [B, L, Hkv, 128] bf16, L a multiple of block_k (64 or 128)
- *   centroids  out [B, Hkv, L/block_k, 128] fp32, contiguous
- *   radii      out [B, Hkv, L/block_k] fp32, contiguous
+ * block's keys of ||k - c_b||_2.  fp32 accumulation of the bf16 keys.  With
+ * nKB = ceil(L / block_k), a last block shorter than block_k (L not a block
+ * multiple) has the mean and maximum of its L - (nKB - 1) block_k keys.
+ *   K          [B, L, Hkv, 128] bf16, block_k 64 or 128
+ *   centroids  out [B, Hkv, nKB, 128] fp32, contiguous
+ *   radii      out [B, Hkv, nKB] fp32, contiguous
  */
 RBS_API rbs_status rbs_block_stats(const rbs_bf16_tensor* K, int32_t block_k, float* centroids, float* radii,
                            rbs_stream_t stream);
@@ -184,8 +186,9 @@ RBS_API rbs_status rbs_block_beta(const float* radii, int64_t batch, int64_t kv_
                           const rbs_select_params* p, float* beta, float* radius_range, rbs_stream_t stream);
 
 /* ---- query-block representative  ([RBS-en] "The Fix": the q of q^T c_b)
- * qbar [B, Hq, L/block_q, 128] fp32 = mean of each query block's queries;
- * qnorm [B, Hq, L/block_q] fp32 = ||qbar||_2.  Both contiguous. */
+ * qbar [B, Hq, nQB, 128] fp32 = mean of each query block's queries (nQB =
+ * ceil(L / block_q); a last, shorter block averages its own queries);
+ * qnorm [B, Hq, nQB] fp32 = ||qbar||_2.  Both contiguous. */
 RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, float* qbar, float* qnorm,
                             rbs_stream_t stream);
 
@@ -197,13 +200,14 @@ RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, f
  * branch keeps its own top ceil(rho * n_i) blocks (or, in MAX_RELATIVE mode,
  * the blocks within its delta of the row maximum); the row's list is the
  * union of both kept sets plus the forced blocks, ascending.
- *   Q            [B, Lq, Hq, 128] bf16, Lq a multiple of block_q
+ *   Q            [B, Lq, Hq, 128] bf16; nQB = ceil(Lq / block_q) query blocks,
+ *                the last one shorter when Lq is not a block multiple
  *   centroids    [B, Hkv, num_kv_blocks, 128] fp32 (rbs_block_stats)
  *   radii        [B, Hkv, num_kv_blocks] fp32
  *   workspace    device scratch of at least rbs_select_workspace_bytes(...)
  *                bytes, 256-byte aligned; its contents need no initialisation
- *   out          lists with num_rows = B * Hq * Lq / block_q (B * Hkv * Lq /
- *                block_q when list_mode is KV_GROUP) and capacity >=
+ *   out          lists with num_rows = B * Hq * nQB (B * Hkv * nQB when
+ *                list_mode is KV_GROUP) and capacity >=
  *                rbs_select_capacity(...), which bounds both modes;
  *                row_ptr, col_idx and flags written
  *   beta_out     optional [B, Hkv, num_kv_blocks] fp32 copy of beta (or NULL)
@@ -273,10 +277,12 @@ RBS_API rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t n
  *   Q         [B, Lq, Hq, 128] bf16; K, V [B, Lk, Hkv, 128] bf16; each with
  *             stride_h <= stride_s (heads inside tokens, as in a packed QKV
  *             projection; else RBS_ERR_UNSUPPORTED)
- *   lists     num_rows = B * Hq * Lq / block_q (row (b, h, i) serves q head
- *             h) or B * Hkv * Lq / block_q (row (b, g, i) serves every q
- *             head of KV head g); indices in [0, Lk / block_k)
- *   block_q == block_k, 64 or 128; q_offset a multiple of block_k
+ *   lists     num_rows = B * Hq * nQB (row (b, h, i) serves q head h) or
+ *             B * Hkv * nQB (row (b, g, i) serves every q head of KV head
+ *             g), nQB = ceil(Lq / block_q); indices in [0, ceil(Lk / block_k))
+ *   block_q == block_k, 64 or 128; q_offset a multiple of block_k.  Lq and
+ *             Lk need not be block multiples: query rows past Lq are not
+ *             written and keys past Lk are never attended.
  *   softmax_scale  <= 0 selects 1/sqrt(128)
  *   O         out [B, Lq, Hq, 128] bf16 (may not alias Q, K or V)
  *   lse       optional out [B, Hq, Lq] fp32 = ln sum_s exp(scale q_t.k_s)

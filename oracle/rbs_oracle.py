@@ -107,22 +107,25 @@ FLAG_FORCED = 4
 def block_stats(K: np.ndarray, block_k: int):
     """Centroid and radius of every key block.
 
-    K: [B, L, Hkv, d] (bf16 bits or float), L a multiple of block_k.
+    K: [B, L, Hkv, d] (bf16 bits or float).  Block b holds keys
+    b*block_k .. min((b+1)*block_k, L) - 1, so n_b = block_k except for a
+    last, shorter block when L is not a multiple of block_k.
     c_b = (1/n_b) sum_{k in b} k ;  r_b = max_{k in b} ||k - c_b||_2.
-    Returns centroids [B, Hkv, nKB, d] and radii [B, Hkv, nKB], float64.
+    Returns centroids [B, Hkv, nKB, d] and radii [B, Hkv, nKB], float64,
+    nKB = ceil(L / block_k).
     """
     B, L, H, d = K.shape
-    assert L % block_k == 0
-    nkb = L // block_k
+    nkb = -(-L // block_k)
     C = np.empty((B, H, nkb, d))
     R = np.empty((B, H, nkb))
     for b in range(B):
         for h in range(H):
-            kb = as_f64(K[b, :, h, :]).reshape(nkb, block_k, d)
-            c = kb.sum(axis=1) / block_k
-            dist = np.sqrt(((kb - c[:, None, :]) ** 2).sum(axis=2))
-            C[b, h] = c
-            R[b, h] = dist.max(axis=1)
+            x = as_f64(K[b, :, h, :])
+            for j in range(nkb):
+                kb = x[j * block_k:min((j + 1) * block_k, L)]
+                c = kb.sum(axis=0) / kb.shape[0]
+                C[b, h, j] = c
+                R[b, h, j] = np.sqrt(((kb - c) ** 2).sum(axis=1)).max()
     return C, R
 
 
@@ -175,15 +178,20 @@ def rescue_beta(R: np.ndarray, p: SelectParams):
 def pooled_queries(Q: np.ndarray, block_q: int):
     """Mean query of every query block and its Euclidean norm.
 
-    Q: [B, L, Hq, d].  Returns qbar [B, Hq, nQB, d] and qnorm [B, Hq, nQB].
+    Q: [B, L, Hq, d].  Query block i holds queries i*block_q ..
+    min((i+1)*block_q, L) - 1 (a last, shorter block when L is not a
+    multiple of block_q).  Returns qbar [B, Hq, nQB, d] and qnorm [B, Hq, nQB],
+    nQB = ceil(L / block_q).
     """
     B, L, H, d = Q.shape
-    assert L % block_q == 0
-    nqb = L // block_q
+    nqb = -(-L // block_q)
     qbar = np.empty((B, H, nqb, d))
     for b in range(B):
         for h in range(H):
-            qbar[b, h] = as_f64(Q[b, :, h, :]).reshape(nqb, block_q, d).sum(axis=1) / block_q
+            x = as_f64(Q[b, :, h, :])
+            for i in range(nqb):
+                blk = x[i * block_q:min((i + 1) * block_q, L)]
+                qbar[b, h, i] = blk.sum(axis=0) / blk.shape[0]
     qnorm = np.sqrt((qbar ** 2).sum(axis=-1))
     return qbar, qnorm
 
@@ -470,7 +478,8 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
     B, Lq, Hq, d = Q.shape
     Hkv = K.shape[2]
     G = Hq // Hkv
-    nqb = Lq // block_q
+    Lk = K.shape[1]
+    nqb = -(-Lq // block_q)  # a last, shorter query block when Lq is not a block multiple
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     O = np.full((B, Lq, Hq, d), np.nan)
@@ -484,26 +493,27 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
         kvh = hq // G
         lrow = (b * Hkv + kvh) * nqb + i if group_lists else row
         blocks = col_idx[row_ptr[lrow]:row_ptr[lrow + 1]]
-        t0 = i * block_q
-        q = as_f64(Q[b, t0:t0 + block_q, hq, :])
+        t0, t1 = i * block_q, min((i + 1) * block_q, Lq)
+        q = as_f64(Q[b, t0:t1, hq, :])
         if len(blocks) == 0:
-            O[b, t0:t0 + block_q, hq] = 0.0
-            lse[b, hq, t0:t0 + block_q] = -np.inf
+            O[b, t0:t1, hq] = 0.0
+            lse[b, hq, t0:t1] = -np.inf
             continue
-        kpos = np.concatenate([np.arange(j * block_k, (j + 1) * block_k) for j in blocks])
+        # key positions of the listed blocks (a last, shorter block ends at Lk)
+        kpos = np.concatenate([np.arange(j * block_k, min((j + 1) * block_k, Lk)) for j in blocks])
         k = as_f64(K[b, kpos, kvh, :])
         v = as_f64(V[b, kpos, kvh, :])
         logits = scale * (q @ k.T)
         if causal:
-            qpos = np.arange(t0, t0 + block_q) + q_offset
+            qpos = np.arange(t0, t1) + q_offset
             logits = np.where(kpos[None, :] <= qpos[:, None], logits, -np.inf)
         m = logits.max(axis=1, keepdims=True)
         m = np.where(np.isfinite(m), m, 0.0)
         w = np.exp(logits - m)
         z = w.sum(axis=1, keepdims=True)
         with np.errstate(invalid="ignore", divide="ignore"):
-            O[b, t0:t0 + block_q, hq] = np.where(z > 0, (w @ v) / z, 0.0)
-            lse[b, hq, t0:t0 + block_q] = (np.log(z) + m)[:, 0]
+            O[b, t0:t1, hq] = np.where(z > 0, (w @ v) / z, 0.0)
+            lse[b, hq, t0:t1] = (np.log(z) + m)[:, 0]
     return O, lse
 
 

@@ -757,3 +757,75 @@ def test_rescue_weight_closed_form_two_keys_forced_and_rescue():
     s1 = float(Q[0, 1, 0] @ K[0, 1, 0]) / math.sqrt(d)
     want = (math.exp(s1) * V[0, 1, 0] + 0.25 * math.exp(s0) * V[0, 0, 0]) / (math.exp(s1) + 0.25 * math.exp(s0))
     np.testing.assert_allclose(a[0, 1, 0], want, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Sequence lengths that are not block multiples: the last block is shorter
+
+
+def test_partial_last_key_block_closed_form():
+    # 2 full blocks of 64 plus a last block of 3 keys {x, x, y}:
+    # c = (2x + y) / 3 and r = |y - c| = (2/3) |x - y|
+    rng = np.random.default_rng(41)
+    d, bk = 128, 64
+    x, y = rng.standard_normal((2, d))
+    K = rng.standard_normal((1, 2 * bk + 3, 1, d))
+    K[0, 2 * bk:2 * bk + 2, 0] = x
+    K[0, 2 * bk + 2, 0] = y
+    C, R = O.block_stats(K, bk)
+    assert C.shape == (1, 1, 3, d) and R.shape == (1, 1, 3)
+    np.testing.assert_allclose(C[0, 0, 2], (2 * x + y) / 3, atol=1e-14)
+    assert R[0, 0, 2] == pytest.approx(2 / 3 * np.linalg.norm(x - y), rel=1e-13)
+    full, _ = O.block_stats(K[:, :2 * bk], bk)  # the full blocks are unaffected by the tail
+    np.testing.assert_array_equal(C[0, 0, :2], full[0, 0])
+    Kone = K[:, :2 * bk + 1]  # a last block of a single key: c = k, r = 0
+    C1, R1 = O.block_stats(Kone, bk)
+    np.testing.assert_array_equal(C1[0, 0, 2], Kone[0, 2 * bk, 0])
+    assert R1[0, 0, 2] == 0.0
+
+
+def test_partial_last_query_block_is_numpy_mean():
+    rng = np.random.default_rng(42)
+    Q = rng.standard_normal((2, 300, 3, 128))
+    qbar, qnorm = O.pooled_queries(Q, 128)
+    assert qbar.shape == (2, 3, 3, 128)
+    np.testing.assert_allclose(qbar[1, 2, 2], Q[1, 256:300, 2].mean(axis=0), atol=1e-15)
+    np.testing.assert_allclose(qbar[0, 1, 0], Q[0, 0:128, 1].mean(axis=0), atol=1e-15)
+    np.testing.assert_allclose(qnorm, np.linalg.norm(qbar, axis=-1), atol=1e-15)
+
+
+def test_ragged_full_lists_equal_dense_attention():
+    # 1000 query and key tokens in 128-token blocks (the last holds 104):
+    # full causal lists give textbook causal attention; non-causal full lists
+    # give plain softmax attention over all 1000 keys (torch SDPA, no mask)
+    rng = np.random.default_rng(43)
+    L, d = 1000, 128
+    Q, K, V = (rng.standard_normal((1, L, h, d)) for h in (4, 2, 2))
+    nqb = 8
+    rp, ci = O.causal_full_lists(1, 4, nqb)
+    Om, lm = O.masked_attention(Q, K, V, rp, ci, 128, 128)
+    Od = O.dense_causal_attention(Q, K, V)
+    np.testing.assert_allclose(Om, Od, atol=1e-12)
+    rpn = np.arange(0, 4 * nqb * nqb + 1, nqb)
+    cin = np.tile(np.arange(nqb), 4 * nqb)
+    On, _ = O.masked_attention(Q, K, V, rpn, cin, 128, 128, causal=0)
+    t = lambda a: torch.from_numpy(a).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(t(Q), t(K).repeat_interleave(2, 1),
+                                                           t(V).repeat_interleave(2, 1)).permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(On, ref, atol=1e-12)
+
+
+def test_ragged_pins_catch_planted_mistakes(monkeypatch):
+    good = O.block_stats
+
+    def full_block_divisor(K, bk):
+        C, R = good(K, bk)
+        L = K.shape[1]
+        nb = L - (C.shape[2] - 1) * bk
+        if nb < bk:  # the tail's sum divided by block_k instead of n_b
+            C = C.copy()
+            C[:, :, -1] *= nb / bk
+        return C, R
+    monkeypatch.setattr(O, "block_stats", full_block_divisor)
+    with pytest.raises(AssertionError):
+        test_partial_last_key_block_closed_form()
