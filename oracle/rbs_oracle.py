@@ -93,6 +93,9 @@ class SelectParams:
     # per (batch, KV head, query block), the union of the lists of the q heads
     # that share the KV head (they then attend to the same key blocks)
     list_mode: int = 0
+    # query representative: 0 = MEAN (the mean of the query block's queries);
+    # 1 = TOKEN_MAX (each branch scores a key block by its best query token)
+    query_pool: int = 0
 
 
 FLAG_CENTROID = 1
@@ -234,6 +237,38 @@ def branch_scores(qbar: np.ndarray, qnorm: np.ndarray, C: np.ndarray, R: np.ndar
     return s_c, s_r
 
 
+def token_max_scores(Qbh: np.ndarray, C: np.ndarray, R: np.ndarray, beta: np.ndarray, block_q: int):
+    """Per-token scoring of one (prompt, q head): every query token scores the
+    key blocks, and a query block keeps each branch's best token score.
+
+    Qbh [L, d] (the q head's queries), C [nKB, d], R, beta [nKB].  For query
+    block i (tokens i*block_q .. min((i+1)*block_q, L) - 1):
+      s_c(i, j) = max_t q_t . c_j
+      s_r(i, j) = max_t (q_t . c_j + |q_t| r_j beta_j)
+    ([RBS-en] "The Fix" writes both branch scores for a query q; here q runs
+    over the block's query tokens instead of their mean).
+    """
+    L = Qbh.shape[0]
+    nqb = -(-L // block_q)
+    q = as_f64(Qbh)
+    rb = R * beta
+    s_c = np.empty((nqb, C.shape[0]))
+    s_r = np.empty((nqb, C.shape[0]))
+    for i in range(nqb):
+        qi = q[i * block_q:min((i + 1) * block_q, L)]
+        dots = qi @ C.T  # [tokens, nKB]
+        s_c[i] = dots.max(axis=0)
+        s_r[i] = (dots + np.sqrt((qi ** 2).sum(axis=1))[:, None] * rb[None, :]).max(axis=0)
+    return s_c, s_r
+
+
+def branch_scores_for(Q, qbar, qnorm, C, R, beta, b: int, hq: int, kvh: int, p: SelectParams):
+    """The two branches' scores of one (prompt, q head) under p.query_pool."""
+    if p.query_pool == 1:
+        return token_max_scores(Q[b, :, hq, :], C[b, kvh], R[b, kvh], beta[b, kvh], p.block_q)
+    return branch_scores(qbar[b, hq], qnorm[b, hq], C[b, kvh], R[b, kvh], beta[b, kvh])
+
+
 def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, keep_scores: bool = False):
     """Per-query-block KV-block lists (CSR), rows ordered (batch, q head, query block).
 
@@ -272,7 +307,7 @@ def select_blocks(Q: np.ndarray, C: np.ndarray, R: np.ndarray, p: SelectParams, 
     for b in range(B):
         for hq in range(Hq):
             kvh = hq // G
-            s_c, s_r = branch_scores(qbar[b, hq], qnorm[b, hq], C[b, kvh], R[b, kvh], beta[b, kvh])
+            s_c, s_r = branch_scores_for(Q, qbar, qnorm, C, R, beta, b, hq, kvh, p)
             if keep_scores:
                 scores[(b, hq)] = (s_c, s_r)
             for i in range(nqb):
@@ -365,7 +400,7 @@ def union_ranks(Q, C, R, p: SelectParams):
     for b in range(B):
         for hq in range(Hq):
             kvh = hq // G
-            s_c, s_r = branch_scores(qbar[b, hq], qnorm[b, hq], C[b, kvh], R[b, kvh], beta[b, kvh])
+            s_c, s_r = branch_scores_for(Q, qbar, qnorm, C, R, beta, b, hq, kvh, p)
             for i in range(nqb):
                 n = visible_blocks(i, nkb, p)
                 rank_c = np.empty(n, dtype=np.int64)

@@ -829,3 +829,91 @@ def test_ragged_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "block_stats", full_block_divisor)
     with pytest.raises(AssertionError):
         test_partial_last_key_block_closed_form()
+
+
+# --------------------------------------------------------------------------
+# Per-token-max query scoring (query_pool = 1)
+
+
+def test_token_max_brute_force_tiny():
+    # pure-Python loops over tokens, blocks and dims on a tiny case (7 tokens,
+    # 3-token query blocks: the last holds one token)
+    rng = np.random.default_rng(51)
+    L, d, nkb = 7, 5, 3
+    Q = rng.standard_normal((L, d))
+    C = rng.standard_normal((nkb, d))
+    R = rng.uniform(0.5, 2.0, nkb)
+    beta = rng.uniform(0.0, 1.0, nkb)
+    s_c, s_r = O.token_max_scores(Q, C, R, beta, 3)
+    for i, toks in enumerate(([0, 1, 2], [3, 4, 5], [6])):
+        for j in range(nkb):
+            dots = [sum(Q[t, e] * C[j, e] for e in range(d)) for t in toks]
+            norms = [math.sqrt(sum(Q[t, e] ** 2 for e in range(d))) for t in toks]
+            assert s_c[i, j] == pytest.approx(max(dots), abs=1e-12)
+            assert s_r[i, j] == pytest.approx(max(x + n * R[j] * beta[j] for x, n in zip(dots, norms)), abs=1e-12)
+
+
+def test_token_max_equals_mean_when_a_block_repeats_one_query():
+    # every query block made of one repeated query: max over its tokens = its
+    # mean, so both representatives give the same scores and lists
+    inp = make_mixture(L=2048, Hq=4, Hkv=2, block=128, seed=52)
+    Q = inp["Q"].copy()
+    Q[:] = np.repeat(Q[:, ::128], 128, axis=1)
+    C, R = O.block_stats(inp["K"], 128)
+    kw = dict(block_q=128, block_k=128, rho_centroid=0.2, rho_rescue=0.2)
+    a = O.select_blocks(Q, C, R, O.SelectParams(**kw), keep_scores=True)
+    b = O.select_blocks(Q, C, R, O.SelectParams(query_pool=1, **kw), keep_scores=True)
+    for key in ("row_ptr", "col_idx", "flags"):
+        assert np.array_equal(a[key], b[key])
+    for hk in a["scores"]:
+        np.testing.assert_allclose(a["scores"][hk][0], b["scores"][hk][0], atol=1e-12)
+        np.testing.assert_allclose(a["scores"][hk][1], b["scores"][hk][1], atol=1e-12)
+
+
+def test_token_max_bounds():
+    # the best token beats the mean query (the dot is linear in q), the rescue
+    # score bounds the centroid score, and with beta = 1 the rescue score bounds
+    # every (token, key) logit of the pair (Cauchy-Schwarz per token, [RBS-en]
+    # "The Fix")
+    inp = make_tiny(L=1024, seed=53)
+    C, R = O.block_stats(inp["K"], 64)
+    p = O.SelectParams(block_q=64, block_k=64, beta_mode=1, beta_const=1.0, query_pool=1)
+    beta, _ = O.rescue_beta(R, p)
+    Qf = O.as_f64(inp["Q"])
+    Kf = O.as_f64(inp["K"])
+    qbar, qnorm = O.pooled_queries(inp["Q"], 64)
+    for hq in range(2):
+        s_c, s_r = O.token_max_scores(inp["Q"][0, :, hq], C[0, 0], R[0, 0], beta[0, 0], 64)
+        m_c, _ = O.branch_scores(qbar[0, hq], qnorm[0, hq], C[0, 0], R[0, 0], beta[0, 0])
+        assert np.all(s_c >= m_c - 1e-12) and np.all(s_r >= s_c)
+        for i in (3, 9, 15):
+            for j in (0, 5, 15):
+                logits = Qf[0, i * 64:(i + 1) * 64, hq] @ Kf[0, j * 64:(j + 1) * 64, 0].T
+                assert logits.max() <= s_r[i, j] + 1e-9
+
+
+def test_token_max_pins_catch_planted_mistakes(monkeypatch):
+    good = O.token_max_scores
+
+    def mean_not_max(Qbh, C, R, beta, block_q):
+        L = Qbh.shape[0]
+        nqb = -(-L // block_q)
+        q = O.as_f64(Qbh)
+        s_c = np.stack([(q[i * block_q:(i + 1) * block_q] @ C.T).mean(axis=0) for i in range(nqb)])
+        return s_c, good(Qbh, C, R, beta, block_q)[1]
+    monkeypatch.setattr(O, "token_max_scores", mean_not_max)
+    with pytest.raises(AssertionError):
+        test_token_max_brute_force_tiny()
+
+    def norm_of_mean(Qbh, C, R, beta, block_q):  # rescue term with |qbar| instead of |q_t|
+        s_c, _ = good(Qbh, C, R, beta, block_q)
+        L = Qbh.shape[0]
+        q = O.as_f64(Qbh)
+        nqb = -(-L // block_q)
+        s_r = np.stack([((q[i * block_q:(i + 1) * block_q] @ C.T)
+                         + np.linalg.norm(q[i * block_q:(i + 1) * block_q].mean(axis=0)) * (R * beta)).max(axis=0)
+                        for i in range(nqb)])
+        return s_c, s_r
+    monkeypatch.setattr(O, "token_max_scores", norm_of_mean)
+    with pytest.raises(AssertionError):
+        test_token_max_bounds()
