@@ -14,8 +14,8 @@ end-to-end number through the same calls with host buffers, the Block-
 attention RAG flow (cache build, RoPE re-encoding, final block), a density
 sweep at 64K (selection and attention time at 2-100% kept density), the same
 prompt with KV-group lists (one list per KV head shared by its q heads), the
-same lists with the rescue blocks' contribution weighted by 0.5, and the CPU
-oracle baseline.
+same lists with the rescue blocks' contribution weighted by 0.5, selection
+with per-token-max query scoring, and the CPU oracle baseline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 N > 1 runs under torchrun: every rank processes its own prompt (weak
@@ -306,6 +306,8 @@ def run_ours(args, ws, rank):
         out["dense"] = dense_measure(rbs, Q, K, V, B, Hq, nqb, peak)
         out["dense"]["speedup_attn_only"] = round(out["dense"]["ms"] / attn_ms, 2)
         out["dense"]["speedup_with_selection"] = round(out["dense"]["ms"] / (attn_ms + select_ms + stats_ms), 2)
+    if args.token_max and rank == 0:
+        out["token_max_select"] = token_max_measure(rbs, Q, C, R, w.rho, B, Hq, Hkv, nqb, nkb)
     if args.rescue_weighted and rank == 0:
         out["rescue_weighted"] = rescue_weighted_measure(rbs, Q, K, V, lists, flops, attn_ms, peak)
     if args.group_lists and rank == 0:
@@ -644,6 +646,27 @@ def block_attention_measure(rbs, peaks):
     return res
 
 
+def token_max_measure(rbs, Q, C, R, rho, B, Hq, Hkv, nqb, nkb):
+    """Selection of the same prompt with each key block scored by the query
+    block's best token (query_pool 1; the token-by-centroid products run on
+    the tensor core).  Algorithmic work: 2 bf16 parts x 2 x 128 x d FLOPs per
+    (token block, key block) pair visited in 128-block tiles."""
+    import torch
+    p = rbs.SelectParams(block_q=BLOCK, block_k=BLOCK, rho_centroid=rho, rho_rescue=rho, query_pool=1)
+    lists = rbs.BlockLists.empty(B * Hq * nqb, rbs.rbs_select_capacity(B, Hq, nqb, nkb, p), "cuda")
+    ws_buf = torch.empty(rbs.rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, p), dtype=torch.uint8, device="cuda")
+    fn = lambda: rbs.rbs_select(Q, C, R, p, workspace=ws_buf, out=lists)
+    fn()
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    ms = _time_ms(fn, 10)
+    tiles = B * Hq * sum(-(-(i + 1) // 128) for i in range(nqb))
+    flops = tiles * 2 * 2 * 128 * BLOCK * HEAD_DIM
+    visible = B * Hq * nqb * (nqb + 1) // 2
+    return {"ms": round(ms, 4), "nnz_pairs": lists.nnz(), "density": round(lists.nnz() / visible, 5),
+            "mma_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
+
+
 def rescue_weighted_measure(rbs, Q, K, V, lists, flops, attn_ms, peak, weight: float = 0.5):
     """The same prompt and lists with the rescue-only blocks' softmax mass scaled
     by `weight` (one pass: a log2(weight) offset on those tiles' logits)."""
@@ -857,6 +880,7 @@ def main():
     ap.add_argument("--no-selector-quality", dest="selector_quality", action="store_false")
     ap.add_argument("--no-group-lists", dest="group_lists", action="store_false")
     ap.add_argument("--no-rescue-weighted", dest="rescue_weighted", action="store_false")
+    ap.add_argument("--no-token-max", dest="token_max", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--seq-len", type=int, default=None,

@@ -56,6 +56,7 @@ class SelectParams:
     delta_centroid: float = 0.0
     delta_rescue: float = 0.0
     list_mode: int = 0  # 0 = one list per q head, 1 = one per KV head (union of its q heads)
+    query_pool: int = 0  # 0 = mean query of the block, 1 = best query token of the block
 
     def c(self) -> SelectParamsC:
         return SelectParamsC(*[getattr(self, f.name) for f in dataclasses.fields(self)])

@@ -33,7 +33,7 @@ class SelectParamsC(ctypes.Structure):
                 ("beta_p_lo", ctypes.c_float), ("beta_p_hi", ctypes.c_float), ("force_diag", ctypes.c_int32),
                 ("force_sink", ctypes.c_int32), ("causal", ctypes.c_int32), ("q_block_offset", ctypes.c_int32),
                 ("threshold_mode", ctypes.c_int32), ("delta_centroid", ctypes.c_float), ("delta_rescue", ctypes.c_float),
-                ("list_mode", ctypes.c_int32)]
+                ("list_mode", ctypes.c_int32), ("query_pool", ctypes.c_int32)]
 
 
 class BlockListsC(ctypes.Structure):
@@ -77,7 +77,7 @@ class RbsError(RuntimeError):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
 
 
-ABI_VERSION = 3  # RBS_ABI_VERSION of include/rbs.h that these structures match
+ABI_VERSION = 4  # RBS_ABI_VERSION of include/rbs.h that these structures match
 _lib = None
 
 

@@ -17,6 +17,7 @@
 #include "rope.cuh"
 #include "select.cuh"
 #include "stats.cuh"
+#include "tokmax.cuh"
 
 using namespace rbs;
 
@@ -82,6 +83,15 @@ rbs_status device_info(DeviceInfo** out) {
     RBS_SEL_ATTR(64)
     RBS_SEL_ATTR(128)
 #undef RBS_SEL_ATTR
+#define RBS_TOK_ATTR(KPL)                                                                                      \
+  e = e ? e : cudaFuncSetAttribute(select_tokmax_kernel<64, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                   TokSmem<64>::kAlloc);                                                        \
+  e = e ? e : cudaFuncSetAttribute(select_tokmax_kernel<128, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                   TokSmem<128>::kAlloc);
+    RBS_TOK_ATTR(8)
+    RBS_TOK_ATTR(32)
+    RBS_TOK_ATTR(64)
+#undef RBS_TOK_ATTR
     e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
     if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     d.attrs_set = true;
@@ -182,6 +192,55 @@ rbs_status make_pool_tensor_map(const rbs_bf16_tensor* t, int R, CUtensorMap* ma
   return RBS_OK;
 }
 
+// Per-token-max selection scores (query_pool TOKEN_MAX): split the centroids
+// into bf16 hi / lo parts in the workspace, then one persistent CTA per SM
+// scores and thresholds rows (select_tokmax_kernel), writing the same mask
+// words and counts as the mean-query kernel.
+rbs_status launch_token_max(const rbs_bf16_tensor* Q, const float* centroids, int64_t B, int32_t Hkv, int64_t nkb,
+                            const rbs_select_params* p, const SelectArgs& sa, uint8_t* c_hi, uint8_t* c_lo,
+                            DeviceInfo* di, rbs_stream_t stream) {
+  rbs_status st;
+  const int64_t n = B * Hkv * nkb * RBS_HEAD_DIM;
+  auto* hi = reinterpret_cast<__nv_bfloat16*>(c_hi);
+  auto* lo = reinterpret_cast<__nv_bfloat16*>(c_lo);
+  split_centroids_kernel<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 4 * di->sms)), 256, 0, stream>>>(
+      centroids, n, hi, lo);
+  if ((st = check_launch("split_centroids_kernel")) != RBS_OK) return st;
+  TokArgs ta;
+  int si = 0;
+  if ((st = make_tensor_map(Q, p->block_q, &ta.tmQ, &si)) != RBS_OK) return st;
+  RBS_REQUIRE(si == 0, RBS_ERR_UNSUPPORTED,
+              "query_pool TOKEN_MAX needs Q with the head stride no larger than the token stride");
+  // the centroid parts as [B, nkb "tokens", Hkv "heads", 128]: block j of KV head h at (j, h)
+  for (int part = 0; part < 2; ++part) {
+    rbs_bf16_tensor v;
+    v.data = part == 0 ? c_hi : c_lo;
+    v.batch = B;
+    v.seqlen = nkb;
+    v.heads = Hkv;
+    v.head_dim = RBS_HEAD_DIM;
+    v.stride_b = Hkv * nkb * RBS_HEAD_DIM;
+    v.stride_s = RBS_HEAD_DIM;
+    v.stride_h = nkb * RBS_HEAD_DIM;
+    if ((st = make_tensor_map(&v, 128, part == 0 ? &ta.tmChi : &ta.tmClo, &si)) != RBS_OK) return st;
+  }
+  ta.s = sa;
+  ta.rows = static_cast<int>(B * sa.Hq * sa.nqb);
+  const int grid = static_cast<int>(std::min<int64_t>(ta.rows, di->sms));
+#define RBS_TOK_LAUNCH(KPL)                                                                                  \
+  do {                                                                                                       \
+    if (p->block_q == 128)                                                                                   \
+      select_tokmax_kernel<128, KPL><<<grid, kTokThreads, TokSmem<128>::kAlloc, stream>>>(ta);               \
+    else                                                                                                     \
+      select_tokmax_kernel<64, KPL><<<grid, kTokThreads, TokSmem<64>::kAlloc, stream>>>(ta);                 \
+  } while (0)
+  if (nkb <= 256) RBS_TOK_LAUNCH(8);
+  else if (nkb <= 1024) RBS_TOK_LAUNCH(32);
+  else RBS_TOK_LAUNCH(64);
+#undef RBS_TOK_LAUNCH
+  return check_launch("select_tokmax_kernel");
+}
+
 int keep_count_host(float rho, int64_t n) {
   int64_t k = static_cast<int64_t>(std::ceil(static_cast<double>(rho) * static_cast<double>(n) - 1e-4));
   if (k < 1) k = 1;
@@ -192,10 +251,11 @@ int keep_count_host(float rho, int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct SelectLayout {
-  size_t mask_c, mask_r, counts, beta, total;
+  size_t mask_c, mask_r, counts, beta, c_hi, c_lo, total;
 };
 
-SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int64_t nkb) {
+// token_max: room for the bf16 hi / lo parts of the centroids as well
+SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int64_t nkb, bool token_max) {
   SelectLayout l{};
   const int64_t rows = B * Hq * nqb;
   const int64_t nwords = (nkb + 31) / 32;
@@ -204,6 +264,10 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
   l.mask_r = off; off += align256(rows * nwords * 4);
   l.counts = off; off += align256(rows * 4);
   l.beta = off; off += align256(B * Hkv * nkb * 4);
+  if (token_max) {
+    l.c_hi = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
+    l.c_lo = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
+  }
   l.total = off;
   return l;
 }
@@ -255,6 +319,7 @@ void rbs_select_params_default(rbs_select_params* p) {
   p->delta_centroid = 0.0f;
   p->delta_rescue = 0.0f;
   p->list_mode = 0;
+  p->query_pool = 0;
 }
 
 rbs_status rbs_get_device_error(int32_t* code_host, rbs_stream_t stream) {
@@ -359,7 +424,7 @@ size_t rbs_select_workspace_bytes(int64_t batch, int64_t heads_q, int64_t num_q_
                                   int64_t num_kv_blocks, const rbs_select_params* p) {
   (void)p;
   if (batch <= 0 || heads_q <= 0 || num_q_blocks <= 0 || kv_heads <= 0 || num_kv_blocks <= 0) return 0;
-  return select_layout(batch, heads_q, num_q_blocks, kv_heads, num_kv_blocks).total;
+  return select_layout(batch, heads_q, num_q_blocks, kv_heads, num_kv_blocks, p != nullptr && p->query_pool == 1).total;
 }
 
 rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const float* radii, int32_t kv_heads,
@@ -381,6 +446,9 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
               RBS_ERR_INVALID_ARG, "delta must be >= 0 (and not NaN)");
   RBS_REQUIRE(p->q_block_offset >= 0, RBS_ERR_INVALID_ARG, "q_block_offset < 0");
   RBS_REQUIRE(p->list_mode == 0 || p->list_mode == 1, RBS_ERR_INVALID_ARG, "list_mode must be 0 or 1");
+  RBS_REQUIRE(p->query_pool == 0 || p->query_pool == 1, RBS_ERR_INVALID_ARG, "query_pool must be 0 or 1");
+  RBS_REQUIRE(p->query_pool == 0 || num_kv_blocks <= kTokMaxKV, RBS_ERR_UNSUPPORTED,
+              "query_pool TOKEN_MAX takes at most %d key blocks", kTokMaxKV);
   RBS_REQUIRE(aligned16(centroids), RBS_ERR_INVALID_ARG, "centroids not 16-byte aligned");
   const int64_t B = Q->batch, Hq = Q->heads, nqb = (Q->seqlen + p->block_q - 1) / p->block_q, nkb = num_kv_blocks;
   const int64_t rows = B * Hq * nqb;                                       // one per q head
@@ -389,7 +457,7 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   const int64_t cap = rbs_select_capacity(B, Hq, nqb, nkb, p);
   RBS_REQUIRE(out->capacity >= cap, RBS_ERR_CAPACITY, "list capacity %lld < %lld", static_cast<long long>(out->capacity),
               static_cast<long long>(cap));
-  const SelectLayout lay = select_layout(B, Hq, nqb, kv_heads, nkb);
+  const SelectLayout lay = select_layout(B, Hq, nqb, kv_heads, nkb, p->query_pool == 1);
   RBS_REQUIRE(workspace != nullptr && workspace_bytes >= lay.total, RBS_ERR_CAPACITY, "workspace %zu < %zu bytes",
               workspace_bytes, lay.total);
   RBS_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, RBS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
@@ -406,7 +474,7 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
     if (G % r == 0) R = r;
   CUtensorMap qmap;
   int seq_inner = 0;
-  if ((st = make_pool_tensor_map(Q, R, &qmap, &seq_inner)) != RBS_OK) return st;
+  if (p->query_pool == 0 && (st = make_pool_tensor_map(Q, R, &qmap, &seq_inner)) != RBS_OK) return st;
   SelectArgs sa;
   sa.C = centroids;
   sa.rad = radii;
@@ -433,27 +501,32 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   sa.mask_c = reinterpret_cast<uint32_t*>(ws + lay.mask_c);
   sa.mask_r = reinterpret_cast<uint32_t*>(ws + lay.mask_r);
   sa.counts = reinterpret_cast<int*>(ws + lay.counts);
-  const int npad = static_cast<int>((nkb + 31) & ~31ll);
-  const size_t smem = sel_smem_bytes(npad);
-  // persistent: as many CTAs as fit on the device at once, each walking the
-  // work items with a stride of the grid
-  auto launch = [&](auto kern) -> rbs_status {
-    int per_sm = 0;
-    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSelThreads, smem);
-    if (e != cudaSuccess || per_sm < 1) return fail(RBS_ERR_CUDA, "select_rows_kernel does not fit on an SM");
-    const int grid = static_cast<int>(std::min<int64_t>(sa.items, static_cast<int64_t>(per_sm) * di->sms));
-    kern<<<grid, kSelThreads, smem, stream>>>(qmap, sa);
-    return check_launch("select_rows_kernel");
-  };
+  if (p->query_pool == 1) {
+    if ((st = launch_token_max(Q, centroids, B, kv_heads, nkb, p, sa, ws + lay.c_hi, ws + lay.c_lo, di, stream)) != RBS_OK)
+      return st;
+  } else {
+    const int npad = static_cast<int>((nkb + 31) & ~31ll);
+    const size_t smem = sel_smem_bytes(npad);
+    // persistent: as many CTAs as fit on the device at once, each walking the
+    // work items with a stride of the grid
+    auto launch = [&](auto kern) -> rbs_status {
+      int per_sm = 0;
+      const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSelThreads, smem);
+      if (e != cudaSuccess || per_sm < 1) return fail(RBS_ERR_CUDA, "select_rows_kernel does not fit on an SM");
+      const int grid = static_cast<int>(std::min<int64_t>(sa.items, static_cast<int64_t>(per_sm) * di->sms));
+      kern<<<grid, kSelThreads, smem, stream>>>(qmap, sa);
+      return check_launch("select_rows_kernel");
+    };
 #define RBS_SEL_LAUNCH(KPL) \
-  st = p->block_q == 128 ? launch(select_rows_kernel<KPL, 128>) : launch(select_rows_kernel<KPL, 64>)
-  if (nkb <= 64) RBS_SEL_LAUNCH(2);
-  else if (nkb <= 256) RBS_SEL_LAUNCH(8);
-  else if (nkb <= 1024) RBS_SEL_LAUNCH(32);
-  else if (nkb <= 2048) RBS_SEL_LAUNCH(64);
-  else RBS_SEL_LAUNCH(128);
+    st = p->block_q == 128 ? launch(select_rows_kernel<KPL, 128>) : launch(select_rows_kernel<KPL, 64>)
+    if (nkb <= 64) RBS_SEL_LAUNCH(2);
+    else if (nkb <= 256) RBS_SEL_LAUNCH(8);
+    else if (nkb <= 1024) RBS_SEL_LAUNCH(32);
+    else if (nkb <= 2048) RBS_SEL_LAUNCH(64);
+    else RBS_SEL_LAUNCH(128);
 #undef RBS_SEL_LAUNCH
-  if (st != RBS_OK) return st;
+    if (st != RBS_OK) return st;
+  }
 
   CompactArgs ca;
   ca.mask_c = sa.mask_c;

@@ -262,33 +262,30 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
   return true;
 }
 
-// Both branches' top-k of one row (warp-wide) -> mask words and the row's
-// union count.  Keys hold KP slots per lane (block 32t + lane in slot t); the
-// row's mask words cover all nwords <= (KPMAX + 31) / 32 * 32 words.
-template <int KP, int KPMAX>
-__device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float* sc, const float* rb, float qnv,
-                                                int warp, int lane, int hq0, int b, int i, int gi, int n, int npad,
-                                                uint32_t* scratch) {
-  const int hq = hq0 + warp;
-  const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
+// Both branches' top-k of one list row (warp-wide) -> mask words and the
+// row's union count.  score_c(j), score_r(j) give the branches' scores of the
+// visible block j < n; keys hold KP slots per lane (block 32t + lane in slot
+// t); the row's mask words cover all nwords <= (KPMAX + 31) / 32 * 32 words.
+template <int KP, int KPMAX, typename SC, typename SR>
+__device__ __forceinline__ void select_row(const SelectArgs& a, SC score_c, SR score_r, int64_t row, int lane,
+                                           int gi, int n, uint32_t* scratch) {
   uint32_t* words_c = scratch + 4 * kTopkCap;
   uint32_t* words_r = words_c + a.nwords;
-  const float* srow = sc + warp * npad;
   auto key_c = [&](int t) -> uint32_t {
     const int j = 32 * t + lane;
-    return j < n ? order_key(srow[j]) : 0u;
+    return j < n ? order_key(score_c(j)) : 0u;
   };
   auto key_r = [&](int t) -> uint32_t {
     const int j = 32 * t + lane;
-    return j < n ? order_key(fmaf(qnv, rb[j], srow[j])) : 0u;
+    return j < n ? order_key(score_r(j)) : 0u;
   };
   if (a.threshold_mode == 1) {
     // Each branch keeps every visible block scoring at least its row maximum
     // minus delta; the threshold is formed in fp32 from the maximum score.
     float mc = -INFINITY, mr = -INFINITY;
     for (int j = lane; j < n; j += 32) {
-      mc = fmaxf(mc, srow[j]);
-      mr = fmaxf(mr, fmaf(qnv, rb[j], srow[j]));
+      mc = fmaxf(mc, score_c(j));
+      mr = fmaxf(mr, score_r(j));
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
@@ -301,9 +298,8 @@ __device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float
       for (int bit = 0; bit < 32; ++bit) {
         const int j = 32 * w + bit;
         if (j < n) {
-          const float sv = srow[j];
-          if (order_key(sv) >= tc) wc |= 1u << bit;
-          if (order_key(fmaf(qnv, rb[j], sv)) >= tr) wr |= 1u << bit;
+          if (order_key(score_c(j)) >= tc) wc |= 1u << bit;
+          if (order_key(score_r(j)) >= tr) wr |= 1u << bit;
         }
       }
       words_c[w] = wc;
@@ -343,6 +339,19 @@ __device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float
   }
   cnt = __reduce_add_sync(0xffffffffu, cnt);
   if (lane == 0) a.counts[row] = cnt;
+}
+
+// The mean-pooled scores of row `warp` of the CTA's item:
+//   s_c(j) = sc[warp][j], s_r(j) = s_c(j) + |qbar| r_j beta_j.
+template <int KP, int KPMAX>
+__device__ __forceinline__ void select_topk_row(const SelectArgs& a, const float* sc, const float* rb, float qnv,
+                                                int warp, int lane, int hq0, int b, int i, int gi, int n, int npad,
+                                                uint32_t* scratch) {
+  const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq0 + warp) * a.nqb + i;
+  const float* srow = sc + warp * npad;
+  select_row<KP, KPMAX>(
+      a, [&](int j) { return srow[j]; }, [&](int j) { return fmaf(qnv, rb[j], srow[j]); }, row, lane, gi, n,
+      scratch);
 }
 
 // Work item w -> (batch, query block, first q head): longest rows first.

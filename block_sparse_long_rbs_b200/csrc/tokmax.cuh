@@ -1,0 +1,326 @@
+// Per-token-max scoring of the two branches on the tensor core
+// ([RBS-en] "The Fix" scores a key block against a query q; here q runs over
+// the query block's tokens and the block keeps each branch's best token):
+//   s_c(i, j) = max_t q_t . c_j
+//   s_r(i, j) = max_t (q_t . c_j + |q_t| r_j beta_j)
+// over the (valid) tokens t of query block i.  The dot products of a query
+// block's BQ tokens with 128 centroids at a time are one 128 x BQ x 128 MMA:
+// A = the centroid tile (128 key blocks x 128 dims, K-major), B = the query
+// tile (BQ tokens x 128 dims, K-major), D = 128 key blocks (TMEM lanes) x BQ
+// tokens (columns), fp32.  The fp32 centroids enter as two bf16 parts, c =
+// hi + lo with hi = bf16(c), lo = bf16(c - hi), and both products accumulate
+// into D, so with bf16 queries every product is exact and only the fp32
+// accumulation and lo's rounding (2^-17 of c) remain.  Each epilogue thread
+// owns one key block (its TMEM lane) and takes the two maxima over its row of
+// BQ columns in registers.  Selection then proceeds as for the mean query.
+//
+// Roles (256 threads, one CTA per SM, persistent over rows (batch, q head,
+// query block), longest rows first):
+//   warps 0-3  token norms |q_t| from the query tile in shared memory, then
+//              per key tile the two maxima of their TMEM lane quarter; scores
+//              to a double-buffered shared row
+//   warp 4     TMA producer: the query tile (once per row) and the hi / lo
+//              centroid tiles (2-stage ring), no multicast
+//   warp 5     TMEM allocation and the MMA issue (one elected lane)
+//   warps 6-7  both branches' top-k of alternate rows (select_row)
+#pragma once
+
+#include "common.cuh"
+#include "select.cuh"
+
+namespace rbs {
+
+constexpr int kTokThreads = 256;
+constexpr int kTokCStages = 2;
+constexpr int kTokMaxKV = 2048;  // key blocks per sequence in this mode
+
+template <int BQ>
+struct TokSmem {
+  static constexpr int kQBytes = BQ * 256;       // BQ tokens x 128 dims (two 64-dim halves of BQ x 128 B)
+  static constexpr int kCHalf = 128 * 128;       // 128 key blocks x 64 dims, bf16
+  static constexpr int kCPart = 2 * kCHalf;      // one part (hi or lo): 32 KB
+  static constexpr int kCStage = 2 * kCPart;     // hi then lo
+  static constexpr int kQ = 0;
+  static constexpr int kC = kQ + kQBytes;        // 1024-aligned: kQBytes is 16 or 32 KB
+  static constexpr int kScores = kC + kTokCStages * kCStage;  // float [2 rows][2 branches][kTokMaxKV]
+  static constexpr int kQn = kScores + 2 * 2 * kTokMaxKV * 4;  // float [2 rows][128]
+  static constexpr int kScratch = kQn + 2 * 128 * 4;           // top-k scratch of warps 6 and 7
+  static constexpr int kScratchWords = sel_topk_scratch_words(kTokMaxKV / 32);
+  static constexpr int kBar = kScratch + 2 * kScratchWords * 4;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kTotal = kBar + kBarBytes;
+  static constexpr int kAlloc = kTotal + 1024;  // slack to align the base to 1024
+  static constexpr uint32_t kTmemCols = 256;    // two D buffers of BQ columns
+};
+
+enum : int {
+  kTokQFull = 0,
+  kTokQEmpty = 1,                   // MMA commit + 4 norm warps
+  kTokCFull = 2,                    // + stage
+  kTokCEmpty = kTokCFull + kTokCStages,
+  kTokDFull = kTokCEmpty + kTokCStages,  // + D buffer
+  kTokDEmpty = kTokDFull + 2,
+  kTokSFull = kTokDEmpty + 2,       // + score row buffer
+  kTokSEmpty = kTokSFull + 2,
+  kTokNumBars = kTokSEmpty + 2
+};
+
+struct TokArgs {
+  CUtensorMap tmQ, tmChi, tmClo;  // Q [B, Lq, Hq, 128]; centroid parts [B, Hkv, nkb, 128] (token index = block)
+  SelectArgs s;
+  int rows;  // work items: B * Hq * nqb
+};
+
+// Row w -> (batch, q head, query block): the last query blocks first.
+__device__ __forceinline__ void tok_item(const SelectArgs& a, int w, int& b, int& hq, int& i) {
+  const int per_i = a.B * a.Hq;
+  i = a.nqb - 1 - w / per_i;
+  const int rem = w % per_i;
+  b = rem / a.Hq;
+  hq = rem % a.Hq;
+}
+
+template <int BQ, int KPL>
+__global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __grid_constant__ TokArgs ta) {
+  using L = TokSmem<BQ>;
+  const SelectArgs& a = ta.s;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + L::kQ, sC = sbase + L::kC;
+  float* scores = reinterpret_cast<float*>(smem + L::kScores);
+  float* qn_s = reinterpret_cast<float*>(smem + L::kQn);
+  const uint32_t bars = sbase + L::kBar;
+  auto bar = [&](int k) -> uint32_t { return bars + 8u * k; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kTokNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + kTokNumBars * 8 + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.Hq / a.Hkv;
+  const int nitems = ta.rows > static_cast<int>(blockIdx.x)
+                         ? (ta.rows - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                         : 0;
+  auto visible = [&](int i) { return a.causal ? min(a.nkb, i + a.q_block_offset + 1) : a.nkb; };
+
+  if (tid == 0) {
+    mbar_init(bar(kTokQFull), 1);
+    mbar_init(bar(kTokQEmpty), 1 + 4);
+    for (int s = 0; s < kTokCStages; ++s) {
+      mbar_init(bar(kTokCFull + s), 1);
+      mbar_init(bar(kTokCEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kTokDFull + s), 1);
+      mbar_init(bar(kTokDEmpty + s), 4);
+      mbar_init(bar(kTokSFull + s), 4);
+      mbar_init(bar(kTokSEmpty + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&ta.tmQ);
+      tma_prefetch_desc(&ta.tmChi);
+      tma_prefetch_desc(&ta.tmClo);
+      uint32_t gt = 0, nq = 0;  // centroid tiles and query tiles issued
+      bool ok = true;
+      for (int k = 0; k < nitems && ok; ++k) {
+        int b, hq, i;
+        tok_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq, i);
+        // the previous row's MMAs and token norms are done with the query tile
+        if (k > 0 && !mbar_wait(bar(kTokQEmpty), (k - 1) & 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(kTokQFull), BQ * 256);
+        tma_load_4d(sQ, &ta.tmQ, bar(kTokQFull), 0, hq, i * BQ, b);
+        tma_load_4d(sQ + BQ * 128, &ta.tmQ, bar(kTokQFull), 64, hq, i * BQ, b);
+        ++nq;
+        const int kvh = hq / G;
+        const int T = (visible(i) + 127) / 128;
+        for (int m = 0; m < T; ++m, ++gt) {
+          const int s = gt % kTokCStages;
+          // the stage's previous tile, gt - 2, must be consumed by its MMAs
+          if (gt >= kTokCStages && !mbar_wait(bar(kTokCEmpty + s), ((gt / kTokCStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sC + s * L::kCStage;
+          mbar_arrive_expect_tx(bar(kTokCFull + s), L::kCStage);
+          tma_load_4d(dst, &ta.tmChi, bar(kTokCFull + s), 0, m * 128, kvh, b);
+          tma_load_4d(dst + L::kCHalf, &ta.tmChi, bar(kTokCFull + s), 64, m * 128, kvh, b);
+          tma_load_4d(dst + L::kCPart, &ta.tmClo, bar(kTokCFull + s), 0, m * 128, kvh, b);
+          tma_load_4d(dst + L::kCPart + L::kCHalf, &ta.tmClo, bar(kTokCFull + s), 64, m * 128, kvh, b);
+        }
+      }
+      // every load issued must land before the CTA exits: stage s was filled
+      // at tile numbers s, s + 2, ...; its last fill completes phase (uses - 1)
+      for (uint32_t s = 0; s < kTokCStages; ++s)
+        if (s < gt) mbar_drain(bar(kTokCFull + s), ((gt - s + kTokCStages - 1) / kTokCStages - 1) & 1);
+      if (nq > 0) mbar_drain(bar(kTokQFull), (nq - 1) & 1);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer (whole warp, one elected lane)
+    constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 0, 0);
+    const uint64_t cdesc0 = smem_desc(sC, 16, 1024, kLayoutSW128);
+    const uint64_t qdesc0 = smem_desc(sQ, 16, 1024, kLayoutSW128);
+    constexpr uint32_t kCHalfU = L::kCHalf >> 4, kCPartU = L::kCPart >> 4, kCStageU = L::kCStage >> 4;
+    constexpr uint32_t kQHalfU = (BQ * 128) >> 4;
+    auto wait = [&](int k, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar(k), parity, abort_flag)); };
+    uint32_t gt = 0;
+    bool ok = true;
+    for (int k = 0; k < nitems && ok; ++k) {
+      int b, hq, i;
+      tok_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq, i);
+      if (!wait(kTokQFull, k & 1)) break;
+      const int T = (visible(i) + 127) / 128;
+      for (int m = 0; m < T; ++m, ++gt) {
+        const int s = gt % kTokCStages, db = gt & 1;
+        if (!wait(kTokCFull + s, (gt / kTokCStages) & 1)) { ok = false; break; }
+        // D buffer db held tile gt - 2: its epilogue must have read it
+        if (gt >= 2 && !wait(kTokDEmpty + db, ((gt >> 1) - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = cdesc0 + s * kCStageU + part * kCPartU + (kk >> 2) * kCHalfU + (kk & 3) * 2;
+            const uint64_t bd = qdesc0 + (kk >> 2) * kQHalfU + (kk & 3) * 2;
+            umma_ss_warp(tmem + db * BQ, ad, bd, idesc, (part | kk) != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit_warp(bar(kTokCEmpty + s));
+        umma_commit_warp(bar(kTokDFull + db));
+      }
+      if (ok) umma_commit_warp(bar(kTokQEmpty));
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ token norms and the per-block maxima
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t gt = 0;
+    bool ok = true;
+    for (int k = 0; k < nitems && ok; ++k) {
+      int b, hq, i;
+      tok_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq, i);
+      const int n = visible(i), T = (n + 127) / 128;
+      const int nq = min(BQ, a.Lq - i * BQ);  // valid tokens of this query block
+      const int kvh = hq / G;
+      const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
+      float* qn = qn_s + (k & 1) * 128;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokQFull), k & 1, abort_flag))) break;
+      if (tid < BQ) {
+        // token tid: 16-byte chunk c of its 128-byte row in each half sits at
+        // chunk position c ^ (tid % 8) (128-byte swizzle)
+        float s2 = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kQ + h * BQ * 128 + tid * 128 +
+                                                            ((c ^ (tid & 7)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              s2 = fmaf(bf16lo(w[q]), bf16lo(w[q]), s2);
+              s2 = fmaf(bf16hi(w[q]), bf16hi(w[q]), s2);
+            }
+          }
+        }
+        qn[tid] = sqrtf(s2);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kTokQEmpty));
+      named_bar_sync(1, 128);  // qn complete
+      const int sb = k & 1;
+      float* sc_c = scores + sb * 2 * kTokMaxKV;
+      float* sc_r = sc_c + kTokMaxKV;
+      // the top-k of row k - 2 must be done with this score buffer
+      if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(kTokSEmpty + sb), ((k >> 1) - 1) & 1, abort_flag))) break;
+      for (int m = 0; m < T; ++m, ++gt) {
+        const int db = gt & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokDFull + db), (gt >> 1) & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        const int j = m * 128 + warp * 32 + lane;
+        const float rho = j < n ? a.rad[kv_off + j] * a.beta[kv_off + j] : 0.f;
+        float mc = -INFINITY, mr = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BQ / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + db * BQ + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (32 * c + e < nq) {
+              const float d = __uint_as_float(v[e]);
+              mc = fmaxf(mc, d);
+              mr = fmaxf(mr, fmaf(qn[32 * c + e], rho, d));
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kTokDEmpty + db));
+        if (j < n) {
+          sc_c[j] = mc;
+          sc_r[j] = mr;
+        }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kTokSFull + sb));
+    }
+  } else {
+    // ------------------------------------------------------------ top-k of alternate rows
+    const int tk = warp - 6;
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(smem + L::kScratch) + tk * L::kScratchWords;
+    for (int k = tk; k < nitems; k += 2) {
+      int b, hq, i;
+      tok_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq, i);
+      const int sb = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokSFull + sb), (k >> 1) & 1, abort_flag))) break;
+      const float* sc_c = scores + sb * 2 * kTokMaxKV;
+      const float* sc_r = sc_c + kTokMaxKV;
+      const int n = visible(i), gi = i + a.q_block_offset;
+      const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
+      auto fc = [&](int j) { return sc_c[j]; };
+      auto fr = [&](int j) { return sc_r[j]; };
+      if (KPL > 2 && n <= 64) select_row<2, KPL>(a, fc, fr, row, lane, gi, n, scratch);
+      else if (KPL > 8 && n <= 256) select_row<8, KPL>(a, fc, fr, row, lane, gi, n, scratch);
+      else if (KPL > 16 && n <= 512) select_row<16, KPL>(a, fc, fr, row, lane, gi, n, scratch);
+      else if (KPL > 32 && n <= 1024) select_row<32, KPL>(a, fc, fr, row, lane, gi, n, scratch);
+      else select_row<KPL, KPL>(a, fc, fr, row, lane, gi, n, scratch);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kTokSEmpty + sb));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// c -> (hi, lo) bf16 parts: hi = bf16(c), lo = bf16(c - hi), both rounded to
+// nearest even, so hi + lo carries c to about 2^-17 of its size.
+__global__ void __launch_bounds__(256) split_centroids_kernel(const float* __restrict__ C, int64_t n,
+                                                              __nv_bfloat16* __restrict__ hi,
+                                                              __nv_bfloat16* __restrict__ lo) {
+  for (int64_t k = blockIdx.x * 256ll + threadIdx.x; k < n; k += static_cast<int64_t>(gridDim.x) * 256) {
+    const float c = C[k];
+    const __nv_bfloat16 h = __float2bfloat16_rn(c);
+    hi[k] = h;
+    lo[k] = __float2bfloat16_rn(c - __bfloat162float(h));
+  }
+}
+
+}  // namespace rbs

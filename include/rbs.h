@@ -59,7 +59,7 @@ extern "C" {
 #define RBS_API
 #endif
 
-#define RBS_ABI_VERSION 3
+#define RBS_ABI_VERSION 4
 #define RBS_HEAD_DIM 128
 #define RBS_MAX_SEGMENTS 512 /* Block-attention segments per call */
 #define RBS_MAX_KV_BLOCKS 4096 /* key blocks per sequence for rbs_select */
@@ -122,6 +122,14 @@ typedef struct {
  *                      [RBS-en] "How This Fits Into the Broader Sparse
  *                      Attention Landscape"; shared key blocks across queries,
  *                      [QUILT] Abstract) (0)
+ *   query_pool         the query side of the scores: 0 = MEAN: the mean of
+ *                      the query block's queries, qbar (as above); 1 =
+ *                      TOKEN_MAX: each branch takes the best token of the
+ *                      block, s_c = max_t q_t . c_j and s_r = max_t (q_t . c_j
+ *                      + ||q_t|| r_j beta_j) ([RBS-en] "The Fix" scores a query
+ *                      q; here q runs over the block's tokens).  TOKEN_MAX
+ *                      needs num_kv_blocks <= 2048, Q with stride_h <=
+ *                      stride_s, and a larger workspace (0)
  * Scores are raw dot products (no 1/sqrt(d)); ties between equal scores go
  * to the lower block index.  Forced blocks do not count toward a branch's k.
  */
@@ -136,6 +144,7 @@ typedef struct {
   int32_t threshold_mode;
   float delta_centroid, delta_rescue;
   int32_t list_mode;
+  int32_t query_pool;
 } rbs_select_params;
 
 /* Per-query-block key-block lists in CSR form (all device memory). */

@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_housekeeping(L):
-    assert L.rbs_abi_version() == 3
+    assert L.rbs_abi_version() == 4
     assert L.rbs_status_string(0) == b"ok"
     assert L.rbs_status_string(3) == b"capacity"
     p = _abi.SelectParamsC()
