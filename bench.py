@@ -52,9 +52,9 @@ SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
 # dram__bytes_write.sum, one single-pass ncu capture of the default workload;
 # profiles/launches_gqa_rbs_128k.md gives the command), valid for the kernel
 # sources with this digest; any other build reports null.
-ATTN_TRAFFIC_BYTES = 3.345e9 + 1.039e9
+ATTN_TRAFFIC_BYTES = 3.306e9 + 1.040e9
 ATTN_TRAFFIC_SOURCES = ("block_sparse_long_rbs_b200/csrc/attention.cuh", "block_sparse_long_rbs_b200/csrc/common.cuh")
-ATTN_TRAFFIC_DIGEST = "af8b21ab5100c5b2"
+ATTN_TRAFFIC_DIGEST = "ef6c3e5cf172632b"
 
 
 def attn_traffic(seq_len: int):
@@ -824,8 +824,9 @@ def cpu_baseline(Qh, Kh, Vh, w, budget_s: float = 20.0, heads_q: int | None = No
     t_sel = time.perf_counter() - t0
     rp, ci = sel["row_ptr"], sel["col_idx"]
     lens = np.diff(rp)
-    # attention on rows spread over the causal range until the time budget is used
-    order = np.linspace(nqb - 1, 0, 64).astype(int)
+    # attention on rows spread over the causal range (every 16th row, longest
+    # first, then the rows in between) until the time budget is used
+    order = np.concatenate([np.arange(nqb - 1 - s, -1, -16) for s in range(16)])
     done_pairs, t_attn, nrows = 0, 0.0, 0
     for row in order:
         t0 = time.perf_counter()

@@ -688,6 +688,12 @@ __device__ __forceinline__ uint32_t forced_word(int t, int gi, int nkb, int forc
 // Mask word t of list row (b, hl, i): the OR over the row's q heads.
 __device__ __forceinline__ void list_row_word(const CompactArgs& a, int b, int hl, int i, int t, uint32_t& c,
                                               uint32_t& r) {
+  if (a.glist == 1) {  // one list per q head: the list row is the mask row
+    const int64_t m = ((static_cast<int64_t>(b) * a.Hq + hl) * a.nqb + i) * a.nwords + t;
+    c = a.mask_c[m];
+    r = a.mask_r[m];
+    return;
+  }
   c = r = 0;
   for (int hh = 0; hh < a.glist; ++hh) {
     const int64_t m = ((static_cast<int64_t>(b) * a.Hq + hl * a.glist + hh) * a.nqb + i) * a.nwords + t;
