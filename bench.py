@@ -45,8 +45,9 @@ WORKLOAD = "gqa_rbs_128k"
 BLOCK = 128
 HEAD_DIM = 128
 FLOP_PER_PAIR = 4 * BLOCK * BLOCK * HEAD_DIM  # QK^T and PV on one 128x128 block pair
-# kernels one step launches: block stats; beta, scoring + top-k, scan, compaction; attention
-LAUNCHES_PER_STEP = 6
+# kernels one step launches: block stats; selection (beta, centroid split,
+# pooling, score MMAs, top-k, scan, compaction); attention
+LAUNCHES_PER_STEP = 9
 SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
 # DRAM traffic of one 131072-token attention launch (dram__bytes_read.sum +
 # dram__bytes_write.sum, one single-pass ncu capture of the default workload;

@@ -17,6 +17,7 @@
 #include "rope.cuh"
 #include "select.cuh"
 #include "stats.cuh"
+#include "select_mma.cuh"
 #include "tokmax.cuh"
 
 using namespace rbs;
@@ -92,6 +93,14 @@ rbs_status device_info(DeviceInfo** out) {
     RBS_TOK_ATTR(32)
     RBS_TOK_ATTR(64)
 #undef RBS_TOK_ATTR
+    e = e ? e : cudaFuncSetAttribute(pool_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kPoolKStages * kPoolChunkBytes);
+    e = e ? e : cudaFuncSetAttribute(pool_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kPoolKStages * kPoolChunkBytes);
+    e = e ? e : cudaFuncSetAttribute(score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem::kAlloc);
+    for (auto kern : {topk_rows_kernel<2>, topk_rows_kernel<8>, topk_rows_kernel<32>, topk_rows_kernel<64>})
+      e = e ? e : cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(topk_smem_bytes(kTokMaxKV, kTokMaxKV / 32)));
     e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
     if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     d.attrs_set = true;
@@ -192,6 +201,41 @@ rbs_status make_pool_tensor_map(const rbs_bf16_tensor* t, int R, CUtensorMap* ma
   return RBS_OK;
 }
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct SelectLayout {
+  size_t mask_c, mask_r, counts, beta, c_hi, c_lo, q_hi, q_lo, qnorm, scores;
+  size_t base;   // bytes the fused mean-query kernel needs
+  size_t total;  // bytes of the full layout
+};
+
+// The parts every path uses, then the bf16 hi / lo centroids (per-token and
+// tensor-core mean scoring) and, for the tensor-core mean scoring, the pooled
+// queries' parts and norms and the score matrix [rows, nkb rounded up to 32].
+SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int64_t nkb, bool token_max) {
+  SelectLayout l{};
+  const int64_t rows = B * Hq * nqb;
+  const int64_t nwords = (nkb + 31) / 32;
+  size_t off = 0;
+  l.mask_c = off; off += align256(rows * nwords * 4);
+  l.mask_r = off; off += align256(rows * nwords * 4);
+  l.counts = off; off += align256(rows * 4);
+  l.beta = off; off += align256(B * Hkv * nkb * 4);
+  l.base = off;
+  l.c_hi = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
+  l.c_lo = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
+  if (token_max) {
+    l.base = off;  // the per-token kernel needs the centroid parts
+  } else {
+    l.q_hi = off; off += align256(rows * RBS_HEAD_DIM * 2);
+    l.q_lo = off; off += align256(rows * RBS_HEAD_DIM * 2);
+    l.qnorm = off; off += align256(rows * 4);
+    l.scores = off; off += align256(rows * nwords * 32 * 4);
+  }
+  l.total = off;
+  return l;
+}
+
 // Per-token-max selection scores (query_pool TOKEN_MAX): split the centroids
 // into bf16 hi / lo parts in the workspace, then one persistent CTA per SM
 // scores and thresholds rows (select_tokmax_kernel), writing the same mask
@@ -241,35 +285,131 @@ rbs_status launch_token_max(const rbs_bf16_tensor* Q, const float* centroids, in
   return check_launch("select_tokmax_kernel");
 }
 
+// 4-D map over a contiguous [B, H, n, 128] bf16 array with a box of 64 dims x
+// rows x heads (128-byte swizzle): the pooled-query parts, R heads x QB blocks.
+rbs_status make_rows_heads_map(void* data, int64_t B, int64_t H, int64_t n, int rows, int heads, CUtensorMap* map) {
+  PFN_encodeTiled enc = encode_fn();
+  if (enc == nullptr) return fail(RBS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[4] = {RBS_HEAD_DIM, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {RBS_HEAD_DIM * 2, static_cast<cuuint64_t>(n) * RBS_HEAD_DIM * 2,
+                                 static_cast<cuuint64_t>(H * n) * RBS_HEAD_DIM * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), static_cast<cuuint32_t>(heads), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, data, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RBS_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return RBS_OK;
+}
+
+// Mean-query scores on the tensor core: pool the query blocks into bf16 hi /
+// lo parts, split the centroids, one 128 x 128 x 128 MMA tile per (128 pooled
+// queries, 128 key blocks) into the score matrix, then one warp per row for
+// the top-k (pool_split_kernel, score_gemm_kernel, topk_rows_kernel).
+rbs_status launch_mma_select(const rbs_bf16_tensor* Q, const float* centroids, int64_t B, int32_t Hkv, int64_t nkb,
+                             const rbs_select_params* p, const SelectArgs& sa, int R, uint8_t* ws,
+                             const SelectLayout& lay, DeviceInfo* di, rbs_stream_t stream) {
+  rbs_status st;
+  const int64_t Hq = Q->heads, nqb = sa.nqb, rows = B * Hq * nqb;
+  const int npad = static_cast<int>((nkb + 31) & ~31ll);
+  auto* c_hi = reinterpret_cast<__nv_bfloat16*>(ws + lay.c_hi);
+  auto* c_lo = reinterpret_cast<__nv_bfloat16*>(ws + lay.c_lo);
+  auto* q_hi = reinterpret_cast<__nv_bfloat16*>(ws + lay.q_hi);
+  auto* q_lo = reinterpret_cast<__nv_bfloat16*>(ws + lay.q_lo);
+  float* qnorm = reinterpret_cast<float*>(ws + lay.qnorm);
+  float* scores = reinterpret_cast<float*>(ws + lay.scores);
+
+  const int64_t nc = B * Hkv * nkb * RBS_HEAD_DIM;
+  split_centroids_kernel<<<static_cast<unsigned>(std::min<int64_t>((nc + 255) / 256, 4 * di->sms)), 256, 0, stream>>>(
+      centroids, nc, c_hi, c_lo);
+  if ((st = check_launch("split_centroids_kernel")) != RBS_OK) return st;
+
+  // pooling
+  PoolArgs pa;
+  CUtensorMap qmap;
+  int seq_inner = 0;
+  if ((st = make_pool_tensor_map(Q, R, &qmap, &seq_inner)) != RBS_OK) return st;
+  pa.B = static_cast<int>(B);
+  pa.Hq = static_cast<int>(Hq);
+  pa.nqb = static_cast<int>(nqb);
+  pa.R = R;
+  pa.items = static_cast<int>(B * nqb * (Hq / R));
+  pa.Lq = static_cast<int>(Q->seqlen);
+  pa.seq_inner = seq_inner;
+  pa.qhi = q_hi;
+  pa.qlo = q_lo;
+  pa.qnorm = qnorm;
+  {
+    const size_t smem = kPoolKStages * kPoolChunkBytes;
+    auto launch = [&](auto kern) -> rbs_status {
+      int per_sm = 0;
+      const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPoolKThreads, smem);
+      if (e != cudaSuccess || per_sm < 1) return fail(RBS_ERR_CUDA, "pool_split_kernel does not fit on an SM");
+      const int grid = static_cast<int>(std::min<int64_t>(pa.items, static_cast<int64_t>(per_sm) * di->sms));
+      kern<<<grid, kPoolKThreads, smem, stream>>>(qmap, pa);
+      return check_launch("pool_split_kernel");
+    };
+    st = p->block_q == 128 ? launch(pool_split_kernel<128>) : launch(pool_split_kernel<64>);
+    if (st != RBS_OK) return st;
+  }
+
+  // scores
+  GemmArgs ga;
+  for (int part = 0; part < 2; ++part) {
+    rbs_bf16_tensor v;
+    v.data = part == 0 ? static_cast<void*>(c_hi) : static_cast<void*>(c_lo);
+    v.batch = B;
+    v.seqlen = nkb;
+    v.heads = Hkv;
+    v.head_dim = RBS_HEAD_DIM;
+    v.stride_b = Hkv * nkb * RBS_HEAD_DIM;
+    v.stride_s = RBS_HEAD_DIM;
+    v.stride_h = nkb * RBS_HEAD_DIM;
+    int si = 0;
+    if ((st = make_tensor_map(&v, 128, part == 0 ? &ga.tmChi : &ga.tmClo, &si)) != RBS_OK) return st;
+  }
+  const int QB = 128 / R;
+  if ((st = make_rows_heads_map(q_hi, B, Hq, nqb, QB, R, &ga.tmQhi)) != RBS_OK) return st;
+  if ((st = make_rows_heads_map(q_lo, B, Hq, nqb, QB, R, &ga.tmQlo)) != RBS_OK) return st;
+  ga.scores = scores;
+  ga.B = static_cast<int>(B);
+  ga.Hq = static_cast<int>(Hq);
+  ga.Hkv = Hkv;
+  ga.nqb = static_cast<int>(nqb);
+  ga.nkb = static_cast<int>(nkb);
+  ga.nkbp = npad;
+  ga.R = R;
+  ga.QB = QB;
+  ga.ngroups = static_cast<int>((nqb + QB - 1) / QB);
+  ga.items = static_cast<int>(B * (Hq / R) * ga.ngroups);
+  ga.q_block_offset = p->q_block_offset;
+  ga.causal = p->causal;
+  score_gemm_kernel<<<static_cast<unsigned>(std::min<int64_t>(ga.items, di->sms)), kGemmThreads, GemmSmem::kAlloc,
+                      stream>>>(ga);
+  if ((st = check_launch("score_gemm_kernel")) != RBS_OK) return st;
+
+  // top-k
+  TopkArgs ta;
+  ta.s = sa;
+  ta.scores = scores;
+  ta.qnorm = qnorm;
+  ta.nkbp = npad;
+  ta.rows = static_cast<int>(rows);
+  const size_t tsm = topk_smem_bytes(npad, sa.nwords);
+  const unsigned tgrid = static_cast<unsigned>((rows + 7) / 8);
+  if (nkb <= 64) topk_rows_kernel<2><<<tgrid, 256, tsm, stream>>>(ta);
+  else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, 256, tsm, stream>>>(ta);
+  else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, 256, tsm, stream>>>(ta);
+  else topk_rows_kernel<64><<<tgrid, 256, tsm, stream>>>(ta);
+  return check_launch("topk_rows_kernel");
+}
+
 int keep_count_host(float rho, int64_t n) {
   int64_t k = static_cast<int64_t>(std::ceil(static_cast<double>(rho) * static_cast<double>(n) - 1e-4));
   if (k < 1) k = 1;
   if (k > n) k = n;
   return static_cast<int>(k);
-}
-
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-struct SelectLayout {
-  size_t mask_c, mask_r, counts, beta, c_hi, c_lo, total;
-};
-
-// token_max: room for the bf16 hi / lo parts of the centroids as well
-SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int64_t nkb, bool token_max) {
-  SelectLayout l{};
-  const int64_t rows = B * Hq * nqb;
-  const int64_t nwords = (nkb + 31) / 32;
-  size_t off = 0;
-  l.mask_c = off; off += align256(rows * nwords * 4);
-  l.mask_r = off; off += align256(rows * nwords * 4);
-  l.counts = off; off += align256(rows * 4);
-  l.beta = off; off += align256(B * Hkv * nkb * 4);
-  if (token_max) {
-    l.c_hi = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
-    l.c_lo = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
-  }
-  l.total = off;
-  return l;
 }
 
 rbs_status check_lists(const rbs_block_lists* out, int64_t rows) {
@@ -458,8 +598,11 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   RBS_REQUIRE(out->capacity >= cap, RBS_ERR_CAPACITY, "list capacity %lld < %lld", static_cast<long long>(out->capacity),
               static_cast<long long>(cap));
   const SelectLayout lay = select_layout(B, Hq, nqb, kv_heads, nkb, p->query_pool == 1);
-  RBS_REQUIRE(workspace != nullptr && workspace_bytes >= lay.total, RBS_ERR_CAPACITY, "workspace %zu < %zu bytes",
-              workspace_bytes, lay.total);
+  // the full layout enables the tensor-core mean scoring; a workspace of at
+  // least the base part runs the fused kernel
+  RBS_REQUIRE(workspace != nullptr && workspace_bytes >= lay.base, RBS_ERR_CAPACITY, "workspace %zu < %zu bytes",
+              workspace_bytes, lay.base);
+  const bool mma_path = p->query_pool == 0 && workspace_bytes >= lay.total && nkb <= kTokMaxKV;
   RBS_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, RBS_ERR_INVALID_ARG, "workspace not 256-byte aligned");
   DeviceInfo* di;
   if ((st = device_info(&di)) != RBS_OK) return st;
@@ -504,6 +647,8 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   if (p->query_pool == 1) {
     if ((st = launch_token_max(Q, centroids, B, kv_heads, nkb, p, sa, ws + lay.c_hi, ws + lay.c_lo, di, stream)) != RBS_OK)
       return st;
+  } else if (mma_path) {
+    if ((st = launch_mma_select(Q, centroids, B, kv_heads, nkb, p, sa, R, ws, lay, di, stream)) != RBS_OK) return st;
   } else {
     const int npad = static_cast<int>((nkb + 31) & ~31ll);
     const size_t smem = sel_smem_bytes(npad);
@@ -601,8 +746,10 @@ rbs_status rbs_select_noalloc(const rbs_bf16_tensor* Q, const float* centroids, 
   RBS_REQUIRE(p != nullptr && (p->block_q == 64 || p->block_q == 128), RBS_ERR_UNSUPPORTED,
               "block_q must be 64 or 128");
   RBS_REQUIRE(kv_heads > 0 && num_kv_blocks > 0, RBS_ERR_INVALID_ARG, "empty KV shape");
-  const size_t need = rbs_select_workspace_bytes(Q->batch, Q->heads, (Q->seqlen + p->block_q - 1) / p->block_q, kv_heads,
-                                                 num_kv_blocks, p);
+  const size_t need = (Q->batch > 0 && Q->heads > 0 && kv_heads > 0 && num_kv_blocks > 0)
+                          ? select_layout(Q->batch, Q->heads, (Q->seqlen + p->block_q - 1) / p->block_q, kv_heads,
+                                          num_kv_blocks, p->query_pool == 1).base
+                          : 0;
   RBS_REQUIRE(need > 0 && need <= RBS_NOALLOC_SCRATCH_BYTES, RBS_ERR_CAPACITY,
               "this selection needs %zu bytes of scratch; the built-in buffer holds %zu (use rbs_select with a "
               "workspace)", need, static_cast<size_t>(RBS_NOALLOC_SCRATCH_BYTES));

@@ -148,6 +148,15 @@ __device__ __forceinline__ void warp_topk2(const uint32_t (&kc)[KPL], const uint
   }
 }
 
+// For a search value known to lie in [lo, hi] (lo <= hi): start = the bits
+// above the highest bit where lo and hi differ (shared by every value in the
+// range), top = that bit (-1 when lo == hi, nothing left to search).
+__device__ __forceinline__ void common_prefix(uint32_t lo, uint32_t hi, uint32_t& start, int& top) {
+  const int p = __clz(lo ^ hi);  // leading bits shared by lo and hi (32 when equal)
+  start = p == 32 ? lo : (p == 0 ? 0u : lo & ~(0xffffffffu >> p));
+  top = 31 - p;
+}
+
 // Insert x into the descending list (t0 >= t1 >= t2 >= t3).
 __device__ __forceinline__ void top4_insert(uint32_t& t0, uint32_t& t1, uint32_t& t2, uint32_t& t3, uint32_t x) {
   const uint32_t y0 = min(t0, x);
@@ -188,14 +197,21 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
     top4_insert(c0, c1, c2, c3, key_c(t));
     top4_insert(r0, r1, r2, r3, key_r(t));
   }
-  uint32_t Lc = 0, Lr = 0;
+  // L lies between the subset's smallest lane second-largest key (each lane
+  // has two keys at least that large: 64 >= k of them), rounded down to 8
+  // bits, and the subset's largest key, so it carries their common leading
+  // bits and the search starts below them.
+  uint32_t Lc, Lr;
+  int topc, topr;
+  common_prefix(__reduce_min_sync(0xffffffffu, c1) & ~255u, __reduce_max_sync(0xffffffffu, c0), Lc, topc);
+  common_prefix(__reduce_min_sync(0xffffffffu, r1) & ~255u, __reduce_max_sync(0xffffffffu, r0), Lr, topr);
 #pragma unroll 1
-  for (int bit = 31; bit >= 8; --bit) {
+  for (int bit = max(topc, topr); bit >= 8; --bit) {
     const uint32_t xc = Lc | (1u << bit), xr = Lr | (1u << bit);
     const int nc = __reduce_add_sync(0xffffffffu, (c0 >= xc) + (c1 >= xc) + (c2 >= xc) + (c3 >= xc));
     const int nr = __reduce_add_sync(0xffffffffu, (r0 >= xr) + (r1 >= xr) + (r2 >= xr) + (r3 >= xr));
-    if (nc >= k_c) Lc = xc;
-    if (nr >= k_r) Lr = xr;
+    if (bit <= topc && nc >= k_c) Lc = xc;
+    if (bit <= topr && nr >= k_r) Lr = xr;
   }
   // Every float's key but one NaN pattern is >= 256, so L > 0 and no absent
   // slot (key 0) becomes a candidate.
@@ -231,14 +247,19 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
     bk[s] = p < base_r ? ck_r[p] : 0u;
     ib[s] = p < base_r ? ci_r[p] : 0;
   }
-  uint32_t Tc = 0, Tr = 0;
+  // T lies between L (at least k candidates reach it) and the largest
+  // candidate: it carries their common leading bits
+  uint32_t Tc, Tr;
+  int tpc, tpr;
+  common_prefix(Lc, __reduce_max_sync(0xffffffffu, max(max(a[0], a[1]), max(a[2], a[3]))), Tc, tpc);
+  common_prefix(Lr, __reduce_max_sync(0xffffffffu, max(max(bk[0], bk[1]), max(bk[2], bk[3]))), Tr, tpr);
 #pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
+  for (int bit = max(tpc, tpr); bit >= 0; --bit) {
     const uint32_t xc = Tc | (1u << bit), xr = Tr | (1u << bit);
     const int nc = __reduce_add_sync(0xffffffffu, (a[0] >= xc) + (a[1] >= xc) + (a[2] >= xc) + (a[3] >= xc));
     const int nr = __reduce_add_sync(0xffffffffu, (bk[0] >= xr) + (bk[1] >= xr) + (bk[2] >= xr) + (bk[3] >= xr));
-    if (nc >= k_c) Tc = xc;
-    if (nr >= k_r) Tr = xr;
+    if (bit <= tpc && nc >= k_c) Tc = xc;
+    if (bit <= tpr && nr >= k_r) Tr = xr;
   }
   const int need_c = k_c - __reduce_add_sync(0xffffffffu, (a[0] > Tc) + (a[1] > Tc) + (a[2] > Tc) + (a[3] > Tc));
   const int need_r = k_r - __reduce_add_sync(0xffffffffu, (bk[0] > Tr) + (bk[1] > Tr) + (bk[2] > Tr) + (bk[3] > Tr));
@@ -262,26 +283,66 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
   return true;
 }
 
-// Both branches' top-k of one list row (warp-wide) -> mask words and the
+// The row's mask words (and forced blocks) -> the mask arrays and the row's
+// union count.  Warp-wide.
+__device__ __forceinline__ void emit_row(const SelectArgs& a, const uint32_t* words_c, const uint32_t* words_r,
+                                         int64_t row, int lane, int gi) {
+  int cnt = 0;
+  for (int t = lane; t < a.nwords; t += 32) {
+    const uint32_t wc = words_c[t], wr = words_r[t];
+    uint32_t f = 0;
+    if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
+    if (a.force_sink && t == 0) f |= 1u;
+    cnt += __popc(wc | wr | f);
+    a.mask_c[row * a.nwords + t] = wc;
+    a.mask_r[row * a.nwords + t] = wr;
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) a.counts[row] = cnt;
+}
+
+// Both branches' top-k (TOPK_FRACTION) of one list row from order-preserving
+// keys: key_c(t), key_r(t) = the keys of block 32t + lane (0 past the n
+// visible blocks); KP slots per lane, mask words covering nwords <=
+// (KPMAX + 31) / 32 * 32 words.  Warp-wide.
+template <int KP, int KPMAX, typename KC, typename KR>
+__device__ __forceinline__ void select_row_keys(const SelectArgs& a, KC key_c, KR key_r, int64_t row, int lane,
+                                                int gi, int n, uint32_t* scratch) {
+  uint32_t* words_c = scratch + 4 * kTopkCap;
+  uint32_t* words_r = words_c + a.nwords;
+  const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
+  const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, scratch, words_c, words_r);
+  if (!done) {
+    uint32_t kc[KP], kr[KP];
+#pragma unroll
+    for (int t = 0; t < KP; ++t) {
+      kc[t] = key_c(t);
+      kr[t] = key_r(t);
+    }
+    constexpr int NO = (KP + 31) / 32;
+    uint32_t own_c[NO], own_r[NO];
+    warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
+    for (int w = lane; w < a.nwords; w += 32) {
+      const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
+      words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+      words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+    }
+    __syncwarp();
+  }
+  emit_row(a, words_c, words_r, row, lane, gi);
+}
+
+// Both branches' selection of one list row (warp-wide) -> mask words and the
 // row's union count.  score_c(j), score_r(j) give the branches' scores of the
-// visible block j < n; keys hold KP slots per lane (block 32t + lane in slot
-// t); the row's mask words cover all nwords <= (KPMAX + 31) / 32 * 32 words.
+// visible block j < n; the top-k runs on KP key slots per lane.
 template <int KP, int KPMAX, typename SC, typename SR>
 __device__ __forceinline__ void select_row(const SelectArgs& a, SC score_c, SR score_r, int64_t row, int lane,
                                            int gi, int n, uint32_t* scratch) {
-  uint32_t* words_c = scratch + 4 * kTopkCap;
-  uint32_t* words_r = words_c + a.nwords;
-  auto key_c = [&](int t) -> uint32_t {
-    const int j = 32 * t + lane;
-    return j < n ? order_key(score_c(j)) : 0u;
-  };
-  auto key_r = [&](int t) -> uint32_t {
-    const int j = 32 * t + lane;
-    return j < n ? order_key(score_r(j)) : 0u;
-  };
   if (a.threshold_mode == 1) {
     // Each branch keeps every visible block scoring at least its row maximum
     // minus delta; the threshold is formed in fp32 from the maximum score.
+    uint32_t* words_c = scratch + 4 * kTopkCap;
+    uint32_t* words_r = words_c + a.nwords;
     float mc = -INFINITY, mr = -INFINITY;
     for (int j = lane; j < n; j += 32) {
       mc = fmaxf(mc, score_c(j));
@@ -306,39 +367,18 @@ __device__ __forceinline__ void select_row(const SelectArgs& a, SC score_c, SR s
       words_r[w] = wr;
     }
     __syncwarp();
-  } else {
-    const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
-    const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, scratch, words_c, words_r);
-    if (!done) {
-      uint32_t kc[KP], kr[KP];
-#pragma unroll
-      for (int t = 0; t < KP; ++t) {
-        kc[t] = key_c(t);
-        kr[t] = key_r(t);
-      }
-      constexpr int NO = (KP + 31) / 32;
-      uint32_t own_c[NO], own_r[NO];
-      warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
-      for (int w = lane; w < a.nwords; w += 32) {
-        const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
-        words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
-        words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
-      }
-      __syncwarp();
-    }
+    emit_row(a, words_c, words_r, row, lane, gi);
+    return;
   }
-  int cnt = 0;
-  for (int t = lane; t < a.nwords; t += 32) {
-    const uint32_t wc = words_c[t], wr = words_r[t];
-    uint32_t f = 0;
-    if (a.force_diag && gi < a.nkb && (gi >> 5) == t) f |= 1u << (gi & 31);
-    if (a.force_sink && t == 0) f |= 1u;
-    cnt += __popc(wc | wr | f);
-    a.mask_c[row * a.nwords + t] = wc;
-    a.mask_r[row * a.nwords + t] = wr;
-  }
-  cnt = __reduce_add_sync(0xffffffffu, cnt);
-  if (lane == 0) a.counts[row] = cnt;
+  auto key_c = [&](int t) -> uint32_t {
+    const int j = 32 * t + lane;
+    return j < n ? order_key(score_c(j)) : 0u;
+  };
+  auto key_r = [&](int t) -> uint32_t {
+    const int j = 32 * t + lane;
+    return j < n ? order_key(score_r(j)) : 0u;
+  };
+  select_row_keys<KP, KPMAX>(a, key_c, key_r, row, lane, gi, n, scratch);
 }
 
 // The mean-pooled scores of row `warp` of the CTA's item:

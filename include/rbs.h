@@ -213,8 +213,12 @@ RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, f
  *                the last one shorter when Lq is not a block multiple
  *   centroids    [B, Hkv, num_kv_blocks, 128] fp32 (rbs_block_stats)
  *   radii        [B, Hkv, num_kv_blocks] fp32
- *   workspace    device scratch of at least rbs_select_workspace_bytes(...)
- *                bytes, 256-byte aligned; its contents need no initialisation
+ *   workspace    device scratch, 256-byte aligned, contents need no
+ *                initialisation.  rbs_select_workspace_bytes(...) bytes
+ *                enable the tensor-core scoring of the mean query (the score
+ *                matrix lives there); a smaller workspace runs the fused
+ *                CUDA-core scoring kernel, down to the masks and counts it
+ *                needs (RBS_ERR_CAPACITY below that)
  *   out          lists with num_rows = B * Hq * nQB (B * Hkv * nQB when
  *                list_mode is KV_GROUP) and capacity >=
  *                rbs_select_capacity(...), which bounds both modes;

@@ -128,7 +128,12 @@ def test_select_rejects_small_capacity_and_workspace(L):
                       None, None)
     assert st == 3
     ok = _abi.BlockListsC(0x40000, 0x50000, None, need, rows)
+    # a workspace below the full size still runs (the fused scoring kernel) ...
     st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, ws - 1, ctypes.byref(ok),
+                      None, None)
+    assert st == 4  # past validation: no GPU here
+    # ... down to the masks and counts it needs
+    st = L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(pc), 0x60000, 256, ctypes.byref(ok),
                       None, None)
     assert st == 3
     wrong_rows = _abi.BlockListsC(0x40000, 0x50000, None, need, rows + 1)

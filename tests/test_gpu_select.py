@@ -112,3 +112,34 @@ def test_select_max_relative_mixture_gqa(cuda_ok):
     inp = make_mixture(L=8192, Hq=16, Hkv=2, block=128, seed=201)
     rep = _run(inp, 128, 0.05, 0.05, threshold_mode=1, delta_centroid=0.5, delta_rescue=2.0)
     print("max-relative mixture", rep)
+
+
+@pytest.mark.parametrize("case", ["mixture", "32k"])
+def test_select_fused_kernel_with_smaller_workspace(cuda_ok, case):
+    # a workspace one byte short of rbs_select_workspace_bytes has no room for
+    # the score matrix: the fused CUDA-core scoring kernel runs instead of the
+    # tensor-core scores; both must match the oracle
+    if case == "mixture":
+        inp, block, rho = make_mixture(L=8192, Hq=8, Hkv=2, block=128, seed=205, batch=2), 128, 0.1
+    else:
+        inp, block, rho = make_inputs(WORKLOADS["gqa_rbs_32k"]), 128, 0.05
+    Q, K = inp["Q"], inp["K"]
+    B, L, Hq, _ = Q.shape
+    Hkv, nqb, nkb = K.shape[2], L // block, K.shape[1] // block
+    p = rbs.SelectParams(block_q=block, block_k=block, rho_centroid=rho, rho_rescue=rho)
+    Cg, Rg = rbs.rbs_block_stats(dev(K), block)
+    full = rbs.rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, p)
+    ws = torch.empty(full + 255, dtype=torch.uint8, device="cuda")
+    off = (-ws.data_ptr()) % 256
+    small = ws[off:off + full - 1]
+    lists = rbs.rbs_select(dev(Q), Cg, Rg, p, workspace=small)
+    ref = rbs.rbs_select(dev(Q), Cg, Rg, p)
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    Co, Ro = O.block_stats(K, block)
+    po = O.SelectParams(block_q=block, block_k=block, rho_centroid=float(np.float32(rho)),
+                        rho_rescue=float(np.float32(rho)))
+    ora = O.select_blocks(Q, Co, Ro, po, keep_scores=True)
+    rep_small = compare_selection(lists, ora, Hq, nqb, nkb)
+    rep_full = compare_selection(ref, ora, Hq, nqb, nkb)
+    print("fused", rep_small, "tensor-core", rep_full)
