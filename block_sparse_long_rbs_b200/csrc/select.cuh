@@ -88,6 +88,11 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float whose order_key is k (order_key is a bijection).
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 __device__ __forceinline__ int keep_count(float rho, int n) {
   // k = ceil(rho * n) within [1, n]; rho is the float32 parameter widened to
   // double, and the 1e-4 slack absorbs its float32 representation error.

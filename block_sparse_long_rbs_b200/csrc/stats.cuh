@@ -16,6 +16,20 @@
 
 namespace rbs {
 
+// The same unpacking as opaque instructions: a kernel that reads packed data
+// held in registers twice uses these in its second pass, so the compiler does
+// not keep the first pass's unpacked floats alive (twice the registers).
+__device__ __forceinline__ float bf16lo_again(uint32_t v) {
+  uint32_t u;
+  asm volatile("shl.b32 %0, %1, 16;" : "=r"(u) : "r"(v));
+  return __uint_as_float(u);
+}
+__device__ __forceinline__ float bf16hi_again(uint32_t v) {
+  uint32_t u;
+  asm volatile("and.b32 %0, %1, 0xFFFF0000;" : "=r"(u) : "r"(v));
+  return __uint_as_float(u);
+}
+
 template <int BK>
 __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* __restrict__ K, int64_t sb,
                                                           int64_t ss, int64_t sh, int nkb, int H, int L,
@@ -72,8 +86,8 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
     float d2 = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float a = bf16lo(w[q]) - cl[2 * q];
-      const float bb = bf16hi(w[q]) - cl[2 * q + 1];
+      const float a = bf16lo_again(w[q]) - cl[2 * q];
+      const float bb = bf16hi_again(w[q]) - cl[2 * q + 1];
       d2 = fmaf(a, a, d2);
       d2 = fmaf(bb, bb, d2);
     }

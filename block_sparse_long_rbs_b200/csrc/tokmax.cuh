@@ -11,18 +11,20 @@
 // hi + lo with hi = bf16(c), lo = bf16(c - hi), and both products accumulate
 // into D, so with bf16 queries every product is exact and only the fp32
 // accumulation and lo's rounding (2^-17 of c) remain.  Each epilogue thread
-// owns one key block (its TMEM lane) and takes the two maxima over its row of
-// BQ columns in registers.  Selection then proceeds as for the mean query.
+// owns one key block (its TMEM lane) and takes the two maxima over half of
+// its row of BQ columns in registers.  Selection then proceeds as for the
+// mean query.
 //
-// Roles (256 threads, one CTA per SM, persistent over rows (batch, q head,
+// Roles (384 threads, one CTA per SM, persistent over rows (batch, q head,
 // query block), longest rows first):
-//   warps 0-3  token norms |q_t| from the query tile in shared memory, then
-//              per key tile the two maxima of their TMEM lane quarter; scores
-//              to a double-buffered shared row
-//   warp 4     TMA producer: the query tile (once per row) and the hi / lo
+//   warps 0-7  token norms |q_t| from the query tile in shared memory, then
+//              per key tile the two maxima over half the tokens (two warps
+//              per TMEM lane quarter); the halves meet through atomicMax on
+//              order-preserving keys in a double-buffered shared row
+//   warp 8     TMA producer: the query tile (once per row) and the hi / lo
 //              centroid tiles (2-stage ring), no multicast
-//   warp 5     TMEM allocation and the MMA issue (one elected lane)
-//   warps 6-7  both branches' top-k of alternate rows (select_row)
+//   warp 9     TMEM allocation and the MMA issue (one elected lane)
+//   warps 10-11 both branches' top-k of alternate rows from those keys
 #pragma once
 
 #include "common.cuh"
@@ -30,7 +32,7 @@
 
 namespace rbs {
 
-constexpr int kTokThreads = 256;
+constexpr int kTokThreads = 384;
 constexpr int kTokCStages = 2;
 constexpr int kTokMaxKV = 2048;  // key blocks per sequence in this mode
 
@@ -42,9 +44,9 @@ struct TokSmem {
   static constexpr int kCStage = 2 * kCPart;     // hi then lo
   static constexpr int kQ = 0;
   static constexpr int kC = kQ + kQBytes;        // 1024-aligned: kQBytes is 16 or 32 KB
-  static constexpr int kScores = kC + kTokCStages * kCStage;  // float [2 rows][2 branches][kTokMaxKV]
-  static constexpr int kQn = kScores + 2 * 2 * kTokMaxKV * 4;  // float [2 rows][128]
-  static constexpr int kScratch = kQn + 2 * 128 * 4;           // top-k scratch of warps 6 and 7
+  static constexpr int kScores = kC + kTokCStages * kCStage;  // uint32 keys [2 rows][2 branches][kTokMaxKV]
+  static constexpr int kQn = kScores + 2 * 2 * kTokMaxKV * 4;  // float [8 epilogue warps][64 tokens]
+  static constexpr int kScratch = kQn + 8 * 64 * 4;            // top-k scratch of warps 10 and 11
   static constexpr int kScratchWords = sel_topk_scratch_words(kTokMaxKV / 32);
   static constexpr int kBar = kScratch + 2 * kScratchWords * 4;
   static constexpr int kBarBytes = 256;
@@ -55,7 +57,7 @@ struct TokSmem {
 
 enum : int {
   kTokQFull = 0,
-  kTokQEmpty = 1,                   // MMA commit + 4 norm warps
+  kTokQEmpty = 1,                   // MMA commit + 8 epilogue warps
   kTokCFull = 2,                    // + stage
   kTokCEmpty = kTokCFull + kTokCStages,
   kTokDFull = kTokCEmpty + kTokCStages,  // + D buffer
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::kQ, sC = sbase + L::kC;
-  float* scores = reinterpret_cast<float*>(smem + L::kScores);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L::kScores);
   float* qn_s = reinterpret_cast<float*>(smem + L::kQn);
   const uint32_t bars = sbase + L::kBar;
   auto bar = [&](int k) -> uint32_t { return bars + 8u * k; };
@@ -104,21 +106,24 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
 
   if (tid == 0) {
     mbar_init(bar(kTokQFull), 1);
-    mbar_init(bar(kTokQEmpty), 1 + 4);
+    mbar_init(bar(kTokQEmpty), 1 + 8);
     for (int s = 0; s < kTokCStages; ++s) {
       mbar_init(bar(kTokCFull + s), 1);
       mbar_init(bar(kTokCEmpty + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kTokDFull + s), 1);
-      mbar_init(bar(kTokDEmpty + s), 4);
-      mbar_init(bar(kTokSFull + s), 4);
+      mbar_init(bar(kTokDEmpty + s), 8);
+      mbar_init(bar(kTokSFull + s), 8);
       mbar_init(bar(kTokSEmpty + s), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  // the key rows start at 0 (below every float's key); the top-k warps
+  // clear each row they consume
+  for (int o = tid; o < 2 * 2 * kTokMaxKV; o += kTokThreads) keys[o] = 0u;
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
     tmem_relinquish();
   }
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&ta.tmQ);
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
         if (s < gt) mbar_drain(bar(kTokCFull + s), ((gt - s + kTokCStages - 1) / kTokCStages - 1) & 1);
       if (nq > 0) mbar_drain(bar(kTokQFull), (nq - 1) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer (whole warp, one elected lane)
     constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 0, 0);
     const uint64_t cdesc0 = smem_desc(sC, 16, 1024, kLayoutSW128);
@@ -202,9 +207,10 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
       }
       if (ok) umma_commit_warp(bar(kTokQEmpty));
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ token norms and the per-block maxima
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int quarter = warp & 3, thalf = warp >> 2;  // TMEM lane quarter, half of the tokens
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t gt = 0;
     bool ok = true;
     for (int k = 0; k < nitems && ok; ++k) {
@@ -214,18 +220,21 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
       const int nq = min(BQ, a.Lq - i * BQ);  // valid tokens of this query block
       const int kvh = hq / G;
       const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
-      float* qn = qn_s + (k & 1) * 128;
+      // this warp's tokens: t0 .. t0 + BQ/2 - 1; their norms in its own array
+      // (no barrier between the epilogue warps)
+      const int t0 = thalf * (BQ / 2);
+      float* qn = qn_s + warp * 64 - t0;  // qn[t] for t in this warp's half
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokQFull), k & 1, abort_flag))) break;
-      if (tid < BQ) {
-        // token tid: 16-byte chunk c of its 128-byte row in each half sits at
-        // chunk position c ^ (tid % 8) (128-byte swizzle)
+      for (int t = t0 + lane; t < t0 + BQ / 2; t += 32) {
+        // token t: 16-byte chunk c of its 128-byte row in each half sits at
+        // chunk position c ^ (t % 8) (128-byte swizzle)
         float s2 = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kQ + h * BQ * 128 + tid * 128 +
-                                                            ((c ^ (tid & 7)) << 4));
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kQ + h * BQ * 128 + t * 128 +
+                                                            ((c ^ (t & 7)) << 4));
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -234,25 +243,24 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
             }
           }
         }
-        qn[tid] = sqrtf(s2);
+        qn[t] = sqrtf(s2);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kTokQEmpty));
-      named_bar_sync(1, 128);  // qn complete
       const int sb = k & 1;
-      float* sc_c = scores + sb * 2 * kTokMaxKV;
-      float* sc_r = sc_c + kTokMaxKV;
+      uint32_t* kc = keys + sb * 2 * kTokMaxKV;
+      uint32_t* kr = kc + kTokMaxKV;
       // the top-k of row k - 2 must be done with this score buffer
       if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(kTokSEmpty + sb), ((k >> 1) - 1) & 1, abort_flag))) break;
       for (int m = 0; m < T; ++m, ++gt) {
         const int db = gt & 1;
+        const int j = m * 128 + quarter * 32 + lane;
+        const float rho = j < n ? a.rad[kv_off + j] * a.beta[kv_off + j] : 0.f;  // in flight during the wait
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokDFull + db), (gt >> 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
-        const int j = m * 128 + warp * 32 + lane;
-        const float rho = j < n ? a.rad[kv_off + j] * a.beta[kv_off + j] : 0.f;
         float mc = -INFINITY, mr = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BQ / 32; ++c) {
+        for (int c = thalf * (BQ / 64); c < (thalf + 1) * (BQ / 64); ++c) {
           uint32_t v[32];
           tmem_ld32(lane_base + db * BQ + 32 * c, v);
           tmem_wait_ld();
@@ -268,9 +276,9 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kTokDEmpty + db));
-        if (j < n) {
-          sc_c[j] = mc;
-          sc_r[j] = mr;
+        if (j < n) {  // the other half of the tokens meets this one here
+          atomicMax(&kc[j], order_key(mc));
+          atomicMax(&kr[j], order_key(mr));
         }
       }
       if (!ok) break;
@@ -279,24 +287,38 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
     }
   } else {
     // ------------------------------------------------------------ top-k of alternate rows
-    const int tk = warp - 6;
+    const int tk = warp - 10;
     uint32_t* scratch = reinterpret_cast<uint32_t*>(smem + L::kScratch) + tk * L::kScratchWords;
     for (int k = tk; k < nitems; k += 2) {
       int b, hq, i;
       tok_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq, i);
       const int sb = k & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokSFull + sb), (k >> 1) & 1, abort_flag))) break;
-      const float* sc_c = scores + sb * 2 * kTokMaxKV;
-      const float* sc_r = sc_c + kTokMaxKV;
+      uint32_t* kc = keys + sb * 2 * kTokMaxKV;
+      uint32_t* kr = kc + kTokMaxKV;
       const int n = visible(i), gi = i + a.q_block_offset;
       const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
-      auto fc = [&](int j) { return sc_c[j]; };
-      auto fr = [&](int j) { return sc_r[j]; };
-      if (KPL > 2 && n <= 64) select_row<2, KPL>(a, fc, fr, row, lane, gi, n, scratch);
-      else if (KPL > 8 && n <= 256) select_row<8, KPL>(a, fc, fr, row, lane, gi, n, scratch);
-      else if (KPL > 16 && n <= 512) select_row<16, KPL>(a, fc, fr, row, lane, gi, n, scratch);
-      else if (KPL > 32 && n <= 1024) select_row<32, KPL>(a, fc, fr, row, lane, gi, n, scratch);
-      else select_row<KPL, KPL>(a, fc, fr, row, lane, gi, n, scratch);
+      if (a.threshold_mode == 1) {
+        auto fc = [&](int j) { return key_to_float(kc[j]); };
+        auto fr = [&](int j) { return key_to_float(kr[j]); };
+        select_row<2, KPL>(a, fc, fr, row, lane, gi, n, scratch);  // no key slots used in this mode
+      } else {
+        auto sc = [&](int s) -> uint32_t {
+          const int j = 32 * s + lane;
+          return j < n ? kc[j] : 0u;
+        };
+        auto sr = [&](int s) -> uint32_t {
+          const int j = 32 * s + lane;
+          return j < n ? kr[j] : 0u;
+        };
+        if (KPL > 2 && n <= 64) select_row_keys<2, KPL>(a, sc, sr, row, lane, gi, n, scratch);
+        else if (KPL > 8 && n <= 256) select_row_keys<8, KPL>(a, sc, sr, row, lane, gi, n, scratch);
+        else if (KPL > 16 && n <= 512) select_row_keys<16, KPL>(a, sc, sr, row, lane, gi, n, scratch);
+        else if (KPL > 32 && n <= 1024) select_row_keys<32, KPL>(a, sc, sr, row, lane, gi, n, scratch);
+        else select_row_keys<KPL, KPL>(a, sc, sr, row, lane, gi, n, scratch);
+      }
+      __syncwarp();
+      for (int j = lane; j < n; j += 32) kc[j] = kr[j] = 0u;  // ready for the buffer's next row
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kTokSEmpty + sb));
     }
@@ -304,7 +326,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
