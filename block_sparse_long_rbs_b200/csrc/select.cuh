@@ -100,6 +100,14 @@ __device__ __forceinline__ int keep_count(float rho, int n) {
   return k < 1 ? 1 : (k > n ? n : k);
 }
 
+// Warp sums of two small counts (each total below 2^16) in one reduction:
+// the first in the low 16 bits, the second in the high 16 bits.
+__device__ __forceinline__ void sum2(int x, int y, int& sx, int& sy) {
+  const uint32_t s = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(x) | (static_cast<uint32_t>(y) << 16));
+  sx = static_cast<int>(s & 0xFFFFu);
+  sy = static_cast<int>(s >> 16);
+}
+
 // Exact top-k of the warp's keys for two branches at once (key 0 = not a
 // candidate; k <= #candidates).  The k-th largest key T is built bit by bit
 // from the top (the largest T with at least k keys >= T); keys above T are
@@ -120,8 +128,8 @@ __device__ __forceinline__ void warp_topk2(const uint32_t (&kc)[KPL], const uint
       nc2[t & 1] += kc[t] >= cc ? 1 : 0;
       nr2[t & 1] += kr[t] >= cr ? 1 : 0;
     }
-    const int nc = __reduce_add_sync(0xffffffffu, nc2[0] + nc2[1]);
-    const int nr = __reduce_add_sync(0xffffffffu, nr2[0] + nr2[1]);
+    int nc, nr;
+    sum2(nc2[0] + nc2[1], nr2[0] + nr2[1], nc, nr);
     if (nc >= k_c) Tc = cc;
     if (nr >= k_r) Tr = cr;
   }
@@ -131,8 +139,9 @@ __device__ __forceinline__ void warp_topk2(const uint32_t (&kc)[KPL], const uint
     gc += kc[t] > Tc ? 1 : 0;
     gr += kr[t] > Tr ? 1 : 0;
   }
-  const int need_c = k_c - __reduce_add_sync(0xffffffffu, gc);  // ties at T to keep, lowest index first
-  const int need_r = k_r - __reduce_add_sync(0xffffffffu, gr);
+  int above_c, above_r;
+  sum2(gc, gr, above_c, above_r);
+  const int need_c = k_c - above_c, need_r = k_r - above_r;  // ties at T to keep, lowest index first
   const uint32_t lt_mask = (1u << lane) - 1u;
   int base_c = 0, base_r = 0;
 #pragma unroll
@@ -213,8 +222,9 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
 #pragma unroll 1
   for (int bit = max(topc, topr); bit >= 8; --bit) {
     const uint32_t xc = Lc | (1u << bit), xr = Lr | (1u << bit);
-    const int nc = __reduce_add_sync(0xffffffffu, (c0 >= xc) + (c1 >= xc) + (c2 >= xc) + (c3 >= xc));
-    const int nr = __reduce_add_sync(0xffffffffu, (r0 >= xr) + (r1 >= xr) + (r2 >= xr) + (r3 >= xr));
+    int nc, nr;
+    sum2((c0 >= xc) + (c1 >= xc) + (c2 >= xc) + (c3 >= xc), (r0 >= xr) + (r1 >= xr) + (r2 >= xr) + (r3 >= xr), nc,
+         nr);
     if (bit <= topc && nc >= k_c) Lc = xc;
     if (bit <= topr && nr >= k_r) Lr = xr;
   }
@@ -261,13 +271,16 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
 #pragma unroll 1
   for (int bit = max(tpc, tpr); bit >= 0; --bit) {
     const uint32_t xc = Tc | (1u << bit), xr = Tr | (1u << bit);
-    const int nc = __reduce_add_sync(0xffffffffu, (a[0] >= xc) + (a[1] >= xc) + (a[2] >= xc) + (a[3] >= xc));
-    const int nr = __reduce_add_sync(0xffffffffu, (bk[0] >= xr) + (bk[1] >= xr) + (bk[2] >= xr) + (bk[3] >= xr));
+    int nc, nr;
+    sum2((a[0] >= xc) + (a[1] >= xc) + (a[2] >= xc) + (a[3] >= xc),
+         (bk[0] >= xr) + (bk[1] >= xr) + (bk[2] >= xr) + (bk[3] >= xr), nc, nr);
     if (bit <= tpc && nc >= k_c) Tc = xc;
     if (bit <= tpr && nr >= k_r) Tr = xr;
   }
-  const int need_c = k_c - __reduce_add_sync(0xffffffffu, (a[0] > Tc) + (a[1] > Tc) + (a[2] > Tc) + (a[3] > Tc));
-  const int need_r = k_r - __reduce_add_sync(0xffffffffu, (bk[0] > Tr) + (bk[1] > Tr) + (bk[2] > Tr) + (bk[3] > Tr));
+  int above_c, above_r;
+  sum2((a[0] > Tc) + (a[1] > Tc) + (a[2] > Tc) + (a[3] > Tc), (bk[0] > Tr) + (bk[1] > Tr) + (bk[2] > Tr) + (bk[3] > Tr),
+       above_c, above_r);
+  const int need_c = k_c - above_c, need_r = k_r - above_r;
   for (int w = lane; w < nwords; w += 32) words_c[w] = words_r[w] = 0u;
   __syncwarp();
   // positions ascend with the block index, so a tie's rank is the number of
