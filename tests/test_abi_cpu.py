@@ -224,3 +224,41 @@ def test_kv_group_lists_validation(L):
     odd = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, 1 * 3 * 8)
     assert f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(odd), 64, 64, 0, 0.0, 1,
              ctypes.byref(o), None, s) == 1
+
+
+def test_rescue_weighted_validation(L):
+    """bsa_prefill_rescue_weighted: the weight must be finite and >= 0, and
+    any weight but 1 needs the lists' branch flags."""
+    s = ctypes.c_void_p(0)
+    q = _fake(Lq=256, H=4)
+    k = _fake(Lq=256, H=2)
+    o = _fake(Lq=256, H=4)
+    flagged = _abi.BlockListsC(0x40000, 0x50000, 0x70000, 100, 1 * 4 * 2)
+    bare = _abi.BlockListsC(0x40000, 0x50000, None, 100, 1 * 4 * 2)
+    f = L.bsa_prefill_rescue_weighted
+    call = lambda lists, w: f(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(lists), 128, 128, 0,
+                              0.0, 1, w, ctypes.byref(o), None, s)
+    for bad in (-1.0, float("nan"), float("inf")):
+        assert call(flagged, bad) == 1, bad
+    assert call(bare, 0.5) == 1  # no flags to tell the rescue blocks apart
+    assert call(bare, 1.0) == 4  # weight 1 is bsa_prefill: past validation, no GPU here
+    assert call(flagged, 0.0) == 4
+
+
+def test_query_pool_validation(L):
+    """query_pool TOKEN_MAX: a field value outside {0, 1} is rejected, and more
+    key blocks than the per-token kernel holds are unsupported."""
+    s = None
+    q = _fake(Lq=512)
+    rows = 1 * 2 * 8
+    ok = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, rows)
+    sel = lambda p, nkb: L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, nkb, ctypes.byref(p), 0x60000, 1 << 26,
+                                      ctypes.byref(ok), None, s)
+    assert sel(SelectParams(block_q=64, block_k=64, query_pool=2).c(), 8) == 1
+    assert sel(SelectParams(block_q=64, block_k=64, query_pool=1).c(), 8) == 4  # past validation
+    assert sel(SelectParams(block_q=64, block_k=64, query_pool=1).c(), 4096) == 2
+    # the per-token path's workspace includes the centroid parts
+    p0 = SelectParams(block_q=64, block_k=64).c()
+    p1 = SelectParams(block_q=64, block_k=64, query_pool=1).c()
+    assert L.rbs_select_workspace_bytes(1, 2, 8, 1, 8, ctypes.byref(p1)) > 0
+    assert L.rbs_select_workspace_bytes(1, 2, 8, 1, 8, ctypes.byref(p0)) > 0
