@@ -143,3 +143,38 @@ def test_select_fused_kernel_with_smaller_workspace(cuda_ok, case):
     rep_small = compare_selection(lists, ora, Hq, nqb, nkb)
     rep_full = compare_selection(ref, ora, Hq, nqb, nkb)
     print("fused", rep_small, "tensor-core", rep_full)
+
+
+@pytest.mark.parametrize("layout", ["fused_qkv_view", "head_major"])
+@pytest.mark.parametrize("small_ws", [False, True])
+def test_select_strided_and_head_major_q(cuda_ok, layout, small_ws):
+    # Q as a slice of a fused [B, L, 3 * Hq, 128] buffer (token stride > Hq * 128)
+    # or as a head-major [B, Hq, L, 128] buffer seen as [B, L, Hq, 128] (token
+    # stride 128): the lists must equal those of the contiguous Q, on the
+    # tensor-core path and on the fused kernel (a workspace without room for
+    # the score matrix)
+    inp = make_mixture(L=8192, Hq=8, Hkv=2, block=128, seed=206)
+    Qc = dev(inp["Q"])
+    if layout == "fused_qkv_view":
+        big = torch.zeros(1, 8192, 24, 128, dtype=torch.bfloat16, device="cuda")
+        big[:, :, 8:16] = Qc
+        Qv = big[:, :, 8:16]
+    else:
+        Qv = Qc.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+        assert Qv.stride(1) == 128
+    assert torch.equal(Qv, Qc) and not Qv.is_contiguous()
+    p = rbs.SelectParams(block_q=128, block_k=128, rho_centroid=0.1, rho_rescue=0.1)
+    Cg, Rg = rbs.rbs_block_stats(dev(inp["K"]), 128)
+    ws = None
+    if small_ws:
+        full = rbs.rbs_select_workspace_bytes(1, 8, 64, 2, 64, p)
+        buf = torch.empty(full + 255, dtype=torch.uint8, device="cuda")
+        off = (-buf.data_ptr()) % 256
+        ws = buf[off:off + full - 1]
+    a = rbs.rbs_select(Qc, Cg, Rg, p, workspace=ws)
+    b = rbs.rbs_select(Qv, Cg, Rg, p, workspace=ws)
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    assert torch.equal(a.row_ptr, b.row_ptr)
+    n = a.nnz()
+    assert torch.equal(a.col_idx[:n], b.col_idx[:n]) and torch.equal(a.flags[:n], b.flags[:n])
