@@ -216,7 +216,8 @@ RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, f
  *   workspace    device scratch, 256-byte aligned, contents need no
  *                initialisation.  rbs_select_workspace_bytes(...) bytes
  *                enable the tensor-core scoring of the mean query (the score
- *                matrix lives there); a smaller workspace runs the fused
+ *                matrix lives there) when num_kv_blocks <= 2048; a smaller
+ *                workspace, or more key blocks, runs the fused
  *                CUDA-core scoring kernel, down to the masks and counts it
  *                needs (RBS_ERR_CAPACITY below that)
  *   out          lists with num_rows = B * Hq * nQB (B * Hkv * nQB when
@@ -242,11 +243,15 @@ RBS_API rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, 
  * fixed buffer of RBS_NOALLOC_SCRATCH_BYTES compiled into the library, which
  * every GPU that loads the library holds until the process exits.
  * The caller still passes all inputs and outputs (same meaning as
- * rbs_select).  A selection whose scratch would exceed the buffer
- * (rbs_select_workspace_bytes > RBS_NOALLOC_SCRATCH_BYTES; the 131072-token,
- * 32-head, 128-block case needs about 24 MiB) returns RBS_ERR_CAPACITY and
- * launches nothing.  The first call on each device looks up the buffer's
- * device address (a CUDA runtime query, no allocation); make that first call
+ * rbs_select).  The buffer is handed to rbs_select as its workspace, so
+ * the same rule picks the scoring path: when the full workspace
+ * (rbs_select_workspace_bytes) fits in RBS_NOALLOC_SCRATCH_BYTES (and
+ * num_kv_blocks <= 2048) the tensor-core scoring runs, otherwise the fused
+ * CUDA-core scoring kernel,
+ * which needs only the masks, counts and beta.  Only a selection whose masks,
+ * counts and beta alone (plus the split centroids, for per-token-max query
+ * scoring) exceed the buffer returns RBS_ERR_CAPACITY and launches nothing.
+ * The first call on each device looks up the buffer's device address (a CUDA runtime query, no allocation); make that first call
  * before any stream capture.  All calls on a device share the one buffer:
  * every scratch region is fully written before it is read, so nothing needs
  * clearing between calls, but two calls that may overlap on the GPU (other
