@@ -226,6 +226,7 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
   l.c_lo = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
   if (token_max) {
     l.base = off;  // the per-token kernel needs the centroid parts
+    l.scores = off; off += align256(rows * 2 * nwords * 32 * 4);  // both branches' keys, for the separate top-k
   } else {
     l.q_hi = off; off += align256(rows * RBS_HEAD_DIM * 2);
     l.q_lo = off; off += align256(rows * RBS_HEAD_DIM * 2);
@@ -236,13 +237,26 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
   return l;
 }
 
+// Both branches' top-k of every row from the stored scores or keys, eight
+// rows per CTA, with as many key slots per lane as the longest row needs.
+void launch_topk_rows(const TopkArgs& t, int64_t nkb, rbs_stream_t stream) {
+  const size_t tsm = topk_smem_bytes(t.nkbp, t.s.nwords);
+  const unsigned tgrid = static_cast<unsigned>((t.rows + 7) / 8);
+  if (nkb <= 64) topk_rows_kernel<2><<<tgrid, 256, tsm, stream>>>(t);
+  else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, 256, tsm, stream>>>(t);
+  else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, 256, tsm, stream>>>(t);
+  else topk_rows_kernel<64><<<tgrid, 256, tsm, stream>>>(t);
+}
+
 // Per-token-max selection scores (query_pool TOKEN_MAX): split the centroids
 // into bf16 hi / lo parts in the workspace, then one persistent CTA per SM
-// scores and thresholds rows (select_tokmax_kernel), writing the same mask
-// words and counts as the mean-query kernel.
+// scores rows (select_tokmax_kernel).  With room in the workspace for both
+// branches' key matrix the kernel stores the keys and topk_rows_kernel
+// selects from them; otherwise two warps of each CTA select in place.  Both
+// write the same mask words and counts as the mean-query kernels.
 rbs_status launch_token_max(const rbs_bf16_tensor* Q, const float* centroids, int64_t B, int32_t Hkv, int64_t nkb,
                             const rbs_select_params* p, const SelectArgs& sa, uint8_t* c_hi, uint8_t* c_lo,
-                            DeviceInfo* di, rbs_stream_t stream) {
+                            uint32_t* keys, DeviceInfo* di, rbs_stream_t stream) {
   rbs_status st;
   const int64_t n = B * Hkv * nkb * RBS_HEAD_DIM;
   auto* hi = reinterpret_cast<__nv_bfloat16*>(c_hi);
@@ -270,6 +284,8 @@ rbs_status launch_token_max(const rbs_bf16_tensor* Q, const float* centroids, in
   }
   ta.s = sa;
   ta.rows = static_cast<int>(B * sa.Hq * sa.nqb);
+  ta.keys_out = keys;
+  ta.nkbp = static_cast<int>((nkb + 31) & ~31ll);
   const int grid = static_cast<int>(std::min<int64_t>(ta.rows, di->sms));
 #define RBS_TOK_LAUNCH(KPL)                                                                                  \
   do {                                                                                                       \
@@ -282,7 +298,17 @@ rbs_status launch_token_max(const rbs_bf16_tensor* Q, const float* centroids, in
   else if (nkb <= 1024) RBS_TOK_LAUNCH(32);
   else RBS_TOK_LAUNCH(64);
 #undef RBS_TOK_LAUNCH
-  return check_launch("select_tokmax_kernel");
+  if ((st = check_launch("select_tokmax_kernel")) != RBS_OK || keys == nullptr) return st;
+  // the stored keys -> masks and counts, one warp per row
+  TopkArgs tk;
+  tk.s = sa;
+  tk.scores = nullptr;
+  tk.qnorm = nullptr;
+  tk.keys = keys;
+  tk.nkbp = ta.nkbp;
+  tk.rows = ta.rows;
+  launch_topk_rows(tk, nkb, stream);
+  return check_launch("topk_rows_kernel");
 }
 
 // 4-D map over a contiguous [B, H, n, 128] bf16 array with a box of 64 dims x
@@ -394,14 +420,10 @@ rbs_status launch_mma_select(const rbs_bf16_tensor* Q, const float* centroids, i
   ta.s = sa;
   ta.scores = scores;
   ta.qnorm = qnorm;
+  ta.keys = nullptr;
   ta.nkbp = npad;
   ta.rows = static_cast<int>(rows);
-  const size_t tsm = topk_smem_bytes(npad, sa.nwords);
-  const unsigned tgrid = static_cast<unsigned>((rows + 7) / 8);
-  if (nkb <= 64) topk_rows_kernel<2><<<tgrid, 256, tsm, stream>>>(ta);
-  else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, 256, tsm, stream>>>(ta);
-  else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, 256, tsm, stream>>>(ta);
-  else topk_rows_kernel<64><<<tgrid, 256, tsm, stream>>>(ta);
+  launch_topk_rows(ta, nkb, stream);
   return check_launch("topk_rows_kernel");
 }
 
@@ -645,7 +667,9 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   sa.mask_r = reinterpret_cast<uint32_t*>(ws + lay.mask_r);
   sa.counts = reinterpret_cast<int*>(ws + lay.counts);
   if (p->query_pool == 1) {
-    if ((st = launch_token_max(Q, centroids, B, kv_heads, nkb, p, sa, ws + lay.c_hi, ws + lay.c_lo, di, stream)) != RBS_OK)
+    uint32_t* keys = workspace_bytes >= lay.total ? reinterpret_cast<uint32_t*>(ws + lay.scores) : nullptr;
+    if ((st = launch_token_max(Q, centroids, B, kv_heads, nkb, p, sa, ws + lay.c_hi, ws + lay.c_lo, keys, di,
+                               stream)) != RBS_OK)
       return st;
   } else if (mma_path) {
     if ((st = launch_mma_select(Q, centroids, B, kv_heads, nkb, p, sa, R, ws, lay, di, stream)) != RBS_OK) return st;

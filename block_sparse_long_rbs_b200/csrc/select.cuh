@@ -196,18 +196,22 @@ __device__ __forceinline__ void top4_insert(uint32_t& t0, uint32_t& t1, uint32_t
 // false, having written nothing the caller uses, when k > 64 or a branch has
 // more candidates (many near-equal keys); the caller then runs the full
 // search.  Both branches advance together so their reduction chains overlap.
-// Warp-uniform.
+// Slots from ceil(n / 32) on hold only absent keys (blocks >= n): they can
+// neither enter a lane's top four nor become candidates, so both passes stop
+// before them.  Warp-uniform.
 template <int KP, typename KeyC, typename KeyR>
-__device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_c, int k_r, int lane, int nwords,
-                                                  uint32_t* scratch, uint32_t* words_c, uint32_t* words_r) {
+__device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_c, int k_r, int n, int lane,
+                                                  int nwords, uint32_t* scratch, uint32_t* words_c,
+                                                  uint32_t* words_r) {
   if (k_c > 64 || k_r > 64) return false;
+  const int nt = min(KP, (n + 31) >> 5);  // slots holding a visible block
   uint32_t* ck_c = scratch;  // candidate keys and blocks of each branch
   int* ci_c = reinterpret_cast<int*>(scratch + kTopkCap);
   uint32_t* ck_r = scratch + 2 * kTopkCap;
   int* ci_r = reinterpret_cast<int*>(scratch + 3 * kTopkCap);
   uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0, r0 = 0, r1 = 0, r2 = 0, r3 = 0;
 #pragma unroll 4
-  for (int t = 0; t < KP; ++t) {
+  for (int t = 0; t < nt; ++t) {
     top4_insert(c0, c1, c2, c3, key_c(t));
     top4_insert(r0, r1, r2, r3, key_r(t));
   }
@@ -233,7 +237,7 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
   const uint32_t lt_mask = (1u << lane) - 1u;
   int base_c = 0, base_r = 0;
 #pragma unroll 4
-  for (int t = 0; t < KP; ++t) {
+  for (int t = 0; t < nt; ++t) {
     const uint32_t uc = key_c(t), ur = key_r(t);
     const bool cand_c = uc >= Lc, cand_r = ur >= Lr;
     const uint32_t bc = __ballot_sync(0xffffffffu, cand_c), br = __ballot_sync(0xffffffffu, cand_r);
@@ -329,7 +333,7 @@ __device__ __forceinline__ void select_row_keys(const SelectArgs& a, KC key_c, K
   uint32_t* words_c = scratch + 4 * kTopkCap;
   uint32_t* words_r = words_c + a.nwords;
   const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
-  const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, scratch, words_c, words_r);
+  const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, n, lane, a.nwords, scratch, words_c, words_r);
   if (!done) {
     uint32_t kc[KP], kr[KP];
 #pragma unroll

@@ -17,7 +17,9 @@
 //                       the scores to the workspace.
 //   topk_rows_kernel    one warp per row: both branches' exact top-k
 //                       (select_row) from the stored scores, the rescue score
-//                       s_r = s_c + |qbar| r_j beta_j formed on the fly.
+//                       s_r = s_c + |qbar| r_j beta_j formed on the fly; or,
+//                       for per-token-max scoring, from both branches' keys
+//                       as select_tokmax_kernel stored them.
 //
 // ([RBS-en] "The Fix: A Radius-Adaptive Rescue Branch"; [RBS-id]
 // "Dual-Branch Selection".)  The mask words and counts they leave are the
@@ -386,6 +388,9 @@ struct TopkArgs {
   SelectArgs s;
   const float* scores;  // [rows, nkbp]
   const float* qnorm;   // [rows]
+  // instead of scores: [rows][2 branches][nkbp] order-preserving keys of
+  // both branches' scores (per-token-max scoring), or null
+  const uint32_t* keys;
   int nkbp, rows;
 };
 
@@ -415,29 +420,42 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(TopkArgs t) {
   float* ssc = topk_smem + warp * 2 * t.nkbp;
   float* srb = ssc + t.nkbp;
   uint32_t* scratch = reinterpret_cast<uint32_t*>(topk_smem + 8 * 2 * t.nkbp) + warp * sel_topk_scratch_words(a.nwords);
-  // stage the row: scores with 16-byte loads (the row starts 128-byte
-  // aligned and is padded to nkbp), r_j beta_j with 4-byte loads
-  const float4* src = reinterpret_cast<const float4*>(t.scores + row * t.nkbp);
-  for (int q = lane; q < (n + 3) / 4; q += 32) reinterpret_cast<float4*>(ssc)[q] = src[q];
-  for (int jj = lane; jj < n; jj += 32) srb[jj] = a.rad[kv_off + jj] * a.beta[kv_off + jj];
+  // both branches' order-preserving keys of blocks 0 .. n-1, in place
+  uint32_t* kcs = reinterpret_cast<uint32_t*>(ssc);
+  uint32_t* krs = reinterpret_cast<uint32_t*>(srb);
+  if (t.keys != nullptr) {
+    // the keys as stored, 16 bytes at a time (each row starts 128-byte
+    // aligned; 4 ceil(n / 4) <= nkbp)
+    const uint4* srcc = reinterpret_cast<const uint4*>(t.keys + row * 2 * t.nkbp);
+    const uint4* srcr = reinterpret_cast<const uint4*>(t.keys + row * 2 * t.nkbp + t.nkbp);
+    for (int q = lane; q < (n + 3) / 4; q += 32) {
+      reinterpret_cast<uint4*>(kcs)[q] = srcc[q];
+      reinterpret_cast<uint4*>(krs)[q] = srcr[q];
+    }
+  } else {
+    // stage the row: scores with 16-byte loads (the row starts 128-byte
+    // aligned and is padded to nkbp), r_j beta_j with 4-byte loads; then
+    // the keys of s_c and of s_r = s_c + |qbar| r_j beta_j over them
+    const float4* src = reinterpret_cast<const float4*>(t.scores + row * t.nkbp);
+    for (int q = lane; q < (n + 3) / 4; q += 32) reinterpret_cast<float4*>(ssc)[q] = src[q];
+    for (int jj = lane; jj < n; jj += 32) srb[jj] = a.rad[kv_off + jj] * a.beta[kv_off + jj];
+    __syncwarp();
+    const float qn = t.qnorm[row];
+    for (int jj = lane; jj < n; jj += 32) {
+      const float sv = ssc[jj];
+      const uint32_t kr = order_key(fmaf(qn, srb[jj], sv));
+      kcs[jj] = order_key(sv);
+      krs[jj] = kr;
+    }
+  }
   __syncwarp();
-  const float qn = t.qnorm[row];
   if (a.threshold_mode == 1) {
-    auto fc = [&](int j) { return ssc[j]; };
-    auto fr = [&](int j) { return fmaf(qn, srb[j], ssc[j]); };
+    // the scores back from their keys (an exact inverse)
+    auto fc = [&](int j) { return key_to_float(kcs[j]); };
+    auto fr = [&](int j) { return key_to_float(krs[j]); };
     select_row<2, KPL>(a, fc, fr, row, lane, gi, n, scratch);  // no key slots used in this mode
     return;
   }
-  // both branches' order-preserving keys, once, in place of the staged values
-  uint32_t* kcs = reinterpret_cast<uint32_t*>(ssc);
-  uint32_t* krs = reinterpret_cast<uint32_t*>(srb);
-  for (int jj = lane; jj < n; jj += 32) {
-    const float sv = ssc[jj];
-    const uint32_t kr = order_key(fmaf(qn, srb[jj], sv));
-    kcs[jj] = order_key(sv);
-    krs[jj] = kr;
-  }
-  __syncwarp();
   auto kc = [&](int s) -> uint32_t {
     const int j = 32 * s + lane;
     return j < n ? kcs[j] : 0u;

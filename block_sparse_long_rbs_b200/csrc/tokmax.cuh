@@ -24,7 +24,10 @@
 //   warp 8     TMA producer: the query tile (once per row) and the hi / lo
 //              centroid tiles (2-stage ring), no multicast
 //   warp 9     TMEM allocation and the MMA issue (one elected lane)
-//   warps 10-11 both branches' top-k of alternate rows from those keys
+//   warps 10-11 alternate rows: with a key matrix in the workspace they copy
+//              the row's keys there (topk_rows_kernel selects from them
+//              afterwards, eight rows per CTA); without one they run both
+//              branches' top-k of the row themselves
 #pragma once
 
 #include "common.cuh"
@@ -71,6 +74,10 @@ struct TokArgs {
   CUtensorMap tmQ, tmChi, tmClo;  // Q [B, Lq, Hq, 128]; centroid parts [B, Hkv, nkb, 128] (token index = block)
   SelectArgs s;
   int rows;  // work items: B * Hq * nqb
+  // [rows][2 branches][nkbp] order-preserving keys of the blocks' maxima
+  // (row as for the masks), or null to select inside this kernel
+  uint32_t* keys_out;
+  int nkbp;  // multiple of 32, >= nkb
 };
 
 // Row w -> (batch, q head, query block): the last query blocks first.
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
       if (lane == 0) mbar_arrive(bar(kTokSFull + sb));
     }
   } else {
-    // ------------------------------------------------------------ top-k of alternate rows
+    // ------------------------------------------------------------ alternate rows: key copy-out or top-k
     const int tk = warp - 10;
     uint32_t* scratch = reinterpret_cast<uint32_t*>(smem + L::kScratch) + tk * L::kScratchWords;
     for (int k = tk; k < nitems; k += 2) {
@@ -298,7 +305,16 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
       uint32_t* kr = kc + kTokMaxKV;
       const int n = visible(i), gi = i + a.q_block_offset;
       const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
-      if (a.threshold_mode == 1) {
+      if (ta.keys_out != nullptr) {
+        // both key rows, 16 bytes at a time: slots n .. 4 ceil(n / 4) - 1
+        // hold 0 (never raised), and 4 ceil(n / 4) <= nkbp
+        uint4* dc = reinterpret_cast<uint4*>(ta.keys_out + row * 2 * ta.nkbp);
+        uint4* dr = reinterpret_cast<uint4*>(ta.keys_out + row * 2 * ta.nkbp + ta.nkbp);
+        for (int q = lane; q < (n + 3) >> 2; q += 32) {
+          dc[q] = reinterpret_cast<const uint4*>(kc)[q];
+          dr[q] = reinterpret_cast<const uint4*>(kr)[q];
+        }
+      } else if (a.threshold_mode == 1) {
         auto fc = [&](int j) { return key_to_float(kc[j]); };
         auto fr = [&](int j) { return key_to_float(kr[j]); };
         select_row<2, KPL>(a, fc, fr, row, lane, gi, n, scratch);  // no key slots used in this mode

@@ -129,7 +129,10 @@ typedef struct {
  *                      + ||q_t|| r_j beta_j) ([RBS-en] "The Fix" scores a query
  *                      q; here q runs over the block's tokens).  TOKEN_MAX
  *                      needs num_kv_blocks <= 2048, Q with stride_h <=
- *                      stride_s, and a larger workspace (0)
+ *                      stride_s, and a larger workspace: the split
+ *                      centroids at least; the full size adds both
+ *                      branches' per-block maxima, so a separate top-k
+ *                      kernel can select from them (0)
  * Scores are raw dot products (no 1/sqrt(d)); ties between equal scores go
  * to the lower block index.  Forced blocks do not count toward a branch's k.
  */
@@ -219,7 +222,11 @@ RBS_API rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, f
  *                matrix lives there) when num_kv_blocks <= 2048; a smaller
  *                workspace, or more key blocks, runs the fused
  *                CUDA-core scoring kernel, down to the masks and counts it
- *                needs (RBS_ERR_CAPACITY below that)
+ *                needs (RBS_ERR_CAPACITY below that).  For TOKEN_MAX the
+ *                full size holds both branches' per-block maxima for the
+ *                separate top-k kernel; down to the split centroids the
+ *                scoring kernel selects in place.  Both choices give the
+ *                same lists.
  *   out          lists with num_rows = B * Hq * nQB (B * Hkv * nQB when
  *                list_mode is KV_GROUP) and capacity >=
  *                rbs_select_capacity(...), which bounds both modes;

@@ -97,3 +97,41 @@ def test_tokmax_128k_sampled_rows(cuda_ok):
                 assert abs(s[j] - tau) <= TOL_NEAR_TAU * max(1.0, abs(tau)), (hq, i, bi, j)
                 excused += 1
     print("tokmax 128k sampled rows, excused", excused, "nnz", int(rp[-1]))
+
+
+@pytest.mark.parametrize("case", ["mixture", "max_relative", "32k"])
+def test_tokmax_both_topk_paths(cuda_ok, case):
+    # with the full workspace the token-max kernel stores both branches' keys
+    # and the separate top-k kernel selects from them; one byte short, two
+    # warps of the token-max kernel select in place.  Both read the same keys
+    # with the same selection code, so their lists must be identical, and
+    # both must match the oracle.
+    kw = {}
+    if case == "mixture":
+        inp, block, rho = make_mixture(L=8192, Hq=8, Hkv=2, block=128, seed=704, batch=2), 128, 0.1
+    elif case == "max_relative":
+        inp, block, rho = make_mixture(L=8192, Hq=4, Hkv=1, block=128, seed=705), 128, 0.1
+        kw = dict(threshold_mode=1, delta_centroid=4.0, delta_rescue=4.0)
+    else:
+        inp, block, rho = make_inputs(WORKLOADS["gqa_rbs_32k"]), 128, 0.05
+    Q, K = inp["Q"], inp["K"]
+    B, L, Hq, _ = Q.shape
+    Hkv, nqb, nkb = K.shape[2], L // block, K.shape[1] // block
+    p = rbs.SelectParams(block_q=block, block_k=block, rho_centroid=rho, rho_rescue=rho, query_pool=1, **kw)
+    Cg, Rg = rbs.rbs_block_stats(dev(K), block)
+    full = rbs.rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, p)
+    ws = torch.empty(full + 255, dtype=torch.uint8, device="cuda")
+    off = (-ws.data_ptr()) % 256
+    lists_sep = rbs.rbs_select(dev(Q), Cg, Rg, p, workspace=ws[off:off + full])
+    lists_in = rbs.rbs_select(dev(Q), Cg, Rg, p, workspace=ws[off:off + full - 1])
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    for a, b in zip(lists_np(lists_sep), lists_np(lists_in)):
+        np.testing.assert_array_equal(a, b)
+    Co, Ro = O.block_stats(K, block)
+    f32 = lambda v: float(np.float32(v)) if isinstance(v, float) else v
+    po = O.SelectParams(block_q=block, block_k=block, rho_centroid=f32(rho), rho_rescue=f32(rho), query_pool=1,
+                        **{k: f32(v) for k, v in kw.items()})
+    ora = O.select_blocks(Q, Co, Ro, po, keep_scores=True)
+    rep = compare_selection(lists_sep, ora, Hq, nqb, nkb, exact_k=kw.get("threshold_mode", 0) == 0)
+    print("tokmax both top-k paths", case, rep)
