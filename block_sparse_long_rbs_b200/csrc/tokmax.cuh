@@ -271,12 +271,27 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
           uint32_t v[32];
           tmem_ld32(lane_base + db * BQ + 32 * c, v);
           tmem_wait_ld();
+          if (32 * c + 32 <= nq) {
+            // all 32 tokens valid (every query block but a short last one):
+            // two tokens per 3-input max, four norms per shared load
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (32 * c + e < nq) {
-              const float d = __uint_as_float(v[e]);
-              mc = fmaxf(mc, d);
-              mr = fmaxf(mr, fmaf(qn[32 * c + e], rho, d));
+            for (int e = 0; e < 32; e += 4) {
+              const float4 q4 = *reinterpret_cast<const float4*>(qn + 32 * c + e);
+              const float d0 = __uint_as_float(v[e]), d1 = __uint_as_float(v[e + 1]);
+              const float d2 = __uint_as_float(v[e + 2]), d3 = __uint_as_float(v[e + 3]);
+              mc = fmax3(mc, d0, d1);
+              mc = fmax3(mc, d2, d3);
+              mr = fmax3(mr, fmaf(q4.x, rho, d0), fmaf(q4.y, rho, d1));
+              mr = fmax3(mr, fmaf(q4.z, rho, d2), fmaf(q4.w, rho, d3));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (32 * c + e < nq) {
+                const float d = __uint_as_float(v[e]);
+                mc = fmaxf(mc, d);
+                mr = fmaxf(mr, fmaf(qn[32 * c + e], rho, d));
+              }
             }
           }
         }
