@@ -17,10 +17,12 @@
 //
 // Roles (384 threads, one CTA per SM, persistent over rows (batch, q head,
 // query block), longest rows first):
-//   warps 0-7  token norms |q_t| from the query tile in shared memory, then
-//              per key tile the two maxima over half the tokens (two warps
-//              per TMEM lane quarter); the halves meet through atomicMax on
-//              order-preserving keys in a double-buffered shared row
+//   warps 0-7  token norms |q_t| from the query tile in shared memory (the
+//              four warps of a token half a quarter each, shared through a
+//              double-buffered array), then per key tile the two maxima over
+//              half the tokens (two warps per TMEM lane quarter); the halves
+//              meet through atomicMax on order-preserving keys in a
+//              double-buffered shared row
 //   warp 8     TMA producer: the query tile (once per row) and the hi / lo
 //              centroid tiles (2-stage ring), no multicast
 //   warp 9     TMEM allocation and the MMA issue (one elected lane)
@@ -48,7 +50,7 @@ struct TokSmem {
   static constexpr int kQ = 0;
   static constexpr int kC = kQ + kQBytes;        // 1024-aligned: kQBytes is 16 or 32 KB
   static constexpr int kScores = kC + kTokCStages * kCStage;  // uint32 keys [2 rows][2 branches][kTokMaxKV]
-  static constexpr int kQn = kScores + 2 * 2 * kTokMaxKV * 4;  // float [8 epilogue warps][64 tokens]
+  static constexpr int kQn = kScores + 2 * 2 * kTokMaxKV * 4;  // token norms, float [2 row buffers][128 tokens]
   static constexpr int kScratch = kQn + 8 * 64 * 4;            // top-k scratch of warps 10 and 11
   static constexpr int kScratchWords = sel_topk_scratch_words(kTokMaxKV / 32);
   static constexpr int kBar = kScratch + 2 * kScratchWords * 4;
@@ -67,7 +69,8 @@ enum : int {
   kTokDEmpty = kTokDFull + 2,
   kTokSFull = kTokDEmpty + 2,       // + score row buffer
   kTokSEmpty = kTokSFull + 2,
-  kTokNumBars = kTokSEmpty + 2
+  kTokNFull = kTokSEmpty + 2,       // + 2 * token half + norm buffer: the half's 4 epilogue warps
+  kTokNumBars = kTokNFull + 4
 };
 
 struct TokArgs {
@@ -124,6 +127,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
       mbar_init(bar(kTokSFull + s), 8);
       mbar_init(bar(kTokSEmpty + s), 1);
     }
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kTokNFull + s), 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -227,38 +231,49 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
       const int nq = min(BQ, a.Lq - i * BQ);  // valid tokens of this query block
       const int kvh = hq / G;
       const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
-      // this warp's tokens: t0 .. t0 + BQ/2 - 1; their norms in its own array
-      // (no barrier between the epilogue warps)
-      const int t0 = thalf * (BQ / 2);
-      float* qn = qn_s + warp * 64 - t0;  // qn[t] for t in this warp's half
+      // this row's token norms, shared by the four warps of a token half
+      // through norm buffer k & 1: warp (quarter q) takes tokens
+      // t0 + q TPW .. t0 + q TPW + TPW - 1, LPT lanes per token, each lane
+      // summing CPL of the token's sixteen 16-byte chunks (two 64-dim halves)
+      constexpr int TPW = BQ / 8, LPT = 32 / TPW, CPL = 16 / LPT;
+      const int t0 = thalf * (BQ / 2), nb = k & 1;
+      float* qn = qn_s + nb * 128;  // qn[t] for the tokens t of this row
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokQFull), k & 1, abort_flag))) break;
-      for (int t = t0 + lane; t < t0 + BQ / 2; t += 32) {
-        // token t: 16-byte chunk c of its 128-byte row in each half sits at
-        // chunk position c ^ (t % 8) (128-byte swizzle)
+      {
+        const int t = t0 + quarter * TPW + lane / LPT, sl = lane % LPT;
         float s2 = 0.f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int cc = 0; cc < CPL; ++cc) {
+          // chunk c of the token's 128-byte row in half h sits at chunk
+          // position c ^ (t % 8) (128-byte swizzle)
+          const int chunk = sl * CPL + cc, h = chunk >> 3, c = chunk & 7;
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(smem + L::kQ + h * BQ * 128 + t * 128 + ((c ^ (t & 7)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kQ + h * BQ * 128 + t * 128 +
-                                                            ((c ^ (t & 7)) << 4));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              s2 = fmaf(bf16lo(w[q]), bf16lo(w[q]), s2);
-              s2 = fmaf(bf16hi(w[q]), bf16hi(w[q]), s2);
-            }
+          for (int q = 0; q < 4; ++q) {
+            s2 = fmaf(bf16lo(w[q]), bf16lo(w[q]), s2);
+            s2 = fmaf(bf16hi(w[q]), bf16hi(w[q]), s2);
           }
         }
-        qn[t] = sqrtf(s2);
+#pragma unroll
+        for (int o = 1; o < LPT; o <<= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        if (sl == 0) qn[t] = sqrtf(s2);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kTokQEmpty));
+      if (lane == 0) {
+        mbar_arrive(bar(kTokQEmpty));
+        mbar_arrive(bar(kTokNFull + 2 * thalf + nb));
+      }
       const int sb = k & 1;
       uint32_t* kc = keys + sb * 2 * kTokMaxKV;
       uint32_t* kr = kc + kTokMaxKV;
       // the top-k of row k - 2 must be done with this score buffer
       if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(kTokSEmpty + sb), ((k >> 1) - 1) & 1, abort_flag))) break;
+      // the other three warps' norms of this half.  Norm buffer nb is written
+      // again two rows later, by a warp past the next row's wait: all four
+      // warps have finished this row by then.
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kTokNFull + 2 * thalf + nb), (k >> 1) & 1, abort_flag))) break;
       for (int m = 0; m < T; ++m, ++gt) {
         const int db = gt & 1;
         const int j = m * 128 + quarter * 32 + lane;
