@@ -262,3 +262,27 @@ def test_query_pool_validation(L):
     p1 = SelectParams(block_q=64, block_k=64, query_pool=1).c()
     assert L.rbs_select_workspace_bytes(1, 2, 8, 1, 8, ctypes.byref(p1)) > 0
     assert L.rbs_select_workspace_bytes(1, 2, 8, 1, 8, ctypes.byref(p0)) > 0
+
+
+def test_token_max_workspace_holds_the_key_matrix(L):
+    """query_pool TOKEN_MAX: the full workspace adds both branches' key rows
+    ([rows][2][nKB padded to 32] uint32) for the separate top-k kernel; a
+    workspace one byte short still runs (the scoring kernel selects in
+    place), one without room for the split centroids is refused."""
+    p1 = SelectParams(block_q=64, block_k=64, query_pool=1).c()
+    nkb = 64
+    small = L.rbs_select_workspace_bytes(1, 2, 8, 1, nkb, ctypes.byref(p1))
+    large = L.rbs_select_workspace_bytes(1, 2, 16, 1, nkb, ctypes.byref(p1))
+    extra_rows = 1 * 2 * 8
+    # at least the extra rows' key rows (2 x 4 B per block); the smaller
+    # regions are rounded up to 256 bytes
+    assert large - small >= extra_rows * 2 * nkb * 4
+    q = _fake(Lq=512)
+    rows = 1 * 2 * 8
+    ok = _abi.BlockListsC(0x40000, 0x50000, None, 1 << 20, rows)
+    sel = lambda ws: L.rbs_select(ctypes.byref(q), 0x20000, 0x30000, 1, 8, ctypes.byref(p1), 0x60000, ws,
+                                  ctypes.byref(ok), None, None)
+    full = L.rbs_select_workspace_bytes(1, 2, 8, 1, 8, ctypes.byref(p1))
+    assert sel(full) == 4  # past validation: no GPU here
+    assert sel(full - 1) == 4
+    assert sel(256) == 3
