@@ -844,24 +844,33 @@ def cpu_baseline(Qh, Kh, Vh, w, budget_s: float = 20.0, heads_q: int | None = No
             "sample": (f"numpy fp64 oracle: stats of KV head 0 ({t_stats:.2f}s), selection of q head 0 "
                        f"({t_sel:.2f}s), attention of {nrows} rows ({done_pairs} block pairs, {t_attn:.2f}s); "
                        f"step time extrapolated x{Hkv} / x{Hq} / by selected pairs = {step_s:.1f}s"),
-            "measured_s": round(t_stats + t_sel + t_attn, 2)}
+            "measured_s": round(t_stats + t_sel + t_attn, 2), "step_s": round(step_s, 3)}
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step a bounded sample of the 128K workload."""
+    """The oracle as the reference arm: each step a bounded sample of the 128K workload.
+
+    Each step's attention sample gets --ref-step-budget seconds, lowered so
+    that the warm-up and timed steps together stay near --ref-total-budget
+    (a sample never has fewer than eight rows).  ms_per_step is the median
+    extrapolated time of one whole step.
+    """
     w = WORKLOADS[WORKLOAD]
-    inp = make_inputs(w)
+    inp = make_inputs(w, seqlen=args.seq_len)
+    n = args.warmup + args.steps
+    budget = min(args.ref_step_budget, args.ref_total_budget / max(1, n))
     vals = []
-    for k in range(args.warmup + args.steps):
-        r = cpu_baseline(inp["Q"], inp["K"], inp["V"], w, budget_s=args.ref_step_budget)
+    for k in range(n):
+        r = cpu_baseline(inp["Q"], inp["K"], inp["V"], w, budget_s=budget)
         if k >= args.warmup:
             vals.append(r)
     v = statistics.median(x["value"] for x in vals)
+    step_ms = statistics.median(x["step_s"] for x in vals) * 1e3
     base = vals[-1]
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic (seeded compact/dispersed key mixture, planted keys)",
-            "config": bench_config(WORKLOADS[WORKLOAD].seqlen, 1, 1),
+            "warmup": args.warmup, "ms_per_step": round(step_ms, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded compact/dispersed key mixture, planted keys)",
+            "config": bench_config(inp["Q"].shape[1], 1, 1),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
                              "sample": base["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -885,6 +894,8 @@ def main():
     ap.add_argument("--no-token-max", dest="token_max", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
+    ap.add_argument("--ref-total-budget", type=float, default=100.0,
+                    help="seconds of oracle sampling for the whole reference run")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="shorter prompt of the same workload (profiling captures only; not the headline)")
     args = ap.parse_args()

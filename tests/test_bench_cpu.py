@@ -34,3 +34,28 @@ def test_radius_quintile_share_is_a_distribution():
     assert len(share) == 5
     assert abs(sum(share) - 1.0) < 1e-3
     assert all(0.0 <= x <= 1.0 for x in share)
+
+
+def test_reference_arm_line():
+    # the oracle arm on a short prompt of the same workload: one JSON-ready
+    # line with the contract's keys, its own cpu_baseline and e2e, and a
+    # sampling time bounded by the total budget
+    import argparse
+    import json
+    import time
+    args = argparse.Namespace(steps=2, warmup=3, ref_step_budget=3.0, ref_total_budget=2.5, seq_len=4096)
+    t0 = time.perf_counter()
+    line = bench.run_reference(args)
+    took = time.perf_counter() - t0
+    json.dumps(line)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert line["steps"] == 2 and line["warmup"] == 3
+    assert line["config"]["seq_len"] == 4096
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert took < 60
