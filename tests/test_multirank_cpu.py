@@ -54,3 +54,22 @@ def test_single_rank_is_identity():
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import bench
     assert bench.aggregate(5.0, 2e12, 1) == (5.0, 2e12, pytest.approx(400.0))
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    # launched like the scaling run (torchrun, two ranks on this host): rank 0
+    # alone runs the oracle and prints one JSON line; the other rank exits 0
+    # without work
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "3", "--seq-len", "4096", "--ref-total-budget", "2"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=240)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["value"] > 0
