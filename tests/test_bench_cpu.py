@@ -59,3 +59,22 @@ def test_reference_arm_line():
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert took < 60
+
+
+def test_attention_traffic_only_for_the_captured_build(tmp_path, monkeypatch):
+    # the DRAM traffic figure is reported only for the 128K workload and only
+    # while the attention sources hash to the build it was captured on
+    import os
+    import shutil
+    assert bench.attn_traffic(32768) is None
+    full = bench.WORKLOADS[bench.WORKLOAD].seqlen
+    now = bench.attn_traffic(full)
+    assert now in (bench.ATTN_TRAFFIC_BYTES, None)
+    for f in bench.ATTN_TRAFFIC_SOURCES:
+        os.makedirs(tmp_path / os.path.dirname(f), exist_ok=True)
+        shutil.copy(os.path.join(bench.ROOT, f), tmp_path / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.attn_traffic(full) == now
+    with open(tmp_path / bench.ATTN_TRAFFIC_SOURCES[0], "a") as fh:
+        fh.write("\n// edited\n")
+    assert bench.attn_traffic(full) is None
