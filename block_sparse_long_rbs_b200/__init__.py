@@ -72,6 +72,16 @@ class BlockLists:
     num_rows: int
 
     def c(self) -> BlockListsC:
+        # the kernels write row_ptr[0 .. num_rows] and col_idx / flags up to
+        # the capacity: every buffer must be a contiguous CUDA tensor that long
+        if self.row_ptr.numel() < self.num_rows + 1:
+            raise ValueError(f"lists.row_ptr: {self.row_ptr.numel()} entries for {self.num_rows} rows")
+        if self.flags is not None and self.flags.numel() < self.col_idx.numel():
+            raise ValueError(f"lists.flags: {self.flags.numel()} entries, capacity {self.col_idx.numel()}")
+        _dev(self.row_ptr, "lists.row_ptr", torch.int32)
+        _dev(self.col_idx, "lists.col_idx", torch.int32)
+        if self.flags is not None:
+            _dev(self.flags, "lists.flags", torch.uint8)
         return BlockListsC(self.row_ptr.data_ptr(), self.col_idx.data_ptr(),
                            self.flags.data_ptr() if self.flags is not None else None,
                            self.col_idx.numel(), self.num_rows)
@@ -85,6 +95,16 @@ class BlockLists:
                           torch.empty(max(1, capacity), dtype=torch.int32, device=device),
                           torch.empty(max(1, capacity), dtype=torch.uint8, device=device) if flags else None,
                           num_rows)
+
+
+def _dev(x, name: str, dtype: torch.dtype) -> int:
+    """Check a contiguous CUDA tensor of the given dtype and return its
+    device pointer."""
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not x.is_cuda or x.dtype != dtype or not x.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous {dtype} CUDA tensor")
+    return x.data_ptr()
 
 
 def _stream() -> ctypes.c_void_p:
@@ -157,8 +177,18 @@ def rbs_select(Q: torch.Tensor, centroids: torch.Tensor, radii: torch.Tensor, pa
                flags: bool = True) -> BlockLists:
     """Two-branch selection -> CSR key-block lists, rows = (batch, q head, query block), or
     (batch, KV head, query block) when params.list_mode == 1."""
-    B, L, Hq, _ = Q.shape
+    B, L, Hq, D = Q.shape
+    if centroids.dim() != 4:
+        raise ValueError(f"centroids: expected [B, Hkv, nKB, {D}], got {tuple(centroids.shape)}")
     Hkv, nkb = centroids.shape[1], centroids.shape[2]
+    # every shape first, then where the tensors live
+    for x, name, shape in ((centroids, "centroids", (B, Hkv, nkb, D)), (radii, "radii", (B, Hkv, nkb)),
+                           (beta_out, "beta_out", (B, Hkv, nkb))):
+        if x is not None and tuple(x.shape) != shape:
+            raise ValueError(f"{name}: expected shape {shape}, got {tuple(x.shape)}")
+    c_ptr = _dev(centroids, "centroids", torch.float32)
+    r_ptr = _dev(radii, "radii", torch.float32)
+    b_ptr = _dev(beta_out, "beta_out", torch.float32) if beta_out is not None else None
     nqb = -(-L // params.block_q)
     rows = B * (Hkv if params.list_mode == 1 else Hq) * nqb
     if out is None:
@@ -166,11 +196,11 @@ def rbs_select(Q: torch.Tensor, centroids: torch.Tensor, radii: torch.Tensor, pa
     if workspace is None:
         workspace = torch.empty(rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, params), dtype=torch.uint8,
                                 device=Q.device)
+    ws_ptr = _dev(workspace, "workspace", torch.uint8)
     p = params.c()
     lc = out.c()
-    check(lib().rbs_select(ctypes.byref(_t(Q, "Q")), _f32(centroids, "centroids"), _f32(radii, "radii"), Hkv, nkb,
-                           ctypes.byref(p), workspace.data_ptr(), workspace.numel(), ctypes.byref(lc),
-                           beta_out.data_ptr() if beta_out is not None else None, _stream()), "rbs_select")
+    check(lib().rbs_select(ctypes.byref(_t(Q, "Q")), c_ptr, r_ptr, Hkv, nkb, ctypes.byref(p), ws_ptr,
+                           workspace.numel(), ctypes.byref(lc), b_ptr, _stream()), "rbs_select")
     return out
 
 
