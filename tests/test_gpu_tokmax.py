@@ -135,3 +135,49 @@ def test_tokmax_both_topk_paths(cuda_ok, case):
     ora = O.select_blocks(Q, Co, Ro, po, keep_scores=True)
     rep = compare_selection(lists_sep, ora, Hq, nqb, nkb, exact_k=kw.get("threshold_mode", 0) == 0)
     print("tokmax both top-k paths", case, rep)
+
+
+def test_tokmax_2048_key_blocks_sampled_rows(cuda_ok):
+    # 262144 tokens in 128-token blocks: 2048 key blocks, the most the
+    # per-token kernel takes (its 64-slot instantiation).  Sampled rows of
+    # each branch against the oracle's scores, and the separate and in-place
+    # top-k giving identical lists.
+    inp = make_mixture(L=262144, Hq=2, Hkv=1, block=128, seed=706)
+    Q, K = inp["Q"], inp["K"]
+    B, L, Hq, _ = Q.shape
+    nqb = nkb = L // 128
+    rho = 0.02
+    p = rbs.SelectParams(rho_centroid=rho, rho_rescue=rho, query_pool=1)
+    Qd = dev(Q)
+    Cg, Rg = rbs.rbs_block_stats(dev(K), 128)
+    full = rbs.rbs_select_workspace_bytes(B, Hq, nqb, 1, nkb, p)
+    ws = torch.empty(full + 255, dtype=torch.uint8, device="cuda")
+    off = (-ws.data_ptr()) % 256
+    lists = rbs.rbs_select(Qd, Cg, Rg, p, workspace=ws[off:off + full])
+    lists_in = rbs.rbs_select(Qd, Cg, Rg, p, workspace=ws[off:off + full - 1])
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    for a, b in zip(lists_np(lists), lists_np(lists_in)):
+        np.testing.assert_array_equal(a, b)
+    rp, ci, fl = lists_np(lists)
+    _, gc, gr = dense_masks(rp, ci, fl, nkb)
+    C, R = O.block_stats(K, 128)
+    po = O.SelectParams(rho_centroid=float(np.float32(rho)), rho_rescue=float(np.float32(rho)), query_pool=1)
+    beta, _ = O.rescue_beta(R, po)
+    excused = 0
+    for hq, i in ((0, 2047), (1, 2047), (0, 1500), (1, 1100), (0, 1030), (1, 700)):
+        q = Q[0, i * 128:(i + 1) * 128, hq][None]
+        s_c, s_r = O.token_max_scores(q[0], C[0, 0], R[0, 0], beta[0, 0], 128)
+        n = i + 1
+        row = hq * nqb + i
+        for bi, (s, gm, r) in enumerate(((s_c[0, :n], gc, po.rho_centroid), (s_r[0, :n], gr, po.rho_rescue))):
+            k = O.keep_count(r, n)
+            top = O.top_k_desc(s, k)
+            want = np.zeros(n, dtype=bool)
+            want[top] = True
+            tau = s[top[-1]]
+            assert gm[row, :n].sum() == k
+            for j in np.nonzero(gm[row, :n] != want)[0]:
+                assert abs(s[j] - tau) <= TOL_NEAR_TAU * max(1.0, abs(tau)), (hq, i, bi, j)
+                excused += 1
+    print("tokmax 2048 key blocks, sampled rows, excused", excused, "nnz", int(rp[-1]))
