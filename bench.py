@@ -48,11 +48,12 @@ FLOP_PER_PAIR = 4 * BLOCK * BLOCK * HEAD_DIM  # QK^T and PV on one 128x128 block
 # kernels one step launches: block stats; selection (beta, centroid split,
 # pooling, score MMAs, top-k, scan, compaction); attention
 LAUNCHES_PER_STEP = 9
+ATTN_KERNEL = "bsa_prefill_kernel<128,128>"
 SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)
 # DRAM traffic of one 131072-token attention launch (dram__bytes_read.sum +
-# dram__bytes_write.sum, one single-pass ncu capture of the default workload;
-# profiles/launches_gqa_rbs_128k.md gives the command), valid for the kernel
-# sources with this digest; any other build reports null.
+# dram__bytes_write.sum from one single-pass ncu capture of the default
+# workload), valid only for the kernel sources with this digest; any other
+# build reports null.
 ATTN_TRAFFIC_BYTES = 3.306e9 + 1.040e9
 ATTN_TRAFFIC_SOURCES = ("block_sparse_long_rbs_b200/csrc/attention.cuh", "block_sparse_long_rbs_b200/csrc/common.cuh")
 ATTN_TRAFFIC_DIGEST = "ef6c3e5cf172632b"
@@ -77,6 +78,28 @@ def bench_config(L: int, B: int, ws: int) -> dict:
             "l2": "inputs larger than L2 (Q 1 GiB, K and V 128 MiB each); no flush"}
 
 
+def roofline_entry(attn_tflops: float, peaks: dict, traffic) -> dict:
+    """The attention kernel against the tensor peak.  The timed region is a
+    few hundred milliseconds of back-to-back steps, so the kernel is compared
+    with the burst bf16 peak; the sustained (seconds-long, power-capped)
+    figure is reported beside it."""
+    peak, peak_sus = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    return {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peak, 4), "traffic": traffic, "kernel": ATTN_KERNEL,
+            "peak_kind": f"bf16 burst ({peaks['source']})", "peak_sustained": peak_sus,
+            "frac_of_sustained": round(attn_tflops / peak_sus, 4)}
+
+
+def ttft_ratios(final_ms: float, reencode_ms: float, full_ms: float, final_pairs: int, full_pairs: int) -> dict:
+    """The Block-attention page's time-to-first-token comparison: with the
+    passages' KV cached, the prompt costs the final block's pass (plus the
+    re-encoding of the cached keys) instead of a full causal prefill."""
+    return {"time_ratio": round(final_ms / full_ms, 5),
+            "time_ratio_with_reencode": round((final_ms + reencode_ms) / full_ms, 5),
+            "flops_ratio": round(final_pairs / full_pairs, 5),
+            "full_prefill": "bsa_prefill with every causally visible block of the whole prompt"}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -94,10 +117,14 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, log_dir: str | None = None):
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.keep = log_dir is not None
+        if log_dir is None:
+            log_dir = tempfile.mkdtemp(prefix="rbs_clocks_")
+        self.path = os.path.join(log_dir, f"clocks_rank{index}.csv")
 
     def start(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
@@ -109,8 +136,20 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _cleanup(self):
+        f = getattr(self, "f", None)
+        if f is not None and not f.closed:
+            f.close()
+        if not self.keep:
+            for rm in (os.remove, os.rmdir):
+                try:
+                    rm(self.path if rm is os.remove else os.path.dirname(self.path))
+                except OSError:
+                    pass
+
     def stop(self):
         if self.proc is None:
+            self._cleanup()
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         self.proc.wait(timeout=10)
@@ -129,6 +168,7 @@ class ClockSampler:
             for nm, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
+        self._cleanup()
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
@@ -247,7 +287,7 @@ def run_ours(args, ws, rank):
     visible = B * Hq * nqb * (nqb + 1) // 2
     diag_half = B * Hq * nqb * (BLOCK * BLOCK * HEAD_DIM * 2)  # the diagonal counted half (causal-exact)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    clk = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clk = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")), args.clock_log_dir)
     clk.start()
     time.sleep(0.3)
     sync_all(ws)
@@ -266,7 +306,7 @@ def run_ours(args, ws, rank):
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     step_ms, all_flops, value = aggregate(total_ms / args.steps, float(flops), ws)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    peak = peaks["bf16_tflops"]
 
     # bytes for the bandwidth-bound kernels
     stats_bytes = L * Hkv * HEAD_DIM * 2 + nkb * Hkv * (HEAD_DIM + 1) * 4
@@ -280,9 +320,7 @@ def run_ours(args, ws, rank):
         "stats_ms": round(stats_ms, 4), "nnz_pairs": nnz, "density": round(nnz / visible, 5),
         "selected_tflop": round(flops / 1e12, 4),
         "causal_exact_tflop": round((flops - diag_half) / 1e12, 4),
-        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(attn_tflops / peak, 4), "traffic": attn_traffic(L),
-                     "kernel": "bsa_prefill_kernel<128,128>", "peak_kind": f"bf16 sustained ({peaks['source']})"},
+        "roofline": roofline_entry(attn_tflops, peaks, attn_traffic(L)),
         "kernels": {
             "block_stats": {"ms": round(stats_ms, 4), "gbs": round(stats_bytes / (stats_ms * 1e-3) / 1e9, 1),
                             "frac_hbm": round(stats_bytes / (stats_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)},
@@ -608,11 +646,19 @@ def block_attention_measure(rbs, peaks):
     Qf = rbs.rope_reencode(Q[:, P * PL:].contiguous(), zero[:FL], glob[P * PL:], w.rope_theta)
     Op = torch.empty_like(Qc[:, :P * PL])
     Of = torch.empty_like(Qf)
+    # full-attention reference: a causal prefill of all 33,280 tokens encoded
+    # at their global positions (every causally visible block)
+    nb = L // BLOCK
+    full_lists = rbs.rbs_lists_causal_full(1, w.heads_q, nb, 0)
+    Qg = rbs.rope_reencode(Q, zero, glob, w.rope_theta)
+    Kfull = rbs.rope_reencode(K, zero, glob, w.rope_theta)
+    Ofull = torch.empty_like(Qg)
     parts = {
         "cache_build": lambda: rbs.bsa_prefill(Qc[:, :P * PL], Kc[:, :P * PL], V[:, :P * PL], cache_lists, BLOCK,
                                                BLOCK, out=Op),
         "rope_reencode": lambda: rbs.rope_reencode(Kc, loc, glob, w.rope_theta, out=Kg),
         "final_block": lambda: rbs.bsa_prefill(Qf, Kg, V, final_lists, BLOCK, BLOCK, q_offset=P * PL, out=Of),
+        "full_prefill": lambda: rbs.bsa_prefill(Qg, Kfull, V, full_lists, BLOCK, BLOCK, out=Ofull),
     }
     res = {}
     flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
@@ -638,12 +684,12 @@ def block_attention_measure(rbs, peaks):
     gbs = rope_bytes / (res["rope_reencode"]["ms"] * 1e-3) / 1e9
     res["rope_reencode"].update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3),
                                  "bytes": rope_bytes})
-    for name, lists in (("cache_build", cache_lists), ("final_block", final_lists)):
+    for name, lists in (("cache_build", cache_lists), ("final_block", final_lists), ("full_prefill", full_lists)):
         fl = lists.nnz() * FLOP_PER_PAIR
         res[name]["tflops"] = round(fl / (res[name]["ms"] * 1e-3) / 1e12, 2)
         res[name]["pairs"] = lists.nnz()
-    # full-attention reference for the final block: the same 512 queries over all 33,280 keys
-    res["final_block_vs_full_prefill"] = None
+    res["final_block_vs_full_prefill"] = ttft_ratios(res["final_block"]["ms"], res["rope_reencode"]["ms"],
+                                                     res["full_prefill"]["ms"], final_lists.nnz(), full_lists.nnz())
     return res
 
 
@@ -781,7 +827,7 @@ def density_sweep_measure(rbs, peaks):
         tflops = nnz * FLOP_PER_PAIR / (attn_ms * 1e-3) / 1e12
         rows.append({"target": target, "rho": rho, "density": round(nnz / visible, 5), "pairs": nnz,
                      "select_ms": round(sel_ms, 4), "attn_ms": round(attn_ms, 4), "attn_tflops": round(tflops, 1),
-                     "attn_frac_peak": round(tflops / peaks["bf16_tflops_sustained"], 4)})
+                     "attn_frac_peak": round(tflops / peaks["bf16_tflops"], 4)})
     assert rbs.rbs_get_device_error() == 0
     dense_ms = rows[-1]["attn_ms"]
     for r in rows:
@@ -853,7 +899,8 @@ def run_reference(args):
     Each step's attention sample gets --ref-step-budget seconds, lowered so
     that the warm-up and timed steps together stay near --ref-total-budget
     (a sample never has fewer than eight rows).  ms_per_step is the median
-    extrapolated time of one whole step.
+    time one step's sample took; extrapolated_ms_per_full_step is the
+    median time of one whole step extrapolated from the samples.
     """
     w = WORKLOADS[WORKLOAD]
     inp = make_inputs(w, seqlen=args.seq_len)
@@ -865,10 +912,14 @@ def run_reference(args):
         if k >= args.warmup:
             vals.append(r)
     v = statistics.median(x["value"] for x in vals)
+    # ms_per_step is the time each step's sample actually took; the whole
+    # step's time, extrapolated from the sample, is reported beside it
+    sample_ms = statistics.median(x["measured_s"] for x in vals) * 1e3
     step_ms = statistics.median(x["step_s"] for x in vals) * 1e3
     base = vals[-1]
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(step_ms, 1), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(sample_ms, 1),
+            "extrapolated_ms_per_full_step": round(step_ms, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded compact/dispersed key mixture, planted keys)",
             "config": bench_config(inp["Q"].shape[1], 1, 1),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
@@ -896,6 +947,8 @@ def main():
     ap.add_argument("--ref-step-budget", type=float, default=3.0)
     ap.add_argument("--ref-total-budget", type=float, default=100.0,
                     help="seconds of oracle sampling for the whole reference run")
+    ap.add_argument("--clock-log-dir", default=None,
+                    help="keep the nvidia-smi clock samples of the timed region here (default: a temporary file)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="shorter prompt of the same workload (profiling captures only; not the headline)")
     args = ap.parse_args()

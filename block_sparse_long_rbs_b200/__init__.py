@@ -111,6 +111,23 @@ def _stream() -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
+def _one_device(ref_name: str, ref, **others) -> torch.device:
+    """The device every tensor of one call must live on (ref's).  The library
+    launches on the current device and its current stream, so a tensor on
+    another GPU would hand a kernel a pointer it cannot use: refuse it here.
+    None entries (optional arguments) are skipped."""
+    dev = ref.device
+    for name, x in others.items():
+        if x is not None and x.device != dev:
+            raise ValueError(f"{name} is on {x.device} but {ref_name} is on {dev}: "
+                             "every tensor of a call must be on one device")
+    return dev
+
+
+def _lists_tensors(lists) -> dict:
+    return {"lists.row_ptr": lists.row_ptr, "lists.col_idx": lists.col_idx, "lists.flags": lists.flags}
+
+
 def _t(x: torch.Tensor, name: str) -> Bf16Tensor:
     """Describe a [B, L, H, 128] bf16 CUDA tensor (head_dim contiguous) for the C ABI."""
     if not isinstance(x, torch.Tensor) or not x.is_cuda:
@@ -133,8 +150,10 @@ def rbs_block_stats(K: torch.Tensor, block_k: int):
     nkb = -(-L // block_k)  # a last, partial block holds the remaining keys
     C = torch.empty(B, H, nkb, D, dtype=torch.float32, device=K.device)
     R = torch.empty(B, H, nkb, dtype=torch.float32, device=K.device)
-    check(lib().rbs_block_stats(ctypes.byref(_t(K, "K")), block_k, C.data_ptr(), R.data_ptr(), _stream()),
-          "rbs_block_stats")
+    tK = _t(K, "K")
+    with torch.cuda.device(K.device):
+        check(lib().rbs_block_stats(ctypes.byref(tK), block_k, C.data_ptr(), R.data_ptr(), _stream()),
+              "rbs_block_stats")
     return C, R
 
 
@@ -144,8 +163,10 @@ def rbs_block_beta(radii: torch.Tensor, params: SelectParams):
     beta = torch.empty_like(radii)
     rng = torch.empty(B, H, 2, dtype=torch.float32, device=radii.device)
     p = params.c()
-    check(lib().rbs_block_beta(_f32(radii, "radii"), B, H, n, ctypes.byref(p), beta.data_ptr(), rng.data_ptr(),
-                               _stream()), "rbs_block_beta")
+    r_ptr = _f32(radii, "radii")
+    with torch.cuda.device(radii.device):
+        check(lib().rbs_block_beta(r_ptr, B, H, n, ctypes.byref(p), beta.data_ptr(), rng.data_ptr(), _stream()),
+              "rbs_block_beta")
     return beta, rng
 
 
@@ -155,8 +176,10 @@ def rbs_pool_queries(Q: torch.Tensor, block_q: int):
     nqb = -(-L // block_q)
     qbar = torch.empty(B, H, nqb, D, dtype=torch.float32, device=Q.device)
     qnorm = torch.empty(B, H, nqb, dtype=torch.float32, device=Q.device)
-    check(lib().rbs_pool_queries(ctypes.byref(_t(Q, "Q")), block_q, qbar.data_ptr(), qnorm.data_ptr(), _stream()),
-          "rbs_pool_queries")
+    tQ = _t(Q, "Q")
+    with torch.cuda.device(Q.device):
+        check(lib().rbs_pool_queries(ctypes.byref(tQ), block_q, qbar.data_ptr(), qnorm.data_ptr(), _stream()),
+              "rbs_pool_queries")
     return qbar, qnorm
 
 
@@ -199,8 +222,12 @@ def rbs_select(Q: torch.Tensor, centroids: torch.Tensor, radii: torch.Tensor, pa
     ws_ptr = _dev(workspace, "workspace", torch.uint8)
     p = params.c()
     lc = out.c()
-    check(lib().rbs_select(ctypes.byref(_t(Q, "Q")), c_ptr, r_ptr, Hkv, nkb, ctypes.byref(p), ws_ptr,
-                           workspace.numel(), ctypes.byref(lc), b_ptr, _stream()), "rbs_select")
+    tQ = _t(Q, "Q")
+    dev = _one_device("Q", Q, centroids=centroids, radii=radii, beta_out=beta_out, workspace=workspace,
+                      **_lists_tensors(out))
+    with torch.cuda.device(dev):
+        check(lib().rbs_select(ctypes.byref(tQ), c_ptr, r_ptr, Hkv, nkb, ctypes.byref(p), ws_ptr,
+                               workspace.numel(), ctypes.byref(lc), b_ptr, _stream()), "rbs_select")
     return out
 
 
@@ -210,8 +237,9 @@ def rbs_lists_causal_full(batch: int, heads_q: int, num_q_blocks: int, q_block_o
     nnz = int(lib().rbs_lists_causal_full_nnz(batch, heads_q, num_q_blocks, q_block_offset))
     out = BlockLists.empty(batch * heads_q * num_q_blocks, nnz, device, flags)
     lc = out.c()
-    check(lib().rbs_lists_causal_full(batch, heads_q, num_q_blocks, q_block_offset, ctypes.byref(lc), _stream()),
-          "rbs_lists_causal_full")
+    with torch.cuda.device(out.row_ptr.device):
+        check(lib().rbs_lists_causal_full(batch, heads_q, num_q_blocks, q_block_offset, ctypes.byref(lc), _stream()),
+              "rbs_lists_causal_full")
     return out
 
 
@@ -225,8 +253,9 @@ def rbs_lists_block_attention(seg_start, final_start: int, block: int, batch: in
         raise RbsError(1, "rbs_lists_block_attention_nnz", lib().rbs_last_error().decode())
     out = BlockLists.empty(batch * heads_q * q_num_blocks, nnz, device, flags)
     lc = out.c()
-    check(lib().rbs_lists_block_attention(seg, len(seg_start), final_start, block, batch, heads_q, q_first_block,
-                                          q_num_blocks, ctypes.byref(lc), _stream()), "rbs_lists_block_attention")
+    with torch.cuda.device(out.row_ptr.device):
+        check(lib().rbs_lists_block_attention(seg, len(seg_start), final_start, block, batch, heads_q, q_first_block,
+                                              q_num_blocks, ctypes.byref(lc), _stream()), "rbs_lists_block_attention")
     return out
 
 
@@ -241,10 +270,12 @@ def bsa_prefill(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, lists: BlockL
         lse = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], dtype=torch.float32, device=Q.device)
     scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(Q.shape[-1])
     lc = lists.c()
-    check(lib().bsa_prefill(ctypes.byref(_t(Q, "Q")), ctypes.byref(_t(K, "K")), ctypes.byref(_t(V, "V")),
-                            ctypes.byref(lc), block_q, block_k, q_offset, scale, 1 if causal else 0,
-                            ctypes.byref(_t(out, "O")), lse.data_ptr() if lse is not None else None, _stream()),
-          "bsa_prefill")
+    tQ, tK, tV, tO = _t(Q, "Q"), _t(K, "K"), _t(V, "V"), _t(out, "O")
+    dev = _one_device("Q", Q, K=K, V=V, out=out, lse=lse, **_lists_tensors(lists))
+    with torch.cuda.device(dev):
+        check(lib().bsa_prefill(ctypes.byref(tQ), ctypes.byref(tK), ctypes.byref(tV), ctypes.byref(lc), block_q,
+                                block_k, q_offset, scale, 1 if causal else 0, ctypes.byref(tO),
+                                lse.data_ptr() if lse is not None else None, _stream()), "bsa_prefill")
     return (out, lse) if return_lse else out
 
 
@@ -261,10 +292,13 @@ def bsa_prefill_rescue_weighted(Q: torch.Tensor, K: torch.Tensor, V: torch.Tenso
         lse = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], dtype=torch.float32, device=Q.device)
     scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(Q.shape[-1])
     lc = lists.c()
-    check(lib().bsa_prefill_rescue_weighted(
-        ctypes.byref(_t(Q, "Q")), ctypes.byref(_t(K, "K")), ctypes.byref(_t(V, "V")), ctypes.byref(lc), block_q,
-        block_k, q_offset, scale, 1 if causal else 0, float(rescue_weight), ctypes.byref(_t(out, "O")),
-        lse.data_ptr() if lse is not None else None, _stream()), "bsa_prefill_rescue_weighted")
+    tQ, tK, tV, tO = _t(Q, "Q"), _t(K, "K"), _t(V, "V"), _t(out, "O")
+    dev = _one_device("Q", Q, K=K, V=V, out=out, lse=lse, **_lists_tensors(lists))
+    with torch.cuda.device(dev):
+        check(lib().bsa_prefill_rescue_weighted(
+            ctypes.byref(tQ), ctypes.byref(tK), ctypes.byref(tV), ctypes.byref(lc), block_q, block_k, q_offset, scale,
+            1 if causal else 0, float(rescue_weight), ctypes.byref(tO), lse.data_ptr() if lse is not None else None,
+            _stream()), "bsa_prefill_rescue_weighted")
     return (out, lse) if return_lse else out
 
 
@@ -276,8 +310,11 @@ def rope_reencode(x: torch.Tensor, old_pos: torch.Tensor, new_pos: torch.Tensor,
     for name, p in (("old_pos", old_pos), ("new_pos", new_pos)):
         if not p.is_cuda or p.dtype != torch.int32 or p.numel() != x.shape[1]:
             raise TypeError(f"{name}: expected int32 CUDA tensor of length {x.shape[1]}")
-    check(lib().rope_reencode(ctypes.byref(_t(x, "x")), ctypes.byref(_t(out, "out")), old_pos.data_ptr(),
-                              new_pos.data_ptr(), theta, rope_style, _stream()), "rope_reencode")
+    tx, to = _t(x, "x"), _t(out, "out")
+    dev = _one_device("x", x, out=out, old_pos=old_pos, new_pos=new_pos)
+    with torch.cuda.device(dev):
+        check(lib().rope_reencode(ctypes.byref(tx), ctypes.byref(to), old_pos.data_ptr(), new_pos.data_ptr(), theta,
+                                  rope_style, _stream()), "rope_reencode")
     return out
 
 

@@ -732,30 +732,21 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
 // rbs_select normally takes as a workspace is instead a fixed buffer in this
 // library's own device image (RBS_NOALLOC_SCRATCH_BYTES on every device that
 // loads the library, held until the process exits).  Host code cannot use the
-// array's name as a device address, so its address is looked up once per
-// device with that device current and cached.
+// array's name as a device address: its address on the current device is
+// looked up on every call (a runtime query that allocates nothing), so no
+// cached address can outlive a context that was torn down and rebuilt.
 
 }  // extern "C"
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[RBS_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void* g_noalloc_ptr[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
-
 rbs_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return fail(RBS_ERR_CUDA, "cudaGetDevice failed");
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return fail(RBS_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return fail(RBS_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+  *out = p;
   return RBS_OK;
 }
 }  // namespace
@@ -765,18 +756,20 @@ extern "C" {
 rbs_status rbs_select_noalloc(const rbs_bf16_tensor* Q, const float* centroids, const float* radii,
                               int32_t kv_heads, int64_t num_kv_blocks, const rbs_select_params* p,
                               rbs_block_lists* out, float* beta_out, rbs_stream_t stream) {
-  rbs_status st = check_tensor(Q, "Q");
-  if (st != RBS_OK) return st;
+  // The size check needs only the shapes, so it comes first: a selection too
+  // large for the built-in buffer is refused whatever the pointers are.
+  RBS_REQUIRE(Q != nullptr && Q->batch > 0 && Q->seqlen > 0 && Q->heads > 0, RBS_ERR_INVALID_ARG,
+              "Q: null tensor or empty shape");
   RBS_REQUIRE(p != nullptr && (p->block_q == 64 || p->block_q == 128), RBS_ERR_UNSUPPORTED,
               "block_q must be 64 or 128");
   RBS_REQUIRE(kv_heads > 0 && num_kv_blocks > 0, RBS_ERR_INVALID_ARG, "empty KV shape");
-  const size_t need = (Q->batch > 0 && Q->heads > 0 && kv_heads > 0 && num_kv_blocks > 0)
-                          ? select_layout(Q->batch, Q->heads, (Q->seqlen + p->block_q - 1) / p->block_q, kv_heads,
-                                          num_kv_blocks, p->query_pool == 1).base
-                          : 0;
-  RBS_REQUIRE(need > 0 && need <= RBS_NOALLOC_SCRATCH_BYTES, RBS_ERR_CAPACITY,
+  const size_t need = select_layout(Q->batch, Q->heads, (Q->seqlen + p->block_q - 1) / p->block_q, kv_heads,
+                                    num_kv_blocks, p->query_pool == 1).base;
+  RBS_REQUIRE(need <= RBS_NOALLOC_SCRATCH_BYTES, RBS_ERR_CAPACITY,
               "this selection needs %zu bytes of scratch; the built-in buffer holds %zu (use rbs_select with a "
               "workspace)", need, static_cast<size_t>(RBS_NOALLOC_SCRATCH_BYTES));
+  rbs_status st = check_tensor(Q, "Q");
+  if (st != RBS_OK) return st;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != RBS_OK) return st;
   return rbs_select(Q, centroids, radii, kv_heads, num_kv_blocks, p, scratch, RBS_NOALLOC_SCRATCH_BYTES, out,

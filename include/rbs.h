@@ -258,8 +258,12 @@ RBS_API rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, 
  * which needs only the masks, counts and beta.  Only a selection whose masks,
  * counts and beta alone (plus the split centroids, for per-token-max query
  * scoring) exceed the buffer returns RBS_ERR_CAPACITY and launches nothing.
- * The first call on each device looks up the buffer's device address (a CUDA runtime query, no allocation); make that first call
- * before any stream capture.  All calls on a device share the one buffer:
+ * Every call looks up the buffer's address on the current device (a CUDA
+ * runtime query that allocates nothing); the first call on a device may
+ * also load the library's device code there, so make that first call before
+ * any stream capture.  The size check uses only the shapes: a selection too
+ * large for the buffer is refused before any pointer is looked at.  All
+ * calls on a device share the one buffer:
  * every scratch region is fully written before it is read, so nothing needs
  * clearing between calls, but two calls that may overlap on the GPU (other
  * streams, other host threads) race on it and must be serialised by the

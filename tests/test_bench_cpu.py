@@ -78,3 +78,53 @@ def test_attention_traffic_only_for_the_captured_build(tmp_path, monkeypatch):
     with open(tmp_path / bench.ATTN_TRAFFIC_SOURCES[0], "a") as fh:
         fh.write("\n// edited\n")
     assert bench.attn_traffic(full) is None
+
+
+def test_reference_arm_reports_the_measured_sample_time():
+    # ms_per_step is the time a step's sample took (so steps x ms_per_step
+    # fits in the run); the whole-step time extrapolated from it has its own key
+    import argparse
+    import time
+    args = argparse.Namespace(steps=2, warmup=3, ref_step_budget=3.0, ref_total_budget=2.5, seq_len=4096)
+    t0 = time.perf_counter()
+    line = bench.run_reference(args)
+    took_ms = (time.perf_counter() - t0) * 1e3
+    assert line["ms_per_step"] * (args.steps + args.warmup) <= took_ms
+    assert line["extrapolated_ms_per_full_step"] >= line["ms_per_step"]
+
+
+def test_roofline_entry_uses_the_burst_peak():
+    peaks = {"bf16_tflops": 1700.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6400.0, "source": "measured"}
+    r = bench.roofline_entry(850.0, peaks, 2.5e9)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["peak"] == 1700.0 and r["frac"] == 0.5
+    assert r["peak_sustained"] == 1400.0 and abs(r["frac_of_sustained"] - 850.0 / 1400.0) < 1e-4
+    assert r["traffic"] == 2.5e9 and "burst" in r["peak_kind"]
+
+
+def test_ttft_ratios():
+    r = bench.ttft_ratios(final_ms=0.25, reencode_ms=0.03, full_ms=10.0, final_pairs=1040, full_pairs=33930)
+    assert r["time_ratio"] == 0.025
+    assert r["time_ratio_with_reencode"] == 0.028
+    assert abs(r["flops_ratio"] - 1040 / 33930) < 1e-5
+
+
+def test_clock_sampler_leaves_no_file_in_the_repo(monkeypatch, tmp_path):
+    # without a log directory the samples go to a temporary file that is
+    # removed afterwards; nvidia-smi missing gives a labelled empty record
+    import subprocess
+
+    def no_smi(*a, **k):
+        raise OSError("no nvidia-smi")
+    monkeypatch.setattr(subprocess, "Popen", no_smi)
+    c = bench.ClockSampler(0)
+    assert not c.path.startswith(bench.ROOT)
+    c.start()
+    rec = c.stop()
+    assert rec["sm_mhz"] is None and rec["reasons"] == ["nvidia-smi unavailable"]
+    import os
+    assert not os.path.exists(c.path)
+    kept = bench.ClockSampler(0, str(tmp_path))
+    kept.start()
+    kept.stop()
+    assert os.path.exists(kept.path)

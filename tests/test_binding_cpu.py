@@ -34,3 +34,18 @@ def test_select_refuses_mismatched_stats_before_any_call():
         rbs.rbs_select(Q, C, R, p, beta_out=torch.zeros(1, 2, 3))
     with pytest.raises(TypeError, match="centroids"):
         rbs.rbs_select(Q, C, R, p)  # shapes right, but host tensors
+
+
+def test_tensors_of_one_call_must_share_a_device():
+    # the library launches on the current device: a tensor on another GPU is
+    # refused before its pointer can reach a kernel (fake device attributes:
+    # no GPU is needed to check the rule)
+    from types import SimpleNamespace
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    Q = SimpleNamespace(device=d0)
+    assert rbs._one_device("Q", Q, K=SimpleNamespace(device=d0), lse=None) == d0
+    with pytest.raises(ValueError, match="K is on cuda:1 but Q is on cuda:0"):
+        rbs._one_device("Q", Q, K=SimpleNamespace(device=d1))
+    lists = SimpleNamespace(row_ptr=SimpleNamespace(device=d0), col_idx=SimpleNamespace(device=d1), flags=None)
+    with pytest.raises(ValueError, match="lists.col_idx"):
+        rbs._one_device("Q", Q, **rbs._lists_tensors(lists))
