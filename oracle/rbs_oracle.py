@@ -463,30 +463,49 @@ def causal_full_lists(batch: int, heads_q: int, nqb: int, q_block_offset: int = 
     return np.asarray(row_ptr, dtype=np.int64), np.asarray(cols, dtype=np.int64)
 
 
+def block_attention_key_start(seg_start, final_start: int, positions) -> np.ndarray:
+    """Lowest key position each query position may attend to under the
+    Block-attention mask ([BA] 2.1 Main idea, 2.2 Block segmentation, 2.4
+    Block fine-tune): a token of passage s (seg_start[s] <= p < next start,
+    the last passage ending at final_start) sees only its own passage's
+    keys, so the bound is its passage's first token; a token of the final
+    block (p >= final_start) sees the whole prompt, bound 0.  Passage starts
+    are token offsets; nothing requires them to be block multiples."""
+    starts = [int(x) for x in seg_start]
+    assert starts[0] == 0 and all(b > a for a, b in zip(starts, starts[1:])) and final_start > starts[-1]
+    out = []
+    for p in positions:
+        p = int(p)
+        if p >= final_start:
+            out.append(0)
+        else:
+            out.append(max(a for a in starts if a <= p))
+    return np.asarray(out, dtype=np.int64)
+
+
 def block_attention_lists(seg_start, final_start: int, block: int, batch: int, heads_q: int,
                           q_first_block: int, q_num_blocks: int):
     """Block-attention mask as per-query-block lists.
 
     Segments: passage s covers tokens [seg_start[s], next start); the final
     block (the user query) starts at ``final_start`` and runs to the end.
-    A query block inside passage s sees the key blocks of passage s up to
-    itself; a query block inside the final block sees every key block up to
-    itself.  Rows cover query blocks q_first_block .. q_first_block +
+    Query block g holds tokens [g * block, (g + 1) * block); its row lists
+    every key block that holds a key one of those tokens may see: from the
+    block of the smallest key_start over its tokens (block_attention_key_start)
+    up to g itself (causal).  When passages start on block boundaries this is
+    "the key blocks of the passage up to itself" for a passage block and
+    "every key block up to itself" for a block of the final block; a block
+    that straddles a boundary lists the union of its tokens' ranges, and the
+    token-level mask (masked_attention's key_start) removes the keys of the
+    other passage.  Rows cover query blocks q_first_block .. q_first_block +
     q_num_blocks - 1 (global block indices), for every (batch, q head).
     """
-    starts = [int(s) for s in seg_start]
-    for s in starts + [final_start]:
-        assert s % block == 0
-    final_blk = final_start // block
     row_ptr = [0]
     cols = []
     for _ in range(batch * heads_q):
         for gi in range(q_first_block, q_first_block + q_num_blocks):
-            if gi >= final_blk:
-                first = 0
-            else:
-                first = max(s for s in starts if s // block <= gi) // block
-            cols.extend(range(first, gi + 1))
+            lo = block_attention_key_start(seg_start, final_start, range(gi * block, (gi + 1) * block)).min()
+            cols.extend(range(int(lo) // block, gi + 1))
             row_ptr.append(len(cols))
     return np.asarray(row_ptr, dtype=np.int64), np.asarray(cols, dtype=np.int64)
 
@@ -497,7 +516,7 @@ def block_attention_lists(seg_start, final_start: int, block: int, batch: int, h
 
 
 def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_offset: int = 0,
-                     scale: float | None = None, causal: int = 1, rows=None):
+                     scale: float | None = None, causal: int = 1, rows=None, key_start=None):
     """Softmax attention of each query token over the key tokens of its row's blocks.
 
     Q [B, Lq, Hq, d]; K, V [B, Lk, Hkv, d].  The lists hold one row per
@@ -508,7 +527,10 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
     head of q head hq is hq // (Hq / Hkv).  Returns O [B, Lq, Hq, d] (NaN for
     rows not computed) and lse [B, Hq, Lq] = log sum_s exp(scale * q.k_s).
     ``rows``: optional iterable of (b, hq, i) numbers (b * Hq + hq) * nqb + i
-    to compute (default: all).
+    to compute (default: all).  ``key_start``: optional [Lq] array, the lowest
+    key position query token t may see (the Block-attention token mask,
+    block_attention_key_start of the token's position); keys below it are
+    masked like keys after the query.
     """
     B, Lq, Hq, d = Q.shape
     Hkv = K.shape[2]
@@ -542,6 +564,9 @@ def masked_attention(Q, K, V, row_ptr, col_idx, block_q: int, block_k: int, q_of
         if causal:
             qpos = np.arange(t0, t1) + q_offset
             logits = np.where(kpos[None, :] <= qpos[:, None], logits, -np.inf)
+        if key_start is not None:
+            lo = np.asarray(key_start, dtype=np.int64)[t0:t1]
+            logits = np.where(kpos[None, :] >= lo[:, None], logits, -np.inf)
         m = logits.max(axis=1, keepdims=True)
         m = np.where(np.isfinite(m), m, 0.0)
         w = np.exp(logits - m)

@@ -917,3 +917,74 @@ def test_token_max_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "token_max_scores", norm_of_mean)
     with pytest.raises(AssertionError):
         test_token_max_bounds()
+
+
+# --------------------------------------------------------------------------
+# Block-attention with passage boundaries inside blocks: the token-level mask
+
+
+def _token_mask_golden():
+    g = {"list": {}, "mask": {}}
+    for line in open(os.path.join(GOLDEN, "block_attention_token_mask_tiny.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("key_start:"):
+            g["key_start"] = [int(x) for x in line.split(":")[1].split()]
+            continue
+        kind, rest = line.split(" ", 1)
+        idx, val = rest.split(":")
+        g[kind][int(idx)] = val.split() if kind == "list" else val.strip()
+    return g
+
+
+def test_block_attention_token_mask_golden():
+    g = _token_mask_golden()
+    seg, final = [0, 6, 9], 13
+    assert O.block_attention_key_start(seg, final, range(16)).tolist() == g["key_start"]
+    rp, ci = O.block_attention_lists(seg, final, 4, 1, 1, 0, 4)
+    for i in range(4):
+        assert ci[rp[i]:rp[i + 1]].tolist() == [int(x) for x in g["list"][i]]
+    # masked_attention on those lists with the token bound equals a direct
+    # softmax over the hand-enumerated visibility matrix
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal((1, 16, 2, 128))
+    k = rng.standard_normal((1, 16, 1, 128))
+    v = rng.standard_normal((1, 16, 1, 128))
+    got, _ = O.masked_attention(q, k, v, np.concatenate([rp, rp[-1] + rp[1:]]), np.concatenate([ci, ci]), 4, 4,
+                                key_start=g["key_start"])
+    vis = np.array([[c == "1" for c in g["mask"][t]] for t in range(16)])
+    for h in range(2):
+        s = (q[0, :, h] @ k[0, :, 0].T) / math.sqrt(128)
+        s = np.where(vis, s, -np.inf)
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        ref = (w / w.sum(axis=1, keepdims=True)) @ v[0, :, 0]
+        np.testing.assert_allclose(got[0, :, h], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_ragged_passages_are_independent_and_need_the_token_mask():
+    # passages of 100, 37 and 91 tokens and a 29-token final block, 32-token
+    # blocks: every passage boundary falls inside a key block
+    lens, blk = [100, 37, 91], 32
+    inp = make_block_attention(final_len=29, Hq=2, Hkv=1, block=blk, seed=42, passage_lens=lens)
+    other = make_block_attention(final_len=29, Hq=2, Hkv=1, block=blk, seed=43, passage_lens=lens)
+    seg, final = inp["seg_start"], inp["final_start"]
+    L = inp["Q"].shape[1]
+    nqb = -(-L // blk)
+    rp, ci = O.block_attention_lists(seg, final, blk, 1, 2, 0, nqb)
+    ks = O.block_attention_key_start(seg, final, range(L))
+    base, _ = O.masked_attention(inp["Q"], inp["K"], inp["V"], rp, ci, blk, blk, key_start=ks)
+    a, e = 100, 137  # passage 1
+    Q2, K2, V2 = other["Q"].copy(), other["K"].copy(), other["V"].copy()
+    Q2[:, a:e], K2[:, a:e], V2[:, a:e] = inp["Q"][:, a:e], inp["K"][:, a:e], inp["V"][:, a:e]
+    out2, _ = O.masked_attention(Q2, K2, V2, rp, ci, blk, blk, key_start=ks)
+    assert np.array_equal(base[:, a:e], out2[:, a:e])  # passage 1 unchanged, bit for bit
+    assert not np.allclose(base[:, final:], out2[:, final:])  # the final block sees everything
+    # a plausible mistake -- the block lists without the token bound -- lets
+    # passage 1 see the keys of passage 0 that share its first key block
+    bad, _ = O.masked_attention(inp["Q"], inp["K"], inp["V"], rp, ci, blk, blk)
+    bad2, _ = O.masked_attention(Q2, K2, V2, rp, ci, blk, blk)
+    assert not np.allclose(bad[:, a:e], bad2[:, a:e])
+    # block-aligned passages give the same lists with or without the bound
+    rp0, ci0 = O.block_attention_lists([0, 64], 128, blk, 1, 1, 0, 5)
+    assert ci0.tolist() == [0, 0, 1, 2, 2, 3, 0, 1, 2, 3, 4]

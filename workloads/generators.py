@@ -188,25 +188,30 @@ def make_mixture(L: int, Hq: int, Hkv: int, block: int = 128, seed: int = SEED_B
 
 
 def make_block_attention(passages: int = 16, passage_len: int = 2048, final_len: int = 512, Hq: int = 32,
-                         Hkv: int = 8, block: int = 128, seed: int = SEED_BASE + 3, batch: int = 1) -> dict:
+                         Hkv: int = 8, block: int = 128, seed: int = SEED_BASE + 3, batch: int = 1,
+                         passage_lens=None) -> dict:
     """RAG-shaped Block-attention workload: un-rotated Q/K/V ~ N(0,1) and the segment table.
 
-    Tokens [p*passage_len, (p+1)*passage_len) form passage p; the final block
-    (the user query) starts at passages*passage_len.  ``local_pos`` is each
-    token's position inside its own passage (the position its cached key was
-    encoded at); ``global_pos`` is its position in the assembled prompt.
+    Passage p covers its own run of tokens: passage_len each, or the lengths
+    in ``passage_lens`` (any token counts, not necessarily block multiples),
+    one after the other; the final block (the user query) follows them.
+    ``local_pos`` is each token's position inside its own passage (the
+    position its cached key was encoded at); ``global_pos`` is its position
+    in the assembled prompt.
     """
     d = HEAD_DIM
-    L = passages * passage_len + final_len
+    lens = [int(x) for x in passage_lens] if passage_lens is not None else [passage_len] * passages
+    seg_start = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int32)
+    final_start = int(sum(lens))
+    L = final_start + final_len
     rng = np.random.Generator(np.random.PCG64(seed))
     Q = _normal_bf16(rng, (batch, L, Hq, d))
     K = _normal_bf16(rng, (batch, L, Hkv, d))
     V = _normal_bf16(rng, (batch, L, Hkv, d))
-    seg_start = np.arange(passages, dtype=np.int32) * passage_len
-    final_start = passages * passage_len
     global_pos = np.arange(L, dtype=np.int32)
     local_pos = global_pos.copy()
-    local_pos[:final_start] = global_pos[:final_start] % passage_len
+    for a, n in zip(seg_start, lens):
+        local_pos[a:a + n] = np.arange(n, dtype=np.int32)
     return {"Q": Q, "K": K, "V": V, "seg_start": seg_start, "final_start": final_start,
             "local_pos": local_pos, "global_pos": global_pos, "block": block}
 
