@@ -32,7 +32,8 @@ from ._abi import (  # noqa: F401
 __all__ = [
     "SelectParams", "BlockLists", "rbs_block_stats", "rbs_block_beta", "rbs_pool_queries", "rbs_select",
     "rbs_select_capacity", "rbs_select_workspace_bytes", "rbs_lists_causal_full", "rbs_lists_block_attention",
-    "bsa_prefill", "rope_reencode", "rbs_get_device_error", "RbsError",
+    "bsa_prefill", "bsa_prefill_rescue_weighted", "bsa_prefill_segments", "rope_reencode", "rbs_get_device_error",
+    "RbsError",
 ]
 
 
@@ -299,6 +300,31 @@ def bsa_prefill_rescue_weighted(Q: torch.Tensor, K: torch.Tensor, V: torch.Tenso
             ctypes.byref(tQ), ctypes.byref(tK), ctypes.byref(tV), ctypes.byref(lc), block_q, block_k, q_offset, scale,
             1 if causal else 0, float(rescue_weight), ctypes.byref(tO), lse.data_ptr() if lse is not None else None,
             _stream()), "bsa_prefill_rescue_weighted")
+    return (out, lse) if return_lse else out
+
+
+def bsa_prefill_segments(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, lists: BlockLists, seg_start,
+                         final_start: int, block_q: int = 128, block_k: int = 128, q_offset: int = 0,
+                         softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                         return_lse: bool = False):
+    """bsa_prefill with the Block-attention mask applied token by token: a query
+    token of a passage sees only its own passage's earlier keys, a token of the
+    final block every earlier key (passage starts may be any token offsets)."""
+    if out is None:
+        out = torch.empty_like(Q)
+    lse = None
+    if return_lse:
+        lse = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], dtype=torch.float32, device=Q.device)
+    scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(Q.shape[-1])
+    seg = (ctypes.c_int32 * len(seg_start))(*[int(s) for s in seg_start])
+    lc = lists.c()
+    tQ, tK, tV, tO = _t(Q, "Q"), _t(K, "K"), _t(V, "V"), _t(out, "O")
+    dev = _one_device("Q", Q, K=K, V=V, out=out, lse=lse, **_lists_tensors(lists))
+    with torch.cuda.device(dev):
+        check(lib().bsa_prefill_segments(ctypes.byref(tQ), ctypes.byref(tK), ctypes.byref(tV), ctypes.byref(lc),
+                                         block_q, block_k, q_offset, seg, len(seg_start), int(final_start), scale,
+                                         ctypes.byref(tO), lse.data_ptr() if lse is not None else None, _stream()),
+              "bsa_prefill_segments")
     return (out, lse) if return_lse else out
 
 

@@ -67,7 +67,12 @@ SIGNATURES = {
                                    i32, P(Bf16Tensor), vp, vp]),
     "bsa_prefill_rescue_weighted": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), P(Bf16Tensor), P(BlockListsC), i32,
                                                    i32, i64, f32, i32, f32, P(Bf16Tensor), vp, vp]),
+    "bsa_prefill_segments": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), P(Bf16Tensor), P(BlockListsC), i32, i32,
+                                            i64, P(i32), i32, i32, f32, P(Bf16Tensor), vp, vp]),
     "rope_reencode": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), vp, vp, f32, i32, vp]),
+    "rbs_testing_bsa_prefill_stalled": (ctypes.c_int, [P(Bf16Tensor), P(Bf16Tensor), P(Bf16Tensor), P(BlockListsC),
+                                                       i32, i32, ctypes.c_uint64, i32, P(Bf16Tensor), vp]),
+    "rbs_testing_exp2": (ctypes.c_int, [vp, vp, i64, vp]),
 }
 
 
@@ -77,7 +82,7 @@ class RbsError(RuntimeError):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
 
 
-ABI_VERSION = 4  # RBS_ABI_VERSION of include/rbs.h that these structures match
+ABI_VERSION = 5  # RBS_ABI_VERSION of include/rbs.h that these structures match
 _lib = None
 
 

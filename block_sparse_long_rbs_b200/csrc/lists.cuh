@@ -2,8 +2,11 @@
 // point), and the Block-attention mask ([BA] 2.1 Main idea, 2.2 Block
 // segmentation, 2.4 Block fine-tune): a query block of passage s sees the key
 // blocks of passage s up to itself, a query block of the final block sees
-// every key block up to itself.  Row pointers are closed forms, so one warp
-// per row writes its own entries with no scan.
+// every key block up to itself.  Passages may start at any token: a query
+// block then lists every key block holding a key one of its tokens may see,
+// and bsa_prefill_segments masks the other passages' keys token by token.
+// Row pointers are closed forms, so one warp per row writes its own entries
+// with no scan.
 #pragma once
 
 #include "common.cuh"
@@ -31,33 +34,46 @@ __global__ void __launch_bounds__(256) lists_causal_full_kernel(int rows, int nq
 }
 
 struct SegmentTable {
-  int n;                           // passages
-  int final_blk;                   // first block of the final block
-  int start_blk[RBS_MAX_SEGMENTS];  // first block of each passage, ascending, start_blk[0] == 0
+  int n;                            // passages
+  int block;                        // block size (tokens)
+  int final_start;                  // first token of the final block
+  int start_tok[RBS_MAX_SEGMENTS];  // first token of each passage, ascending, start_tok[0] == 0
 };
 
-// First visible key block of global query block g.
+// First visible key block of global query block g: the block of the smallest
+// first-visible-key over g's tokens.  Its first token carries the smallest
+// passage start; a block holding a token of the final block sees key 0.
 __device__ __forceinline__ int ba_first(const SegmentTable& s, int g) {
-  if (g >= s.final_blk) return 0;
-  int lo = 0, hi = s.n - 1;  // last passage whose start <= g
+  if (static_cast<int64_t>(g + 1) * s.block > s.final_start) return 0;
+  const int64_t p = static_cast<int64_t>(g) * s.block;
+  int lo = 0, hi = s.n - 1;  // last passage whose start <= p
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s.start_blk[mid] <= g) lo = mid; else hi = mid - 1;
+    if (s.start_tok[mid] <= p) lo = mid; else hi = mid - 1;
   }
-  return s.start_blk[lo];
+  return s.start_tok[lo] / s.block;
 }
 
-// Entries of global query blocks 0 .. x-1 (one head).
-__device__ __forceinline__ int64_t ba_prefix(const SegmentTable& s, int x) {
+// Entries of global query blocks 0 .. x-1 (one head): the sum over g < x of
+// g - ba_first(g) + 1, in closed form per passage.  Passage s owns the query
+// blocks whose first token it holds, g in [ceil(a_s / B), ceil(a_{s+1} / B)),
+// each listing from block floor(a_s / B); blocks from floor(final_start / B)
+// on hold a token of the final block and list from block 0.
+__device__ __host__ __forceinline__ int64_t ba_prefix(const SegmentTable& s, int64_t x) {
+  const int64_t B = s.block;
+  const int64_t fb = s.final_start / B;
+  const int64_t cap = x < fb ? x : fb;
   int64_t tot = 0;
   for (int p = 0; p < s.n; ++p) {
-    const int a = s.start_blk[p];
-    const int e = p + 1 < s.n ? s.start_blk[p + 1] : s.final_blk;
-    const int64_t m = static_cast<int64_t>(min(max(x, a), e) - a);
-    tot += m * (m + 1) / 2;
+    const int64_t a = s.start_tok[p];
+    const int64_t e = p + 1 < s.n ? s.start_tok[p + 1] : s.final_start;
+    int64_t lo = (a + B - 1) / B, hi = (e + B - 1) / B;
+    if (hi > cap) hi = cap;
+    if (hi <= lo) continue;
+    const int64_t f = a / B;
+    tot += (hi * (hi + 1) / 2 - lo * (lo + 1) / 2) - f * (hi - lo);
   }
-  const int64_t mf = static_cast<int64_t>(max(0, x - s.final_blk));
-  tot += mf * (s.final_blk + 1) + mf * (mf - 1) / 2;
+  if (x > fb) tot += x * (x + 1) / 2 - fb * (fb + 1) / 2;
   return tot;
 }
 

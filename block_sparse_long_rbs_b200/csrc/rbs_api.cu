@@ -50,6 +50,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   int sms = 0;
   bool attrs_set = false;
+  bool attn_regs_ok = false;  // the attention kernels' register split fits their launch
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -103,6 +104,17 @@ rbs_status device_info(DeviceInfo** out) {
                                        static_cast<int>(topk_smem_bytes(kTokMaxKV, kTokMaxKV / 32)));
     e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
     if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    // The attention kernels move registers between warpgroups at run time:
+    // the block must be launched with at least the split's total, or the
+    // softmax warpgroups would wait for registers that never come.
+    d.attn_regs_ok = true;
+    for (const void* kern : {reinterpret_cast<const void*>(bsa_prefill_kernel<128, 128>),
+                             reinterpret_cast<const void*>(bsa_prefill_kernel<64, 64>)}) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+          static_cast<uint32_t>(fa.numRegs) * kAttnThreads < kRegsSplitTotal)
+        d.attn_regs_ok = false;
+    }
     d.attrs_set = true;
   }
   *out = &d;
@@ -799,6 +811,9 @@ rbs_status rbs_lists_causal_full(int32_t batch, int32_t heads_q, int32_t num_q_b
 }
 
 namespace {
+// Passage starts (host array) -> the device segment table.  Starts are token
+// offsets in any position: ascending, the first 0, the final block after the
+// last passage.
 rbs_status segment_table(const int32_t* seg_start, int32_t num_segments, int32_t final_start, int32_t block,
                          SegmentTable* t) {
   RBS_REQUIRE(seg_start != nullptr && num_segments > 0 && num_segments <= RBS_MAX_SEGMENTS, RBS_ERR_INVALID_ARG,
@@ -806,28 +821,15 @@ rbs_status segment_table(const int32_t* seg_start, int32_t num_segments, int32_t
   RBS_REQUIRE(block == 64 || block == 128, RBS_ERR_UNSUPPORTED, "block must be 64 or 128");
   RBS_REQUIRE(seg_start[0] == 0, RBS_ERR_INVALID_ARG, "seg_start[0] must be 0");
   t->n = num_segments;
+  t->block = block;
   for (int s = 0; s < num_segments; ++s) {
-    RBS_REQUIRE(seg_start[s] % block == 0, RBS_ERR_UNSUPPORTED, "segment start %d not a multiple of block", seg_start[s]);
     RBS_REQUIRE(s == 0 || seg_start[s] > seg_start[s - 1], RBS_ERR_INVALID_ARG, "segment starts must ascend");
-    t->start_blk[s] = seg_start[s] / block;
+    t->start_tok[s] = seg_start[s];
   }
-  RBS_REQUIRE(final_start % block == 0 && final_start > seg_start[num_segments - 1], RBS_ERR_INVALID_ARG,
-              "final_start must be a block multiple after the last passage");
-  t->final_blk = final_start / block;
+  RBS_REQUIRE(final_start > seg_start[num_segments - 1], RBS_ERR_INVALID_ARG,
+              "final_start must come after the last passage start");
+  t->final_start = final_start;
   return RBS_OK;
-}
-
-int64_t ba_prefix_host(const SegmentTable& s, int64_t x) {
-  int64_t tot = 0;
-  for (int p = 0; p < s.n; ++p) {
-    const int64_t a = s.start_blk[p];
-    const int64_t e = p + 1 < s.n ? s.start_blk[p + 1] : s.final_blk;
-    const int64_t m = std::min(std::max(x, a), e) - a;
-    tot += m * (m + 1) / 2;
-  }
-  const int64_t mf = std::max<int64_t>(0, x - s.final_blk);
-  tot += mf * (s.final_blk + 1) + mf * (mf - 1) / 2;
-  return tot;
 }
 }  // namespace
 
@@ -838,7 +840,7 @@ int64_t rbs_lists_block_attention_nnz(const int32_t* seg_start, int32_t num_segm
   if (segment_table(seg_start, num_segments, final_start, block, &t) != RBS_OK) return -1;
   if (batch <= 0 || heads_q <= 0 || q_first_block < 0 || q_num_blocks <= 0) return -1;
   return static_cast<int64_t>(batch) * heads_q *
-         (ba_prefix_host(t, q_first_block + q_num_blocks) - ba_prefix_host(t, q_first_block));
+         (ba_prefix(t, static_cast<int64_t>(q_first_block) + q_num_blocks) - ba_prefix(t, q_first_block));
 }
 
 rbs_status rbs_lists_block_attention(const int32_t* seg_start, int32_t num_segments, int32_t final_start,
@@ -867,10 +869,19 @@ namespace {
 
 // bsa_prefill and its rescue-weighted form: flags == nullptr gives every
 // block weight 1; otherwise rescue-only entries get log2(w) = rescue_bias.
+// Extra controls of one attention launch: the Block-attention segment mask
+// (null: none) and, for the library's own tests, the wait limit and a
+// producer that stops early.
+struct BsaExtra {
+  const SegmentTable* seg = nullptr;
+  uint64_t wait_ns = kWaitLimitNs;
+  int stall_after = -1;
+};
+
 rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
                       const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
                       float softmax_scale, int32_t causal, const uint8_t* flags, float rescue_bias,
-                      rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
+                      rbs_bf16_tensor* O, float* lse, rbs_stream_t stream, const BsaExtra& ex = BsaExtra()) {
   rbs_status st;
   if ((st = check_tensor(Q, "Q")) != RBS_OK) return st;
   if ((st = check_tensor(K, "K")) != RBS_OK) return st;
@@ -890,6 +901,8 @@ rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const 
   if ((st = check_lists(lists, group_lists ? Q->batch * K->heads * nqb : rows)) != RBS_OK) return st;
   DeviceInfo* di;
   if ((st = device_info(&di)) != RBS_OK) return st;
+  RBS_REQUIRE(di->attn_regs_ok, RBS_ERR_UNSUPPORTED,
+              "this build's attention kernel has fewer registers per thread than its warpgroup split needs");
 
   AttnArgs a;
   int siq = 0, sik = 0, siv = 0;
@@ -921,7 +934,17 @@ rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const 
   a.rescue_bias = rescue_bias;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(RBS_HEAD_DIM));
   a.scale_log2 = scale * 1.4426950408889634f;
-  const int grid = static_cast<int>(std::min<int64_t>(rows, di->sms));
+  a.wait_ns = ex.wait_ns;
+  a.stall_after = ex.stall_after;
+  a.seg_n = 0;
+  a.seg_final = 0;
+  if (ex.seg != nullptr) {
+    a.seg_n = ex.seg->n;
+    a.seg_final = ex.seg->final_start;
+    for (int k = 0; k < ex.seg->n; ++k) a.seg_start[k] = ex.seg->start_tok[k];
+  }
+  // persistent: one CTA per SM, each taking pairs of rows
+  const int grid = static_cast<int>(std::min<int64_t>((rows + 1) / 2, di->sms));
   if (block_q == 128)
     bsa_prefill_kernel<128, 128><<<grid, kAttnThreads, AttnSmem<128>::kAlloc, stream>>>(a);
   else
@@ -952,6 +975,38 @@ rbs_status bsa_prefill_rescue_weighted(const rbs_bf16_tensor* Q, const rbs_bf16_
   const float bias = rescue_weight > 0.f ? std::log2(rescue_weight) : -INFINITY;
   return launch_bsa(Q, K, V, lists, block_q, block_k, q_offset, softmax_scale, causal, lists->flags, bias, O, lse,
                     stream);
+}
+
+rbs_status bsa_prefill_segments(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                                const rbs_block_lists* lists, int32_t block_q, int32_t block_k, int64_t q_offset,
+                                const int32_t* seg_start, int32_t num_segments, int32_t final_start,
+                                float softmax_scale, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream) {
+  SegmentTable t;
+  const rbs_status st = segment_table(seg_start, num_segments, final_start, block_k, &t);
+  if (st != RBS_OK) return st;
+  BsaExtra ex;
+  ex.seg = &t;
+  return launch_bsa(Q, K, V, lists, block_q, block_k, q_offset, softmax_scale, 1, nullptr, 0.f, O, lse, stream, ex);
+}
+
+rbs_status rbs_testing_bsa_prefill_stalled(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K,
+                                           const rbs_bf16_tensor* V, const rbs_block_lists* lists, int32_t block_q,
+                                           int32_t block_k, uint64_t wait_ns, int32_t stall_after,
+                                           rbs_bf16_tensor* O, rbs_stream_t stream) {
+  RBS_REQUIRE(wait_ns >= 100000ull && wait_ns <= kWaitLimitNs, RBS_ERR_INVALID_ARG,
+              "wait_ns must be in [1e5, %llu]", static_cast<unsigned long long>(kWaitLimitNs));
+  RBS_REQUIRE(stall_after >= 0, RBS_ERR_INVALID_ARG, "stall_after must be >= 0");
+  BsaExtra ex;
+  ex.wait_ns = wait_ns;
+  ex.stall_after = stall_after;
+  return launch_bsa(Q, K, V, lists, block_q, block_k, 0, 0.f, 1, nullptr, 0.f, O, nullptr, stream, ex);
+}
+
+rbs_status rbs_testing_exp2(const float* x, float* y, int64_t n, rbs_stream_t stream) {
+  RBS_REQUIRE(x != nullptr && y != nullptr && n > 0 && n < (1ll << 31), RBS_ERR_INVALID_ARG, "bad exp2 test buffers");
+  const int64_t pairs = (n + 1) / 2;
+  exp2_test_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, stream>>>(x, y, n);
+  return check_launch("exp2_test_kernel");
 }
 
 // ---------------------------------------------------------------------------

@@ -59,7 +59,7 @@ extern "C" {
 #define RBS_API
 #endif
 
-#define RBS_ABI_VERSION 4
+#define RBS_ABI_VERSION 5
 #define RBS_HEAD_DIM 128
 #define RBS_MAX_SEGMENTS 512 /* Block-attention segments per call */
 #define RBS_MAX_KV_BLOCKS 4096 /* key blocks per sequence for rbs_select */
@@ -287,8 +287,12 @@ RBS_API rbs_status rbs_lists_causal_full(int32_t batch, int32_t heads_q, int32_t
  * the final block lists every key block up to itself.  Rows are query blocks
  * q_first_block .. q_first_block + q_num_blocks - 1 (global block indices) of
  * every (batch, q head).  seg_start is a HOST array of num_segments <=
- * RBS_MAX_SEGMENTS ascending token offsets, seg_start[0] == 0, every offset
- * and final_start a multiple of block. */
+ * RBS_MAX_SEGMENTS ascending token offsets, seg_start[0] == 0, final_start
+ * after the last of them.  Offsets need not be block multiples: a query
+ * block then lists every key block holding a key one of its tokens may see
+ * (from the block of the smallest passage start among its tokens, or block
+ * 0 when it holds a token of the final block), and bsa_prefill_segments
+ * applies the mask token by token. */
 RBS_API int64_t rbs_lists_block_attention_nnz(const int32_t* seg_start, int32_t num_segments, int32_t final_start,
                                       int32_t block, int32_t batch, int32_t heads_q, int32_t q_first_block,
                                       int32_t q_num_blocks);
@@ -342,6 +346,28 @@ RBS_API rbs_status bsa_prefill_rescue_weighted(const rbs_bf16_tensor* Q, const r
                                        int32_t block_k, int64_t q_offset, float softmax_scale, int32_t causal,
                                        float rescue_weight, rbs_bf16_tensor* O, float* lse, rbs_stream_t stream);
 
+/* ---- Block-attention with passages at any token offset  ([BA] 2.2 Block
+ * segmentation: each retrieved passage is a block, the user query is the
+ * final block; 2.4 Block fine-tune: a token of a passage attends only to
+ * earlier tokens of its own passage, a token of the final block to every
+ * earlier token)
+ * bsa_prefill with the Block-attention mask applied token by token: the
+ * query token at key position p = t + q_offset sees key s when
+ *   lo(p) <= s <= p,  lo(p) = the last seg_start <= p   (p < final_start)
+ *                     lo(p) = 0                          (p >= final_start).
+ * seg_start / num_segments / final_start as for rbs_lists_block_attention
+ * (a HOST array; offsets need not be block multiples), and lists must hold
+ * every key block a row's tokens may see (rbs_lists_block_attention with the
+ * same segments builds them: a query block straddling a passage boundary
+ * lists both passages' blocks and the bound above removes the keys its
+ * tokens may not see).  Always causal.  Other arguments, layouts and errors
+ * as bsa_prefill. */
+RBS_API rbs_status bsa_prefill_segments(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const rbs_bf16_tensor* V,
+                                        const rbs_block_lists* lists, int32_t block_q, int32_t block_k,
+                                        int64_t q_offset, const int32_t* seg_start, int32_t num_segments,
+                                        int32_t final_start, float softmax_scale, rbs_bf16_tensor* O, float* lse,
+                                        rbs_stream_t stream);
+
 /* ---- RoPE position re-encoding  ([BA] 2.3 Position re-encoding, 2.5 Inference)
  * Keys cached with RoPE at old_pos are moved to new_pos: the rotation is reset
  * to position 0 and applied again at the new position, done as one rotation by
@@ -354,6 +380,22 @@ RBS_API rbs_status bsa_prefill_rescue_weighted(const rbs_bf16_tensor* Q, const r
  * Re-encoding from old_pos = 0 is plain RoPE encoding. */
 RBS_API rbs_status rope_reencode(const rbs_bf16_tensor* x_in, rbs_bf16_tensor* x_out, const int32_t* old_pos,
                          const int32_t* new_pos, float theta, int32_t rope_style, rbs_stream_t stream);
+
+/* ---- testing hooks (no counterpart in the papers; used by the library's
+ * own tests to reach code paths that correct inputs never reach)
+ * rbs_testing_bsa_prefill_stalled: bsa_prefill (causal, default scale, no
+ *   LSE) with every pipeline wait limited to wait_ns (1e5 .. 2e9 ns; the
+ *   product limit is 2e9) and the K/Q producer stopping for good after
+ *   stall_after key tiles.  The waits for the tiles never loaded run out:
+ *   the kernel must set RBS_DEVERR_TIMEOUT, leave no copy or MMA in flight,
+ *   free its tensor memory and return.  O is left partly written.
+ * rbs_testing_exp2: y[i] = the attention kernel's software base-2
+ *   exponential (the FMA-pipe polynomial) of x[i], n values (device). */
+RBS_API rbs_status rbs_testing_bsa_prefill_stalled(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K,
+                                                   const rbs_bf16_tensor* V, const rbs_block_lists* lists,
+                                                   int32_t block_q, int32_t block_k, uint64_t wait_ns,
+                                                   int32_t stall_after, rbs_bf16_tensor* O, rbs_stream_t stream);
+RBS_API rbs_status rbs_testing_exp2(const float* x, float* y, int64_t n, rbs_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_housekeeping(L):
-    assert L.rbs_abi_version() == 4
+    assert L.rbs_abi_version() == 5
     assert L.rbs_status_string(0) == b"ok"
     assert L.rbs_status_string(3) == b"capacity"
     p = _abi.SelectParamsC()
@@ -84,10 +84,31 @@ def test_block_attention_nnz_matches_oracle(L):
 
 
 def test_block_attention_rejects_bad_segments(L):
-    bad = (ctypes.c_int32 * 2)(0, 100)  # not a block multiple
-    assert L.rbs_lists_block_attention_nnz(bad, 2, 512, 128, 1, 1, 0, 4) == -1
     desc = (ctypes.c_int32 * 2)(128, 256)  # does not start at 0
     assert L.rbs_lists_block_attention_nnz(desc, 2, 512, 128, 1, 1, 0, 4) == -1
+    down = (ctypes.c_int32 * 3)(0, 300, 200)  # not ascending
+    assert L.rbs_lists_block_attention_nnz(down, 3, 512, 128, 1, 1, 0, 4) == -1
+    late = (ctypes.c_int32 * 2)(0, 600)  # final block before the last passage
+    assert L.rbs_lists_block_attention_nnz(late, 2, 512, 128, 1, 1, 0, 6) == -1
+
+
+def test_block_attention_nnz_with_ragged_passages(L):
+    # passage starts at any token offset: the library's closed-form row
+    # offsets equal the oracle builder's entry counts
+    rng = np.random.default_rng(77)
+    cases = [([0, 1999, 4099], 4616, 128), ([0, 100, 137], 228, 32), ([0, 6, 9], 13, 4)]
+    for _ in range(20):
+        n = int(rng.integers(1, 8))
+        starts = np.concatenate([[0], np.sort(rng.choice(np.arange(1, 3000), n - 1, replace=False))]).tolist()
+        cases.append((starts, starts[-1] + int(rng.integers(1, 700)), int(rng.choice([64, 128]))))
+    for seg, final, blk in cases:
+        if blk not in (64, 128):
+            continue
+        arr = (ctypes.c_int32 * len(seg))(*seg)
+        nqb = -(-(final + 300) // blk)
+        for first, num in ((0, nqb), (final // blk, nqb - final // blk), (1, max(1, nqb // 2))):
+            rp, ci = O.block_attention_lists(seg, final, blk, 2, 3, first, num)
+            assert L.rbs_lists_block_attention_nnz(arr, len(seg), final, blk, 2, 3, first, num) == ci.size
 
 
 def _fake(B=1, Lq=256, H=2, D=128, sb=None, ss=None, sh=None, ptr=0x10000):
