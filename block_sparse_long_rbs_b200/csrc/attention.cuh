@@ -101,7 +101,7 @@ static_assert(kRegsSplitTotal <= kAttnThreads * kRegsLaunch, "register split");
 // Cody-Waite range reduction 2^x = 2^n * 2^f, n = rint(x) (via the 1.5*2^23
 // shifter), f = x - n in [-1/2, 1/2], then p(f) = 1 + c1 f + c2 f^2 + c3 f^3,
 // a degree-3 fit by the Remez exchange algorithm for minimum relative error
-// (max 4.3e-4; csrc/exp2_poly_fit.py derives the coefficients).  The
+// (max 4.315e-4; csrc/exp2_poly_fit.py derives the coefficients).  The
 // exponent n is added to p's exponent field.  Inputs are clamped at -127, where
 // the result is +0 (p(0) = 1 exactly); inputs above 127 are not expected
 // (the running max keeps them at or below 8).  Below -126 the sum leaves the

@@ -9,7 +9,7 @@ involved: the missing tiles are simply never requested.
 
 The attention kernel's FMA-pipe exponential (a degree-3 Remez fit after
 Cody-Waite range reduction) is checked against exp2 in float64 within its
-fitted relative error."""
+fitted relative error (4.315e-4 by the Remez fit, plus fp32 rounding)."""
 
 import ctypes
 
@@ -86,7 +86,9 @@ def test_software_exp2_within_its_fitted_bound(cuda_ok):
     ref = np.exp2(x.astype(np.float64))
     normal = x >= -126.0
     rel = np.abs(got[normal] - ref[normal]) / ref[normal]
-    assert rel.max() <= 4.3e-4 + 2e-7, rel.max()  # the fit's bound plus fp32 rounding
+    # the fit's maximum relative error (4.315e-4, csrc/exp2_poly_fit.py) plus
+    # the fp32 rounding of the evaluation
+    assert rel.max() <= 4.315e-4 + 5e-7, rel.max()
     # below the normal range the result is only close in absolute terms
     assert np.all(np.abs(got[~normal] - ref[~normal]) <= 2.0 ** -126)
     assert np.all(got[x <= -127.0] == 0.0)
