@@ -97,7 +97,9 @@ def o_rows_close(O_gpu: torch.Tensor, O_ref: np.ndarray, rows, Hq: int, nqb: int
         b, rem = divmod(int(row), Hq * nqb)
         hq, i = divmod(rem, nqb)
         sl = slice(i * block_q, (i + 1) * block_q)
-        d = np.abs(og[b, sl, hq] - O_ref[b, sl, hq]).max()
-        worst = max(worst, float(d))
+        a, r = og[b, sl, hq], O_ref[b, sl, hq]
+        # a NaN on either side is a failure, not a silently skipped comparison
+        assert np.all(np.isfinite(a)) and np.all(np.isfinite(r)), f"non-finite output in row {row}"
+        worst = max(worst, float(np.abs(a - r).max()))
     assert worst <= tol, f"max |O_gpu - O_oracle| = {worst}"
     return worst

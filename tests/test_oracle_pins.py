@@ -988,3 +988,16 @@ def test_ragged_passages_are_independent_and_need_the_token_mask():
     # block-aligned passages give the same lists with or without the bound
     rp0, ci0 = O.block_attention_lists([0, 64], 128, blk, 1, 1, 0, 5)
     assert ci0.tolist() == [0, 0, 1, 2, 2, 3, 0, 1, 2, 3, 4]
+
+
+def test_mixture_generator_fills_a_ragged_tail():
+    # a prompt that is not a block multiple gets a last, shorter key block of
+    # real values (no uninitialised memory), and a block-multiple prompt is the
+    # same whether or not a longer tail exists elsewhere
+    rag = make_mixture(L=2048 + 77, Hq=4, Hkv=2, block=128, seed=61)
+    k = O.bf16_to_f64(rag["K"])
+    assert np.all(np.isfinite(k)) and np.abs(k).max() < 100.0
+    assert all(q_tok < 2048 + 77 for (_, _, _, _, _, q_tok) in rag["plants"])
+    a = make_mixture(L=2048, Hq=4, Hkv=2, block=128, seed=62)
+    b = make_mixture(L=2048, Hq=4, Hkv=2, block=128, seed=62)
+    assert np.array_equal(a["K"], b["K"]) and np.array_equal(a["Q"], b["Q"])

@@ -154,7 +154,7 @@ def make_mixture(L: int, Hq: int, Hkv: int, block: int = 128, seed: int = SEED_B
     uniform q head of the KV group.  Q and V are N(0, 1).
     """
     d = HEAD_DIM
-    nb = L // block
+    nb = -(-L // block)  # a last, shorter block when L is not a block multiple
     G = Hq // Hkv
     rng = np.random.Generator(np.random.PCG64(seed))
     Q = _normal_bf16(rng, (batch, L, Hq, d))
@@ -169,7 +169,8 @@ def make_mixture(L: int, Hq: int, Hkv: int, block: int = 128, seed: int = SEED_B
             eps = eps.reshape(j1 - j0, block, Hkv, d)
             mu = centres[b, :, j0:j1].transpose(1, 0, 2)[:, None, :, :]
             sg = sigma[b, :, j0:j1].transpose(1, 0)[:, None, :, None]
-            K[b, j0 * block:j1 * block] = f32_to_bf16_bits((mu + sg * eps).reshape(-1, Hkv, d))
+            t1 = min(L, j1 * block)
+            K[b, j0 * block:t1] = f32_to_bf16_bits((mu + sg * eps).reshape(-1, Hkv, d)[:t1 - j0 * block])
     V = _normal_bf16(rng, (batch, L, Hkv, d))
     plants = []
     for b in range(batch):
@@ -180,7 +181,7 @@ def make_mixture(L: int, Hq: int, Hkv: int, block: int = 128, seed: int = SEED_B
                 for _ in range(int(rng.integers(1, max_plants + 1))):
                     pos_k = j * block + int(rng.integers(0, block))
                     qi = int(rng.integers(j + 1, nb))
-                    q_tok = qi * block + int(rng.integers(0, block))
+                    q_tok = qi * block + int(rng.integers(0, min(block, L - qi * block)))
                     q_head = h * G + int(rng.integers(0, G))
                     _plant(K, Q, b, h, pos_k, q_tok, q_head, logit)
                     plants.append((b, h, j, pos_k, q_head, q_tok))
