@@ -90,10 +90,10 @@ constexpr int kNS = 2;  // K and V ring depth
 // Registers per thread after set-up.  The block is launched with 168 per
 // thread (384 x 168 = 64512); the producer / issuer warpgroup gives part of
 // its share to the two softmax warpgroups, which hold up to 96 values of a
-// row of S each: 128 x 104 + 256 x 200 = 64512.  The host refuses to launch
+// row of S each: 128 x 120 + 256 x 192 = 64512.  The host refuses to launch
 // a build whose register count per thread makes the block's total smaller
 // than that sum (the softmax warpgroups' increase would never be granted).
-constexpr uint32_t kRegsLaunch = 168, kRegsIO = 104, kRegsSoftmax = 200;
+constexpr uint32_t kRegsLaunch = 168, kRegsIO = 120, kRegsSoftmax = 192;
 constexpr uint32_t kRegsSplitTotal = 128 * kRegsIO + 256 * kRegsSoftmax;
 static_assert(kRegsSplitTotal <= kAttnThreads * kRegsLaunch, "register split");
 
@@ -134,6 +134,11 @@ __global__ void __launch_bounds__(256) exp2_test_kernel(const float* __restrict_
   y[i] = r.x;
   if (i + 1 < n) y[i + 1] = r.y;
 }
+
+template <int N>
+struct integral_c {
+  static constexpr int value = N;
+};
 
 // Softmax helpers on one 32-column chunk of a thread's row of S.
 // Columns c0 + e outside [lo, hi] become -inf.
@@ -182,8 +187,14 @@ struct AttnSmem {
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t col_s(int slot) { return slot * 128; }
   // P of keys 16 kk .. 16 kk + 15 (8 packed columns) within a slot's S
-  // columns: keys 0-63 in columns 0-31, keys 64-127 in columns 64-95
-  __host__ __device__ static constexpr uint32_t col_p(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
+  // columns: the keys of each half of the tile sit at the start of that
+  // half's S columns (BK = 128: keys 0-63 in columns 0-31, keys 64-127 in
+  // columns 64-95), so the S product of one key half never overwrites the
+  // other half's P
+  static constexpr int kStepsHalf = BK / 32;  // 16-key MMA steps per key half
+  __host__ __device__ static constexpr uint32_t col_p(int kk) {
+    return (kk / kStepsHalf) * (BK / 2) + (kk % kStepsHalf) * 8;
+  }
   __host__ __device__ static constexpr uint32_t col_o(int slot) { return 256 + slot * 128; }
 };
 
@@ -193,15 +204,16 @@ enum : int {
   kBarQEmpty = kBarQFull + 2,     // + slot: the row's last S completed
   kBarSFull = kBarQEmpty + 2,     // + slot: S ready (one phase per tile of the slot)
   kBarPFull = kBarSFull + 2,      // + slot: P written (4 warps arrive)
-  kBarPVDone = kBarPFull + 2,     // + slot: PV completed
-  kBarOFull = kBarPVDone + 2,     // + slot: the row's last PV completed
+  kBarPVaDone = kBarPFull + 2,    // + slot: the PV product of the tile's first key half completed
+  kBarPVbDone = kBarPVaDone + 2,  // + slot: the whole PV product completed
+  kBarOFull = kBarPVbDone + 2,    // + slot: the row's last PV completed
   kBarOEmpty = kBarOFull + 2,     // + slot: the epilogue read O (4 warps arrive)
   kBarKFull = kBarOEmpty + 2,     // + stage
   kBarKEmpty = kBarKFull + kNS,   // + stage: the step's S products completed
   kBarVFull = kBarKEmpty + kNS,   // + stage
   kBarVEmpty = kBarVFull + kNS,   // + stage: the step's PV products completed
-  kBarDrain = kBarVEmpty + kNS,   // + issuer (2)
-  kNumBars = kBarDrain + 2
+  kBarDrain = kBarVEmpty + kNS,   // the MMA issuer's last products
+  kNumBars = kBarDrain + 1
 };
 static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
 
@@ -265,9 +277,13 @@ __device__ __forceinline__ Pair next_pair(const AttnArgs& a, int p) {
   return x;
 }
 
-// The pair's two lists as one stream in ascending block order.  A block both
-// rows list (same batch and KV head) is one step feeding both slots; ties
-// between rows of different KV heads go to slot 0 first.
+// The pair's two lists as one stream.  A block that both rows list next
+// (same batch and KV head) is one step feeding both slots.  Otherwise the
+// row that has consumed fewer entries goes next, so single-row steps
+// alternate between the slots (the tensor core then always has the other
+// slot's work while one slot's softmax runs); with equal counts the smaller
+// block index goes first, so lists that advance together meet on their
+// shared blocks.
 struct Merge {
   int n0, n1, beg0, beg1;
   int p0, p1;  // entries of each row consumed
@@ -291,6 +307,7 @@ struct Merge {
     int mask;
     if (h0 && h1) {
       if (share && j0 == j1) mask = 3;
+      else if (p0 != p1) mask = p0 < p1 ? 1 : 2;  // the row that is behind: the slots alternate
       else mask = j0 <= j1 ? 1 : 2;
     } else {
       mask = h0 ? 1 : 2;
@@ -344,7 +361,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       mbar_init(bar(kBarQEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarPFull + s), kWGWarps);
-      mbar_init(bar(kBarPVDone + s), 1);
+      mbar_init(bar(kBarPVaDone + s), 1);
+      mbar_init(bar(kBarPVbDone + s), 1);
       mbar_init(bar(kBarOFull + s), 1);
       mbar_init(bar(kBarOEmpty + s), kWGWarps);
     }
@@ -354,8 +372,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
     }
-    mbar_init(bar(kBarDrain + 0), 1);
-    mbar_init(bar(kBarDrain + 1), 1);
+    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -434,11 +451,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         for (int s = 0; s < 2; ++s)
           if (nq[s] > 0) mbar_drain(bar(kBarQFull + s), (nq[s] - 1) & 1, limit);
     }
-  } else {
-    // ------------------------------------------------------------ S issuer / PV issuer
-    // (the whole warp runs the loop; one elected lane issues each tcgen05 instruction)
-    const bool isS = warp == 10;
-    constexpr uint32_t idS = idesc_bf16_f32(128, BK, 0, 0);
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ MMA issuer
+    // (the whole warp runs the loop; one elected lane issues each tcgen05
+    // instruction).  Order: for each step of the merged stream and each slot
+    // it feeds, first the slot's previous tile's PV product, then the slot's
+    // S for this step.  With the slots alternating, the tensor core runs
+    //   PV_0(t-1)  S_0(t)  PV_1(t-1)  S_1(t)  PV_0(t)  S_0(t+1) ...
+    // so each slot's softmax overlaps the other slot's two products.  S and
+    // PV are each issued as two key halves; the S of one half waits only for
+    // the PV half that read the same TMEM columns, which completes while the
+    // other PV half runs.
+    constexpr uint32_t idS = idesc_bf16_f32(128, BK / 2, 0, 0);
     constexpr uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
     // Descriptors are built once; a buffer or k-step only adds its
     // start-address offset (16-byte units) to the low field (addresses stay
@@ -448,65 +472,125 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
     const uint64_t vdesc0 = smem_desc(sV, BK * 128, 1024, kLayoutSW128);
     constexpr uint32_t kQUnits = L::kQBytes >> 4, kStageUnits = L::kKVBytes >> 4;
     constexpr uint32_t kQHalf = (128 * 128) >> 4, kKHalf = (BK * 128) >> 4;
+    constexpr uint32_t kKRowsHalf = ((BK / 2) * 128) >> 4;  // the second half of the key rows
     auto wait = [&](int k, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar(k), parity, abort_flag, limit));
     };
-    uint32_t g = 0;                   // merged steps
-    uint32_t ts[2] = {0, 0};          // tiles of each slot, over all rows
-    uint32_t rs[2] = {0, 0};          // rows of each slot
+    struct PendingPV {
+      bool v, first, last;
+      uint32_t step;
+    };
+    PendingPV pv0{false, false, false, 0}, pv1{false, false, false, 0};
+    uint32_t ts[2] = {0, 0};  // S products issued per slot (over all rows)
+    uint32_t tp[2] = {0, 0};  // PV products issued per slot
+    uint32_t rs[2] = {0, 0};  // rows of each slot whose last S was issued (Q tiles used)
+    uint32_t ro[2] = {0, 0};  // rows of each slot whose first PV was issued (O used)
+    // The pending PV product of slot S.  Its V stage is released once the
+    // step's last PV is issued (the other slot may still owe one for the
+    // same step).
+    auto issue_pv = [&](auto S_) -> bool {
+      constexpr int s = decltype(S_)::value;
+      PendingPV& p = s == 0 ? pv0 : pv1;
+      const PendingPV& o = s == 0 ? pv1 : pv0;
+      const uint32_t st = p.step % kNS;
+      if (!wait(kBarVFull + st, (p.step / kNS) & 1)) return false;
+      if (!wait(kBarPFull + s, tp[s] & 1)) return false;
+      // the first PV of a row overwrites O: the previous row's epilogue must
+      // have read it
+      if (p.first && ro[s] > 0 && !wait(kBarOEmpty + s, (ro[s] - 1) & 1)) return false;
+      tc_fence_after();
+      const uint64_t vd = vdesc0 + st * kStageUnits;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int k = 0; k < L::kStepsHalf; ++k) {
+          const int kk = h * L::kStepsHalf + k;
+          umma_ts_warp(tmem + L::col_o(s), tmem + L::col_s(s) + L::col_p(kk), vd + kk * (2048 >> 4), idPV,
+                       (p.first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit_warp(bar((h == 0 ? kBarPVaDone : kBarPVbDone) + s));
+      }
+      if (p.last) umma_commit_warp(bar(kBarOFull + s));
+      if (!(o.v && o.step == p.step)) umma_commit_warp(bar(kBarVEmpty + st));
+      if (p.first) ++ro[s];
+      ++tp[s];
+      p.v = false;
+      return true;
+    };
+    // S of slot S for the step in K stage st.
+    auto issue_s = [&](auto S_, uint32_t st, bool first, bool last) -> bool {
+      constexpr int s = decltype(S_)::value;
+      if (first && !wait(kBarQFull + s, rs[s] & 1)) return false;
+      const uint64_t qd = qdesc0 + s * kQUnits;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // S of key half h overwrites that half's P of the slot's previous
+        // tile: its PV half must be complete.  That barrier's next phase
+        // needs this S, so the parity is exact.
+        if (ts[s] > 0 && !wait((h == 0 ? kBarPVaDone : kBarPVbDone) + s, (ts[s] - 1) & 1)) return false;
+        tc_fence_after();
+        const uint64_t kd = kdesc0 + st * kStageUnits + h * kKRowsHalf;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 2, offk = (kk >> 2) * kKHalf + (kk & 3) * 2;
+          umma_ss_warp(tmem + L::col_s(s) + h * (BK / 2), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
+        }
+      }
+      umma_commit_warp(bar(kBarSFull + s));
+      if (last) {
+        umma_commit_warp(bar(kBarQEmpty + s));
+        ++rs[s];
+      }
+      ++ts[s];
+      return true;
+    };
+    using I0 = integral_c<0>;
+    using I1 = integral_c<1>;
+    uint32_t g = 0;  // merged steps
     bool ok = true;
     for (Pair x = next_pair(a, blockIdx.x); x.p < num_pairs(a) && ok; x = next_pair(a, x.p + gridDim.x)) {
       Merge m;
       m.init(a, x);
-      int tr[2] = {0, 0};  // tiles of the current row of each slot
+      int tr0 = 0, tr1 = 0;  // tiles of the current row of each slot
       while (ok && !m.done()) {
         int j;
         const int mask = m.step(a, j);
-        const int st = g % kNS;
-        if (!wait((isS ? kBarKFull : kBarVFull) + st, (g / kNS) & 1)) { ok = false; break; }
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          if (!ok || !((mask >> s) & 1)) continue;
-          const bool last = tr[s] + 1 == x.s[s].n;
-          if (isS) {
-            if (tr[s] == 0 && !wait(kBarQFull + s, rs[s] & 1)) { ok = false; break; }
-            // S_s overwrites the slot's P: its previous PV must be complete.
-            // That barrier's next phase needs this S, so the parity is exact.
-            if (ts[s] > 0 && !wait(kBarPVDone + s, (ts[s] - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t qd = qdesc0 + s * kQUnits, kd = kdesc0 + st * kStageUnits;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 2, offk = (kk >> 2) * kKHalf + (kk & 3) * 2;
-              umma_ss_warp(tmem + L::col_s(s), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
-            }
-            umma_commit_warp(bar(kBarSFull + s));
-            if (last) umma_commit_warp(bar(kBarQEmpty + s));
-          } else {
-            if (!wait(kBarPFull + s, ts[s] & 1)) { ok = false; break; }
-            // the first PV of a row overwrites O: the previous row's epilogue
-            // must have read it
-            if (tr[s] == 0 && rs[s] > 0 && !wait(kBarOEmpty + s, (rs[s] - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t vd = vdesc0 + st * kStageUnits;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_ts_warp(tmem + L::col_o(s), tmem + L::col_s(s) + L::col_p(kk), vd + kk * (2048 >> 4), idPV,
-                           (tr[s] == 0 && kk == 0) ? 0u : 1u);
-            umma_commit_warp(bar(kBarPVDone + s));
-            if (last) umma_commit_warp(bar(kBarOFull + s));
-          }
-          ++ts[s];
-          if (++tr[s] == x.s[s].n) ++rs[s];
+        const uint32_t st = g % kNS;
+        // A product still pending from kNS steps back holds the V stage this
+        // step's V load needs: issue it first (the older one first).
+        const bool old0 = pv0.v && pv0.step + kNS <= g, old1 = pv1.v && pv1.step + kNS <= g;
+        if (old0 && old1 && pv1.step < pv0.step) {
+          ok = issue_pv(I1{}) && issue_pv(I0{});
+        } else {
+          if (old0) ok = issue_pv(I0{});
+          if (ok && old1) ok = issue_pv(I1{});
         }
-        if (!ok) break;
-        umma_commit_warp(bar((isS ? kBarKEmpty : kBarVEmpty) + st));
+        if (!ok || !wait(kBarKFull + st, (g / kNS) & 1)) { ok = false; break; }
+        if (mask & 1) {
+          if (pv0.v && !issue_pv(I0{})) { ok = false; break; }
+          const bool first = tr0 == 0, last = tr0 + 1 == x.s[0].n;
+          if (!issue_s(I0{}, st, first, last)) { ok = false; break; }
+          pv0 = PendingPV{true, first, last, g};
+          ++tr0;
+        }
+        if (mask & 2) {
+          if (pv1.v && !issue_pv(I1{})) { ok = false; break; }
+          const bool first = tr1 == 0, last = tr1 + 1 == x.s[1].n;
+          if (!issue_s(I1{}, st, first, last)) { ok = false; break; }
+          pv1 = PendingPV{true, first, last, g};
+          ++tr1;
+        }
+        umma_commit_warp(bar(kBarKEmpty + st));
         ++g;
       }
     }
-    // drain this issuer's outstanding tensor-core work before TMEM is freed
-    umma_commit_warp(bar(kBarDrain + (isS ? 0 : 1)));
-    mbar_drain(bar(kBarDrain + (isS ? 0 : 1)), 0, limit);
+    // the last products, the older first
+    if (ok && pv0.v && pv1.v && pv1.step < pv0.step) ok = issue_pv(I1{});
+    if (ok && pv0.v) ok = issue_pv(I0{});
+    if (ok && pv1.v) ok = issue_pv(I1{});
+    // drain the outstanding tensor-core work before TMEM is freed
+    umma_commit_warp(bar(kBarDrain));
+    mbar_drain(bar(kBarDrain), 0, limit);
   }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
@@ -645,9 +729,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           }
           const float m_exp = update_max(fmaxf(max_chunk(v[0]), max_chunk(v[1])));
           const float2 nm2 = make_float2(bias - m_exp, bias - m_exp);
-          exp_pack_chunk<0>(v[0], v[0], c2, nm2, acc);
-          exp_pack_chunk<16>(v[1], v[0], c2, nm2, acc);
-          tmem_st32(sc, v[0]);
+          exp_pack_chunk<0>(v[0], v[0], c2, nm2, acc);   // keys 0-31 -> columns 0-15
+          exp_pack_chunk<0>(v[1], v[1], c2, nm2, acc);   // keys 32-63 -> columns 32-47
+          tmem_st16(sc, &v[0][0]);
+          tmem_st16(sc + 32, &v[1][0]);
         }
         l2.x *= factor;
         l2.y *= factor;
@@ -656,7 +741,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           // O is scaled after P is formed, so the wait below overlaps the
           // exponentials.  O must hold every earlier tile's product first;
           // the next phase of that barrier needs this tile's P.
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPVDone + slot), (g - 1) & 1, abort_flag, limit))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPVbDone + slot), (g - 1) & 1, abort_flag, limit))) {
             ok = false;
             break;
           }
