@@ -1,52 +1,59 @@
 // Block-sparse prefill attention on the 5th-generation tensor core.
 // ([RBS-en] "The Fix": exact softmax attention over the selected key blocks,
-// compatible with standard multi-head / grouped-query attention;
-// [QUILT] Abstract: query tiles that select the same key blocks share their
-// loads; [BA] 2.4 Block fine-tune: the Block-attention token mask.)
+// compatible with standard multi-head / grouped-query attention; [BA] 2.4
+// Block fine-tune: the Block-attention token mask.)
 //
-// Work item = a PAIR of list rows (a row is one (batch, q head, query block):
-// a 128-row query tile against the row's listed key blocks).  The rows of a
-// pair are consecutive in a work order that keeps one KV head's rows together
-// and, within it, starts with the last query blocks (the longest causal rows):
-// normally two q heads of one KV head at the same query block.  Persistent
-// CTAs take pairs round-robin.
+// Work item = one list row (batch b, q head h, query block i): a 128-row
+// query tile (BQ valid rows) against the row's listed key blocks, in list
+// order.  Persistent CTAs take non-empty work items round-robin in an order
+// that keeps one KV head's rows together and, within it, starts with the last
+// query blocks (the longest causal rows).
 //
-// Two query tiles per CTA ("slots" 0 and 1), each with its own S and O in
-// TMEM, so the tensor core works on one slot's tile while the softmax warps
-// of the other slot work on theirs (ping-pong).  The two rows' key-block
-// lists are walked as ONE merged stream in ascending block order: a block
-// both rows list (same batch and KV head) is loaded once and feeds both
-// slots' S = Q K^T and O += P V products; a block only one row lists feeds
-// that slot alone.  Every role walks the same merged stream, so they agree
-// on the order without exchanging it.
+// One softmax pipeline with two S buffers in TMEM.  While the softmax warps
+// work on tile t, the tensor core computes S for tile t+1 and accumulates
+// P_{t-1} V_{t-1}, so the tensor core and the softmax overlap without either
+// waiting on the other's latency.
+//
+// Each key tile is split into two column halves, and each half has its own
+// softmax state: running max m_h, row sum l_h and accumulator
+// O_h = sum over tiles of P_h V_h (the P and V rows of that half's keys).
+// The two halves are merged exactly once per row, in the epilogue:
+//   O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)),
+// so the two warps that share a query row never wait for each other inside
+// the key loop.
 //
 // Roles (384 threads):
-//   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1: one thread per
-//              query row (TMEM lane), all BK columns of S.  Per tile: load S,
-//              apply the masks (causal diagonal, keys past Lk, the token-level
-//              segment bound, dead tiles), take the row max, lazily update
-//              the running max m (O rescaled in TMEM only when it grows by
-//              more than 2^8; the final normalisation uses the same m, so the
-//              result is exact), form P = exp2(S*c - m) (3 of every 8 element
-//              pairs on the FMA pipe, see exp2_fma2, the rest on the SFU),
-//              write P as packed bf16 pairs over the first BK/2 columns of the
-//              slot's S.  A tile of a rescue-only block whose contribution is
-//              weighted by w has log2(w) added to its scaled scores.  At the
-//              end of a row: O / l -> bf16, and the LSE.
+//   warps 0-7  softmax: warp w owns query rows 32(w%4) .. 32(w%4)+31 (its
+//              TMEM lane quarter) and column half h = w/4 of every key tile.
+//              Pass 1 reads its half row of S into registers and takes its
+//              maximum; the running max is lazily updated (O_h rescaled in
+//              TMEM only when it grows by more than 2^8; the final
+//              normalisation uses the same max, so the result is exact).
+//              A tile of a rescue-only block whose contribution is weighted
+//              by w has log2(w) added to its scaled scores (max and
+//              exponentials alike), which weights its softmax mass by w.
+//              Pass 2 forms P = exp2(S*c - m_h) from the registers (3 of every
+//              8 element pairs on the FMA pipe, see exp2_fma2, the rest on the
+//              SFU) and writes it as packed bf16 pairs over the first quarter
+//              of its own S columns.  In the epilogue the two warps of a
+//              quarter exchange (m_h, l_h) and each writes 64 of the 128
+//              output dims from both accumulators.
 //   warp 8     Q and K producer, warp 9 V producer (one thread each): TMA
-//              loads of the slots' Q tiles and of the merged stream's K / V
-//              tiles, gathered by block index (4-D tensor maps over
-//              [B, L, H, 128], 128B swizzle, no multicast) into 2-deep rings.
+//              loads of the Q tile (double-buffered) and of the K_j / V_j
+//              tiles gathered by block index (4-D tensor maps over
+//              [B, L, H, 128], 128B swizzle, no multicast) into 2-deep K and
+//              V rings; list indices fetched one tile ahead.
 //   warp 10    TMEM allocator and S issuer, warp 11 PV issuer (each warp runs
 //              its loop; one elected lane issues):
-//                S_s  = Q_s K_u^T    A = Q_s (smem), B = K_u (smem)
-//                O_s += P_s V_u      A = P_s (TMEM), B = V_u (MN-major smem)
-//              for each slot s that step u of the merged stream feeds.  S_s
-//              of a slot's next tile overwrites its P, so the S issuer waits
-//              for that slot's previous PV; otherwise the two issuers run
-//              independently.  A ring stage is refilled when the issuer that
-//              read it commits the stage's "empty" barrier.
-// TMEM columns: S_0 [0, 128), S_1 [128, 256), O_0 [256, 384), O_1 [384, 512).
+//                S_g   = Q K_g^T      into S buffer g%2  A = Q (smem), B = K_g (smem)
+//                O_h  += P_g,h V_g,h  for h = 0, 1       A = P (TMEM), B = V_g (MN-major smem)
+//              over the CTA's tiles g = 0, 1, 2, ... of all its rows in
+//              sequence.  S_{g+2} overwrites P_g, so the S issuer waits for
+//              PV_g to complete; otherwise the two issuers run independently,
+//              so each one's waits and commits overlap the other's MMAs.
+//              The K and V producers refill a ring stage when the S (PV)
+//              barrier of the tile that used it completes.
+// TMEM columns: S buffers [0, BK), [128, 128+BK); O_0 [256, 384), O_1 [384, 512).
 //
 // Every mbarrier wait is bounded (a.wait_ns); on a timeout all roles unwind,
 // in-flight TMA loads and MMAs are drained (bounded), TMEM is freed, and the
@@ -68,7 +75,7 @@ struct AttnArgs {
   float* lse;
   int B, Hq, Hkv, nqb, nkb, Lq;
   int k_tail;  // keys in the last key block (BK unless Lk is not a block multiple)
-  int q_block_off, causal, num_rows;  // num_rows: B * Hq * nqb list rows to compute
+  int q_block_off, causal, num_rows;  // num_rows: work items, B * Hq * nqb
   int group_lists;  // 1: list row (b, KV head, i) serves every q head of the KV head
   // rescue blocks weighted by w: entries whose flags are exactly "rescue
   // branch only" get log2(w) added to their logits (in log2 units); flags is
@@ -87,15 +94,6 @@ struct AttnArgs {
 
 constexpr int kAttnThreads = 384;
 constexpr int kNS = 2;  // K and V ring depth
-// Registers per thread after set-up.  The block is launched with 168 per
-// thread (384 x 168 = 64512); the producer / issuer warpgroup gives part of
-// its share to the two softmax warpgroups, which hold up to 96 values of a
-// row of S each: 128 x 120 + 256 x 192 = 64512.  The host refuses to launch
-// a build whose register count per thread makes the block's total smaller
-// than that sum (the softmax warpgroups' increase would never be granted).
-constexpr uint32_t kRegsLaunch = 168, kRegsIO = 120, kRegsSoftmax = 192;
-constexpr uint32_t kRegsSplitTotal = 128 * kRegsIO + 256 * kRegsSoftmax;
-static_assert(kRegsSplitTotal <= kAttnThreads * kRegsLaunch, "register split");
 
 // Software base-2 exponential of two values at once, on the FMA pipe:
 // Cody-Waite range reduction 2^x = 2^n * 2^f, n = rint(x) (via the 1.5*2^23
@@ -135,93 +133,57 @@ __global__ void __launch_bounds__(256) exp2_test_kernel(const float* __restrict_
   if (i + 1 < n) y[i + 1] = r.y;
 }
 
-template <int N>
-struct integral_c {
-  static constexpr int value = N;
-};
-
-// Softmax helpers on one 32-column chunk of a thread's row of S.
-// Columns c0 + e outside [lo, hi] become -inf.
-__device__ __forceinline__ void mask_chunk(uint32_t (&w)[32], int c0, int lo, int hi) {
-#pragma unroll
-  for (int e = 0; e < 32; ++e)
-    if (c0 + e < lo || c0 + e > hi) w[e] = __float_as_uint(-INFINITY);
-}
-
-__device__ __forceinline__ float max_chunk(const uint32_t (&w)[32]) {
-  float m0 = __uint_as_float(w[0]);
-#pragma unroll
-  for (int e = 1; e < 31; e += 2) m0 = fmax3(m0, __uint_as_float(w[e]), __uint_as_float(w[e + 1]));
-  return fmaxf(m0, __uint_as_float(w[31]));
-}
-
-// P = exp2(s * c + nm) of the chunk's 16 column pairs -> packed bf16 pairs in
-// out[OFF .. OFF + 15] (out may be w itself: pair k is written after it and
-// every earlier pair were read); the values are added into acc.  Pairs 1, 4
-// and 6 of every 8 use the FMA-pipe exponential, the rest the SFU.
-template <int OFF>
-__device__ __forceinline__ void exp_pack_chunk(const uint32_t (&w)[32], uint32_t (&out)[32], float2 c2, float2 nm2,
-                                               float2 (&acc)[4]) {
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const float2 arg = ffma2(make_float2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1])), c2, nm2);
-    const int pi = k & 7;
-    const float2 p = (pi == 1 || pi == 4 || pi == 6) ? exp2_fma2(arg) : make_float2(ptx_exp2(arg.x), ptx_exp2(arg.y));
-    acc[k & 3] = fadd2(acc[k & 3], p);
-    out[OFF + k] = pack_bf16x2(p.x, p.y);
+// First key position query position p may see under the segment mask.
+__device__ __forceinline__ int segment_key_start(const int* seg, int n, int final_start, int p) {
+  if (n <= 0 || p >= final_start) return 0;
+  int lo = 0, hi = n - 1;  // the last passage whose start <= p
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (seg[mid] <= p) lo = mid; else hi = mid - 1;
   }
+  return seg[lo];
 }
 
 template <int BK>
 struct AttnSmem {
   static constexpr int kQBytes = 128 * 128 * 2;  // one Q tile: 128 rows x 128 dims (two 64-dim halves)
   static constexpr int kKVBytes = BK * 128 * 2;  // BK rows x 128 dims (two halves)
-  static constexpr int kQ = 0;                   // Q tiles of slot 0 and slot 1
+  static constexpr int kQ = 0;                   // two Q buffers
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kNS * kKVBytes;
-  static constexpr int kSeg = kV + kNS * kKVBytes;  // int [RBS_MAX_SEGMENTS] passage starts
+  static constexpr int kX = kV + kNS * kKVBytes;  // float [2 exchange parity][2 halves][(m, l)][128 rows]
+  static constexpr int kSeg = kX + 2 * 2 * 2 * 128 * 4;  // int [RBS_MAX_SEGMENTS] passage starts
   static constexpr int kBar = kSeg + RBS_MAX_SEGMENTS * 4;
   static constexpr int kBarBytes = 256;
   static constexpr int kTotal = kBar + kBarBytes;
   static constexpr int kAlloc = kTotal + 1024;  // slack to align the base to 1024
   static constexpr uint32_t kTmemCols = 512;
-  __host__ __device__ static constexpr uint32_t col_s(int slot) { return slot * 128; }
-  // P of keys 16 kk .. 16 kk + 15 (8 packed columns) within a slot's S
-  // columns: the keys of each half of the tile sit at the start of that
-  // half's S columns (BK = 128: keys 0-63 in columns 0-31, keys 64-127 in
-  // columns 64-95), so the S product of one key half never overwrites the
-  // other half's P
-  static constexpr int kStepsHalf = BK / 32;  // 16-key MMA steps per key half
-  __host__ __device__ static constexpr uint32_t col_p(int kk) {
-    return (kk / kStepsHalf) * (BK / 2) + (kk % kStepsHalf) * 8;
-  }
-  __host__ __device__ static constexpr uint32_t col_o(int slot) { return 256 + slot * 128; }
+  static constexpr int kSBufs = 2;
+  __host__ __device__ static constexpr uint32_t col_s(int buf) { return buf * 128; }
+  __host__ __device__ static constexpr uint32_t col_o(int half) { return 256 + half * 128; }
 };
 
 // barrier slots (8 bytes each)
 enum : int {
-  kBarQFull = 0,                  // + slot: the slot's Q tile landed (one phase per row)
-  kBarQEmpty = kBarQFull + 2,     // + slot: the row's last S completed
-  kBarSFull = kBarQEmpty + 2,     // + slot: S ready (one phase per tile of the slot)
-  kBarPFull = kBarSFull + 2,      // + slot: P written (4 warps arrive)
-  kBarPVaDone = kBarPFull + 2,    // + slot: the PV product of the tile's first key half completed
-  kBarPVbDone = kBarPVaDone + 2,  // + slot: the whole PV product completed
-  kBarOFull = kBarPVbDone + 2,    // + slot: the row's last PV completed
-  kBarOEmpty = kBarOFull + 2,     // + slot: the epilogue read O (4 warps arrive)
-  kBarKFull = kBarOEmpty + 2,     // + stage
-  kBarKEmpty = kBarKFull + kNS,   // + stage: the step's S products completed
-  kBarVFull = kBarKEmpty + kNS,   // + stage
-  kBarVEmpty = kBarVFull + kNS,   // + stage: the step's PV products completed
-  kBarDrain = kBarVEmpty + kNS,   // the MMA issuer's last products
-  kNumBars = kBarDrain + 1
+  kBarQFull = 0,                 // + buffer (2)
+  kBarQEmpty = kBarQFull + 2,    // + buffer (2)
+  kBarKFull = kBarQEmpty + 2,    // + stage
+  kBarVFull = kBarKFull + kNS,   // + stage
+  kBarSFull = kBarVFull + kNS,   // + S buffer (2)
+  kBarPFull = kBarSFull + 2,     // + S buffer (2)
+  kBarPVDone = kBarPFull + 2,    // + tile index mod 4: one phase per fourth PV
+  kBarOFull = kBarPVDone + 4,    // one phase per row
+  kBarOEmpty = kBarOFull + 1,    // one phase per row
+  kBarX = kBarOEmpty + 1,        // + lane quarter (4): the two warps' exchanges
+  kBarDrain = kBarX + 4,         // + issuer (2)
+  kNumBars = kBarDrain + 2
 };
 static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
 
-// Work order index w -> (batch, q head, query block) and its list row: batch
-// entry, then KV head, then query block from the last (the longest causal
-// rows first), then the G q heads sharing that KV head.  The CTAs working at
-// the same time therefore read the K/V tiles of one KV head, which fit in L2
-// (64 MiB for 131072 tokens), instead of every head's.
+// Work order: batch entry, then KV head, then query block from the last (the
+// longest causal rows first), then the G q heads sharing that KV head.  The
+// CTAs working at the same time therefore read the K/V tiles of one KV head,
+// which fit in L2 (64 MiB for 131072 tokens), instead of every head's.
 __device__ __forceinline__ void decode_work(const AttnArgs& a, int w, int& b, int& h, int& i, int& row) {
   const int G = a.Hq / a.Hkv;
   const int per_b = a.Hq * a.nqb, per_kvh = G * a.nqb;
@@ -241,116 +203,38 @@ __device__ __forceinline__ int row_extent(const AttnArgs& a, int row, int& beg) 
   return end - beg;
 }
 
-struct Slot {
-  int b, h, i, kvh, beg, n;  // n <= 0: nothing to compute in the main loop
+struct Work {
+  int w, b, h, i, row, beg, n;
 };
 
-struct Pair {
-  int p;  // pair index; rows 2p (slot 0) and 2p + 1 (slot 1) of the work order
-  Slot s[2];
-};
-
-__device__ __forceinline__ Slot load_slot(const AttnArgs& a, int w) {
-  Slot s;
-  s.b = s.h = s.i = s.kvh = s.beg = 0;
-  s.n = 0;
-  if (w < a.num_rows) {
-    int row;
-    decode_work(a, w, s.b, s.h, s.i, row);
-    s.kvh = s.h / (a.Hq / a.Hkv);
-    s.n = row_extent(a, row, s.beg);
+// The first non-empty work item at or after w in this CTA's round-robin order.
+__device__ __forceinline__ Work next_work(const AttnArgs& a, int w) {
+  Work x;
+  for (; w < a.num_rows; w += gridDim.x) {
+    decode_work(a, w, x.b, x.h, x.i, x.row);
+    x.n = row_extent(a, x.row, x.beg);
+    if (x.n > 0) break;
   }
-  return s;
-}
-
-__device__ __forceinline__ int num_pairs(const AttnArgs& a) { return (a.num_rows + 1) >> 1; }
-
-// The first pair at or after p in this CTA's round-robin order with work.
-__device__ __forceinline__ Pair next_pair(const AttnArgs& a, int p) {
-  Pair x;
-  for (; p < num_pairs(a); p += gridDim.x) {
-    x.s[0] = load_slot(a, 2 * p);
-    x.s[1] = load_slot(a, 2 * p + 1);
-    if (x.s[0].n > 0 || x.s[1].n > 0) break;
-  }
-  x.p = p;
+  x.w = w;
   return x;
-}
-
-// The pair's two lists as one stream.  A block that both rows list next
-// (same batch and KV head) is one step feeding both slots.  Otherwise the
-// row that has consumed fewer entries goes next, so single-row steps
-// alternate between the slots (the tensor core then always has the other
-// slot's work while one slot's softmax runs); with equal counts the smaller
-// block index goes first, so lists that advance together meet on their
-// shared blocks.
-struct Merge {
-  int n0, n1, beg0, beg1;
-  int p0, p1;  // entries of each row consumed
-  int j0, j1;  // each row's next entry
-  bool share;
-
-  __device__ __forceinline__ void init(const AttnArgs& a, const Pair& x) {
-    n0 = max(x.s[0].n, 0);
-    n1 = max(x.s[1].n, 0);
-    beg0 = x.s[0].beg;
-    beg1 = x.s[1].beg;
-    p0 = p1 = 0;
-    j0 = n0 > 0 ? __ldg(a.col_idx + beg0) : 0;
-    j1 = n1 > 0 ? __ldg(a.col_idx + beg1) : 0;
-    share = n0 > 0 && n1 > 0 && x.s[0].b == x.s[1].b && x.s[0].kvh == x.s[1].kvh;
-  }
-  __device__ __forceinline__ bool done() const { return p0 >= n0 && p1 >= n1; }
-  // The next step: the slots it feeds (bit s) and its key block.
-  __device__ __forceinline__ int step(const AttnArgs& a, int& j) {
-    const bool h0 = p0 < n0, h1 = p1 < n1;
-    int mask;
-    if (h0 && h1) {
-      if (share && j0 == j1) mask = 3;
-      else if (p0 != p1) mask = p0 < p1 ? 1 : 2;  // the row that is behind: the slots alternate
-      else mask = j0 <= j1 ? 1 : 2;
-    } else {
-      mask = h0 ? 1 : 2;
-    }
-    j = (mask & 1) ? j0 : j1;
-    if (mask & 1) {
-      ++p0;
-      if (p0 < n0) j0 = __ldg(a.col_idx + beg0 + p0);
-    }
-    if (mask & 2) {
-      ++p1;
-      if (p1 < n1) j1 = __ldg(a.col_idx + beg1 + p1);
-    }
-    return mask;
-  }
-};
-
-// First key position query position p may see under the segment mask.
-__device__ __forceinline__ int segment_key_start(const int* seg, int n, int final_start, int p) {
-  if (n <= 0 || p >= final_start) return 0;
-  int lo = 0, hi = n - 1;  // the last passage whose start <= p
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (seg[mid] <= p) lo = mid; else hi = mid - 1;
-  }
-  return seg[lo];
 }
 
 template <int BQ, int BK>
 __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __grid_constant__ AttnArgs a) {
   using L = AttnSmem<BK>;
-  constexpr int kWGWarps = 4;  // barriers a softmax warpgroup completes count one arrival per warp
+  constexpr int kSoftmaxWarps = 8;  // barriers the softmax warps complete count one arrival per warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::kQ;
   const uint32_t sK = sbase + L::kK;
   const uint32_t sV = sbase + L::kV;
-  int* seg = reinterpret_cast<int*>(smem + L::kSeg);
+  float* xch = reinterpret_cast<float*>(smem + L::kX);
   const uint32_t bars = sbase + L::kBar;
   auto bar = [&](int k) -> uint32_t { return bars + 8u * k; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + kNumBars * 8 + 4);
+  int* seg = reinterpret_cast<int*>(smem + L::kSeg);
   const uint64_t limit = a.wait_ns;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -359,20 +243,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarQFull + s), 1);
       mbar_init(bar(kBarQEmpty + s), 1);
-      mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarPFull + s), kWGWarps);
-      mbar_init(bar(kBarPVaDone + s), 1);
-      mbar_init(bar(kBarPVbDone + s), 1);
-      mbar_init(bar(kBarOFull + s), 1);
-      mbar_init(bar(kBarOEmpty + s), kWGWarps);
     }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarVEmpty + s), 1);
     }
-    mbar_init(bar(kBarDrain), 1);
+    for (int s = 0; s < L::kSBufs; ++s) {
+      mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarPFull + s), kSoftmaxWarps);
+    }
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kBarPVDone + s), 1);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOEmpty), kSoftmaxWarps);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(kBarX + q), 2);
+    mbar_init(bar(kBarDrain + 0), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -392,8 +277,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 8) {
-  regs_dec<kRegsIO>();  // the whole warpgroup (warps 8-11), before it splits into roles
   if (warp == 8 || warp == 9) {
     // ------------------------------------------------------------ Q+K / V producers
     if (lane == 0) {
@@ -401,201 +284,123 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       const CUtensorMap* map = isK ? &a.tmK : &a.tmV;
       const uint32_t ring = isK ? sK : sV;
       const int full0 = isK ? kBarKFull : kBarVFull;
-      const int empty0 = isK ? kBarKEmpty : kBarVEmpty;
       tma_prefetch_desc(map);
       if (isK) tma_prefetch_desc(&a.tmQ);
-      uint32_t nf = 0, nq[2] = {0, 0};  // ring fills, Q fills per slot
+      uint32_t nf = 0, nq = 0;  // ring fills, Q fills issued
       bool ok = true;
-      for (Pair x = next_pair(a, blockIdx.x); x.p < num_pairs(a) && ok; x = next_pair(a, x.p + gridDim.x)) {
+      for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
+        int j_next = __ldg(a.col_idx + x.beg);
         if (isK) {
-#pragma unroll
-          for (int s = 0; s < 2; ++s) {
-            if (!ok || x.s[s].n <= 0) continue;
-            // the slot's previous row must be done with its Q tile (its last
-            // S completed); the next phase of that barrier needs this load
-            if (nq[s] > 0 && !mbar_wait(bar(kBarQEmpty + s), (nq[s] - 1) & 1, abort_flag, limit)) { ok = false; break; }
-            const uint32_t dst = sQ + s * L::kQBytes;
-            mbar_arrive_expect_tx(bar(kBarQFull + s), BQ * 256);
-            tma_load_4d(dst, &a.tmQ, bar(kBarQFull + s), 0, x.s[s].h, x.s[s].i * BQ, x.s[s].b);
-            tma_load_4d(dst + 128 * 128, &a.tmQ, bar(kBarQFull + s), 64, x.s[s].h, x.s[s].i * BQ, x.s[s].b);
-            ++nq[s];
-          }
-          if (!ok) break;
+          const int qb = nq & 1;
+          if (nq >= 2 && !mbar_wait(bar(kBarQEmpty + qb), ((nq >> 1) - 1) & 1, abort_flag, limit)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(kBarQFull + qb), BQ * 256);
+          tma_load_4d(sQ + qb * L::kQBytes, &a.tmQ, bar(kBarQFull + qb), 0, x.h, x.i * BQ, x.b);
+          tma_load_4d(sQ + qb * L::kQBytes + 128 * 128, &a.tmQ, bar(kBarQFull + qb), 64, x.h, x.i * BQ, x.b);
+          ++nq;
         }
-        Merge m;
-        m.init(a, x);
-        while (!m.done()) {
+        const int kvh = x.h / (a.Hq / a.Hkv);
+        for (int t = 0; t < x.n; ++t) {
           if (isK && a.stall_after >= 0 && static_cast<int>(nf) >= a.stall_after) { ok = false; break; }
-          int j;
-          const int mask = m.step(a, j);
-          const bool from0 = mask & 1;  // the K/V head and batch of the slot(s) the step feeds
-          const int src_kvh = from0 ? x.s[0].kvh : x.s[1].kvh, src_b = from0 ? x.s[0].b : x.s[1].b;
-          if (j < 0 || j >= a.nkb) j = 0;  // the softmax masks such a tile and reports it
-          const int st = nf % kNS;
-          // the stage's previous step, nf - kNS, must be consumed; the next
-          // phase of its empty barrier needs this load, so the parity is
-          // unambiguous
-          if (nf >= kNS && !mbar_wait(bar(empty0 + st), ((nf / kNS) - 1) & 1, abort_flag, limit)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(full0 + st), BK * 256);
-          tma_load_4d(ring + st * L::kKVBytes, map, bar(full0 + st), 0, src_kvh, j * BK, src_b);
-          tma_load_4d(ring + st * L::kKVBytes + BK * 128, map, bar(full0 + st), 64, src_kvh, j * BK, src_b);
+          int j = j_next;
+          if (t + 1 < x.n) j_next = __ldg(a.col_idx + x.beg + t + 1);
+          if (j < 0 || j >= a.nkb) j = 0;
+          const int s = nf % kNS;
+          // the stage's previous tile, nf - kNS, must be consumed: its S (for
+          // K) or PV (for V) is complete.  Neither barrier can move past that
+          // phase before this load lands, so the parity is unambiguous.
+          if (nf >= kNS) {
+            const uint32_t prev = nf - kNS;
+            const bool done = isK ? mbar_wait(bar(kBarSFull + prev % L::kSBufs), (prev / L::kSBufs) & 1, abort_flag, limit)
+                                  : mbar_wait(bar(kBarPVDone + (prev & 3)), (prev >> 2) & 1, abort_flag, limit);
+            if (!done) { ok = false; break; }
+          }
+          mbar_arrive_expect_tx(bar(full0 + s), BK * 256);
+          tma_load_4d(ring + s * L::kKVBytes, map, bar(full0 + s), 0, kvh, j * BK, x.b);
+          tma_load_4d(ring + s * L::kKVBytes + BK * 128, map, bar(full0 + s), 64, kvh, j * BK, x.b);
           ++nf;
         }
       }
-      // drain: every load issued must land before the CTA exits.  Stage s was
-      // filled at fill numbers s, s + depth, ...; its last fill completes
+      // drain: every load issued must land before the CTA exits.  Buffer s
+      // was filled at fill numbers s, s + depth, ...; its last fill completes
       // phase (uses - 1).
       for (uint32_t s = 0; s < kNS; ++s)
         if (s < nf) mbar_drain(bar(full0 + s), ((nf - s + kNS - 1) / kNS - 1) & 1, limit);
       if (isK)
-        for (int s = 0; s < 2; ++s)
-          if (nq[s] > 0) mbar_drain(bar(kBarQFull + s), (nq[s] - 1) & 1, limit);
+        for (uint32_t s = 0; s < 2; ++s)
+          if (s < nq) mbar_drain(bar(kBarQFull + s), ((nq - s + 1) / 2 - 1) & 1, limit);
     }
-  } else if (warp == 10) {
-    // ------------------------------------------------------------ MMA issuer
-    // (the whole warp runs the loop; one elected lane issues each tcgen05
-    // instruction).  Order: for each step of the merged stream and each slot
-    // it feeds, first the slot's previous tile's PV product, then the slot's
-    // S for this step.  With the slots alternating, the tensor core runs
-    //   PV_0(t-1)  S_0(t)  PV_1(t-1)  S_1(t)  PV_0(t)  S_0(t+1) ...
-    // so each slot's softmax overlaps the other slot's two products.  S and
-    // PV are each issued as two key halves; the S of one half waits only for
-    // the PV half that read the same TMEM columns, which completes while the
-    // other PV half runs.
-    constexpr uint32_t idS = idesc_bf16_f32(128, BK / 2, 0, 0);
-    constexpr uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
-    // Descriptors are built once; a buffer or k-step only adds its
-    // start-address offset (16-byte units) to the low field (addresses stay
-    // below 256 KB: no carry out of the 14-bit field).
-    const uint64_t qdesc0 = smem_desc(sQ, 16, 1024, kLayoutSW128);
-    const uint64_t kdesc0 = smem_desc(sK, 16, 1024, kLayoutSW128);
-    const uint64_t vdesc0 = smem_desc(sV, BK * 128, 1024, kLayoutSW128);
-    constexpr uint32_t kQUnits = L::kQBytes >> 4, kStageUnits = L::kKVBytes >> 4;
-    constexpr uint32_t kQHalf = (128 * 128) >> 4, kKHalf = (BK * 128) >> 4;
-    constexpr uint32_t kKRowsHalf = ((BK / 2) * 128) >> 4;  // the second half of the key rows
-    auto wait = [&](int k, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(bar(k), parity, abort_flag, limit));
-    };
-    struct PendingPV {
-      bool v, first, last;
-      uint32_t step;
-    };
-    PendingPV pv0{false, false, false, 0}, pv1{false, false, false, 0};
-    uint32_t ts[2] = {0, 0};  // S products issued per slot (over all rows)
-    uint32_t tp[2] = {0, 0};  // PV products issued per slot
-    uint32_t rs[2] = {0, 0};  // rows of each slot whose last S was issued (Q tiles used)
-    uint32_t ro[2] = {0, 0};  // rows of each slot whose first PV was issued (O used)
-    // The pending PV product of slot S.  Its V stage is released once the
-    // step's last PV is issued (the other slot may still owe one for the
-    // same step).
-    auto issue_pv = [&](auto S_) -> bool {
-      constexpr int s = decltype(S_)::value;
-      PendingPV& p = s == 0 ? pv0 : pv1;
-      const PendingPV& o = s == 0 ? pv1 : pv0;
-      const uint32_t st = p.step % kNS;
-      if (!wait(kBarVFull + st, (p.step / kNS) & 1)) return false;
-      if (!wait(kBarPFull + s, tp[s] & 1)) return false;
-      // the first PV of a row overwrites O: the previous row's epilogue must
-      // have read it
-      if (p.first && ro[s] > 0 && !wait(kBarOEmpty + s, (ro[s] - 1) & 1)) return false;
-      tc_fence_after();
-      const uint64_t vd = vdesc0 + st * kStageUnits;
+  } else if (warp == 10 || warp == 11) {
+    // ------------------------------------------------------------ S issuer / PV issuer
+    {  // the whole warp runs the loop; one elected lane issues each tcgen05 instruction
+      const bool isS = warp == 10;
+      constexpr uint32_t idS = idesc_bf16_f32(128, BK, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16_f32(128, 128, 0, 1);
+      // Descriptors are built once; a buffer or k-step only adds its
+      // start-address offset (16-byte units) to the low field (addresses
+      // stay below 256 KB: no carry out of the 14-bit field).
+      const uint64_t qdesc0 = smem_desc(sQ, 16, 1024, kLayoutSW128);
+      const uint64_t kdesc0 = smem_desc(sK, 16, 1024, kLayoutSW128);
+      const uint64_t vdesc0 = smem_desc(sV, BK * 128, 1024, kLayoutSW128);
+      constexpr uint32_t kQUnits = L::kQBytes >> 4, kStageUnits = L::kKVBytes >> 4;
+      constexpr uint32_t kQHalf = (128 * 128) >> 4, kKHalf = (BK * 128) >> 4;
+      constexpr int kStepsHalf = BK / 32;  // K16 steps per half of a key tile
+      auto wait = [&](int k, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar(k), parity, abort_flag, limit)); };
+      // Each issuer walks the CTA's (row, tile) sequence: g counts tiles over
+      // all rows, it rows.
+      Work x = next_work(a, blockIdx.x);
+      int t = 0;
+      uint32_t g = 0, it = 0;
+      bool ok = true;
+      for (; ok && x.w < a.num_rows; ++g) {
+        const int b = g % L::kSBufs, s = g % kNS;
+        if (isS) {
+          const int qb = it & 1;
+          if (t == 0 && !wait(kBarQFull + qb, (it >> 1) & 1)) break;
+          if (!wait(kBarKFull + s, (g / kNS) & 1)) break;
+          // S_g overwrites P_{g-2}: PV_{g-2} must be complete.  The next phase
+          // of that barrier is PV_{g+2}, which needs S_{g+2}: not yet issued.
+          if (g >= L::kSBufs && !wait(kBarPVDone + ((g - 2) & 3), ((g - 2) >> 2) & 1)) break;
+          tc_fence_after();
+          const uint64_t qd = qdesc0 + qb * kQUnits, kd = kdesc0 + s * kStageUnits;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int k = 0; k < L::kStepsHalf; ++k) {
-          const int kk = h * L::kStepsHalf + k;
-          umma_ts_warp(tmem + L::col_o(s), tmem + L::col_s(s) + L::col_p(kk), vd + kk * (2048 >> 4), idPV,
-                       (p.first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit_warp(bar((h == 0 ? kBarPVaDone : kBarPVbDone) + s));
-      }
-      if (p.last) umma_commit_warp(bar(kBarOFull + s));
-      if (!(o.v && o.step == p.step)) umma_commit_warp(bar(kBarVEmpty + st));
-      if (p.first) ++ro[s];
-      ++tp[s];
-      p.v = false;
-      return true;
-    };
-    // S of slot S for the step in K stage st.
-    auto issue_s = [&](auto S_, uint32_t st, bool first, bool last) -> bool {
-      constexpr int s = decltype(S_)::value;
-      if (first && !wait(kBarQFull + s, rs[s] & 1)) return false;
-      const uint64_t qd = qdesc0 + s * kQUnits;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        // S of key half h overwrites that half's P of the slot's previous
-        // tile: its PV half must be complete.  That barrier's next phase
-        // needs this S, so the parity is exact.
-        if (ts[s] > 0 && !wait((h == 0 ? kBarPVaDone : kBarPVbDone) + s, (ts[s] - 1) & 1)) return false;
-        tc_fence_after();
-        const uint64_t kd = kdesc0 + st * kStageUnits + h * kKRowsHalf;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 2, offk = (kk >> 2) * kKHalf + (kk & 3) * 2;
-          umma_ss_warp(tmem + L::col_s(s) + h * (BK / 2), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
-        }
-      }
-      umma_commit_warp(bar(kBarSFull + s));
-      if (last) {
-        umma_commit_warp(bar(kBarQEmpty + s));
-        ++rs[s];
-      }
-      ++ts[s];
-      return true;
-    };
-    using I0 = integral_c<0>;
-    using I1 = integral_c<1>;
-    uint32_t g = 0;  // merged steps
-    bool ok = true;
-    for (Pair x = next_pair(a, blockIdx.x); x.p < num_pairs(a) && ok; x = next_pair(a, x.p + gridDim.x)) {
-      Merge m;
-      m.init(a, x);
-      int tr0 = 0, tr1 = 0;  // tiles of the current row of each slot
-      while (ok && !m.done()) {
-        int j;
-        const int mask = m.step(a, j);
-        const uint32_t st = g % kNS;
-        // A product still pending from kNS steps back holds the V stage this
-        // step's V load needs: issue it first (the older one first).
-        const bool old0 = pv0.v && pv0.step + kNS <= g, old1 = pv1.v && pv1.step + kNS <= g;
-        if (old0 && old1 && pv1.step < pv0.step) {
-          ok = issue_pv(I1{}) && issue_pv(I0{});
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 2, offk = (kk >> 2) * kKHalf + (kk & 3) * 2;
+            umma_ss_warp(tmem + L::col_s(b), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit_warp(bar(kBarSFull + b));
+          if (t == x.n - 1) umma_commit_warp(bar(kBarQEmpty + qb));
         } else {
-          if (old0) ok = issue_pv(I0{});
-          if (ok && old1) ok = issue_pv(I1{});
+          if (!wait(kBarPFull + b, (g / L::kSBufs) & 1)) break;
+          if (!wait(kBarVFull + s, (g / kNS) & 1)) break;
+          if (t == 0 && it > 0 && !wait(kBarOEmpty, (it - 1) & 1)) break;
+          tc_fence_after();
+          const uint64_t vd = vdesc0 + s * kStageUnits;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // key half h = kk / kStepsHalf: its P sits at the start of that
+            // half's S columns and accumulates into O_h
+            const int h = kk / kStepsHalf;
+            const uint32_t pcol = L::col_s(b) + h * (BK / 2) + (kk % kStepsHalf) * 8;
+            umma_ts_warp(tmem + L::col_o(h), tmem + pcol, vd + kk * (2048 >> 4), idPV,
+                         (t == 0 && kk % kStepsHalf == 0) ? 0u : 1u);
+          }
+          umma_commit_warp(bar(kBarPVDone + (g & 3)));
+          if (t == x.n - 1) umma_commit_warp(bar(kBarOFull));
         }
-        if (!ok || !wait(kBarKFull + st, (g / kNS) & 1)) { ok = false; break; }
-        if (mask & 1) {
-          if (pv0.v && !issue_pv(I0{})) { ok = false; break; }
-          const bool first = tr0 == 0, last = tr0 + 1 == x.s[0].n;
-          if (!issue_s(I0{}, st, first, last)) { ok = false; break; }
-          pv0 = PendingPV{true, first, last, g};
-          ++tr0;
+        if (++t == x.n) {
+          x = next_work(a, x.w + gridDim.x);
+          t = 0;
+          ++it;
         }
-        if (mask & 2) {
-          if (pv1.v && !issue_pv(I1{})) { ok = false; break; }
-          const bool first = tr1 == 0, last = tr1 + 1 == x.s[1].n;
-          if (!issue_s(I1{}, st, first, last)) { ok = false; break; }
-          pv1 = PendingPV{true, first, last, g};
-          ++tr1;
-        }
-        umma_commit_warp(bar(kBarKEmpty + st));
-        ++g;
       }
+      // drain this issuer's outstanding tensor-core work before TMEM is freed
+      umma_commit_warp(bar(kBarDrain + (isS ? 0 : 1)));
+      mbar_drain(bar(kBarDrain + (isS ? 0 : 1)), 0, limit);
     }
-    // the last products, the older first
-    if (ok && pv0.v && pv1.v && pv1.step < pv0.step) ok = issue_pv(I1{});
-    if (ok && pv0.v) ok = issue_pv(I0{});
-    if (ok && pv1.v) ok = issue_pv(I1{});
-    // drain the outstanding tensor-core work before TMEM is freed
-    umma_commit_warp(bar(kBarDrain));
-    mbar_drain(bar(kBarDrain), 0, limit);
-  }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
-    regs_inc<kRegsSoftmax>();  // each softmax warpgroup as a whole
-    const int slot = warp >> 2, quarter = warp & 3;
+    constexpr int kHalf = BK / 2;  // S columns per warp
+    const int quarter = warp & 3, hf = warp >> 2;
     const int r = quarter * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float c = a.scale_log2;
@@ -603,14 +408,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(k));
     };
+    // exchange (m, l) of each row with the other warp of this lane quarter
+    uint32_t nx = 0;
+    auto exchange = [&](float m, float l, float& mo, float& lo) -> bool {
+      float* xb = xch + (nx & 1) * 512;  // [2 halves][(m, l)][128 rows]
+      xb[hf * 256 + r] = m;
+      xb[hf * 256 + 128 + r] = l;
+      warp_arrive(kBarX + quarter);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarX + quarter), nx & 1, abort_flag, limit))) return false;
+      mo = xb[(hf ^ 1) * 256 + r];
+      lo = xb[(hf ^ 1) * 256 + 128 + r];
+      ++nx;
+      return true;
+    };
 
-    // Rows with no (or a corrupt) list: zeros and LSE = -inf, no pipeline
-    // work.  Each of the 256 softmax threads checks one of this CTA's rows
-    // (pair p, slot e & 1) per pass; a warp then clears the empty rows it
-    // found together.
-    for (int base = 0; blockIdx.x + static_cast<int64_t>(gridDim.x) * (base >> 1) < num_pairs(a); base += 256) {
-      const int e = base + tid;
-      const int64_t w = 2 * (blockIdx.x + static_cast<int64_t>(gridDim.x) * (e >> 1)) + (e & 1);
+    // rows with no (or a corrupt) list: zeros and LSE = -inf, no pipeline
+    // work.  Each softmax thread checks one of this CTA's rows per pass; a
+    // warp then clears the empty rows it found together.
+    for (int base = 0; blockIdx.x + static_cast<int64_t>(gridDim.x) * base < a.num_rows; base += 256) {
+      const int64_t w = blockIdx.x + static_cast<int64_t>(gridDim.x) * (base + tid);
       int b = 0, h = 0, i = 0, n = 1;
       if (w < a.num_rows) {
         int row, beg;
@@ -634,17 +450,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       }
     }
 
-    uint32_t g = 0, item = 0;  // tiles and rows of this slot
+    uint32_t g = 0, item = 0;  // tiles and rows processed by this CTA
     bool ok = true;
-    for (Pair px = next_pair(a, blockIdx.x); px.p < num_pairs(a) && ok; px = next_pair(a, px.p + gridDim.x)) {
-      const Slot x = slot ? px.s[1] : px.s[0];
-      if (x.n <= 0) continue;
+    for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
       const int n = x.n;
       const int gi = x.i + a.q_block_off;
       // the segment mask's first visible key of this thread's query
       const int key_lo = segment_key_start(seg, a.seg_n, a.seg_final, gi * BK + r);
-      float m_used = -INFINITY;  // running max, in log2 units (score * c)
-      float2 l2 = make_float2(0.f, 0.f);  // row sum (two partial sums)
+      float m_used = -INFINITY;  // this half's running max, in log2 units (score * c)
+      float2 l2 = make_float2(0.f, 0.f);  // this half's row sum
       int j_next = __ldg(a.col_idx + x.beg);
       int f_next = a.flags != nullptr ? __ldg(a.flags + x.beg) : 0;
       for (int t = 0; t < n; ++t, ++g) {
@@ -655,93 +469,85 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           j_next = __ldg(a.col_idx + x.beg + t + 1);
           if (a.flags != nullptr) f_next = __ldg(a.flags + x.beg + t + 1);
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + slot), g & 1, abort_flag, limit))) { ok = false; break; }
+        const int b = g % L::kSBufs;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + b), (g / L::kSBufs) & 1, abort_flag, limit))) { ok = false; break; }
         tc_fence_after();
         const bool bad = j < 0 || j >= a.nkb;
         const bool dead = bad || (a.causal && j > gi);
         const bool diag = a.causal && j == gi;
         const bool tail = j == a.nkb - 1 && a.k_tail < BK;  // keys past Lk were loaded as zeros
-        const int lo_col = key_lo - j * BK;                  // columns below are before the passage start
-        if (dead && r == 0) raise_error(bad ? RBS_DEVERR_BLOCK_INDEX : RBS_DEVERR_NONCAUSAL);
-        // column e of the tile is kept when lo_c <= e <= hi_c
-        const bool need_mask = __any_sync(0xffffffffu, dead || diag || tail || lo_col > 0);
-        const int lo_c = lo_col;
-        int hi_c = dead ? -1 : BK - 1;
-        if (diag) hi_c = min(hi_c, r);
-        if (tail) hi_c = min(hi_c, a.k_tail - 1);
-        const uint32_t sc = lane_base + L::col_s(slot);
-        const float2 c2 = make_float2(c, c);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        if (dead && r == 0 && hf == 0) raise_error(bad ? RBS_DEVERR_BLOCK_INDEX : RBS_DEVERR_NONCAUSAL);
+        // pass 1: this warp's half row of S into registers, masked; its maximum
+        const uint32_t scol = L::col_s(b) + hf * kHalf;
+        uint32_t v[kHalf / 32][32];
+#pragma unroll
+        for (int q = 0; q < kHalf / 32; ++q) tmem_ld32(lane_base + scol + 32 * q, v[q]);
+        tmem_wait_ld();
+        const int lo_col = key_lo - j * BK;  // tile columns below are before the query's passage start
+        if (dead || diag || tail || lo_col > hf * kHalf) {
+          // tile column hf * kHalf + 32 q + e is masked when it is above the
+          // diagonal, past the last key, before the query's passage start,
+          // or always (a dead tile)
+#pragma unroll
+          for (int q = 0; q < kHalf / 32; ++q) {
+            const int col0 = hf * kHalf + 32 * q;
+            int lim = dead ? -1 : BK;
+            if (diag) lim = min(lim, r - col0);
+            if (tail) lim = min(lim, a.k_tail - 1 - col0);
+            const int lo = lo_col - col0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (e > lim || e < lo) v[q][e] = __float_as_uint(-INFINITY);
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kHalf / 32; ++q) {
+          float m0 = __uint_as_float(v[q][0]);
+#pragma unroll
+          for (int e = 1; e < 31; e += 2) m0 = fmax3(m0, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
+          mx = fmax3(mx, m0, __uint_as_float(v[q][31]));
+        }
+        const float m_new = fmaxf(m_used, fmaf(mx, c, bias));
         float factor = 1.f;
         bool rescale = false;
-        // The running max after this tile (a lazy update), from the tile's
-        // row maximum mx; P is formed against m_exp.
-        auto update_max = [&](float mx) -> float {
-          const float m_new = fmaxf(m_used, fmaf(mx, c, bias));
-          if (t == 0) {
-            m_used = m_new;
-          } else if (m_new - m_used > 8.f) {
-            factor = ptx_exp2(m_used - m_new);
-            m_used = m_new;
-            rescale = true;
-          }
-          return m_used == -INFINITY ? 0.f : m_used;
-        };
-        if constexpr (BK == 128) {
-          // Keys 64-127 stay in registers from the max pass to the
-          // exponentials; keys 0-63 are read twice (32 columns at a time), so
-          // a thread never holds more than 96 values of S.  P of keys 64-127
-          // goes to columns 64-95, of keys 0-63 to columns 0-31.
-          uint32_t vh[2][32], vc[32];
-          tmem_ld32(sc + 64, vh[0]);
-          tmem_ld32(sc + 96, vh[1]);
-          tmem_ld32(sc, vc);
-          tmem_wait_ld();
-          if (need_mask) {
-            mask_chunk(vh[0], 64, lo_c, hi_c);
-            mask_chunk(vh[1], 96, lo_c, hi_c);
-            mask_chunk(vc, 0, lo_c, hi_c);
-          }
-          float mx = fmaxf(fmaxf(max_chunk(vh[0]), max_chunk(vh[1])), max_chunk(vc));
-          tmem_ld32(sc + 32, vc);
-          tmem_wait_ld();
-          if (need_mask) mask_chunk(vc, 32, lo_c, hi_c);
-          mx = fmaxf(mx, max_chunk(vc));
-          const float m_exp = update_max(mx);
-          const float2 nm2 = make_float2(bias - m_exp, bias - m_exp);
-          exp_pack_chunk<0>(vh[0], vh[0], c2, nm2, acc);
-          exp_pack_chunk<16>(vh[1], vh[0], c2, nm2, acc);
-          tmem_st32(sc + 64, vh[0]);
-          exp_pack_chunk<16>(vc, vh[1], c2, nm2, acc);  // keys 32-63
-          tmem_ld32(sc, vc);                              // keys 0-31 again
-          tmem_wait_ld();
-          if (need_mask) mask_chunk(vc, 0, lo_c, hi_c);
-          exp_pack_chunk<0>(vc, vh[1], c2, nm2, acc);
-          tmem_st32(sc, vh[1]);
-        } else {
-          uint32_t v[2][32];
-          tmem_ld32(sc, v[0]);
-          tmem_ld32(sc + 32, v[1]);
-          tmem_wait_ld();
-          if (need_mask) {
-            mask_chunk(v[0], 0, lo_c, hi_c);
-            mask_chunk(v[1], 32, lo_c, hi_c);
-          }
-          const float m_exp = update_max(fmaxf(max_chunk(v[0]), max_chunk(v[1])));
-          const float2 nm2 = make_float2(bias - m_exp, bias - m_exp);
-          exp_pack_chunk<0>(v[0], v[0], c2, nm2, acc);   // keys 0-31 -> columns 0-15
-          exp_pack_chunk<0>(v[1], v[1], c2, nm2, acc);   // keys 32-63 -> columns 32-47
-          tmem_st16(sc, &v[0][0]);
-          tmem_st16(sc + 32, &v[1][0]);
+        if (t == 0) {
+          m_used = m_new;
+        } else if (m_new - m_used > 8.f) {
+          factor = ptx_exp2(m_used - m_new);
+          m_used = m_new;
+          rescale = true;
         }
+        const float m_exp = m_used == -INFINITY ? 0.f : m_used;
         l2.x *= factor;
         l2.y *= factor;
-        l2 = fadd2(l2, fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])));
+        // pass 2: P = exp2(s*c - m) from the registers, written as packed bf16
+        // pairs over the first kHalf/2 of this warp's S columns (already read)
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(bias - m_exp, bias - m_exp);
+        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        uint32_t pw[kHalf / 2];
+#pragma unroll
+        for (int e = 0; e < kHalf; e += 2) {
+          const float2 sv = make_float2(__uint_as_float(v[e >> 5][e & 31]), __uint_as_float(v[e >> 5][(e & 31) + 1]));
+          const float2 arg = ffma2(sv, c2, nm2);
+          const int pi = (e >> 1) & 7;  // pairs 1, 4 and 6 of every 8 on the FMA pipe
+          const float2 p = (pi == 1 || pi == 4 || pi == 6) ? exp2_fma2(arg)
+                                                             : make_float2(ptx_exp2(arg.x), ptx_exp2(arg.y));
+          acc[(e >> 1) & 1] = fadd2(acc[(e >> 1) & 1], p);
+          pw[e >> 1] = pack_bf16x2(p.x, p.y);
+        }
+        if constexpr (kHalf == 64) {
+          tmem_st32(lane_base + scol, pw);
+        } else {
+          tmem_st16(lane_base + scol, pw);
+        }
+        l2 = fadd2(l2, fadd2(acc[0], acc[1]));
         if (__any_sync(0xffffffffu, rescale)) {
           // O is scaled after P is formed, so the wait below overlaps the
-          // exponentials.  O must hold every earlier tile's product first;
-          // the next phase of that barrier needs this tile's P.
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPVbDone + slot), (g - 1) & 1, abort_flag, limit))) {
+          // exponentials.  O must hold every earlier tile's product first.
+          // The next phase of PV_{g-1}'s barrier is PV_{g+3}, which cannot
+          // start before this tile's P is complete.
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarPVDone + ((g - 1) & 3)), ((g - 1) >> 2) & 1, abort_flag, limit))) {
             ok = false;
             break;
           }
@@ -749,47 +555,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t o[32];
-            tmem_ld32(lane_base + L::col_o(slot) + 32 * q, o);
+            tmem_ld32(lane_base + L::col_o(hf) + 32 * q, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(lane_base + L::col_o(slot) + 32 * q, o);
+            tmem_st32(lane_base + L::col_o(hf) + 32 * q, o);
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        warp_arrive(kBarPFull + slot);
+        warp_arrive(kBarPFull + b);
       }
       if (!ok) break;
 
-      // ---- epilogue: O / l -> bf16, LSE
-      const float lt = l2.x + l2.y;
+      // ---- epilogue: merge the halves, O / l -> bf16 (this warp: dims
+      // [64 hf, 64 hf + 64) of both accumulators), LSE
+      const float lh = l2.x + l2.y;
+      float mo, lo;
+      if (!exchange(m_used, lh, mo, lo)) { ok = false; break; }
+      const float m0 = hf == 0 ? m_used : mo, l0 = hf == 0 ? lh : lo;
+      const float m1 = hf == 0 ? mo : m_used, l1 = hf == 0 ? lo : lh;
+      const float m = fmaxf(m0, m1);
+      const float w0 = l0 > 0.f ? ptx_exp2(m0 - m) : 0.f;
+      const float w1 = l1 > 0.f ? ptx_exp2(m1 - m) : 0.f;
+      const float lt = l0 * w0 + l1 * w1;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarOFull + slot), item & 1, abort_flag, limit))) { ok = false; break; }
+      const float s0 = w0 * inv, s1 = w1 * inv;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBarOFull), item & 1, abort_flag, limit))) { ok = false; break; }
       tc_fence_after();
       const int64_t qrow = static_cast<int64_t>(x.i) * BQ + r;
-      uint4* dst = reinterpret_cast<uint4*>(a.O + x.b * a.ob + qrow * a.os + x.h * a.oh);
+      uint4* dst = reinterpret_cast<uint4*>(a.O + x.b * a.ob + qrow * a.os + x.h * a.oh) + 8 * hf;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[32];
-        tmem_ld32(lane_base + L::col_o(slot) + 32 * q, o);
+      for (int q = 0; q < 2; ++q) {
+        uint32_t va[32], vb[32];
+        tmem_ld32(lane_base + L::col_o(0) + 64 * hf + 32 * q, va);
+        tmem_ld32(lane_base + L::col_o(1) + 64 * hf + 32 * q, vb);
         tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = fmaf(__uint_as_float(vb[e]), s1, __uint_as_float(va[e]) * s0);
         if (r < BQ && qrow < a.Lq) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            dst[4 * q + k] = make_uint4(
-                pack_bf16x2(__uint_as_float(o[8 * k]) * inv, __uint_as_float(o[8 * k + 1]) * inv),
-                pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv),
-                pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv),
-                pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv));
+            dst[4 * q + k] = make_uint4(pack_bf16x2(o[8 * k], o[8 * k + 1]), pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
+                                        pack_bf16x2(o[8 * k + 4], o[8 * k + 5]),
+                                        pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
         }
       }
-      if (a.lse != nullptr && r < BQ && qrow < a.Lq) {
+      if (hf == 0 && a.lse != nullptr && r < BQ && qrow < a.Lq) {
         a.lse[(static_cast<int64_t>(x.b) * a.Hq + x.h) * a.Lq + qrow] =
-            lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+            lt > 0.f ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
       }
       tc_fence_before();
-      warp_arrive(kBarOEmpty + slot);
+      warp_arrive(kBarOEmpty);
       ++item;
     }
   }

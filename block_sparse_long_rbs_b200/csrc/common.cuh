@@ -253,19 +253,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Per-warpgroup register budget (all four warps of an aligned warpgroup
-// execute it).  inc waits until other warpgroups' dec have released enough
-// of the block's registers; the budgets of all warpgroups must add up to at
-// most the registers the block was launched with.
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // ex2.approx (the SFU base-2 exponential), flush-to-zero.
 __device__ __forceinline__ float ptx_exp2(float x) {
   float y;

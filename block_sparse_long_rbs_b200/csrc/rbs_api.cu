@@ -50,7 +50,6 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   int sms = 0;
   bool attrs_set = false;
-  bool attn_regs_ok = false;  // the attention kernels' register split fits their launch
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -104,17 +103,6 @@ rbs_status device_info(DeviceInfo** out) {
                                        static_cast<int>(topk_smem_bytes(kTokMaxKV, kTokMaxKV / 32)));
     e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
     if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    // The attention kernels move registers between warpgroups at run time:
-    // the block must be launched with at least the split's total, or the
-    // softmax warpgroups would wait for registers that never come.
-    d.attn_regs_ok = true;
-    for (const void* kern : {reinterpret_cast<const void*>(bsa_prefill_kernel<128, 128>),
-                             reinterpret_cast<const void*>(bsa_prefill_kernel<64, 64>)}) {
-      cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
-          static_cast<uint32_t>(fa.numRegs) * kAttnThreads < kRegsSplitTotal)
-        d.attn_regs_ok = false;
-    }
     d.attrs_set = true;
   }
   *out = &d;
@@ -901,8 +889,6 @@ rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const 
   if ((st = check_lists(lists, group_lists ? Q->batch * K->heads * nqb : rows)) != RBS_OK) return st;
   DeviceInfo* di;
   if ((st = device_info(&di)) != RBS_OK) return st;
-  RBS_REQUIRE(di->attn_regs_ok, RBS_ERR_UNSUPPORTED,
-              "this build's attention kernel has fewer registers per thread than its warpgroup split needs");
 
   AttnArgs a;
   int siq = 0, sik = 0, siv = 0;
@@ -943,8 +929,8 @@ rbs_status launch_bsa(const rbs_bf16_tensor* Q, const rbs_bf16_tensor* K, const 
     a.seg_final = ex.seg->final_start;
     for (int k = 0; k < ex.seg->n; ++k) a.seg_start[k] = ex.seg->start_tok[k];
   }
-  // persistent: one CTA per SM, each taking pairs of rows
-  const int grid = static_cast<int>(std::min<int64_t>((rows + 1) / 2, di->sms));
+  // persistent: one CTA per SM
+  const int grid = static_cast<int>(std::min<int64_t>(rows, di->sms));
   if (block_q == 128)
     bsa_prefill_kernel<128, 128><<<grid, kAttnThreads, AttnSmem<128>::kAlloc, stream>>>(a);
   else

@@ -1,11 +1,9 @@
-"""GPU parity of the two-row attention schedule (the kernel runs rows in
-pairs and walks their lists as one stream, loading a key block both rows
-list once: "QUILT: Rethinking Sparse-Attention Prefill through Shared Query
-Execution", Abstract).  Random lists exercise the cases the merge must get
-right: pairs of rows of the same KV head with overlapping lists, pairs that
-straddle KV heads or query blocks (3 q heads per KV head), an odd number of
-rows (a last pair with one row), pairs with one empty row, identical lists
-(KV-group lists), and rows of very different lengths."""
+"""GPU parity of block-sparse attention on random lists that exercise the
+cases a fixed selection rarely produces: overlapping lists of neighbouring
+heads, 3 q heads per KV head, an odd number of rows, empty rows between full
+ones, MHA with 5 heads, KV-group lists (one list per KV head), rows of very
+different lengths next to each other, and every row empty; each against the
+fp64 oracle (outputs and log-sum-exps)."""
 
 import numpy as np
 import pytest
@@ -53,12 +51,12 @@ def _check(inp, rp, ci, block=128):
 
 
 @pytest.mark.parametrize("Hq,Hkv,p_keep,p_empty,seed", [
-    (8, 2, 0.4, 0.0, 701),   # pairs of q heads of one KV head, overlapping lists
-    (6, 2, 0.3, 0.0, 702),   # 3 q heads per KV head: pairs straddle KV heads / query blocks
-    (3, 1, 0.5, 0.2, 703),   # odd rows per prompt, empty rows inside pairs
-    (5, 5, 0.6, 0.1, 704),   # MHA, 5 heads: pairs of consecutive query blocks, odd total
+    (8, 2, 0.4, 0.0, 701),   # neighbouring q heads of one KV head, overlapping lists
+    (6, 2, 0.3, 0.0, 702),   # 3 q heads per KV head
+    (3, 1, 0.5, 0.2, 703),   # odd rows per prompt, empty rows in between
+    (5, 5, 0.6, 0.1, 704),   # MHA, 5 heads, odd total
 ])
-def test_pairs_random_lists(cuda_ok, Hq, Hkv, p_keep, p_empty, seed):
+def test_random_lists(cuda_ok, Hq, Hkv, p_keep, p_empty, seed):
     inp = make_mixture(L=2048 + 77, Hq=Hq, Hkv=Hkv, block=128, seed=seed)
     nqb = -(-inp["Q"].shape[1] // 128)
     rng = np.random.default_rng(seed)
@@ -66,7 +64,7 @@ def test_pairs_random_lists(cuda_ok, Hq, Hkv, p_keep, p_empty, seed):
     _check(inp, rp, ci)
 
 
-def test_pairs_very_different_lengths(cuda_ok):
+def test_rows_of_very_different_lengths(cuda_ok):
     # row lengths alternate between 1 and every visible block
     inp = make_mixture(L=4096, Hq=4, Hkv=1, block=128, seed=705)
     nqb = 32
@@ -79,8 +77,8 @@ def test_pairs_very_different_lengths(cuda_ok):
     _check(inp, rp, ci)
 
 
-def test_pairs_kv_group_lists(cuda_ok):
-    # one list per KV head: every pair of q heads shares its whole list
+def test_random_kv_group_lists(cuda_ok):
+    # one list per KV head, shared by its q heads
     inp = make_mixture(L=4096, Hq=8, Hkv=2, block=128, seed=706)
     nqb = 32
     rng = np.random.default_rng(706)
@@ -88,7 +86,7 @@ def test_pairs_kv_group_lists(cuda_ok):
     _check(inp, rp, ci)
 
 
-def test_pairs_all_rows_empty(cuda_ok):
+def test_all_rows_empty(cuda_ok):
     inp = make_mixture(L=1024, Hq=4, Hkv=2, block=128, seed=707)
     rp = np.zeros(4 * 8 + 1, dtype=np.int32)
     lists = rbs.BlockLists(torch.from_numpy(rp).cuda(), torch.zeros(1, dtype=torch.int32, device="cuda"), None, 32)
