@@ -673,25 +673,42 @@ __global__ void __launch_bounds__(kSelThreads, KPL <= 32 ? 2 : 1)
 }
 
 // Exclusive scan of per-row counts into row_ptr (one CTA of 1024 threads;
-// each thread owns a contiguous run of rows, read and written 4 at a time).
+// each thread owns a contiguous run of rows, read 32 at a time with all the
+// loads of a run issued before any is used).
+__device__ __forceinline__ void load_counts32(const int* __restrict__ counts, int c, int s1, int (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 32; u += 4) {
+    if (c + u + 4 <= s1) {
+      const int4 x = *reinterpret_cast<const int4*>(counts + c + u);
+      v[u] = x.x;
+      v[u + 1] = x.y;
+      v[u + 2] = x.z;
+      v[u + 3] = x.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[u + e] = c + u + e < s1 ? counts[c + u + e] : 0;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict__ counts, int rows,
                                                            int* __restrict__ row_ptr, int64_t capacity) {
   __shared__ long long wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = ((rows + 1023) / 1024 + 3) & ~3;  // multiple of 4
+  const int per = ((rows + 1023) / 1024 + 3) & ~3;  // multiple of 4: runs start 16-byte aligned
   const int s0 = min(rows, tid * per), s1 = min(rows, s0 + per);
   long long local = 0;
-  int r = s0;
-  for (; r + 4 <= s1; r += 4) {
-    const int4 c4 = *reinterpret_cast<const int4*>(counts + r);
-    local += static_cast<long long>(c4.x) + c4.y + c4.z + c4.w;
+  for (int c = s0; c < s1; c += 32) {
+    int v[32];
+    load_counts32(counts, c, s1, v);
+#pragma unroll
+    for (int u = 0; u < 32; ++u) local += v[u];
   }
-  for (; r < s1; ++r) local += counts[r];
   long long incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    const long long x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
@@ -700,27 +717,32 @@ __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict
     long long wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const long long v = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += v;
+      const long long x = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += x;
     }
     wsum[lane] = wi - w;
   }
   __syncthreads();
   long long run = wsum[warp] + incl - local;
-  r = s0;
-  for (; r + 4 <= s1; r += 4) {
-    const int4 c4 = *reinterpret_cast<const int4*>(counts + r);
-    int4 o;
-    o.x = static_cast<int>(run);
-    o.y = static_cast<int>(run += c4.x);
-    o.z = static_cast<int>(run += c4.y);
-    o.w = static_cast<int>(run += c4.z);
-    run += c4.w;
-    *reinterpret_cast<int4*>(row_ptr + r) = o;
-  }
-  for (; r < s1; ++r) {
-    row_ptr[r] = static_cast<int>(run);
-    run += counts[r];
+  for (int c = s0; c < s1; c += 32) {
+    int v[32];
+    load_counts32(counts, c, s1, v);
+    int out[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      out[u] = static_cast<int>(run);
+      run += v[u];
+    }
+#pragma unroll
+    for (int u = 0; u < 32; u += 4) {
+      if (c + u + 4 <= s1) {
+        *reinterpret_cast<int4*>(row_ptr + c + u) = make_int4(out[u], out[u + 1], out[u + 2], out[u + 3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (c + u + e < s1) row_ptr[c + u + e] = out[u + e];
+      }
+    }
   }
   if (tid == 1023) {
     row_ptr[rows] = static_cast<int>(run);
@@ -789,6 +811,9 @@ __global__ void __launch_bounds__(256) compact_lists_kernel(CompactArgs a) {
   const int i = row % a.nqb, bh = row / a.nqb;
   const int b = bh / a.Hl, hl = bh % a.Hl;
   const int gi = i + a.q_block_offset;
+  // the row's first mask words are loaded together with its extent
+  uint32_t c0 = 0, r0 = 0;
+  if (lane < a.nwords) list_row_word(a, b, hl, i, lane, c0, r0);
   const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
   if (beg < 0 || end < beg || end > a.capacity) {
     if (lane == 0) raise_error(RBS_DEVERR_ROW_PTR);
@@ -799,7 +824,12 @@ __global__ void __launch_bounds__(256) compact_lists_kernel(CompactArgs a) {
     const int t = w0 + lane;
     uint32_t c = 0, r = 0, f = 0;
     if (t < a.nwords) {
-      list_row_word(a, b, hl, i, t, c, r);
+      if (w0 == 0) {
+        c = c0;
+        r = r0;
+      } else {
+        list_row_word(a, b, hl, i, t, c, r);
+      }
       f = forced_word(t, gi, a.nkb, a.force_diag, a.force_sink);
     }
     uint32_t u = c | r | f;

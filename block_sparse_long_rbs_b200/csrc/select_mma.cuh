@@ -433,19 +433,55 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(TopkArgs t) {
       reinterpret_cast<uint4*>(krs)[q] = srcr[q];
     }
   } else {
-    // stage the row: scores with 16-byte loads (the row starts 128-byte
-    // aligned and is padded to nkbp), r_j beta_j with 4-byte loads; then
-    // the keys of s_c and of s_r = s_c + |qbar| r_j beta_j over them
+    // The row's keys of s_c and of s_r = s_c + |qbar| r_j beta_j, into
+    // shared memory.  Every global load of a chunk of up to 32 x 4 key blocks
+    // is issued before any is used (one memory round trip per chunk, not
+    // per key block): the scores with 16-byte loads (each row starts 128-byte
+    // aligned and is padded to nkbp), r_j and beta_j with 16-byte loads when
+    // their rows are 16-byte aligned (nkb a multiple of 4), else 4-byte ones.
     const float4* src = reinterpret_cast<const float4*>(t.scores + row * t.nkbp);
-    for (int q = lane; q < (n + 3) / 4; q += 32) reinterpret_cast<float4*>(ssc)[q] = src[q];
-    for (int jj = lane; jj < n; jj += 32) srb[jj] = a.rad[kv_off + jj] * a.beta[kv_off + jj];
-    __syncwarp();
     const float qn = t.qnorm[row];
-    for (int jj = lane; jj < n; jj += 32) {
-      const float sv = ssc[jj];
-      const uint32_t kr = order_key(fmaf(qn, srb[jj], sv));
-      kcs[jj] = order_key(sv);
-      krs[jj] = kr;
+    const int nq4 = (n + 3) / 4;
+    constexpr int kU = 8;  // float4 per lane per chunk
+    const bool vec = (a.nkb & 3) == 0;
+    for (int base = 0; base < nq4; base += 32 * kU) {
+      float4 s4[kU], r4[kU], b4[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int q = base + lane + 32 * u;
+        s4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        r4[u] = b4[u] = s4[u];
+        if (q < nq4) {
+          s4[u] = src[q];
+          if (vec) {
+            r4[u] = reinterpret_cast<const float4*>(a.rad + kv_off)[q];
+            b4[u] = reinterpret_cast<const float4*>(a.beta + kv_off)[q];
+          } else {
+            const int j0 = 4 * q;
+            r4[u] = make_float4(a.rad[kv_off + j0], j0 + 1 < n ? a.rad[kv_off + j0 + 1] : 0.f,
+                                j0 + 2 < n ? a.rad[kv_off + j0 + 2] : 0.f, j0 + 3 < n ? a.rad[kv_off + j0 + 3] : 0.f);
+            b4[u] = make_float4(a.beta[kv_off + j0], j0 + 1 < n ? a.beta[kv_off + j0 + 1] : 0.f,
+                                j0 + 2 < n ? a.beta[kv_off + j0 + 2] : 0.f,
+                                j0 + 3 < n ? a.beta[kv_off + j0 + 3] : 0.f);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int q = base + lane + 32 * u;
+        if (q < nq4) {
+          const float sv[4] = {s4[u].x, s4[u].y, s4[u].z, s4[u].w};
+          const float rv[4] = {r4[u].x * b4[u].x, r4[u].y * b4[u].y, r4[u].z * b4[u].z, r4[u].w * b4[u].w};
+          uint4 kc, kr;
+          kc.x = order_key(sv[0]); kc.y = order_key(sv[1]); kc.z = order_key(sv[2]); kc.w = order_key(sv[3]);
+          kr.x = order_key(fmaf(qn, rv[0], sv[0]));
+          kr.y = order_key(fmaf(qn, rv[1], sv[1]));
+          kr.z = order_key(fmaf(qn, rv[2], sv[2]));
+          kr.w = order_key(fmaf(qn, rv[3], sv[3]));
+          reinterpret_cast<uint4*>(kcs)[q] = kc;
+          reinterpret_cast<uint4*>(krs)[q] = kr;
+        }
+      }
     }
   }
   __syncwarp();

@@ -126,6 +126,40 @@ __global__ void __launch_bounds__(1024) block_beta_kernel(const float* __restric
     }
     return;
   }
+  if (p_lo <= 0.f && p_hi == 1.f) {
+    // quantile 0 is the minimum and quantile 1 the maximum: no sort needed
+    // (p_lo < 0 means R_lo = 0, handled below)
+    float mn = INFINITY, mx = -INFINITY;
+    for (int j = tid; j < nkb; j += blockDim.x) {
+      const float r = R[off + j];
+      mn = fminf(mn, r);
+      mx = fmaxf(mx, r);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    __shared__ float wmn[32], wmx[32];
+    if ((tid & 31) == 0) {
+      wmn[tid >> 5] = mn;
+      wmx[tid >> 5] = mx;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) {
+        mn = fminf(mn, wmn[w]);
+        mx = fmaxf(mx, wmx[w]);
+      }
+      lo_hi[0] = p_lo < 0.f ? 0.f : mn;
+      lo_hi[1] = mx;
+      if (range != nullptr) {
+        range[2 * (b * H + h)] = lo_hi[0];
+        range[2 * (b * H + h) + 1] = lo_hi[1];
+      }
+    }
+    __syncthreads();
+  } else {
   int n2 = 1;
   while (n2 < nkb) n2 <<= 1;
   for (int i = tid; i < n2; i += blockDim.x) s[i] = i < nkb ? R[off + i] : __int_as_float(0x7f800000);
@@ -169,6 +203,7 @@ __global__ void __launch_bounds__(1024) block_beta_kernel(const float* __restric
     }
   }
   __syncthreads();
+  }
   const float rlo = lo_hi[0], rhi = lo_hi[1];
   const bool degenerate = (rhi - rlo) <= 1e-12f * fmaxf(rhi, 1e-30f);
   const float inv = degenerate ? 0.f : 1.f / (rhi - rlo);
