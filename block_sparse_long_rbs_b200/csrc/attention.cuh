@@ -597,9 +597,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
         if (r < BQ && qrow < a.Lq) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            dst[4 * q + k] = make_uint4(pack_bf16x2(o[8 * k], o[8 * k + 1]), pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
-                                        pack_bf16x2(o[8 * k + 4], o[8 * k + 5]),
-                                        pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
+            // streaming (evict-first) stores: the output is not read again
+            // here, and the K / V tiles it would otherwise push out of L2
+            // are (as are the next kernel's inputs)
+            __stcs(dst + 4 * q + k, make_uint4(pack_bf16x2(o[8 * k], o[8 * k + 1]),
+                                               pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
+                                               pack_bf16x2(o[8 * k + 4], o[8 * k + 5]),
+                                               pack_bf16x2(o[8 * k + 6], o[8 * k + 7])));
         }
       }
       if (hf == 0 && a.lse != nullptr && r < BQ && qrow < a.Lq) {
