@@ -690,6 +690,45 @@ def block_attention_measure(rbs, peaks):
         res[name]["pairs"] = lists.nnz()
     res["final_block_vs_full_prefill"] = ttft_ratios(res["final_block"]["ms"], res["rope_reencode"]["ms"],
                                                      res["full_prefill"]["ms"], final_lists.nnz(), full_lists.nnz())
+    del Kfull, Ofull, Qg, Kg
+    res["ragged_passages"] = ragged_block_attention_measure(rbs, w)
+    return res
+
+
+def ragged_block_attention_measure(rbs, w):
+    """The same flow with passages that do not end on block boundaries
+    (passages 8, 9 and 10 of the 16 have 1,999, 2,100 and 2,045 tokens, so two
+    passage boundaries fall inside key blocks; the total is unchanged): the
+    cache build and the final block through bsa_prefill_segments, the
+    Block-attention mask applied token by token ("Block-Attention for
+    Efficient Prefilling", 2.2, 2.4)."""
+    import torch
+    lens = [w.passage_len] * 7 + [1999, 2100, 2045] + [w.passage_len] * 6
+    inp = make_block_attention(final_len=w.final_len, Hq=w.heads_q, Hkv=w.heads_kv, block=w.block, seed=w.seed,
+                               passage_lens=lens)
+    L = inp["Q"].shape[1]
+    fs = inp["final_start"]
+    nb = -(-L // BLOCK)
+    f0 = fs // BLOCK
+    Q, K, V = to_dev(inp["Q"]), to_dev(inp["K"]), to_dev(inp["V"])
+    seg = inp["seg_start"].tolist()
+    cache_lists = rbs.rbs_lists_block_attention(seg, fs, BLOCK, 1, w.heads_q, 0, f0)
+    final_lists = rbs.rbs_lists_block_attention(seg, fs, BLOCK, 1, w.heads_q, f0, nb - f0)
+    Op = torch.empty_like(Q[:, :f0 * BLOCK])
+    Qf = Q[:, f0 * BLOCK:].contiguous()
+    Of = torch.empty_like(Qf)
+    parts = {
+        "cache_build": (lambda: rbs.bsa_prefill_segments(Q[:, :f0 * BLOCK], K[:, :f0 * BLOCK], V[:, :f0 * BLOCK],
+                                                         cache_lists, seg, fs, out=Op), cache_lists),
+        "final_block": (lambda: rbs.bsa_prefill_segments(Qf, K, V, final_lists, seg, fs, q_offset=f0 * BLOCK, out=Of),
+                        final_lists),
+    }
+    res = {"passage_lens": "7 x 2048, 1999, 2100, 2045, 6 x 2048; final 512", "passage_starts_off_block": 2}
+    for name, (fn, lists) in parts.items():
+        ms = _time_ms(fn, 10)
+        fl = lists.nnz() * FLOP_PER_PAIR
+        res[name] = {"ms": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 2), "pairs": lists.nnz()}
+    assert rbs.rbs_get_device_error() == 0
     return res
 
 
@@ -775,7 +814,7 @@ def _time_ms(fn, reps: int, warm: int = 2) -> float:
     return statistics.median(times)
 
 
-def density_sweep_measure(rbs, peaks):
+def density_sweep_measure(rbs, peaks, targets=SWEEP_TARGETS, seqlen=None):
     """Selection and attention time against the kept-union density at 64K
     tokens (32 q / 8 KV heads, the compact/dispersed key mixture).  For each
     target density one rho, shared by both branches, is found by bisection on
@@ -783,7 +822,7 @@ def density_sweep_measure(rbs, peaks):
     the achieved density is within 0.25 percentage points; 100% is rho = 1."""
     import torch
     w = WORKLOADS["density_sweep_64k"]
-    inp = make_inputs(w)
+    inp = make_inputs(w, seqlen=seqlen)
     Q, K, V = to_dev(inp["Q"]), to_dev(inp["K"]), to_dev(inp["V"])
     B, L, Hq, _ = Q.shape
     Hkv = K.shape[2]
@@ -804,7 +843,7 @@ def density_sweep_measure(rbs, peaks):
         return lists.nnz() / visible
 
     rows = []
-    for target in SWEEP_TARGETS:
+    for target in targets:
         if target >= 1.0:
             rho, dens = 1.0, density(1.0)
         else:
@@ -829,10 +868,11 @@ def density_sweep_measure(rbs, peaks):
                      "select_ms": round(sel_ms, 4), "attn_ms": round(attn_ms, 4), "attn_tflops": round(tflops, 1),
                      "attn_frac_peak": round(tflops / peaks["bf16_tflops"], 4)})
     assert rbs.rbs_get_device_error() == 0
-    dense_ms = rows[-1]["attn_ms"]
-    for r in rows:
-        r["speedup_vs_dense"] = round(dense_ms / (r["attn_ms"] + r["select_ms"]), 2)
-    return {"workload": "density_sweep_64k: L=65536, 32 q / 8 KV heads, 128x128 blocks, causal", "rows": rows}
+    if rows[-1]["target"] >= 1.0:
+        dense_ms = rows[-1]["attn_ms"]
+        for r in rows:
+            r["speedup_vs_dense"] = round(dense_ms / (r["attn_ms"] + r["select_ms"]), 2)
+    return {"workload": f"density_sweep_64k: L={L}, 32 q / 8 KV heads, 128x128 blocks, causal", "rows": rows}
 
 
 # ---------------------------------------------------------------------------
@@ -949,6 +989,8 @@ def main():
                     help="seconds of oracle sampling for the whole reference run")
     ap.add_argument("--clock-log-dir", default=None,
                     help="keep the nvidia-smi clock samples of the timed region here (default: a temporary file)")
+    ap.add_argument("--sweep-only", default=None,
+                    help="profiling: only the density sweep at these comma-separated densities (with --seq-len)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="shorter prompt of the same workload (profiling captures only; not the headline)")
     args = ap.parse_args()
@@ -959,6 +1001,14 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if args.sweep_only:
+        # profiling captures of the attention kernel at chosen densities (not the headline)
+        import block_sparse_long_rbs_b200 as rbs
+        dist_setup()
+        targets = tuple(float(x) for x in args.sweep_only.split(","))
+        print(json.dumps(density_sweep_measure(rbs, load_peaks(), targets, args.seq_len)), flush=True)
         return
 
     ws, rank, _ = dist_setup()

@@ -286,6 +286,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
       const int full0 = isK ? kBarKFull : kBarVFull;
       tma_prefetch_desc(map);
       if (isK) tma_prefetch_desc(&a.tmQ);
+      // Q tiles are read once; the K / V tiles of a KV head are read by
+      // every row of its q heads and should stay in L2 meanwhile
+      const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
       uint32_t nf = 0, nq = 0;  // ring fills, Q fills issued
       bool ok = true;
       for (Work x = next_work(a, blockIdx.x); x.w < a.num_rows && ok; x = next_work(a, x.w + gridDim.x)) {
@@ -294,8 +297,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
           const int qb = nq & 1;
           if (nq >= 2 && !mbar_wait(bar(kBarQEmpty + qb), ((nq >> 1) - 1) & 1, abort_flag, limit)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(kBarQFull + qb), BQ * 256);
-          tma_load_4d(sQ + qb * L::kQBytes, &a.tmQ, bar(kBarQFull + qb), 0, x.h, x.i * BQ, x.b);
-          tma_load_4d(sQ + qb * L::kQBytes + 128 * 128, &a.tmQ, bar(kBarQFull + qb), 64, x.h, x.i * BQ, x.b);
+          tma_load_4d_hint(sQ + qb * L::kQBytes, &a.tmQ, bar(kBarQFull + qb), 0, x.h, x.i * BQ, x.b, pol_q);
+          tma_load_4d_hint(sQ + qb * L::kQBytes + 128 * 128, &a.tmQ, bar(kBarQFull + qb), 64, x.h, x.i * BQ, x.b,
+                           pol_q);
           ++nq;
         }
         const int kvh = x.h / (a.Hq / a.Hkv);
@@ -315,8 +319,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) bsa_prefill_kernel(const __gr
             if (!done) { ok = false; break; }
           }
           mbar_arrive_expect_tx(bar(full0 + s), BK * 256);
-          tma_load_4d(ring + s * L::kKVBytes, map, bar(full0 + s), 0, kvh, j * BK, x.b);
-          tma_load_4d(ring + s * L::kKVBytes + BK * 128, map, bar(full0 + s), 64, kvh, j * BK, x.b);
+          tma_load_4d_hint(ring + s * L::kKVBytes, map, bar(full0 + s), 0, kvh, j * BK, x.b, pol_kv);
+          tma_load_4d_hint(ring + s * L::kKVBytes + BK * 128, map, bar(full0 + s), 64, kvh, j * BK, x.b, pol_kv);
           ++nf;
         }
       }

@@ -129,6 +129,29 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* des
       : "memory");
 }
 
+// The same load with an L2 cache policy (from make_l2_policy).
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap* desc, uint32_t bar, int c0, int c1,
+                                                 int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
+}
+
+// L2 cache policies for loads: data read once (evict first) and data that
+// should stay resident while it is reused (evict last).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tensor core and TMA reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
