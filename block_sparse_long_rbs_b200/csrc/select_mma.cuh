@@ -442,7 +442,9 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(TopkArgs t) {
     const float4* src = reinterpret_cast<const float4*>(t.scores + row * t.nkbp);
     const float qn = t.qnorm[row];
     const int nq4 = (n + 3) / 4;
-    constexpr int kU = 8;  // float4 per lane per chunk
+    // float4 per lane per chunk: as many as the longest row of this
+    // instantiation needs (up to 8), so short rows issue no idle loads
+    constexpr int kU = KPL / 4 < 1 ? 1 : (KPL / 4 > 8 ? 8 : KPL / 4);
     const bool vec = (a.nkb & 3) == 0;
     for (int base = 0; base < nq4; base += 32 * kU) {
       float4 s4[kU], r4[kU], b4[kU];
