@@ -182,19 +182,212 @@ __device__ __forceinline__ void top4_insert(uint32_t& t0, uint32_t& t1, uint32_t
   t3 = max(t3, y2);
 }
 
+// Bitonic sort across the warp, descending, of the 32 E values x[e] at
+// positions p = lane + 32 e, for two sequences (x and y) at once.  Position p
+// ends up holding the (p + 1)-th largest value.  Warp-uniform.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc2(uint32_t (&x)[E], uint32_t (&y)[E], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32 * E; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+        // partner p + 32: element e + 1 of the same lane (only k = 64 here,
+        // a descending block: the lower position keeps the larger value)
+#pragma unroll
+        for (int e = 0; e + 1 < E; e += 2) {
+          const uint32_t hx = max(x[e], x[e + 1]), lx = min(x[e], x[e + 1]);
+          const uint32_t hy = max(y[e], y[e + 1]), ly = min(y[e], y[e + 1]);
+          x[e] = hx;
+          x[e + 1] = lx;
+          y[e] = hy;
+          y[e + 1] = ly;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int p = lane + 32 * e;
+          // in a descending block (bit k of p clear) the lower position of
+          // the pair keeps the larger value, in an ascending block the smaller
+          const bool keep_max = ((p & j) == 0) == ((p & k) == 0);
+          const uint32_t px = __shfl_xor_sync(0xffffffffu, x[e], j);
+          const uint32_t py = __shfl_xor_sync(0xffffffffu, y[e], j);
+          x[e] = keep_max ? max(x[e], px) : min(x[e], px);
+          y[e] = keep_max ? max(y[e], py) : min(y[e], py);
+        }
+      }
+    }
+  }
+}
+
+// The k-th largest (1 <= k <= 32 E) of the values sorted by warp_sort_desc2.
+template <int E>
+__device__ __forceinline__ uint32_t sorted_kth(const uint32_t (&x)[E], int k) {
+  const int p = k - 1;
+  uint32_t v = x[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e)
+    if ((p >> 5) == e) v = x[e];
+  return __shfl_sync(0xffffffffu, v, p & 31);
+}
+
+// Both branches' selection from lower bounds Lc <= T_c and Lr <= T_r of
+// their k-th largest keys (T), each reached by at least k keys and above
+// key 0 (so no absent slot qualifies).  Every key >= L is a candidate; when
+// at most kTopkCap keys of each branch are, they are compacted in ascending
+// block order into shared memory and T is found among them: by sorting them
+// across the warp when there are at most 64, else by a bitwise search (the
+// largest T with at least k candidates >= T).  The keys above T are kept and
+// of the ties at T the lowest block indices, and the kept blocks are OR-ed
+// into words[0, nwords) (cleared first).  Returns false, having written
+// nothing the caller uses, when a branch has more than kTopkCap candidates.
+// Slots from nt on hold only absent keys.  Warp-uniform.
+template <typename KeyC, typename KeyR>
+__device__ __forceinline__ bool topk2_from_bounds(KeyC key_c, KeyR key_r, uint32_t Lc, uint32_t Lr, int k_c, int k_r,
+                                                  int nt, int lane, int nwords, uint32_t* scratch,
+                                                  uint32_t* words_c, uint32_t* words_r) {
+  uint32_t* ck_c = scratch;  // candidate keys and blocks of each branch
+  int* ci_c = reinterpret_cast<int*>(scratch + kTopkCap);
+  uint32_t* ck_r = scratch + 2 * kTopkCap;
+  int* ci_r = reinterpret_cast<int*>(scratch + 3 * kTopkCap);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base_c = 0, base_r = 0;
+#pragma unroll 4
+  for (int t = 0; t < nt; ++t) {
+    const uint32_t uc = key_c(t), ur = key_r(t);
+    const bool cand_c = uc >= Lc, cand_r = ur >= Lr;
+    const uint32_t bc = __ballot_sync(0xffffffffu, cand_c), br = __ballot_sync(0xffffffffu, cand_r);
+    const int pc = base_c + __popc(bc & lt_mask), pr = base_r + __popc(br & lt_mask);
+    if (cand_c && pc < kTopkCap) {
+      ck_c[pc] = uc;
+      ci_c[pc] = 32 * t + lane;
+    }
+    if (cand_r && pr < kTopkCap) {
+      ck_r[pr] = ur;
+      ci_r[pr] = 32 * t + lane;
+    }
+    base_c += __popc(bc);
+    base_r += __popc(br);
+  }
+  if (base_c > kTopkCap || base_r > kTopkCap) return false;
+  __syncwarp();
+  // candidate position p = lane + 32 s holds slot s of this lane (0 = none)
+  const int cmax = max(base_c, base_r);
+  const int ns = (cmax + 31) >> 5;  // slots holding a candidate of either branch
+  uint32_t a[4], bk[4];
+  int ia[4], ib[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int p = lane + 32 * s;
+    a[s] = p < base_c ? ck_c[p] : 0u;
+    ia[s] = p < base_c ? ci_c[p] : 0;
+    bk[s] = p < base_r ? ck_r[p] : 0u;
+    ib[s] = p < base_r ? ci_r[p] : 0;
+  }
+  uint32_t Tc, Tr;
+  if (cmax <= 32) {
+    uint32_t x[1] = {a[0]}, y[1] = {bk[0]};
+    warp_sort_desc2<1>(x, y, lane);
+    Tc = sorted_kth<1>(x, k_c);
+    Tr = sorted_kth<1>(y, k_r);
+  } else if (cmax <= 64) {
+    uint32_t x[2] = {a[0], a[1]}, y[2] = {bk[0], bk[1]};
+    warp_sort_desc2<2>(x, y, lane);
+    Tc = sorted_kth<2>(x, k_c);
+    Tr = sorted_kth<2>(y, k_r);
+  } else {
+    // T lies between L (at least k candidates reach it) and the largest
+    // candidate: it carries their common leading bits
+    int tpc, tpr;
+    common_prefix(Lc, __reduce_max_sync(0xffffffffu, max(max(a[0], a[1]), max(a[2], a[3]))), Tc, tpc);
+    common_prefix(Lr, __reduce_max_sync(0xffffffffu, max(max(bk[0], bk[1]), max(bk[2], bk[3]))), Tr, tpr);
+#pragma unroll 1
+    for (int bit = max(tpc, tpr); bit >= 0; --bit) {
+      const uint32_t xc = Tc | (1u << bit), xr = Tr | (1u << bit);
+      int nc, nr;
+      sum2((a[0] >= xc) + (a[1] >= xc) + (a[2] >= xc) + (a[3] >= xc),
+           (bk[0] >= xr) + (bk[1] >= xr) + (bk[2] >= xr) + (bk[3] >= xr), nc, nr);
+      if (bit <= tpc && nc >= k_c) Tc = xc;
+      if (bit <= tpr && nr >= k_r) Tr = xr;
+    }
+  }
+  int above_c, above_r;
+  sum2((a[0] > Tc) + (a[1] > Tc) + (a[2] > Tc) + (a[3] > Tc), (bk[0] > Tr) + (bk[1] > Tr) + (bk[2] > Tr) + (bk[3] > Tr),
+       above_c, above_r);
+  const int need_c = k_c - above_c, need_r = k_r - above_r;
+  for (int w = lane; w < nwords; w += 32) words_c[w] = words_r[w] = 0u;
+  __syncwarp();
+  // positions ascend with the block index, so a tie's rank is the number of
+  // ties at lower positions
+  int rank_c = 0, rank_r = 0;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    if (s >= ns) break;
+    const bool tc = a[s] == Tc, tr = bk[s] == Tr;
+    const uint32_t bc = __ballot_sync(0xffffffffu, tc), br = __ballot_sync(0xffffffffu, tr);
+    const bool sc = a[s] > Tc || (tc && rank_c + __popc(bc & lt_mask) < need_c);
+    const bool sr = bk[s] > Tr || (tr && rank_r + __popc(br & lt_mask) < need_r);
+    if (sc) atomicOr(&words_c[ia[s] >> 5], 1u << (ia[s] & 31));
+    if (sr) atomicOr(&words_r[ib[s] >> 5], 1u << (ib[s] & 31));
+    rank_c += __popc(bc);
+    rank_r += __popc(br);
+  }
+  __syncwarp();
+  return true;
+}
+
+// Exact top-k of both branches, for k <= 64, from a sorted subset (key(t) =
+// this lane's key in slot t, block 32 t + lane, 0 for an absent slot).  Each
+// lane keeps its E largest keys per branch (E = 1 when k <= 32, else 2); the
+// subset's k-th largest key L (found by sorting the 32 E keys across the
+// warp) is at most the row's k-th largest, and at least k keys reach it.
+// The subset holds at least k present keys (min(n, 32 E) >= k), so L > 0
+// unless the row's keys are themselves 0 (one NaN pattern), which is left to
+// the caller's other searches like an overflow.  Returns false when k > 64,
+// L = 0, or a branch has more than kTopkCap candidates.  Warp-uniform.
+template <int KP, typename KeyC, typename KeyR>
+__device__ __forceinline__ bool warp_topk2_sorted(KeyC key_c, KeyR key_r, int k_c, int k_r, int n, int lane,
+                                                  int nwords, uint32_t* scratch, uint32_t* words_c,
+                                                  uint32_t* words_r) {
+  if (k_c > 64 || k_r > 64) return false;
+  const int nt = min(KP, (n + 31) >> 5);  // slots holding a visible block
+  uint32_t Lc, Lr;
+  if (max(k_c, k_r) <= 32) {
+    uint32_t x[1] = {0u}, y[1] = {0u};
+#pragma unroll 4
+    for (int t = 0; t < nt; ++t) {
+      x[0] = max(x[0], key_c(t));
+      y[0] = max(y[0], key_r(t));
+    }
+    warp_sort_desc2<1>(x, y, lane);
+    Lc = sorted_kth<1>(x, k_c);
+    Lr = sorted_kth<1>(y, k_r);
+  } else {
+    uint32_t x[2] = {0u, 0u}, y[2] = {0u, 0u};
+#pragma unroll 4
+    for (int t = 0; t < nt; ++t) {
+      const uint32_t uc = key_c(t), ur = key_r(t);
+      x[1] = max(x[1], min(x[0], uc));
+      x[0] = max(x[0], uc);
+      y[1] = max(y[1], min(y[0], ur));
+      y[0] = max(y[0], ur);
+    }
+    warp_sort_desc2<2>(x, y, lane);
+    Lc = sorted_kth<2>(x, k_c);
+    Lr = sorted_kth<2>(y, k_r);
+  }
+  if (Lc == 0u || Lr == 0u) return false;
+  return topk2_from_bounds(key_c, key_r, Lc, Lr, k_c, k_r, nt, lane, nwords, scratch, words_c, words_r);
+}
+
 // Exact top-k of both branches by pruning, for k <= 64 (key(t) = this
 // lane's key in slot t, block 32 t + lane, 0 for an absent slot).  Each lane
 // keeps its four largest keys per branch; that subset of the row holds at
 // least k present keys (all of them when n <= 128, 128 otherwise), so its
 // k-th largest key, rounded down to 24 bits (L), is at most the row's k-th
-// largest key T, and every key >= T is a candidate (key >= L).  When at most
-// kTopkCap keys of each branch are candidates they are compacted in
-// ascending block order into shared memory, T is found among them by a
-// bitwise search (the largest T with at least k candidates >= T), the keys
-// above T are kept and of the ties at T the lowest block indices, and the
-// kept blocks are OR-ed into words[0, nwords) (cleared first).  Returns
-// false, having written nothing the caller uses, when k > 64 or a branch has
-// more candidates (many near-equal keys); the caller then runs the full
+// largest key T, and every key >= T is a candidate (key >= L); the rest is
+// topk2_from_bounds.  Returns false when k > 64 or a branch has more than
+// kTopkCap candidates (many near-equal keys); the caller then runs the full
 // search.  Both branches advance together so their reduction chains overlap.
 // Slots from ceil(n / 32) on hold only absent keys (blocks >= n): they can
 // neither enter a lane's top four nor become candidates, so both passes stop
@@ -205,10 +398,6 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
                                                   uint32_t* words_r) {
   if (k_c > 64 || k_r > 64) return false;
   const int nt = min(KP, (n + 31) >> 5);  // slots holding a visible block
-  uint32_t* ck_c = scratch;  // candidate keys and blocks of each branch
-  int* ci_c = reinterpret_cast<int*>(scratch + kTopkCap);
-  uint32_t* ck_r = scratch + 2 * kTopkCap;
-  int* ci_r = reinterpret_cast<int*>(scratch + 3 * kTopkCap);
   uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0, r0 = 0, r1 = 0, r2 = 0, r3 = 0;
 #pragma unroll 4
   for (int t = 0; t < nt; ++t) {
@@ -234,75 +423,7 @@ __device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_
   }
   // Every float's key but one NaN pattern is >= 256, so L > 0 and no absent
   // slot (key 0) becomes a candidate.
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int base_c = 0, base_r = 0;
-#pragma unroll 4
-  for (int t = 0; t < nt; ++t) {
-    const uint32_t uc = key_c(t), ur = key_r(t);
-    const bool cand_c = uc >= Lc, cand_r = ur >= Lr;
-    const uint32_t bc = __ballot_sync(0xffffffffu, cand_c), br = __ballot_sync(0xffffffffu, cand_r);
-    const int pc = base_c + __popc(bc & lt_mask), pr = base_r + __popc(br & lt_mask);
-    if (cand_c && pc < kTopkCap) {
-      ck_c[pc] = uc;
-      ci_c[pc] = 32 * t + lane;
-    }
-    if (cand_r && pr < kTopkCap) {
-      ck_r[pr] = ur;
-      ci_r[pr] = 32 * t + lane;
-    }
-    base_c += __popc(bc);
-    base_r += __popc(br);
-  }
-  if (base_c > kTopkCap || base_r > kTopkCap) return false;
-  __syncwarp();
-  // candidate position p = lane + 32 s holds slot s of this lane (0 = none)
-  uint32_t a[4], bk[4];
-  int ia[4], ib[4];
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int p = lane + 32 * s;
-    a[s] = p < base_c ? ck_c[p] : 0u;
-    ia[s] = p < base_c ? ci_c[p] : 0;
-    bk[s] = p < base_r ? ck_r[p] : 0u;
-    ib[s] = p < base_r ? ci_r[p] : 0;
-  }
-  // T lies between L (at least k candidates reach it) and the largest
-  // candidate: it carries their common leading bits
-  uint32_t Tc, Tr;
-  int tpc, tpr;
-  common_prefix(Lc, __reduce_max_sync(0xffffffffu, max(max(a[0], a[1]), max(a[2], a[3]))), Tc, tpc);
-  common_prefix(Lr, __reduce_max_sync(0xffffffffu, max(max(bk[0], bk[1]), max(bk[2], bk[3]))), Tr, tpr);
-#pragma unroll 1
-  for (int bit = max(tpc, tpr); bit >= 0; --bit) {
-    const uint32_t xc = Tc | (1u << bit), xr = Tr | (1u << bit);
-    int nc, nr;
-    sum2((a[0] >= xc) + (a[1] >= xc) + (a[2] >= xc) + (a[3] >= xc),
-         (bk[0] >= xr) + (bk[1] >= xr) + (bk[2] >= xr) + (bk[3] >= xr), nc, nr);
-    if (bit <= tpc && nc >= k_c) Tc = xc;
-    if (bit <= tpr && nr >= k_r) Tr = xr;
-  }
-  int above_c, above_r;
-  sum2((a[0] > Tc) + (a[1] > Tc) + (a[2] > Tc) + (a[3] > Tc), (bk[0] > Tr) + (bk[1] > Tr) + (bk[2] > Tr) + (bk[3] > Tr),
-       above_c, above_r);
-  const int need_c = k_c - above_c, need_r = k_r - above_r;
-  for (int w = lane; w < nwords; w += 32) words_c[w] = words_r[w] = 0u;
-  __syncwarp();
-  // positions ascend with the block index, so a tie's rank is the number of
-  // ties at lower positions
-  int rank_c = 0, rank_r = 0;
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const bool tc = a[s] == Tc, tr = bk[s] == Tr;
-    const uint32_t bc = __ballot_sync(0xffffffffu, tc), br = __ballot_sync(0xffffffffu, tr);
-    const bool sc = a[s] > Tc || (tc && rank_c + __popc(bc & lt_mask) < need_c);
-    const bool sr = bk[s] > Tr || (tr && rank_r + __popc(br & lt_mask) < need_r);
-    if (sc) atomicOr(&words_c[ia[s] >> 5], 1u << (ia[s] & 31));
-    if (sr) atomicOr(&words_r[ib[s] >> 5], 1u << (ib[s] & 31));
-    rank_c += __popc(bc);
-    rank_r += __popc(br);
-  }
-  __syncwarp();
-  return true;
+  return topk2_from_bounds(key_c, key_r, Lc, Lr, k_c, k_r, nt, lane, nwords, scratch, words_c, words_r);
 }
 
 // The row's mask words (and forced blocks) -> the mask arrays and the row's
@@ -333,7 +454,9 @@ __device__ __forceinline__ void select_row_keys(const SelectArgs& a, KC key_c, K
   uint32_t* words_c = scratch + 4 * kTopkCap;
   uint32_t* words_r = words_c + a.nwords;
   const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
-  const bool done = warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, n, lane, a.nwords, scratch, words_c, words_r);
+  const bool done =
+      warp_topk2_sorted<KP>(key_c, key_r, k_c, k_r, n, lane, a.nwords, scratch, words_c, words_r) ||
+      warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, n, lane, a.nwords, scratch, words_c, words_r);
   if (!done) {
     uint32_t kc[KP], kr[KP];
 #pragma unroll

@@ -443,8 +443,11 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(TopkArgs t) {
     const float qn = t.qnorm[row];
     const int nq4 = (n + 3) / 4;
     // float4 per lane per chunk: as many as the longest row of this
-    // instantiation needs (up to 8), so short rows issue no idle loads
-    constexpr int kU = KPL / 4 < 1 ? 1 : (KPL / 4 > 8 ? 8 : KPL / 4);
+    // instantiation needs, at most 4 (512 key blocks); a longer row takes
+    // several chunks.  Every slot of a chunk issues its instructions whether
+    // or not it holds a block, so a larger chunk would cost the shorter rows
+    // of an instantiation more than the extra round trip costs the longest.
+    constexpr int kU = KPL / 4 < 1 ? 1 : (KPL / 4 > 4 ? 4 : KPL / 4);
     const bool vec = (a.nkb & 3) == 0;
     for (int base = 0; base < nq4; base += 32 * kU) {
       float4 s4[kU], r4[kU], b4[kU];

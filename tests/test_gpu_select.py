@@ -11,9 +11,9 @@ import pytest
 import torch
 
 import block_sparse_long_rbs_b200 as rbs
-from helpers import compare_selection, dev
+from helpers import compare_selection, dense_masks, dev, lists_np
 from oracle import rbs_oracle as O
-from workloads import WORKLOADS, make_inputs, make_mixture, make_tiny
+from workloads import WORKLOADS, make_inputs, make_mixture, make_tied, make_tiny
 
 pytestmark = pytest.mark.gpu
 
@@ -80,6 +80,38 @@ def test_select_128k_config(cuda_ok):
     print("128k", rep)
 
 
+@pytest.mark.parametrize("n_patterns", [3, 40, 128])
+def test_select_exact_ties(cuda_ok, n_patterns):
+    # Scores tie exactly (repeated integer block contents): each branch must
+    # keep the oracle's set exactly, ties at the threshold going to the lowest
+    # block indices, with no near-threshold excuse.  Few patterns put hundreds
+    # of ties at the threshold (more candidates than the pruned searches
+    # hold), many put a handful.  512 key blocks: the widest top-k rows.
+    block, rho = 128, 0.05
+    inp = make_tied(L=65536, Hq=2, Hkv=1, block=block, n_patterns=n_patterns, seed=211)
+    Q, K = inp["Q"], inp["K"]
+    nqb = nkb = 65536 // block
+    p = rbs.SelectParams(block_q=block, block_k=block, rho_centroid=rho, rho_rescue=rho)
+    Cg, Rg = rbs.rbs_block_stats(dev(K), block)
+    lists = rbs.rbs_select(dev(Q), Cg, Rg, p)
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    Co, Ro = O.block_stats(K, block)
+    ora = O.select_blocks(Q, Co, Ro, O.SelectParams(block_q=block, block_k=block, rho_centroid=float(np.float32(rho)),
+                                                     rho_rescue=float(np.float32(rho))), keep_scores=True)
+    grp, gci, gfl = lists_np(lists)
+    _, gc, gr = dense_masks(grp, gci, gfl, nkb)
+    _, oc, orr = dense_masks(ora["row_ptr"], ora["col_idx"], ora["flags"], nkb)
+    assert np.array_equal(gc, oc) and np.array_equal(gr, orr)
+    # the ties are real: rows whose centroid threshold is shared by more
+    # blocks than the branch keeps
+    s_c = ora["scores"][(0, 0)][0]
+    tau = ora["tau"][0, 0, :, 0]
+    tied = [int((s_c[i, :i + 1] == tau[i]).sum()) for i in range(nqb)]
+    assert max(tied) > 1
+    print("ties", n_patterns, "max tied at tau", max(tied))
+
+
 def test_select_deterministic(cuda_ok):
     inp = make_tiny(L=2048)
     p = rbs.SelectParams(block_q=64, block_k=64, rho_centroid=0.25, rho_rescue=0.25)
@@ -89,6 +121,41 @@ def test_select_deterministic(cuda_ok):
     assert torch.equal(a.row_ptr, b.row_ptr)
     n = a.nnz()
     assert torch.equal(a.col_idx[:n], b.col_idx[:n]) and torch.equal(a.flags[:n], b.flags[:n])
+
+
+def test_select_graph_capture_matches_eager(cuda_ok):
+    # Selection captured into a CUDA graph (every launch on the capturing
+    # stream, no host synchronisation inside the call) gives the eager lists,
+    # and a replayed graph recomputes them from new inputs in the same
+    # buffers.
+    inp = make_mixture(L=8192, Hq=16, Hkv=2, block=128, seed=207)
+    Q, K = dev(inp["Q"]), dev(inp["K"])
+    B, L, Hq, _ = Q.shape
+    Hkv, nqb, nkb = K.shape[2], L // 128, L // 128
+    p = rbs.SelectParams(block_q=128, block_k=128, rho_centroid=0.1, rho_rescue=0.1)
+    C, R = rbs.rbs_block_stats(K, 128)
+    eager = rbs.rbs_select(Q, C, R, p)
+    ws = torch.empty(rbs.rbs_select_workspace_bytes(B, Hq, nqb, Hkv, nkb, p), dtype=torch.uint8, device="cuda")
+    out = rbs.BlockLists.empty(B * Hq * nqb, rbs.rbs_select_capacity(B, Hq, nqb, nkb, p), "cuda")
+    Qg = torch.zeros_like(Q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        rbs.rbs_select(Qg, C, R, p, workspace=ws, out=out)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        rbs.rbs_select(Qg, C, R, p, workspace=ws, out=out)
+    Qg.copy_(Q)
+    g.replay()
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    n = eager.nnz()
+    assert out.nnz() == n
+    assert torch.equal(out.row_ptr, eager.row_ptr)
+    assert torch.equal(out.col_idx[:n], eager.col_idx[:n]) and torch.equal(out.flags[:n], eager.flags[:n])
+    del g
 
 
 def test_select_rho_one_is_causal_full(cuda_ok):

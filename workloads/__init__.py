@@ -14,5 +14,6 @@ from .generators import (  # noqa: F401
     make_block_attention,
     make_inputs,
     make_mixture,
+    make_tied,
     make_tiny,
 )

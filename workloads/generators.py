@@ -106,6 +106,29 @@ def _plant(K: np.ndarray, Q: np.ndarray, b: int, kvh: int, pos_k: int, q_tok: in
     K[b, pos_k, kvh] = f32_to_bf16_bits((scale * q).astype(np.float32))
 
 
+def make_tied(L: int, Hq: int, Hkv: int, block: int, n_patterns: int, seed: int, batch: int = 1) -> dict:
+    """Inputs whose block scores tie exactly: Q and K entries are integers in
+    {-1, 0, 1} (exact in bf16), and the key blocks repeat n_patterns block
+    contents (block j of each KV head takes pattern (7 j + h) % n_patterns).
+    Centroids and pooled queries are then binary fractions, and blocks with
+    the same content score the same, so each selection row holds about
+    n / n_patterns exactly tied scores per value.  V is N(0, 1).
+    """
+    d = HEAD_DIM
+    nb = L // block
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Q = f32_to_bf16_bits(rng.integers(-1, 2, size=(batch, L, Hq, d)).astype(np.float32))
+    pats = rng.integers(-1, 2, size=(batch, Hkv, n_patterns, block, d)).astype(np.float32)
+    Kf = np.empty((batch, L, Hkv, d), dtype=np.float32)
+    for b in range(batch):
+        for h in range(Hkv):
+            for j in range(nb):
+                Kf[b, j * block:(j + 1) * block, h] = pats[b, h, (7 * j + h) % n_patterns]
+    K = f32_to_bf16_bits(Kf)
+    V = _normal_bf16(rng, (batch, L, Hkv, d))
+    return {"Q": Q, "K": K, "V": V}
+
+
 def make_tiny(L: int = 4096, Hq: int = 2, Hkv: int = 1, block: int = 64, seed: int = SEED_BASE + 0,
               batch: int = 1, offset_std: float = 0.5, plant_every: int = 16, logit: float = 8.0) -> dict:
     """Tiny RBS workload: N(0,1) Q/K/V, per-block N(0, offset_std^2) key offsets, planted keys.
