@@ -46,7 +46,7 @@ BLOCK = 128
 HEAD_DIM = 128
 FLOP_PER_PAIR = 4 * BLOCK * BLOCK * HEAD_DIM  # QK^T and PV on one 128x128 block pair
 # kernels one step launches: block stats; selection (beta, centroid split,
-# pooling, score MMAs, top-k, scan, compaction); attention
+# pooling, score MMAs, top-k, tile scan, compaction); attention
 LAUNCHES_PER_STEP = 9
 ATTN_KERNEL = "bsa_prefill_kernel<128,128>"
 SWEEP_TARGETS = (0.02, 0.05, 0.10, 0.25, 0.50, 1.00)

@@ -204,7 +204,8 @@ rbs_status make_pool_tensor_map(const rbs_bf16_tensor* t, int R, CUtensorMap* ma
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct SelectLayout {
-  size_t mask_c, mask_r, counts, beta, c_hi, c_lo, q_hi, q_lo, qnorm, scores;
+  size_t mask_c, mask_r, counts, beta, tiles, c_hi, c_lo, q_hi, q_lo, qnorm, scores;
+  int64_t ntiles;  // partial sums of the row-pointer scan (kScanTile rows each)
   size_t base;   // bytes the fused mean-query kernel needs
   size_t total;  // bytes of the full layout
 };
@@ -221,6 +222,8 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
   l.mask_r = off; off += align256(rows * nwords * 4);
   l.counts = off; off += align256(rows * 4);
   l.beta = off; off += align256(B * Hkv * nkb * 4);
+  l.ntiles = (rows + kScanTile - 1) / kScanTile;  // list rows <= rows
+  l.tiles = off; off += align256(2 * l.ntiles * 4);  // the sums, then their exclusive prefixes
   l.base = off;
   l.c_hi = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
   l.c_lo = off; off += align256(B * Hkv * nkb * RBS_HEAD_DIM * 2);
@@ -666,6 +669,13 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   sa.mask_c = reinterpret_cast<uint32_t*>(ws + lay.mask_c);
   sa.mask_r = reinterpret_cast<uint32_t*>(ws + lay.mask_r);
   sa.counts = reinterpret_cast<int*>(ws + lay.counts);
+  int* tile_sums = reinterpret_cast<int*>(ws + lay.tiles);
+  int* tile_prefix = tile_sums + lay.ntiles;
+  const int64_t list_tiles = (list_rows + kScanTile - 1) / kScanTile;
+  // KV_GROUP lists sum the group unions' counts instead (group_counts_kernel)
+  sa.tile_sums = p->list_mode == 1 ? nullptr : tile_sums;
+  if (cudaMemsetAsync(tile_sums, 0, static_cast<size_t>(list_tiles) * 4, stream) != cudaSuccess)
+    return fail(RBS_ERR_CUDA, "cudaMemsetAsync failed");
   if (p->query_pool == 1) {
     uint32_t* keys = workspace_bytes >= lay.total ? reinterpret_cast<uint32_t*>(ws + lay.scores) : nullptr;
     if ((st = launch_token_max(Q, centroids, B, kv_heads, nkb, p, sa, ws + lay.c_hi, ws + lay.c_lo, keys, di,
@@ -700,7 +710,6 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   CompactArgs ca;
   ca.mask_c = sa.mask_c;
   ca.mask_r = sa.mask_r;
-  ca.row_ptr = out->row_ptr;
   ca.col_idx = out->col_idx;
   ca.flags = out->flags;
   ca.capacity = out->capacity;
@@ -718,12 +727,13 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
   if (p->list_mode == 1) {
     // the per-head counts written by the selection are replaced by the
     // counts of the group unions (list_rows <= rows entries)
-    group_counts_kernel<<<list_grid, 256, 0, stream>>>(ca, sa.counts);
+    group_counts_kernel<<<list_grid, 256, 0, stream>>>(ca, sa.counts, tile_sums);
     if ((st = check_launch("group_counts_kernel")) != RBS_OK) return st;
   }
-  scan_counts_kernel<<<1, 1024, 0, stream>>>(sa.counts, static_cast<int>(list_rows), out->row_ptr, out->capacity);
-  if ((st = check_launch("scan_counts_kernel")) != RBS_OK) return st;
-  compact_lists_kernel<<<list_grid, 256, 0, stream>>>(ca);
+  scan_tiles_kernel<<<1, 1024, 0, stream>>>(tile_sums, static_cast<int>(list_tiles), tile_prefix, out->row_ptr,
+                                            static_cast<int>(list_rows), out->capacity);
+  if ((st = check_launch("scan_tiles_kernel")) != RBS_OK) return st;
+  compact_lists_kernel<<<list_grid, 256, 0, stream>>>(ca, sa.counts, tile_prefix, out->row_ptr);
   return check_launch("compact_lists_kernel");
 }
 

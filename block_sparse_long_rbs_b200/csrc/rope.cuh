@@ -5,7 +5,7 @@
 // evaluated in fp64 once per (token, m) and shared by all heads of the token;
 // the rotation is applied in fp32 and rounded once to bf16.
 //
-// One 256-thread CTA per 8 tokens of one batch entry.  Rotate-half pairs
+// One 256-thread CTA per 16 tokens of one batch entry.  Rotate-half pairs
 // (m, m + 64): a thread task is (token, head, chunk c in 0..7) and moves the
 // two 16-byte chunks c and c + 8 of the head's row.  Interleaved pairs
 // (2m, 2m + 1): a task is (token, head, chunk c in 0..15) and moves chunk c.
@@ -25,7 +25,7 @@ struct RopeArgs {
   double inv_freq[64];
 };
 
-constexpr int kRopeTokens = 8;
+constexpr int kRopeTokens = 16;
 
 __device__ __forceinline__ void rot8(const uint4& a, const uint4& bsrc, const float* c, const float* s, uint4& oa,
                                      uint4& ob) {
@@ -44,12 +44,41 @@ __device__ __forceinline__ void rot8(const uint4& a, const uint4& bsrc, const fl
   ob = make_uint4(rb[0], rb[1], rb[2], rb[3]);
 }
 
+// Tasks per thread and pass: their loads are issued together, and the first
+// pass's loads before the sine/cosine table is formed, so the table's fp64
+// arithmetic runs under the memory latency instead of ahead of it.  The
+// output is stored with the default policy: the attention pass that follows
+// reads it, and it may still be in L2.
+constexpr int kRopeUnroll = 4;
+
 template <int STYLE>
 __global__ void __launch_bounds__(256) rope_reencode_kernel(const __grid_constant__ RopeArgs a) {
   __shared__ float cs[kRopeTokens][64];
   __shared__ float sn[kRopeTokens][64];
   __shared__ double inv[64];
   const int t0 = blockIdx.x * kRopeTokens, b = blockIdx.y, tid = threadIdx.x;
+  constexpr int CPH = STYLE == 0 ? 8 : 16;  // tasks per head
+  const int tasks = kRopeTokens * a.H * CPH;
+  // task k -> (token tl, head h, chunk c); false past the last token
+  auto task = [&](int k, int& tl, int& h, int& c) {
+    c = k % CPH;
+    h = (k / CPH) % a.H;
+    tl = k / (CPH * a.H);
+    return k < tasks && t0 + tl < a.L;
+  };
+  uint4 va[kRopeUnroll], vb[kRopeUnroll];
+  auto load = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      int tl, h, c;
+      if (task(base + tid + 256 * u, tl, h, c)) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + b * a.xb + (t0 + tl) * a.xs + h * a.xh);
+        va[u] = src[c];
+        if (STYLE == 0) vb[u] = src[c + 8];
+      }
+    }
+  };
+  load(0);
   // the frequency table to shared memory with uniform (non-divergent) reads of
   // the parameter block
   if (tid < 64) {
@@ -87,36 +116,32 @@ __global__ void __launch_bounds__(256) rope_reencode_kernel(const __grid_constan
     }
   }
   __syncthreads();
-  constexpr int CPH = STYLE == 0 ? 8 : 16;  // tasks per head
-  const int tasks = kRopeTokens * a.H * CPH;
-  for (int k = tid; k < tasks; k += blockDim.x) {
-    const int c = k % CPH;
-    const int h = (k / CPH) % a.H;
-    const int tl = k / (CPH * a.H);
-    const int t = t0 + tl;
-    if (t >= a.L) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + b * a.xb + t * a.xs + h * a.xh);
-    uint4* dst = reinterpret_cast<uint4*>(a.y + b * a.yb + t * a.ys + h * a.yh);
-    if (STYLE == 0) {
-      const uint4 lo = src[c], hi = src[c + 8];
-      uint4 olo, ohi;
-      rot8(lo, hi, &cs[tl][8 * c], &sn[tl][8 * c], olo, ohi);
-      dst[c] = olo;
-      dst[c + 8] = ohi;
-    } else {
-      // chunk c holds pairs (2m, 2m+1), m = 4c .. 4c+3: even lanes are the
-      // first member of a pair, odd lanes the second.
-      const uint4 v = src[c];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t r[4];
+  for (int base = 0; base < tasks; base += 256 * kRopeUnroll) {
+    if (base > 0) load(base);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int m = 4 * c + q;
-        const float x0 = bf16lo(w[q]), x1 = bf16hi(w[q]);
-        const float cv = cs[tl][m], sv = sn[tl][m];
-        r[q] = pack_bf16x2(fmaf(x0, cv, -x1 * sv), fmaf(x0, sv, x1 * cv));
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      int tl, h, c;
+      if (!task(base + tid + 256 * u, tl, h, c)) continue;
+      uint4* dst = reinterpret_cast<uint4*>(a.y + b * a.yb + (t0 + tl) * a.ys + h * a.yh);
+      if (STYLE == 0) {
+        uint4 olo, ohi;
+        rot8(va[u], vb[u], &cs[tl][8 * c], &sn[tl][8 * c], olo, ohi);
+        dst[c] = olo;
+        dst[c + 8] = ohi;
+      } else {
+        // chunk c holds pairs (2m, 2m+1), m = 4c .. 4c+3: even lanes are the
+        // first member of a pair, odd lanes the second.
+        const uint32_t w[4] = {va[u].x, va[u].y, va[u].z, va[u].w};
+        uint32_t r[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int m = 4 * c + q;
+          const float x0 = bf16lo(w[q]), x1 = bf16hi(w[q]);
+          const float cv = cs[tl][m], sv = sn[tl][m];
+          r[q] = pack_bf16x2(fmaf(x0, cv, -x1 * sv), fmaf(x0, sv, x1 * cv));
+        }
+        dst[c] = make_uint4(r[0], r[1], r[2], r[3]);
       }
-      dst[c] = make_uint4(r[0], r[1], r[2], r[3]);
     }
   }
 }

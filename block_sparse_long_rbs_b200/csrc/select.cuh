@@ -25,8 +25,11 @@
 //                       32-bit mask word per 32 blocks.
 //   group_counts_kernel (KV_GROUP lists) one warp per (batch, KV head, query
 //                       block) counts the union of its q heads' masks.
-//   scan_counts_kernel  exclusive scan of the per-row counts -> row_ptr.
-//   compact_lists_kernel one warp per list row turns mask words (OR-ed over
+//   scan_tiles_kernel   exclusive scan of the sums of 256 rows' counts (the
+//                       selection kernels add each row's count to its tile's
+//                       sum as they write it).
+//   compact_lists_kernel one warp per list row: its row pointer (tile prefix +
+//                       the tile's earlier counts), and its mask words (OR-ed over
 //                       the q heads of a KV_GROUP row) into ascending block
 //                       indices and per-entry branch flags.
 #pragma once
@@ -50,7 +53,13 @@ struct SelectArgs {
   uint32_t* mask_c;  // [rows, nwords]
   uint32_t* mask_r;  // [rows, nwords]
   int* counts;       // [rows]
+  // [ceil(rows / kScanTile)] sums of the counts of kScanTile consecutive rows
+  // (zero on entry, added to as rows finish), or null when another kernel
+  // forms the list rows' counts
+  int* tile_sums;
 };
+
+constexpr int kScanTile = 256;  // rows per partial sum of the row-pointer scan
 
 constexpr int kSelComputeThreads = 256;  // warps 0-7: scores and top-k
 constexpr int kSelPoolThreads = 64;      // warps 8-9: pooling of the next item
@@ -441,7 +450,10 @@ __device__ __forceinline__ void emit_row(const SelectArgs& a, const uint32_t* wo
     a.mask_r[row * a.nwords + t] = wr;
   }
   cnt = __reduce_add_sync(0xffffffffu, cnt);
-  if (lane == 0) a.counts[row] = cnt;
+  if (lane == 0) {
+    a.counts[row] = cnt;
+    if (a.tile_sums != nullptr) atomicAdd(a.tile_sums + row / kScanTile, cnt);
+  }
 }
 
 // Both branches' top-k (TOPK_FRACTION) of one list row from order-preserving
@@ -795,38 +807,18 @@ __global__ void __launch_bounds__(kSelThreads, KPL <= 32 ? 2 : 1)
   }
 }
 
-// Exclusive scan of per-row counts into row_ptr (one CTA of 1024 threads;
-// each thread owns a contiguous run of rows, read 32 at a time with all the
-// loads of a run issued before any is used).
-__device__ __forceinline__ void load_counts32(const int* __restrict__ counts, int c, int s1, int (&v)[32]) {
-#pragma unroll
-  for (int u = 0; u < 32; u += 4) {
-    if (c + u + 4 <= s1) {
-      const int4 x = *reinterpret_cast<const int4*>(counts + c + u);
-      v[u] = x.x;
-      v[u + 1] = x.y;
-      v[u + 2] = x.z;
-      v[u + 3] = x.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) v[u + e] = c + u + e < s1 ? counts[c + u + e] : 0;
-    }
-  }
-}
-
-__global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict__ counts, int rows,
-                                                           int* __restrict__ row_ptr, int64_t capacity) {
+// Exclusive scan of the tile sums (one CTA of 1024 threads; each thread owns
+// a contiguous run of tiles) into tile_prefix, and the total into
+// row_ptr[rows].  The row pointers themselves are formed by the compaction.
+__global__ void __launch_bounds__(1024) scan_tiles_kernel(const int* __restrict__ tile_sums, int ntiles,
+                                                          int* __restrict__ tile_prefix, int* __restrict__ row_ptr,
+                                                          int rows, int64_t capacity) {
   __shared__ long long wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = ((rows + 1023) / 1024 + 3) & ~3;  // multiple of 4: runs start 16-byte aligned
-  const int s0 = min(rows, tid * per), s1 = min(rows, s0 + per);
+  const int per = (ntiles + 1023) / 1024;
+  const int s0 = min(ntiles, tid * per), s1 = min(ntiles, s0 + per);
   long long local = 0;
-  for (int c = s0; c < s1; c += 32) {
-    int v[32];
-    load_counts32(counts, c, s1, v);
-#pragma unroll
-    for (int u = 0; u < 32; ++u) local += v[u];
-  }
+  for (int t = s0; t < s1; ++t) local += tile_sums[t];
   long long incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -836,7 +828,7 @@ __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    long long w = wsum[lane];
+    const long long w = wsum[lane];
     long long wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -847,36 +839,19 @@ __global__ void __launch_bounds__(1024) scan_counts_kernel(const int* __restrict
   }
   __syncthreads();
   long long run = wsum[warp] + incl - local;
-  for (int c = s0; c < s1; c += 32) {
-    int v[32];
-    load_counts32(counts, c, s1, v);
-    int out[32];
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      out[u] = static_cast<int>(run);
-      run += v[u];
-    }
-#pragma unroll
-    for (int u = 0; u < 32; u += 4) {
-      if (c + u + 4 <= s1) {
-        *reinterpret_cast<int4*>(row_ptr + c + u) = make_int4(out[u], out[u + 1], out[u + 2], out[u + 3]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (c + u + e < s1) row_ptr[c + u + e] = out[u + e];
-      }
-    }
+  for (int t = s0; t < s1; ++t) {
+    tile_prefix[t] = static_cast<int>(run);
+    run += tile_sums[t];
   }
   if (tid == 1023) {
     row_ptr[rows] = static_cast<int>(run);
-    if (run > capacity) raise_error(RBS_DEVERR_ROW_PTR);
+    if (run > capacity || run > 0x7fffffffll) raise_error(RBS_DEVERR_ROW_PTR);
   }
 }
 
 struct CompactArgs {
   const uint32_t* mask_c;  // [B * Hq * nqb, nwords], one row per q head
   const uint32_t* mask_r;
-  const int* row_ptr;
   int32_t* col_idx;
   uint8_t* flags;
   int64_t capacity;
@@ -910,7 +885,8 @@ __device__ __forceinline__ void list_row_word(const CompactArgs& a, int b, int h
 }
 
 // KV_GROUP lists: the entry count of every list row (b, g, i).
-__global__ void __launch_bounds__(256) group_counts_kernel(CompactArgs a, int* __restrict__ counts) {
+__global__ void __launch_bounds__(256) group_counts_kernel(CompactArgs a, int* __restrict__ counts,
+                                                           int* __restrict__ tile_sums) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= a.rows) return;
@@ -924,10 +900,17 @@ __global__ void __launch_bounds__(256) group_counts_kernel(CompactArgs a, int* _
     cnt += __popc(c | r | forced_word(t, gi, a.nkb, a.force_diag, a.force_sink));
   }
   cnt = __reduce_add_sync(0xffffffffu, cnt);
-  if (lane == 0) counts[row] = cnt;
+  if (lane == 0) {
+    counts[row] = cnt;
+    atomicAdd(tile_sums + row / kScanTile, cnt);
+  }
 }
 
-__global__ void __launch_bounds__(256) compact_lists_kernel(CompactArgs a) {
+// One warp per list row: its row pointer (the tile's prefix plus the counts
+// of the tile's earlier rows) and its entries.
+__global__ void __launch_bounds__(256) compact_lists_kernel(CompactArgs a, const int* __restrict__ counts,
+                                                            const int* __restrict__ tile_prefix,
+                                                            int* __restrict__ row_ptr) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= a.rows) return;
@@ -937,11 +920,22 @@ __global__ void __launch_bounds__(256) compact_lists_kernel(CompactArgs a) {
   // the row's first mask words are loaded together with its extent
   uint32_t c0 = 0, r0 = 0;
   if (lane < a.nwords) list_row_word(a, b, hl, i, lane, c0, r0);
-  const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
-  if (beg < 0 || end < beg || end > a.capacity) {
+  const int t0 = row - row % kScanTile;
+  int before = 0;  // counts of rows t0 .. row - 1
+#pragma unroll
+  for (int u = 0; u < kScanTile / 32; ++u) {
+    const int r = t0 + u * 32 + lane;
+    before += r < row ? counts[r] : 0;
+  }
+  before = __reduce_add_sync(0xffffffffu, before);
+  const long long beg64 = static_cast<long long>(tile_prefix[row / kScanTile]) + before;
+  const long long end64 = beg64 + counts[row];
+  if (end64 > a.capacity || end64 > 0x7fffffffll) {
     if (lane == 0) raise_error(RBS_DEVERR_ROW_PTR);
     return;
   }
+  const int beg = static_cast<int>(beg64), end = static_cast<int>(end64);
+  if (lane == 0) row_ptr[row] = beg;
   int run = beg;
   for (int w0 = 0; w0 < a.nwords; w0 += 32) {
     const int t = w0 + lane;

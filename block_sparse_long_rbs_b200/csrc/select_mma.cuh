@@ -209,6 +209,13 @@ __device__ __forceinline__ void gemm_item(const GemmArgs& a, int w, int& b, int&
   i0 = g * a.QB;
 }
 
+// The k-th item of CTA c of G: a snake over the longest-first item order
+// (c, 2G - 1 - c, 2G + c, 4G - 1 - c, ...), so a CTA that takes one of the
+// longest items of a round takes one of the shortest of the next: the items'
+// tile counts fall from 8 to 1 at 128K, and the busiest CTA's total drops
+// from half again the mean (round-robin) to about the mean.  Increasing in k.
+__device__ __forceinline__ int gemm_work(int k, int c, int G) { return (k & 1) ? (k + 1) * G - 1 - c : k * G + c; }
+
 __device__ __forceinline__ int gemm_tiles(const GemmArgs& a, int i0) {
   const int i_last = min(a.nqb - 1, i0 + a.QB - 1);
   const int n = a.causal ? min(a.nkb, i_last + a.q_block_offset + 1) : a.nkb;
@@ -227,9 +234,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) score_gemm_kernel(const __gri
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + kGmNumBars * 8 + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.Hq / a.Hkv;
-  const int nitems = a.items > static_cast<int>(blockIdx.x)
-                         ? (a.items - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-                         : 0;
+  const int cta = static_cast<int>(blockIdx.x), grid = static_cast<int>(gridDim.x);
+  int nitems = 0;
+  while (gemm_work(nitems, cta, grid) < a.items) ++nitems;
 
   if (tid == 0) {
     mbar_init(bar(kGmBFull), 1);
@@ -264,7 +271,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) score_gemm_kernel(const __gri
       bool ok = true;
       for (int k = 0; k < nitems && ok; ++k) {
         int b, hq0, i0;
-        gemm_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq0, i0);
+        gemm_item(a, gemm_work(k, cta, grid), b, hq0, i0);
         if (k > 0 && !mbar_wait(bar(kGmBEmpty), (k - 1) & 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(bar(kGmBFull), 2 * b_bytes);
         // box rows (R heads x QB blocks) land as 128-byte rows h * QB + ii of each half
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) score_gemm_kernel(const __gri
     bool ok = true;
     for (int k = 0; k < nitems && ok; ++k) {
       int b, hq0, i0;
-      gemm_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq0, i0);
+      gemm_item(a, gemm_work(k, cta, grid), b, hq0, i0);
       if (!wait(kGmBFull, k & 1)) break;
       const int T = gemm_tiles(a, i0);
       for (int m = 0; m < T; ++m, ++gt) {
@@ -339,7 +346,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) score_gemm_kernel(const __gri
     bool ok = true;
     for (int k = 0; k < nitems; ++k) {
       int b, hq0, i0;
-      gemm_item(a, static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x), b, hq0, i0);
+      gemm_item(a, gemm_work(k, cta, grid), b, hq0, i0);
       const int T = gemm_tiles(a, i0);
       named_bar_sync(1, 256);  // the previous item's columns are no longer read
       if (etid < 128) {
