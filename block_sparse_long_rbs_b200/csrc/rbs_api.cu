@@ -102,6 +102,7 @@ rbs_status device_info(DeviceInfo** out) {
       e = e ? e : cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(topk_smem_bytes(kTokMaxKV, kTokMaxKV / 32)));
     e = e ? e : cudaFuncSetAttribute(block_beta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
+    e = e ? e : cudaFuncSetAttribute(select_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RBS_MAX_KV_BLOCKS * 4);
     if (e != cudaSuccess) return fail(RBS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     d.attrs_set = true;
   }
@@ -240,15 +241,16 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
   return l;
 }
 
-// Both branches' top-k of every row from the stored scores or keys, eight
+// Both branches' top-k of every row from the stored scores or keys, kTopkWarps
 // rows per CTA, with as many key slots per lane as the longest row needs.
 void launch_topk_rows(const TopkArgs& t, int64_t nkb, rbs_stream_t stream) {
   const size_t tsm = topk_smem_bytes(t.nkbp, t.s.nwords);
-  const unsigned tgrid = static_cast<unsigned>((t.rows + 7) / 8);
-  if (nkb <= 64) topk_rows_kernel<2><<<tgrid, 256, tsm, stream>>>(t);
-  else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, 256, tsm, stream>>>(t);
-  else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, 256, tsm, stream>>>(t);
-  else topk_rows_kernel<64><<<tgrid, 256, tsm, stream>>>(t);
+  const unsigned tgrid = static_cast<unsigned>((t.rows + kTopkWarps - 1) / kTopkWarps);
+  constexpr int kThreads = kTopkWarps * 32;
+  if (nkb <= 64) topk_rows_kernel<2><<<tgrid, kThreads, tsm, stream>>>(t);
+  else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, kThreads, tsm, stream>>>(t);
+  else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, kThreads, tsm, stream>>>(t);
+  else topk_rows_kernel<64><<<tgrid, kThreads, tsm, stream>>>(t);
 }
 
 // Per-token-max selection scores (query_pool TOKEN_MAX): split the centroids
@@ -261,12 +263,6 @@ rbs_status launch_token_max(const rbs_bf16_tensor* Q, const float* centroids, in
                             const rbs_select_params* p, const SelectArgs& sa, uint8_t* c_hi, uint8_t* c_lo,
                             uint32_t* keys, DeviceInfo* di, rbs_stream_t stream) {
   rbs_status st;
-  const int64_t n = B * Hkv * nkb * RBS_HEAD_DIM;
-  auto* hi = reinterpret_cast<__nv_bfloat16*>(c_hi);
-  auto* lo = reinterpret_cast<__nv_bfloat16*>(c_lo);
-  split_centroids_kernel<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 4 * di->sms)), 256, 0, stream>>>(
-      centroids, n, hi, lo);
-  if ((st = check_launch("split_centroids_kernel")) != RBS_OK) return st;
   TokArgs ta;
   int si = 0;
   if ((st = make_tensor_map(Q, p->block_q, &ta.tmQ, &si)) != RBS_OK) return st;
@@ -349,10 +345,6 @@ rbs_status launch_mma_select(const rbs_bf16_tensor* Q, const float* centroids, i
   float* qnorm = reinterpret_cast<float*>(ws + lay.qnorm);
   float* scores = reinterpret_cast<float*>(ws + lay.scores);
 
-  const int64_t nc = B * Hkv * nkb * RBS_HEAD_DIM;
-  split_centroids_kernel<<<static_cast<unsigned>(std::min<int64_t>((nc + 255) / 256, 4 * di->sms)), 256, 0, stream>>>(
-      centroids, nc, c_hi, c_lo);
-  if ((st = check_launch("split_centroids_kernel")) != RBS_OK) return st;
 
   // pooling
   PoolArgs pa;
@@ -525,8 +517,14 @@ rbs_status rbs_block_stats(const rbs_bf16_tensor* K, int32_t block_k, float* cen
   return check_launch("block_stats_kernel");
 }
 
-rbs_status rbs_block_beta(const float* radii, int64_t batch, int64_t kv_heads, int64_t num_blocks,
-                          const rbs_select_params* p, float* beta, float* radius_range, rbs_stream_t stream) {
+}  // extern "C"
+
+// Validates the beta parameters, then launches beta alone (block_beta_kernel)
+// or, with split_n > 0, beta and the centroids' bf16 hi / lo split as one
+// launch (select_prep_kernel).
+rbs_status launch_beta(const float* radii, int64_t batch, int64_t kv_heads, int64_t num_blocks,
+                       const rbs_select_params* p, float* beta, float* radius_range, const float* centroids,
+                       int64_t split_n, void* c_hi, void* c_lo, rbs_stream_t stream) {
   RBS_REQUIRE(radii != nullptr && beta != nullptr && p != nullptr, RBS_ERR_INVALID_ARG, "null argument");
   RBS_REQUIRE(batch > 0 && kv_heads > 0 && num_blocks > 0, RBS_ERR_INVALID_ARG, "empty shape");
   RBS_REQUIRE(num_blocks <= RBS_MAX_KV_BLOCKS, RBS_ERR_UNSUPPORTED, "num_blocks > %d", RBS_MAX_KV_BLOCKS);
@@ -539,10 +537,34 @@ rbs_status rbs_block_beta(const float* radii, int64_t batch, int64_t kv_heads, i
   if (st != RBS_OK) return st;
   int n2 = 1;
   while (n2 < num_blocks) n2 <<= 1;
-  block_beta_kernel<<<dim3(static_cast<unsigned>(kv_heads), static_cast<unsigned>(batch)), 1024, n2 * 4, stream>>>(
-      radii, static_cast<int>(num_blocks), static_cast<int>(kv_heads), p->beta_mode, p->beta_const, p->beta_p_lo,
-      p->beta_p_hi, beta, radius_range);
-  return check_launch("block_beta_kernel");
+  BetaArgs ba;
+  ba.R = radii;
+  ba.nkb = static_cast<int>(num_blocks);
+  ba.H = static_cast<int>(kv_heads);
+  ba.mode = p->beta_mode;
+  ba.beta_const = p->beta_const;
+  ba.p_lo = p->beta_p_lo;
+  ba.p_hi = p->beta_p_hi;
+  ba.beta = beta;
+  ba.range = radius_range;
+  if (split_n == 0) {
+    block_beta_kernel<<<dim3(static_cast<unsigned>(kv_heads), static_cast<unsigned>(batch)), 1024, n2 * 4, stream>>>(
+        ba);
+    return check_launch("block_beta_kernel");
+  }
+  const int64_t nbeta = batch * kv_heads;
+  const int64_t nsplit = std::min<int64_t>((split_n + 1023) / 1024, di->sms);
+  select_prep_kernel<<<static_cast<unsigned>(nbeta + nsplit), 1024, n2 * 4, stream>>>(
+      ba, static_cast<int>(nbeta), centroids, split_n, static_cast<__nv_bfloat16*>(c_hi),
+      static_cast<__nv_bfloat16*>(c_lo));
+  return check_launch("select_prep_kernel");
+}
+
+extern "C" {
+
+rbs_status rbs_block_beta(const float* radii, int64_t batch, int64_t kv_heads, int64_t num_blocks,
+                          const rbs_select_params* p, float* beta, float* radius_range, rbs_stream_t stream) {
+  return launch_beta(radii, batch, kv_heads, num_blocks, p, beta, radius_range, nullptr, 0, nullptr, nullptr, stream);
 }
 
 rbs_status rbs_pool_queries(const rbs_bf16_tensor* Q, int32_t block_q, float* qbar, float* qnorm,
@@ -634,7 +656,12 @@ rbs_status rbs_select(const rbs_bf16_tensor* Q, const float* centroids, const fl
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* beta = beta_out != nullptr ? beta_out : reinterpret_cast<float*>(ws + lay.beta);
-  if ((st = rbs_block_beta(radii, B, kv_heads, nkb, p, beta, nullptr, stream)) != RBS_OK) return st;
+  // the tensor-core and per-token scoring need the centroids' bf16 hi / lo
+  // parts: split them in the same launch as beta
+  const int64_t split_n = (p->query_pool == 1 || mma_path) ? B * kv_heads * nkb * RBS_HEAD_DIM : 0;
+  if ((st = launch_beta(radii, B, kv_heads, nkb, p, beta, nullptr, centroids, split_n, ws + lay.c_hi, ws + lay.c_lo,
+                        stream)) != RBS_OK)
+    return st;
 
   const int G = static_cast<int>(Hq / kv_heads);
   int R = 1;

@@ -401,18 +401,24 @@ struct TopkArgs {
   int nkbp, rows;
 };
 
+// Rows (one warp each) per CTA of topk_rows_kernel.  The kernel is bound by
+// instruction issue, so the more warps an SM holds the better; its shared
+// memory (two key rows per warp) and registers cap that near 20 warps, which
+// CTAs of four warps reach (five per SM) and CTAs of eight (two) do not.
+constexpr int kTopkWarps = 4;
+
 // Shared memory of topk_rows_kernel: per warp the row's scores and the KV
 // head's r_j beta_j (nkbp floats each), then per warp the top-k scratch.
 __host__ __device__ constexpr size_t topk_smem_bytes(int nkbp, int nwords) {
-  return static_cast<size_t>(8) * (2 * nkbp + sel_topk_scratch_words(nwords)) * 4;
+  return static_cast<size_t>(kTopkWarps) * (2 * nkbp + sel_topk_scratch_words(nwords)) * 4;
 }
 
 template <int KPL>
-__global__ void __launch_bounds__(256) topk_rows_kernel(TopkArgs t) {
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(TopkArgs t) {
   extern __shared__ __align__(16) float topk_smem[];
   const SelectArgs& a = t.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int w = blockIdx.x * 8 + warp;
+  const int w = blockIdx.x * kTopkWarps + warp;
   if (w >= t.rows) return;
   // rows with the last query blocks (the longest) first
   const int per_i = a.B * a.Hq;
@@ -426,7 +432,8 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(TopkArgs t) {
   const int64_t kv_off = static_cast<int64_t>(b * a.Hkv + kvh) * a.nkb;
   float* ssc = topk_smem + warp * 2 * t.nkbp;
   float* srb = ssc + t.nkbp;
-  uint32_t* scratch = reinterpret_cast<uint32_t*>(topk_smem + 8 * 2 * t.nkbp) + warp * sel_topk_scratch_words(a.nwords);
+  uint32_t* scratch =
+      reinterpret_cast<uint32_t*>(topk_smem + kTopkWarps * 2 * t.nkbp) + warp * sel_topk_scratch_words(a.nwords);
   // both branches' order-preserving keys of blocks 0 .. n-1, in place
   uint32_t* kcs = reinterpret_cast<uint32_t*>(ssc);
   uint32_t* krs = reinterpret_cast<uint32_t*>(srb);

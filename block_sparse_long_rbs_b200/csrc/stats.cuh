@@ -111,12 +111,24 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
 // (R_hi - R_lo), 0, 1) with R_lo / R_hi linear-interpolation quantiles of that
 // head's radii (a bitonic sort of the radii in shared memory), or a constant.
 
-__global__ void __launch_bounds__(1024) block_beta_kernel(const float* __restrict__ R, int nkb, int H, int mode,
-                                                          float beta_const, float p_lo, float p_hi,
-                                                          float* __restrict__ beta, float* __restrict__ range) {
-  extern __shared__ float s[];
+struct BetaArgs {
+  const float* R;
+  int nkb, H, mode;
+  float beta_const, p_lo, p_hi;
+  float* beta;
+  float* range;
+};
+
+// beta of KV head h of batch entry b; the whole CTA (up to 1024 threads)
+// takes part, with s[] holding a power of two >= nkb floats for the sort.
+__device__ __forceinline__ void block_beta_body(const BetaArgs& ba, int h, int b, float* s) {
+  const float* __restrict__ R = ba.R;
+  const int nkb = ba.nkb, H = ba.H, mode = ba.mode;
+  const float beta_const = ba.beta_const, p_lo = ba.p_lo, p_hi = ba.p_hi;
+  float* __restrict__ beta = ba.beta;
+  float* __restrict__ range = ba.range;
   __shared__ float lo_hi[2];
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int64_t off = static_cast<int64_t>(b * H + h) * nkb;
   if (mode == 1) {
     for (int j = tid; j < nkb; j += blockDim.x) beta[off + j] = beta_const;
@@ -211,6 +223,11 @@ __global__ void __launch_bounds__(1024) block_beta_kernel(const float* __restric
     const float r = R[off + j];
     beta[off + j] = degenerate ? 1.f : fminf(fmaxf((r - rlo) * inv, 0.f), 1.f);
   }
+}
+
+__global__ void __launch_bounds__(1024) block_beta_kernel(const __grid_constant__ BetaArgs ba) {
+  extern __shared__ float beta_sort[];
+  block_beta_body(ba, blockIdx.x, blockIdx.y, beta_sort);
 }
 
 // ---------------------------------------------------------------------------

@@ -34,6 +34,7 @@
 
 #include "common.cuh"
 #include "select.cuh"
+#include "stats.cuh"
 
 namespace rbs {
 
@@ -378,12 +379,22 @@ __global__ void __launch_bounds__(kTokThreads, 1) select_tokmax_kernel(const __g
   }
 }
 
-// c -> (hi, lo) bf16 parts: hi = bf16(c), lo = bf16(c - hi), both rounded to
-// nearest even, so hi + lo carries c to about 2^-17 of its size.
-__global__ void __launch_bounds__(256) split_centroids_kernel(const float* __restrict__ C, int64_t n,
-                                                              __nv_bfloat16* __restrict__ hi,
-                                                              __nv_bfloat16* __restrict__ lo) {
-  for (int64_t k = blockIdx.x * 256ll + threadIdx.x; k < n; k += static_cast<int64_t>(gridDim.x) * 256) {
+// The selection's first launch when it scores on the tensor core: beta of
+// every (batch, KV head) in CTAs 0 .. nbeta - 1 (block_beta_body, nbeta =
+// B Hkv), in the rest the centroids' bf16 parts c -> (hi, lo): hi = bf16(c),
+// lo = bf16(c - hi), both rounded to nearest even, so hi + lo carries c to
+// about 2^-17 of its size.
+__global__ void __launch_bounds__(1024) select_prep_kernel(const __grid_constant__ BetaArgs ba, int nbeta,
+                                                           const float* __restrict__ C, int64_t n,
+                                                           __nv_bfloat16* __restrict__ hi,
+                                                           __nv_bfloat16* __restrict__ lo) {
+  extern __shared__ float prep_sort[];
+  if (static_cast<int>(blockIdx.x) < nbeta) {
+    block_beta_body(ba, static_cast<int>(blockIdx.x) % ba.H, static_cast<int>(blockIdx.x) / ba.H, prep_sort);
+    return;
+  }
+  const int64_t stride = static_cast<int64_t>(gridDim.x - nbeta) * 1024;
+  for (int64_t k = static_cast<int64_t>(blockIdx.x - nbeta) * 1024 + threadIdx.x; k < n; k += stride) {
     const float c = C[k];
     const __nv_bfloat16 h = __float2bfloat16_rn(c);
     hi[k] = h;
