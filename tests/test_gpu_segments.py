@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import block_sparse_long_rbs_b200 as rbs
-from helpers import dev, lists_np, o_rows_close
+from helpers import TOL_O_ABS, dev, lists_np, o_rows_close
 from oracle import rbs_oracle as O
 from workloads import make_block_attention
 
@@ -103,3 +103,57 @@ def test_block_aligned_segments_equal_plain_prefill(cuda_ok):
     a = rbs.bsa_prefill_segments(Q, K, V, lists, seg, final)
     b = rbs.bsa_prefill(Q, K, V, lists, BLK, BLK)
     assert torch.equal(a, b)
+
+
+FULL_RAGGED = [2048] * 7 + [1999, 2100, 2045] + [2048] * 6  # the bench's ragged variant (same total)
+
+
+@pytest.mark.parametrize("ragged", [False, True])
+def test_block_attention_full_config_sampled_rows(cuda_ok, ragged):
+    # The Block-attention workload at its full size: 16 passages (2048 tokens
+    # each, or three of 1,999 / 2,100 / 2,045 tokens), a 512-token final
+    # block, 32 q / 8 KV heads.  Cache build at local positions, re-encoding
+    # of the cached keys, final pass at global positions, as the bench runs
+    # them; sampled rows against the oracle (keys encoded directly at their
+    # positions), including query blocks that straddle a passage boundary.
+    theta = 500000.0
+    inp = make_block_attention(passages=16, passage_len=2048, final_len=512, Hq=32, Hkv=8, block=BLK,
+                               passage_lens=FULL_RAGGED if ragged else None)
+    seg, final = inp["seg_start"].tolist(), inp["final_start"]
+    L = inp["Q"].shape[1]
+    nqb, fb = L // BLK, final // BLK
+    Qraw, Kraw, V = dev(inp["Q"]), dev(inp["K"]), dev(inp["V"])
+    zero = torch.zeros(L, dtype=torch.int32, device="cuda")
+    loc = torch.from_numpy(inp["local_pos"]).cuda()
+    glob = torch.from_numpy(inp["global_pos"]).cuda()
+    Kc = rbs.rope_reencode(Kraw, zero, loc, theta)
+    Qc = rbs.rope_reencode(Qraw, zero, loc, theta)
+    cache = rbs.rbs_lists_block_attention(seg, final, BLK, 1, 32, 0, fb)
+    Opass = rbs.bsa_prefill_segments(Qc[:, :final], Kc[:, :final], V[:, :final], cache, seg, final)
+    Kg = rbs.rope_reencode(Kc, loc, glob, theta)
+    Qf = rbs.rope_reencode(Qraw[:, final:].contiguous(), zero[:L - final], glob[final:], theta)
+    fin = rbs.rbs_lists_block_attention(seg, final, BLK, 1, 32, fb, nqb - fb)
+    Ofin = rbs.bsa_prefill_segments(Qf, Kg, V, fin, seg, final, q_offset=final)
+    torch.cuda.synchronize()
+    assert rbs.rbs_get_device_error() == 0
+    Vf = O.bf16_to_f64(inp["V"])
+    # final block: every key of the prompt, causally, at global positions
+    Kglob = O.rope_rotate(inp["K"], inp["global_pos"], theta)
+    Qg = O.rope_rotate(inp["Q"][:, final:], inp["global_pos"][final:], theta)
+    rp, ci = O.block_attention_lists(seg, final, BLK, 1, 32, fb, nqb - fb)
+    ks = O.block_attention_key_start(seg, final, range(final, L))
+    rows = [0 * 4 + 0, 7 * 4 + 3, 19 * 4 + 1, 31 * 4 + 3]  # (q head, final query block)
+    Oo, _ = O.masked_attention(Qg, Kglob, Vf, rp, ci, BLK, BLK, q_offset=final, rows=rows, key_start=ks)
+    o_rows_close(Ofin, Oo, rows, 32, nqb - fb, BLK)
+    # passages: each token sees only its own passage, at local positions
+    Kloc = O.rope_rotate(inp["K"][:, :final], inp["local_pos"][:final], theta)
+    og = Opass.float().cpu().numpy()
+    for i0, h in ((0, 0), (127, 5), (128, 12), (143, 30), (160, 21), (fb - 1, 9)):
+        sl = slice(i0 * BLK, (i0 + 1) * BLK)
+        Qs = O.rope_rotate(inp["Q"][:, sl], inp["local_pos"][sl], theta)
+        rp, ci = O.block_attention_lists(seg, final, BLK, 1, 32, i0, 1)
+        ks = O.block_attention_key_start(seg, final, range(i0 * BLK, (i0 + 1) * BLK))
+        Oo, _ = O.masked_attention(Qs, Kloc, Vf[:, :final], rp, ci, BLK, BLK, q_offset=i0 * BLK, rows=[h], key_start=ks)
+        got, ref = og[0, sl, h], Oo[0, :, h]
+        assert np.all(np.isfinite(got)) and np.all(np.isfinite(ref))
+        assert np.abs(got - ref).max() <= TOL_O_ABS, (i0, h, float(np.abs(got - ref).max()))
