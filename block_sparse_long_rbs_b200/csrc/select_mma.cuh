@@ -362,16 +362,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) score_gemm_kernel(const __gri
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kGmDFull + db), (gt >> 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
         const int j = m * 128 + quarter * 32 + lane;
-#pragma unroll 1
-        for (int c0 = 64 * chalf; c0 < 64 * chalf + 64; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + db * 128 + c0, v);
-          tmem_wait_ld();
+        // both 32-column chunks of this warp's half in flight before one wait
+        uint32_t va[32], vb[32];
+        tmem_ld32(lane_base + db * 128 + 64 * chalf, va);
+        tmem_ld32(lane_base + db * 128 + 64 * chalf + 32, vb);
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int row = col_row[c0 + e], n = col_n[c0 + e];
-            if (j < n) a.scores[static_cast<int64_t>(row) * a.nkbp + j] = __uint_as_float(v[e]);
-          }
+        for (int e4 = 0; e4 < 16; ++e4) {
+          // the column tables four columns at a time (broadcast reads)
+          const int4 rw = reinterpret_cast<const int4*>(col_row + 64 * chalf)[e4];
+          const int4 nn = reinterpret_cast<const int4*>(col_n + 64 * chalf)[e4];
+          const int rows4[4] = {rw.x, rw.y, rw.z, rw.w}, ns4[4] = {nn.x, nn.y, nn.z, nn.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (j < ns4[q])
+              a.scores[static_cast<int64_t>(rows4[q]) * a.nkbp + j] =
+                  __uint_as_float(e4 < 8 ? va[4 * e4 + q] : vb[4 * (e4 - 8) + q]);
         }
         tc_fence_before();
         __syncwarp();
