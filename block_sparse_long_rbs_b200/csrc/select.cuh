@@ -402,7 +402,7 @@ __device__ __forceinline__ bool warp_topk2_sorted(KeyC key_c, KeyR key_r, int k_
 // neither enter a lane's top four nor become candidates, so both passes stop
 // before them.  Warp-uniform.
 template <int KP, typename KeyC, typename KeyR>
-__device__ __forceinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_c, int k_r, int n, int lane,
+__device__ __noinline__ bool warp_topk2_pruned(KeyC key_c, KeyR key_r, int k_c, int k_r, int n, int lane,
                                                   int nwords, uint32_t* scratch, uint32_t* words_c,
                                                   uint32_t* words_r) {
   if (k_c > 64 || k_r > 64) return false;
@@ -456,6 +456,28 @@ __device__ __forceinline__ void emit_row(const SelectArgs& a, const uint32_t* wo
   }
 }
 
+// The full 32-step bitwise search of both branches (the last fallback: k > 64
+// or many equal keys), into the mask words.  Warp-wide.
+template <int KP, typename KC, typename KR>
+__device__ __noinline__ void select_row_full(KC key_c, KR key_r, int k_c, int k_r, int lane, int nwords,
+                                             uint32_t* words_c, uint32_t* words_r) {
+  uint32_t kc[KP], kr[KP];
+#pragma unroll
+  for (int t = 0; t < KP; ++t) {
+    kc[t] = key_c(t);
+    kr[t] = key_r(t);
+  }
+  constexpr int NO = (KP + 31) / 32;
+  uint32_t own_c[NO], own_r[NO];
+  warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
+  for (int w = lane; w < nwords; w += 32) {
+    const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
+    words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+    words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
+  }
+  __syncwarp();
+}
+
 // Both branches' top-k (TOPK_FRACTION) of one list row from order-preserving
 // keys: key_c(t), key_r(t) = the keys of block 32t + lane (0 past the n
 // visible blocks); KP slots per lane, mask words covering nwords <=
@@ -466,26 +488,11 @@ __device__ __forceinline__ void select_row_keys(const SelectArgs& a, KC key_c, K
   uint32_t* words_c = scratch + 4 * kTopkCap;
   uint32_t* words_r = words_c + a.nwords;
   const int k_c = keep_count(a.rho_c, n), k_r = keep_count(a.rho_r, n);
+  // the fallbacks (rare) are separate functions, out of the hot path's code
   const bool done =
       warp_topk2_sorted<KP>(key_c, key_r, k_c, k_r, n, lane, a.nwords, scratch, words_c, words_r) ||
       warp_topk2_pruned<KP>(key_c, key_r, k_c, k_r, n, lane, a.nwords, scratch, words_c, words_r);
-  if (!done) {
-    uint32_t kc[KP], kr[KP];
-#pragma unroll
-    for (int t = 0; t < KP; ++t) {
-      kc[t] = key_c(t);
-      kr[t] = key_r(t);
-    }
-    constexpr int NO = (KP + 31) / 32;
-    uint32_t own_c[NO], own_r[NO];
-    warp_topk2<KP>(kc, kr, k_c, k_r, lane, own_c, own_r);
-    for (int w = lane; w < a.nwords; w += 32) {
-      const bool mine = w < KP;  // word w is owned by lane w % 32 as own[w / 32]
-      words_c[w] = mine ? own_c[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
-      words_r[w] = mine ? own_r[(w >> 5) < NO ? (w >> 5) : 0] : 0u;
-    }
-    __syncwarp();
-  }
+  if (!done) select_row_full<KP>(key_c, key_r, k_c, k_r, lane, a.nwords, words_c, words_r);
   emit_row(a, words_c, words_r, row, lane, gi);
 }
 
