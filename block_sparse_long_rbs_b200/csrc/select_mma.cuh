@@ -1,5 +1,6 @@
 // Two-branch selection in three kernels (the mean-query scores on the tensor
-// core), used when the caller's workspace holds the score matrix:
+// core), used when the caller's workspace holds the score matrix, after
+// select_prep_kernel (beta, and the centroids' bf16 hi / lo parts):
 //
 //   pool_split_kernel   qbar_i = mean of query block i's queries for every
 //                       (batch, q head), streamed from HBM through a 4-stage
@@ -14,7 +15,8 @@
 //                       products hi.hi + lo.hi + hi.lo accumulated in fp32;
 //                       eight epilogue warps (two per TMEM lane quarter, one
 //                       key block per thread, half the columns each) write
-//                       the scores to the workspace.
+//                       the scores to the workspace.  Persistent CTAs take
+//                       the items in a snake over the longest-first order.
 //   topk_rows_kernel    one warp per row: both branches' exact top-k
 //                       (select_row) from the stored scores, the rescue score
 //                       s_r = s_c + |qbar| r_j beta_j formed on the fly; or,
@@ -22,9 +24,9 @@
 //                       as select_tokmax_kernel stored them.
 //
 // ([RBS-en] "The Fix: A Radius-Adaptive Rescue Branch"; [RBS-id]
-// "Dual-Branch Selection".)  The mask words and counts they leave are the
-// ones the fused select_rows_kernel writes; the scan and the compaction
-// follow unchanged.
+// "Dual-Branch Selection".)  The mask words, counts and tile sums they leave
+// are the ones the fused select_rows_kernel writes; the tile scan and the
+// compaction follow unchanged.
 #pragma once
 
 #include "common.cuh"
