@@ -243,14 +243,21 @@ SelectLayout select_layout(int64_t B, int64_t Hq, int64_t nqb, int64_t Hkv, int6
 
 // Both branches' top-k of every row from the stored scores or keys, kTopkWarps
 // rows per CTA, with as many key slots per lane as the longest row needs.
-void launch_topk_rows(const TopkArgs& t, int64_t nkb, rbs_stream_t stream) {
+void launch_topk_rows(const TopkArgs& t0, int64_t nkb, rbs_stream_t stream) {
+  TopkArgs t = t0;
   const size_t tsm = topk_smem_bytes(t.nkbp, t.s.nwords);
-  const unsigned tgrid = static_cast<unsigned>((t.rows + kTopkWarps - 1) / kTopkWarps);
+  t.nhg = (t.s.Hq + kTopkWarps - 1) / kTopkWarps;
+  t.inv_nhg = 1.0f / static_cast<float>(t.nhg);
+  t.inv_g = 1.0f / static_cast<float>(t.s.Hq / t.s.Hkv);
   constexpr int kThreads = kTopkWarps * 32;
-  if (nkb <= 64) topk_rows_kernel<2><<<tgrid, kThreads, tsm, stream>>>(t);
-  else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, kThreads, tsm, stream>>>(t);
-  else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, kThreads, tsm, stream>>>(t);
-  else topk_rows_kernel<64><<<tgrid, kThreads, tsm, stream>>>(t);
+  for (int y0 = 0; y0 < t.s.nqb; y0 += 65535) {
+    t.y0 = y0;
+    const dim3 tgrid(static_cast<unsigned>(t.s.B * t.nhg), static_cast<unsigned>(std::min(65535, t.s.nqb - y0)));
+    if (nkb <= 64) topk_rows_kernel<2><<<tgrid, kThreads, tsm, stream>>>(t);
+    else if (nkb <= 256) topk_rows_kernel<8><<<tgrid, kThreads, tsm, stream>>>(t);
+    else if (nkb <= 1024) topk_rows_kernel<32><<<tgrid, kThreads, tsm, stream>>>(t);
+    else topk_rows_kernel<64><<<tgrid, kThreads, tsm, stream>>>(t);
+  }
 }
 
 // Per-token-max selection scores (query_pool TOKEN_MAX): split the centroids

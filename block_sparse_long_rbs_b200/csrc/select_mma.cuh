@@ -407,6 +407,12 @@ struct TopkArgs {
   // both branches' scores (per-token-max scoring), or null
   const uint32_t* keys;
   int nkbp, rows;
+  // grid (B * nhg, nqb): x = (batch, group of kTopkWarps q heads), y = the
+  // query block counted from the last; reciprocals for exact small-integer
+  // division, (x + 0.5) * (1 / d) (launch_topk_rows sets these)
+  int nhg;
+  float inv_nhg, inv_g;
+  int y0;  // the query-block index (from the last) of blockIdx.y = 0 (launches of at most 65535 rows of the grid)
 };
 
 // Rows (one warp each) per CTA of topk_rows_kernel.  The kernel is bound by
@@ -426,14 +432,15 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(TopkArgs t) 
   extern __shared__ __align__(16) float topk_smem[];
   const SelectArgs& a = t.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int w = blockIdx.x * kTopkWarps + warp;
-  if (w >= t.rows) return;
-  // rows with the last query blocks (the longest) first
-  const int per_i = a.B * a.Hq;
-  const int i = a.nqb - 1 - w / per_i;
-  const int bh = w % per_i;
-  const int b = bh / a.Hq, hq = bh % a.Hq;
-  const int kvh = hq / (a.Hq / a.Hkv);
+  // rows with the last query blocks (the longest) first; no integer
+  // division: (x + 0.5) / d is at least 0.5 / d from the next integer, far
+  // beyond the float error for these sizes
+  const int bx = static_cast<int>(blockIdx.x);
+  const int b = __float2int_rz((static_cast<float>(bx) + 0.5f) * t.inv_nhg);
+  const int hq = (bx - b * t.nhg) * kTopkWarps + warp;
+  if (hq >= a.Hq) return;
+  const int i = a.nqb - 1 - (t.y0 + static_cast<int>(blockIdx.y));
+  const int kvh = __float2int_rz((static_cast<float>(hq) + 0.5f) * t.inv_g);
   const int gi = i + a.q_block_offset;
   const int n = a.causal ? min(a.nkb, gi + 1) : a.nkb;
   const int64_t row = (static_cast<int64_t>(b) * a.Hq + hq) * a.nqb + i;
